@@ -1,0 +1,312 @@
+"""CPU oracle for the SLA2 / SLA sparse-linear attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+CPU-baseline / reference leg may import this module.  The library
+(sparse_linear_attention_b200) never imports it and shares no code with it.
+
+Plain, slow and written to be checked by eye against the pages:
+
+  [SLA2-sum]  "SLA2: Sparse-Linear Attention with Learnable Routing and QAT"
+              (gist.science summary), section 2 "Methodology: SLA2".
+  [SLA2-deep] "SLA2 深度解读：97% 稀疏、18.7 倍注意力加速，它和 DeepSeek DSA 的可学习
+              Indexer 到底差在哪" (jefxiong.cn), sections 04 (formulation),
+              05 (learnable router), 07 (QAT), 08 (inference kernel).
+  [SLA]       "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+              Sparse-Linear Attention" (papernotes.org), 方法详解 / 关键设计 2
+              (compressed map and three labels), 3 (linear branch and Proj),
+              4 (fused kernel), 损失函数/训练策略 (phi, k_h, k_l, block sizes).
+
+Precision.  Attention arithmetic is fp64 on the exact values of the input bytes.
+The router is fixed-order fp32 (below) because a hard top-k must be reproduced
+bit for bit; every fp32 step is one IEEE round-to-nearest-even operation:
+  pooled mean : sum tokens in ascending order from +0.0, then divide by count;
+  projection  : y[c] = sum_e fl(xbar[e] * W[e,c]), e ascending, from +0.0
+                (product rounded, then sum rounded: no fused multiply-add);
+  score       : s[i,j] = sum_c fl(qt[i,c] * kt[j,c]), c ascending, from +0.0.
+Neither 1/sqrt(d) nor the softmax of the SLA compressed map is applied before
+ranking: both are strictly increasing per row, so they cannot change a top-k.
+
+Block conventions.  Query block i holds tokens [i*bq, min((i+1)*bq, N)), key
+block j holds [j*bkv, min((j+1)*bkv, N)).  Tokens past N do not exist: they are
+left out of every mean, softmax and sum.
+
+Every function here has pins in tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F32 = np.float32
+F64 = np.float64
+
+
+# ----------------------------------------------------------------------------
+# Router  [SLA2-deep §05], [SLA 关键设计 2], [SLA2-sum §2.B]
+# ----------------------------------------------------------------------------
+
+def keep_count(ratio: float, n_kv: int) -> int:
+    """Blocks kept per row for a keep fraction "k%" [SLA2-deep §05]: the pages
+    give only the percentage, so this reads it as round-half-up(ratio*n_kv),
+    at least 1 when ratio > 0, clamped to [0, n_kv]."""
+    if ratio <= 0.0:
+        return 0
+    k = int(math.floor(ratio * n_kv + 0.5))
+    return max(1, min(n_kv, k))
+
+
+def pool_blocks(x32: np.ndarray, b: int) -> np.ndarray:
+    """Block mean-pooling pool(X) [SLA2-deep §05, SLA 关键设计 2].
+
+    x32: float32 [B,H,N,d] -> float32 [B,H,ceil(N/b),d], fixed-order fp32.
+    """
+    x32 = np.asarray(x32, dtype=F32)
+    B, H, N, d = x32.shape
+    nb = -(-N // b)
+    acc = np.zeros((B, H, nb, d), dtype=F32)
+    counts = np.array([min((i + 1) * b, N) - i * b for i in range(nb)], dtype=np.int64)
+    for t in range(b):
+        live = np.nonzero(counts > t)[0]          # blocks that have a token at offset t
+        rows = live * b + t
+        acc[:, :, live, :] = acc[:, :, live, :] + x32[:, :, rows, :]
+    return acc / counts.astype(F32)[None, None, :, None]
+
+
+def project(xbar32: np.ndarray, w32) -> np.ndarray:
+    """Learnable projection proj(X) = X W (no bias) [SLA2-deep §05]; W = None is
+    the identity, which turns the router into SLA's pooled heuristic."""
+    if w32 is None:
+        return np.array(xbar32, dtype=F32, copy=True)
+    xbar32 = np.asarray(xbar32, dtype=F32)
+    w32 = np.asarray(w32, dtype=F32)
+    d = xbar32.shape[-1]
+    acc = np.zeros(xbar32.shape[:-1] + (w32.shape[1],), dtype=F32)
+    for e in range(d):
+        acc = acc + xbar32[..., e:e + 1] * w32[e, :]
+    return acc
+
+
+def block_scores(qt32: np.ndarray, kt32: np.ndarray) -> np.ndarray:
+    """Compressed score map P_c = proj_q(Qbar) proj_k(Kbar)^T [SLA2-deep §05],
+    fixed-order fp32, without the monotone 1/sqrt(d) and softmax of
+    [SLA 关键设计 2].  qt32 [B,H,nq,d], kt32 [B,H,nkv,d] -> [B,H,nq,nkv]."""
+    qt32 = np.asarray(qt32, dtype=F32)
+    kt32 = np.asarray(kt32, dtype=F32)
+    d = qt32.shape[-1]
+    acc = np.zeros(qt32.shape[:-1] + (kt32.shape[-2],), dtype=F32)
+    for c in range(d):
+        acc = acc + qt32[..., :, c, None] * kt32[..., None, :, c]
+    return acc
+
+
+def rank_order(scores: np.ndarray) -> np.ndarray:
+    """Per row, key-block indices from best to worst: score descending, lower
+    index first among equal scores (the pages do not say how ties break)."""
+    return np.argsort(-scores, axis=-1, kind="stable")
+
+
+def topk_blocks(scores: np.ndarray, k: int) -> np.ndarray:
+    """Hard Top-k(k%, P_c) block mask as kept indices [SLA2-deep §05], ascending.
+    Returns int32 [..., k]."""
+    order = rank_order(scores)[..., :k]
+    return np.sort(order, axis=-1).astype(np.int32)
+
+
+def three_way_labels(scores: np.ndarray, k_h: int, k_l: int) -> np.ndarray:
+    """SLA labels [SLA 关键设计 2]: top k_h blocks of each row critical (+1),
+    bottom k_l negligible (-1), the rest marginal (0).  int8 [..., nkv]."""
+    n_kv = scores.shape[-1]
+    if k_h + k_l > n_kv:
+        raise ValueError("k_h + k_l exceeds the number of key blocks")
+    order = rank_order(scores)
+    lab = np.zeros(scores.shape, dtype=np.int8)
+    np.put_along_axis(lab, order[..., :k_h], np.int8(1), axis=-1)
+    if k_l > 0:
+        np.put_along_axis(lab, order[..., n_kv - k_l:], np.int8(-1), axis=-1)
+    return lab
+
+
+def route(q, k, wq, wk, bq, bkv, mode="sla2", k_keep=0, k_neg=0):
+    """Whole router: pool, project, score, select.  q, k: float32 views of the
+    input bytes [B,H,N,d].  Returns (kept int32 [B,H,nq,k_keep] ascending,
+    labels int8 [B,H,nq,nkv], scores float32 [B,H,nq,nkv]).  For mode "sla2"
+    labels are 1 on kept blocks and 0 elsewhere; for "sla" kept lists the
+    critical blocks."""
+    qt = project(pool_blocks(q, bq), wq)
+    kt = project(pool_blocks(k, bkv), wk)
+    s = block_scores(qt, kt)
+    if mode == "sla2":
+        kept = topk_blocks(s, k_keep)
+        lab = np.zeros(s.shape, dtype=np.int8)
+        if k_keep > 0:
+            np.put_along_axis(lab, kept.astype(np.int64), np.int8(1), axis=-1)
+        return kept, lab, s
+    lab = three_way_labels(s, k_keep, k_neg)
+    kept = topk_blocks(s, k_keep)
+    return kept, lab, s
+
+
+# ----------------------------------------------------------------------------
+# Feature map phi  [SLA 损失函数/训练策略, SLA 关键设计 3]
+# ----------------------------------------------------------------------------
+
+def phi(x: np.ndarray, kind: str = "elu1") -> np.ndarray:
+    """Linear-attention feature map.  "elu1": ELU(x)+1 = x+1 for x>0, exp(x)
+    otherwise.  "softmax": softmax over the channel axis of each token."""
+    x = np.asarray(x, dtype=F64)
+    if kind == "elu1":
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    if kind == "softmax":
+        e = np.exp(x - x.max(axis=-1, keepdims=True))
+        return e / e.sum(axis=-1, keepdims=True)
+    raise ValueError(kind)
+
+
+# ----------------------------------------------------------------------------
+# Attention branches (fp64)
+# ----------------------------------------------------------------------------
+
+def _rows(i, b, N):
+    return np.arange(i * b, min((i + 1) * b, N))
+
+
+def _tokens_of(blocks, b, N):
+    if len(blocks) == 0:
+        return np.zeros(0, dtype=np.int64)
+    return np.concatenate([_rows(int(j), b, N) for j in blocks])
+
+
+def sparse_branch(q, k, v, rows, keys):
+    """O_s = P_s V with P_s the softmax of Q K^T/sqrt(d) over the selected keys
+    only, i.e. P_1 renormalised per row [SLA2-deep §04, §08].  No selected key
+    -> O_s = 0."""
+    d = q.shape[-1]
+    if len(keys) == 0:
+        return np.zeros((len(rows), v.shape[-1]), dtype=F64)
+    s = (q[rows] @ k[keys].T) / math.sqrt(d)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ v[keys]
+
+
+def linear_branch(q, k, v, rows, keys, phi_kind="elu1"):
+    """O_l = phi(Q) H / (phi(Q) Z) with H = sum phi(K_m)^T V_m and Z = sum phi(K_m)
+    over the given (unselected) keys [SLA 关键设计 3], summed directly.  No key ->
+    O_l = 0."""
+    if len(keys) == 0:
+        return np.zeros((len(rows), v.shape[-1]), dtype=F64)
+    pk = phi(k[keys], phi_kind)
+    Hm = pk.T @ v[keys]            # [d, dv]
+    Z = pk.sum(axis=0)             # [d]
+    pq = phi(q[rows], phi_kind)
+    return (pq @ Hm) / (pq @ Z)[:, None]
+
+
+def _blocks_to_do(B, H, nq, blocks):
+    if blocks is None:
+        return [(b, h, i) for b in range(B) for h in range(H) for i in range(nq)]
+    return list(blocks)
+
+
+def sla2_forward(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None):
+    """SLA2 output O = alpha*O_s + (1-alpha)*O_l [SLA2-deep §04, SLA2-sum §2.A],
+    alpha per (batch, head, query block) as in the kernel description
+    [SLA2-deep §08].  O_s runs over the kept key blocks, O_l over all others.
+
+    q, k, v: float64 [B,H,N,d]; kept: int [B,H,nq,k]; alpha: [B,H,nq].
+    blocks: optional list of (b,h,i) to compute (others stay NaN).
+    Returns dict with "o", "o_s", "o_l" (float64 [B,H,N,d])."""
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    n_kv = -(-N // bkv)
+    out = {n: np.full(v.shape, np.nan) for n in ("o", "o_s", "o_l")}
+    for (b, h, i) in _blocks_to_do(B, H, nq, blocks):
+        rows = _rows(i, bq, N)
+        sel = sorted(int(j) for j in kept[b, h, i])
+        uns = [j for j in range(n_kv) if j not in set(sel)]
+        qs, ks, vs = q[b, h], k[b, h], v[b, h]
+        o_s = sparse_branch(qs, ks, vs, rows, _tokens_of(sel, bkv, N))
+        o_l = linear_branch(qs, ks, vs, rows, _tokens_of(uns, bkv, N), phi_kind)
+        a = float(alpha[b, h, i])
+        out["o_s"][b, h, rows] = o_s
+        out["o_l"][b, h, rows] = o_l
+        out["o"][b, h, rows] = a * o_s + (1.0 - a) * o_l
+    return out
+
+
+def sla_forward(q, k, v, labels, wproj, bq, bkv, phi_kind="elu1", blocks=None):
+    """SLA output O = O_s + Proj(O_l) [SLA 关键设计 3]: sparse softmax over the
+    critical blocks (+1), linear attention over the marginal blocks (0),
+    negligible blocks (-1) skipped [SLA 关键设计 2].  Proj(x) = x @ wproj with
+    wproj [d_in, d_out], no bias, shared by all heads.  Same layout as
+    sla2_forward."""
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    wp = np.asarray(wproj, dtype=F64)
+    out = {n: np.full(v.shape, np.nan) for n in ("o", "o_s", "o_l")}
+    for (b, h, i) in _blocks_to_do(B, H, nq, blocks):
+        rows = _rows(i, bq, N)
+        lab = labels[b, h, i]
+        crit = [int(j) for j in np.nonzero(lab == 1)[0]]
+        marg = [int(j) for j in np.nonzero(lab == 0)[0]]
+        qs, ks, vs = q[b, h], k[b, h], v[b, h]
+        o_s = sparse_branch(qs, ks, vs, rows, _tokens_of(crit, bkv, N))
+        o_l = linear_branch(qs, ks, vs, rows, _tokens_of(marg, bkv, N), phi_kind)
+        out["o_s"][b, h, rows] = o_s
+        out["o_l"][b, h, rows] = o_l
+        out["o"][b, h, rows] = o_s + o_l @ wp
+    return out
+
+
+# ----------------------------------------------------------------------------
+# FP8 e4m3 codec (OCP 8-bit floating point spec, E4M3: bias 7, no infinities,
+# max finite 448, NaN = S.1111.111), round to nearest even, saturating.
+# ----------------------------------------------------------------------------
+
+def e4m3_encode(x32: np.ndarray) -> np.ndarray:
+    """float32 -> uint8 e4m3 codes, round-to-nearest-even, finite values beyond
+    448 saturate to +-448, NaN -> 0x7F with the sign bit."""
+    x = np.asarray(x32, dtype=F32).astype(F64)
+    sign = np.signbit(x).astype(np.uint8) << 7
+    a = np.abs(x)
+    code = np.zeros(x.shape, dtype=np.uint8)
+    nan = np.isnan(a)
+    sat = (~nan) & (a >= 448.0)
+    sub = (~nan) & (~sat) & (a < 2.0 ** -6)
+    nor = (~nan) & (~sat) & (~sub)
+    # subnormals (and zero): multiples of 2^-9, code = m, m in 0..8 (8 -> min normal)
+    m_sub = np.rint(a[sub] / 2.0 ** -9).astype(np.int64)
+    code[sub] = m_sub.astype(np.uint8)
+    # normals: a = f * 2^e with f in [1,2)
+    fr, ex = np.frexp(a[nor])          # a = fr * 2^ex, fr in [0.5, 1)
+    e = ex - 1
+    f = fr * 2.0
+    q = np.rint((f - 1.0) * 8.0).astype(np.int64)
+    carry = q == 8
+    e = np.where(carry, e + 1, e)
+    q = np.where(carry, 0, q)
+    big = e > 8                        # cannot happen for a < 448, kept for clarity
+    c = ((e + 7) << 3) | q
+    c = np.where(big, 0x7E, c)
+    code[nor] = c.astype(np.uint8)
+    code[sat] = 0x7E
+    code[nan] = 0x7F
+    return code | sign
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    """uint8 e4m3 codes -> float64 values."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return s * val
+
+
+def e4m3_round(x32: np.ndarray) -> np.ndarray:
+    """Value of x after an e4m3 round trip, float64."""
+    return e4m3_decode(e4m3_encode(x32))

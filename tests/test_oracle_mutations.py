@@ -1,0 +1,53 @@
+"""Each pin set must catch a plausible mistake planted in the oracle.
+
+A mutation is a textual edit of oracle/sla_oracle.py, executed as a separate
+module on the CPU; the real oracle is untouched.  Every mutation must make at
+least one pin fail.
+"""
+import os
+import types
+
+import pytest
+
+from tests.oracle_pins import ALL_PINS
+
+SRC = open(os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "sla_oracle.py")).read()
+
+MUTATIONS = {
+    "phi_drops_plus_one": ("np.where(x > 0, x + 1.0, np.exp", "np.where(x > 0, x, np.exp"),
+    "sparse_no_sqrt_d": ("(q[rows] @ k[keys].T) / math.sqrt(d)", "(q[rows] @ k[keys].T)"),
+    "linear_H_transposed": ("Hm = pk.T @ v[keys]", "Hm = (pk.T @ v[keys]).T"),
+    "linear_no_denominator": ("(pq @ Hm) / (pq @ Z)[:, None]", "(pq @ Hm)"),
+    "alpha_swapped": ("a * o_s + (1.0 - a) * o_l", "(1.0 - a) * o_s + a * o_l"),
+    "pool_divides_by_block_size": ("return acc / counts.astype(F32)[None, None, :, None]",
+                                   "return acc / F32(b)"),
+    "project_uses_W_transpose": ("xbar32[..., e:e + 1] * w32[e, :]", "xbar32[..., e:e + 1] * w32[:, e]"),
+    "ties_prefer_higher_index": ('return np.argsort(-scores, axis=-1, kind="stable")',
+                                 'return scores.shape[-1] - 1 - np.argsort(-scores[..., ::-1], axis=-1, kind="stable")'),
+    "negligible_taken_from_top": ("order[..., n_kv - k_l:]", "order[..., k_h:k_h + k_l]"),
+    "sla_proj_transposed": ("o_s + o_l @ wp", "o_s + o_l @ wp.T"),
+    "sla_linear_includes_negligible": ("np.nonzero(lab == 0)", "np.nonzero(lab <= 0)"),
+    "keep_count_truncates": ("ratio * n_kv + 0.5", "ratio * n_kv"),
+    "e4m3_truncates": ("q = np.rint((f - 1.0) * 8.0)", "q = np.floor((f - 1.0) * 8.0)"),
+    "unselected_uses_kept": ("uns = [j for j in range(n_kv) if j not in set(sel)]",
+                             "uns = [j for j in range(n_kv)]"),
+}
+
+
+def _mutant(old, new):
+    assert SRC.count(old) == 1, old
+    mod = types.ModuleType("sla_oracle_mutant")
+    exec(compile(SRC.replace(old, new), "sla_oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name):
+    mod = _mutant(*MUTATIONS[name])
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(mod)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutation {name}"
