@@ -1,0 +1,168 @@
+/*
+ * sla.h -- C ABI of libsla: SLA2 / SLA sparse-linear attention forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The pages this follows:
+ *   [SLA2-deep] "SLA2 深度解读：97% 稀疏、18.7 倍注意力加速，它和 DeepSeek DSA 的可学习
+ *               Indexer 到底差在哪" (jefxiong.cn), sections 04 (formulation),
+ *               05 (learnable router), 07 (QAT), 08 (inference kernel).
+ *   [SLA2-sum]  "SLA2: Sparse-Linear Attention with Learnable Routing and QAT"
+ *               (gist.science), section 2 "Methodology: SLA2".
+ *   [SLA]       "SLA: Beyond Sparsity in Diffusion Transformers via
+ *               Fine-Tunable Sparse-Linear Attention" (papernotes.org),
+ *               关键设计 2 (compressed map, three labels), 3 (linear branch,
+ *               O = O_s + Proj(O_l)), 4 (fused kernel).
+ *
+ * Conventions for every entry point
+ *   - Q, K, V are contiguous [B, H, N, d] (row-major, d fastest) in device
+ *     memory, dtype SLA_BF16 or SLA_F32, base addresses 16-byte aligned.
+ *     Query block i holds tokens [i*bq, min((i+1)*bq, N)); key block j holds
+ *     [j*bkv, min((j+1)*bkv, N)); tokens past N do not exist (ragged last
+ *     blocks are masked, never padded).
+ *   - Ownership: the caller allocates and owns every buffer (inputs, outputs
+ *     and the workspace `ws`).  The library allocates nothing, frees nothing,
+ *     keeps no state between calls and does not synchronise the stream
+ *     (except sla_read_device_status).  Every call only enqueues kernels on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Errors: invalid arguments are reported before anything is launched
+ *     (SLA_ERR_INVALID_ARG, SLA_ERR_UNSUPPORTED, SLA_ERR_ALIGNMENT,
+ *     SLA_ERR_WORKSPACE).  A failed launch returns SLA_ERR_CUDA.  Errors found
+ *     on the device (a bounded wait that ran out, an out-of-range block index)
+ *     are written to a status word in `ws` and read with
+ *     sla_read_device_status.  No call traps, asserts or hangs the device.
+ *   - Supported: 8 <= d <= 128 with d % 8 == 0; bq in {64, 128}; bkv == 64;
+ *     1 <= N <= 131072; B*H >= 1.
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad enum value */
+  SLA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported set above */
+  SLA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+  SLA_ERR_WORKSPACE = 4,     /* ws too small (see sla_workspace_size) */
+  SLA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  SLA_ERR_TIMEOUT = 6,       /* device: a bounded wait ran out */
+  SLA_ERR_DEVICE_INDEX = 7   /* device: a block index out of [0, n_kv) */
+} sla_status;
+
+typedef enum { SLA_F32 = 0, SLA_BF16 = 1 } sla_dtype;
+
+/* Linear-attention feature map phi [SLA 损失函数/训练策略, 关键设计 3]:
+ * ELU(x)+1, or a softmax over the d channels of each token. */
+typedef enum { SLA_PHI_ELU1 = 0, SLA_PHI_SOFTMAX = 1 } sla_phi;
+
+/* Router output kind: SLA2 hard top-k [SLA2-deep §05], or SLA's three labels
+ * critical / marginal / negligible [SLA 关键设计 2]. */
+typedef enum { SLA_MODE_SLA2_TOPK = 0, SLA_MODE_SLA_3WAY = 1 } sla_route_mode;
+
+/* flags for the attention entry points */
+#define SLA_FLAG_PREPARED 1u  /* ws already holds sla_prepare's results for these K, V */
+#define SLA_FLAG_FP8 2u       /* low-bit (e4m3) sparse branch [SLA2-deep §07]; reserved */
+
+typedef struct {
+  int B, H, N, d;   /* batch, heads, tokens, head dim */
+  int bq, bkv;      /* query / key block sizes (tokens) */
+  int in_dtype;     /* sla_dtype of Q, K, V */
+} sla_shape;
+
+/* Human-readable name of a status code (static storage). */
+const char* sla_status_string(sla_status s);
+
+/* One line on the last host-side failure of this thread (which argument was
+ * rejected, or which CUDA call failed and why); "" if none yet. */
+const char* sla_last_error_detail(void);
+
+/* Blocks kept per query block for a keep fraction "k%" [SLA2-deep §05]:
+ * round-half-up(ratio * n_kv), at least 1 when ratio > 0, clamped to
+ * [0, n_kv].  (The pages give only the percentage.) */
+int sla_keep_count(double ratio, int n_kv);
+
+/* Bytes of device workspace the calls below need for this shape and mode.
+ * Returns 0 for an invalid shape.  One workspace serves sla_route,
+ * sla_prepare and the attention calls; calls that share it must be ordered
+ * on one stream. */
+size_t sla_workspace_size(const sla_shape* shape, int mode);
+
+/* Zero the workspace's device status word (enqueued on stream).  Call once
+ * after allocating ws (a zero-filled allocation also works). */
+sla_status sla_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Router [SLA2-deep §05; SLA 关键设计 2; SLA2-sum §2.B]:
+ *   Qbar = pool_bq(Q), Kbar = pool_bkv(K)          (block means, valid tokens)
+ *   Qt = Qbar Wq, Kt = Kbar Wk                     (Wq, Wk: d x d row-major fp32,
+ *                                                   shared by all heads; NULL =
+ *                                                   identity = SLA heuristic)
+ *   s[i,j] = Qt_i . Kt_j
+ * then per query block i, with key blocks ordered by (s desc, index asc):
+ *   SLA2: the first k_keep are kept;
+ *   SLA : the first k_keep are critical (+1), the last k_neg negligible (-1).
+ * All of this is fixed-order fp32 (sums in ascending index order from +0.0,
+ * each multiply and add rounded separately, no fused multiply-add), so the
+ * selection is reproducible bit for bit.  The 1/sqrt(d) and softmax of SLA's
+ * compressed map are not applied: both are monotone per row.
+ * Outputs (device):
+ *   kept_idx   int32 [B,H,n_q,k_keep], ascending per row (k_keep may be 0)
+ *   labels     int8  [B,H,n_q,n_kv] (nullable): SLA2 1/0; SLA +1/0/-1
+ *   scores_dbg fp32  [B,H,n_q,n_kv] (nullable): the raw scores s
+ * Requires n_kv <= 2048 and k_keep + k_neg <= n_kv (k_neg = 0 for SLA2). */
+sla_status sla_route(const sla_shape* shape, const void* q, const void* k,
+                     const float* Wq, const float* Wk, int mode, int k_keep,
+                     int k_neg, int32_t* kept_idx, int8_t* labels,
+                     float* scores_dbg, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Linear-branch totals [SLA 关键设计 3, 4; SLA2-deep §08]: per (b,h)
+ *   H_tot = sum_n phi(k_n)^T v_n  (d x d),  Z_tot = sum_n phi(k_n)  (d)
+ * over all N tokens, plus the per-token phi(K) and V staged in ws for the
+ * attention kernel.  The attention calls run this themselves unless
+ * SLA_FLAG_PREPARED is passed.  K, V as in the conventions. */
+sla_status sla_prepare(const sla_shape* shape, const void* k, const void* v,
+                       int phi, void* ws, size_t ws_bytes, void* stream);
+
+/* SLA2 attention forward [SLA2-deep §04, §08; SLA2-sum §2.A]:
+ *   O_s = softmax over the kept key blocks of Q K^T / sqrt(d), times V
+ *   O_l = phi(Q) H_i / (phi(Q) Z_i),  H_i, Z_i over the key blocks not kept
+ *   O   = alpha_i * O_s + (1 - alpha_i) * O_l
+ * kept_idx: int32 [B,H,n_q,k_keep], ascending per row, values in [0, n_kv)
+ *   (as written by sla_route).  k_keep == 0 -> O_s = 0; k_keep == n_kv ->
+ *   O_l = 0.
+ * alpha: fp32 [B,H,n_q], one mixing ratio per query block, already in [0,1].
+ * out: [B,H,N,d] of out_dtype (SLA_F32 or SLA_BF16), fully overwritten.
+ * flags: SLA_FLAG_PREPARED to skip the sla_prepare step. */
+sla_status sla2_attn_fwd(const sla_shape* shape, const void* q, const void* k,
+                         const void* v, const int32_t* kept_idx, int k_keep,
+                         const float* alpha, int phi, unsigned flags,
+                         void* out, int out_dtype, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* SLA attention forward [SLA 关键设计 2, 3, 4]:
+ *   O_s = softmax attention over the critical blocks (label +1)
+ *   O_l = linear attention over the marginal blocks (label 0); negligible
+ *         blocks (label -1) are skipped
+ *   O   = O_s + O_l W_proj,  W_proj bf16 [d_in][d_out] row-major, no bias
+ * labels: int8 [B,H,n_q,n_kv] with values in {-1, 0, 1} (any counts per row).
+ * ws must be sized with mode SLA_MODE_SLA_3WAY.  Other arguments as above. */
+sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k,
+                        const void* v, const int8_t* labels, const void* Wproj,
+                        int phi, unsigned flags, void* out, int out_dtype,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then return (and clear) the device status word that
+ * kernels write when a bounded wait runs out or a block index is out of
+ * range.  SLA_OK when no device error happened. */
+sla_status sla_read_device_status(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

@@ -1,0 +1,322 @@
+// prepare.cu -- linear-branch totals and the operand staging of the attention
+// kernel.
+//
+// "SLA: Beyond Sparsity in Diffusion Transformers …" (papernotes.org) 关键设计 3
+// defines the linear branch through H_i = sum_j phi(K_j)^T V_j and
+// Z_i = sum_j colsum phi(K_j) over the marginal blocks; 关键设计 4 precomputes
+// the per-block h_j, z_j.  Here the totals over all N tokens are formed once
+// per (b,h); the attention kernel subtracts the blocks it does not treat
+// linearly.  "SLA2 深度解读 …" (jefxiong.cn) §08 describes the same aggregation
+// of (K^phi)^T V for the blocks the mask misses.
+//
+// lin_prepass_kernel: per (b,h) and a contiguous range of 64-token key blocks,
+//   phi(K) -> fp16 and V -> fp16 (written to the workspace for the attention
+//   kernel, channels past d zero), and the partial sums
+//   H_part = phi(K)^T V (tcgen05, fp16 in / fp32 accumulate in TMEM) and
+//   Z_part = phi(K)^T 1 (same, against a column of ones).
+// reduce_kernel: H_tot, Z_tot = sum of the partials in split order (fixed, so
+//   deterministic).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "sla_device.cuh"
+#include "sla_internal.h"
+#include "sla_kernels.h"
+
+namespace sla {
+
+namespace {
+
+constexpr int kPreThreads = 128;
+constexpr uint32_t kTileBytes = 64 * 128 * 2;  // 64 tokens x 128 channels x 2 B
+constexpr uint32_t kOffPhi0 = 0;
+constexpr uint32_t kOffV0 = kTileBytes;
+constexpr uint32_t kBufBytes = 2 * kTileBytes;       // phi(K) + V for one buffer
+constexpr uint32_t kOffOnes = 2 * kBufBytes;          // 65536
+constexpr uint32_t kOffBar = kOffOnes + 2048;         // 2 mma barriers + done
+constexpr uint32_t kOffMisc = kOffBar + 64;           // tmem base, abort flag
+constexpr uint32_t kPreSmem = kOffMisc + 64 + 1024;   // + alignment slack
+constexpr uint32_t kPreTmemCols = 256;                // H: 0..127, Z: 128..143
+
+// 8 consecutive channels [8u, 8u+8) of token row `row` as fp32; zero past d.
+template <typename T>
+__device__ __forceinline__ void load8(const T* __restrict__ base, long long row, int d, int u, bool valid,
+                                      float* f) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+  if (!valid || 8 * u >= d) return;
+  if constexpr (sizeof(T) == 2) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(base + row * d + 8 * u));
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 p = unpack_bf162(w[i]);
+      f[2 * i] = p.x;
+      f[2 * i + 1] = p.y;
+    }
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(base + row * d + 8 * u));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(base + row * d + 8 * u + 4));
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
+    const T* __restrict__ k, const T* __restrict__ v, __half* __restrict__ phik, __half* __restrict__ v16,
+    __nv_bfloat16* __restrict__ khat, float* __restrict__ hpart, float* __restrict__ zpart, int N, int d,
+    int nkv, int nsplit, int phi_kind, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [0], [1]
+  uint64_t* done_bar = mma_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int split = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const int jb0 = static_cast<int>((static_cast<long long>(split) * nkv) / nsplit);
+  const int jb1 = static_cast<int>((static_cast<long long>(split + 1) * nkv) / nsplit);
+
+  // ones column for Z: K-major 16 x 64 tile, row 0 = 1.0, rows 1..15 = 0
+  for (int i = tid; i < 2048 / 4; i += kPreThreads) {
+    const uint32_t one2 = 0x3C003C00u;  // two fp16 ones
+    reinterpret_cast<uint32_t*>(sm + kOffOnes)[i] = (i < 32) ? one2 : 0u;
+  }
+  if (tid == 0) {
+    mbar_init(&mma_bar[0], 1);
+    mbar_init(&mma_bar[1], 1);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kPreTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const T* kb = k + bh * static_cast<long long>(N) * d;
+  const T* vb = v + bh * static_cast<long long>(N) * d;
+  __half* phib = phik + bh * static_cast<long long>(N) * kDPad;
+  __half* v16b = v16 + bh * static_cast<long long>(N) * kDPad;
+  __nv_bfloat16* khb = khat ? khat + bh * static_cast<long long>(N) * kDPad : nullptr;
+
+  const uint32_t idesc_h = idesc_f16(0, 1, 1, 128, 128);  // phi(K)^T (MN-major) x V (MN-major)
+  const uint32_t idesc_z = idesc_f16(0, 1, 0, 128, 16);   // phi(K)^T x ones (K-major)
+  bool ok = true;
+
+  for (int jb = jb0; jb < jb1; ++jb) {
+    const int it = jb - jb0;
+    const int buf = it & 1;
+    uint8_t* sphi = sm + buf * kBufBytes + kOffPhi0;
+    uint8_t* sv = sm + buf * kBufBytes + kOffV0;
+    // this thread's 8 units: row m = tid/16 + 8*i, unit u = tid % 16
+    float kf[8][8], vf[8][8];
+    const int u = tid % 16;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int m = tid / 16 + 8 * i;
+      const int tok = jb * 64 + m;
+      load8<T>(kb, tok, d, u, tok < N, kf[i]);
+      load8<T>(vb, tok, d, u, tok < N, vf[i]);
+    }
+    // buffer reuse: the MMA that read this buffer two tiles ago must be done
+    if (it >= 2) {
+      if (!mbar_wait(&mma_bar[buf], ((it - 2) >> 1) & 1, abort_flag, status)) ok = false;
+    }
+    ok = __syncthreads_and(ok) != 0;  // CTA-uniform verdict
+    if (!ok) break;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int m = tid / 16 + 8 * i;
+      const int tok = jb * 64 + m;
+      const bool valid = tok < N;
+      float ph[8];
+      if (phi_kind == SLA_PHI_SOFTMAX) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (8 * u + e < d) mx = fmaxf(mx, kf[i][e]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ph[e] = (8 * u + e < d) ? expf(kf[i][e] - mx) : 0.0f;
+          sum += ph[e];
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ph[e] *= inv;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ph[e] = (8 * u + e < d) ? elu1(kf[i][e]) : 0.0f;
+      }
+      uint4 pu, vu;
+      if (valid) {
+        pu = make_uint4(pack_half2(ph[0], ph[1]), pack_half2(ph[2], ph[3]), pack_half2(ph[4], ph[5]),
+                        pack_half2(ph[6], ph[7]));
+        vu = make_uint4(pack_half2(vf[i][0], vf[i][1]), pack_half2(vf[i][2], vf[i][3]),
+                        pack_half2(vf[i][4], vf[i][5]), pack_half2(vf[i][6], vf[i][7]));
+        const long long g = static_cast<long long>(tok) * kDPad + 8 * u;
+        *reinterpret_cast<uint4*>(phib + g) = pu;
+        *reinterpret_cast<uint4*>(v16b + g) = vu;
+        if (khb) {
+          const uint4 ku = make_uint4(pack_bf162(kf[i][0], kf[i][1]), pack_bf162(kf[i][2], kf[i][3]),
+                                      pack_bf162(kf[i][4], kf[i][5]), pack_bf162(kf[i][6], kf[i][7]));
+          *reinterpret_cast<uint4*>(khb + g) = ku;
+        }
+      } else {
+        pu = make_uint4(0, 0, 0, 0);
+        vu = pu;
+      }
+      const uint32_t off = (u >> 3) * 8192u + sw128_off(m, u & 7);
+      *reinterpret_cast<uint4*>(sphi + off) = pu;
+      *reinterpret_cast<uint4*>(sv + off) = vu;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t aphi = smem_u32(sphi), av = smem_u32(sv), aones = smem_u32(sm + kOffOnes);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = sdesc_sw128(aphi + kk * 2048, 8192, 1024);
+        const uint64_t b = sdesc_sw128(av + kk * 2048, 8192, 1024);
+        const uint64_t bo = sdesc_sw128(aones + kk * 32, 16, 1024);
+        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+        mma_f16_ss(tmem + 0, a, b, idesc_h, acc);
+        mma_f16_ss(tmem + 128, a, bo, idesc_z, acc);
+      }
+      mma_commit(&mma_bar[buf]);
+    }
+  }
+  // all MMAs of this CTA done -> read the partial sums out of TMEM
+  if (tid == 0) mma_commit(done_bar);
+  __syncwarp();
+  bool have = ok && (jb1 > jb0);
+  {
+    // warp-uniform wait: lane 0 waits, the warp follows its verdict
+    int w_ok = 0;
+    if ((tid & 31) == 0) w_ok = mbar_wait(done_bar, 0, abort_flag, status) ? 1 : 0;
+    w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+    have = have && w_ok;
+  }
+  tc_fence_after();
+  if (have) {
+    float* hp = hpart + ((bh * nsplit + split) * kDPad + tid) * kDPad;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      float x[32];
+      tmem_ld32(tmem + ((warp * 32) << 16) + cc * 32, x);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(hp + cc * 32 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+    }
+    float z[32];
+    tmem_ld32(tmem + ((warp * 32) << 16) + 128, z);
+    tmem_wait_ld();
+    zpart[(bh * nsplit + split) * kDPad + tid] = z[0];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kPreTmemCols);
+  }
+}
+
+// H_tot[bh] = sum over splits (ascending) of H_part; Z_tot likewise.
+__global__ void __launch_bounds__(256) reduce_kernel(const float* __restrict__ hpart,
+                                                     const float* __restrict__ zpart, float* __restrict__ htot,
+                                                     float* __restrict__ ztot, int BH, int nsplit) {
+  const long long per = kDPad * kDPad + kDPad;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= per * BH) return;
+  const long long bh = idx / per, r = idx % per;
+  float acc = 0.0f;
+  if (r < kDPad * kDPad) {
+    for (int s = 0; s < nsplit; ++s) acc += hpart[(bh * nsplit + s) * kDPad * kDPad + r];
+    htot[bh * kDPad * kDPad + r] = acc;
+  } else {
+    const long long e = r - kDPad * kDPad;
+    for (int s = 0; s < nsplit; ++s) acc += zpart[(bh * nsplit + s) * kDPad + e];
+    ztot[bh * kDPad + e] = acc;
+  }
+}
+
+// Q as bf16 with the head dim padded to 128 (needed when d != 128 or the
+// input is fp32).  One thread per 8 output channels.
+template <typename T>
+__global__ void __launch_bounds__(256) qhat_kernel(const T* __restrict__ q, __nv_bfloat16* __restrict__ qhat,
+                                                   long long rows, int d) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= rows * 16) return;
+  const long long row = idx / 16;
+  const int u = static_cast<int>(idx % 16);
+  float f[8];
+  load8<T>(q, row, d, u, true, f);
+  *reinterpret_cast<uint4*>(qhat + row * kDPad + 8 * u) =
+      make_uint4(pack_bf162(f[0], f[1]), pack_bf162(f[2], f[3]), pack_bf162(f[4], f[5]), pack_bf162(f[6], f[7]));
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
+                           char* ws, cudaStream_t st) {
+  const int BH = s.B * s.H;
+  const int nkv = ceil_div(s.N, s.bkv);
+  __half* phik = reinterpret_cast<__half*>(ws + L.phik);
+  __half* v16 = reinterpret_cast<__half*>(ws + L.v16);
+  __nv_bfloat16* khat = L.need_hat ? reinterpret_cast<__nv_bfloat16*>(ws + L.khat) : nullptr;
+  float* hpart = reinterpret_cast<float*>(ws + L.hpart);
+  float* zpart = reinterpret_cast<float*>(ws + L.zpart);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  dim3 grid(L.nsplit, BH);
+  cudaError_t e;
+  if (s.in_dtype == SLA_BF16) {
+    e = cudaFuncSetAttribute(lin_prepass_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPreSmem);
+    if (e != cudaSuccess) return e;
+    lin_prepass_kernel<__nv_bfloat16><<<grid, kPreThreads, kPreSmem, st>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), phik, v16, khat, hpart,
+        zpart, s.N, s.d, nkv, L.nsplit, phi, status);
+  } else {
+    e = cudaFuncSetAttribute(lin_prepass_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmem);
+    if (e != cudaSuccess) return e;
+    lin_prepass_kernel<float><<<grid, kPreThreads, kPreSmem, st>>>(
+        static_cast<const float*>(k), static_cast<const float*>(v), phik, v16, khat, hpart, zpart, s.N, s.d,
+        nkv, L.nsplit, phi, status);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n = static_cast<long long>(BH) * (kDPad * kDPad + kDPad);
+  reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      hpart, zpart, reinterpret_cast<float*>(ws + L.htot), reinterpret_cast<float*>(ws + L.ztot), BH, L.nsplit);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qhat(const sla_shape& s, const void* q, const WsLayout& L, char* ws, cudaStream_t st) {
+  const long long rows = static_cast<long long>(s.B) * s.H * s.N;
+  __nv_bfloat16* qhat = reinterpret_cast<__nv_bfloat16*>(ws + L.qhat);
+  const unsigned blocks = static_cast<unsigned>((rows * 16 + 255) / 256);
+  if (s.in_dtype == SLA_BF16)
+    qhat_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qhat, rows, s.d);
+  else
+    qhat_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(q), qhat, rows, s.d);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,74 @@
+// sla_internal.h -- definitions shared by the libsla host code and kernels.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sla.h"
+
+namespace sla {
+
+constexpr int kDPad = 128;        // head dim as stored for the tensor-core path
+constexpr int kBlockKV = 64;      // key block size (tokens)
+constexpr int kMaxNKV = 2048;     // router limit on key blocks per head
+constexpr int kMaxN = 131072;     // token limit (n_kv <= 2048 at bkv = 64)
+constexpr int kNumSMs = 148;
+
+// Device workspace layout.  All offsets are 256-byte aligned.
+struct WsLayout {
+  size_t status = 0;  // int32 status word (+ padding)
+  size_t qbar = 0, kbar = 0;  // fp32 [BH, n_q, d], [BH, n_kv, d]   pooled means
+  size_t qt = 0, kt = 0;      // fp32, same shapes                  projected
+  size_t phik = 0;            // fp16 [BH, N, 128]  phi(K), zero past d
+  size_t v16 = 0;             // fp16 [BH, N, 128]  V, zero past d
+  size_t qhat = 0, khat = 0;  // bf16 [BH, N, 128]  Q, K (only when need_hat)
+  size_t hpart = 0, zpart = 0;  // fp32 [BH, nsplit, 128, 128], [BH, nsplit, 128]
+  size_t htot = 0, ztot = 0;    // fp32 [BH, 128, 128], [BH, 128]
+  size_t lists = 0;             // SLA: int32 [BH, n_q, 2, n_kv] critical / negligible lists
+  size_t counts = 0;            // SLA: int32 [BH, n_q, 2]
+  size_t total = 0;
+  int nsplit = 1;
+  bool need_hat = false;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+inline WsLayout ws_layout(const sla_shape& s, int mode) {
+  WsLayout L;
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
+  L.need_hat = (s.d != kDPad) || (s.in_dtype == SLA_F32);
+  int ns = ceil_div(2 * kNumSMs, static_cast<int>(BH > 0 ? BH : 1));
+  L.nsplit = ns < 1 ? 1 : (ns > nkv ? nkv : ns);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.status = take(256);
+  L.qbar = take(BH * nq * s.d * 4);
+  L.kbar = take(BH * nkv * s.d * 4);
+  L.qt = take(BH * nq * s.d * 4);
+  L.kt = take(BH * nkv * s.d * 4);
+  L.phik = take(BH * s.N * kDPad * 2);
+  L.v16 = take(BH * s.N * kDPad * 2);
+  if (L.need_hat) {
+    L.qhat = take(BH * s.N * kDPad * 2);
+    L.khat = take(BH * s.N * kDPad * 2);
+  }
+  L.hpart = take(BH * L.nsplit * kDPad * kDPad * 4);
+  L.zpart = take(BH * L.nsplit * kDPad * 4);
+  L.htot = take(BH * kDPad * kDPad * 4);
+  L.ztot = take(BH * kDPad * 4);
+  if (mode == SLA_MODE_SLA_3WAY) {
+    L.lists = take(BH * nq * 2 * static_cast<size_t>(nkv) * 4);
+    L.counts = take(BH * nq * 2 * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace sla

@@ -1,0 +1,48 @@
+// sla_kernels.h -- host-side launchers of the libsla kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sla_internal.h"
+
+namespace sla {
+
+cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const float* Wq, const float* Wk,
+                         int mode, int k_keep, int k_neg, int32_t* kept_idx, int8_t* labels,
+                         float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st);
+
+cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
+                           char* ws, cudaStream_t st);
+
+cudaError_t launch_qhat(const sla_shape& s, const void* q, const WsLayout& L, char* ws, cudaStream_t st);
+
+cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, const WsLayout& L, char* ws,
+                                   cudaStream_t st);
+
+struct SparseArgs {
+  int BH, N, d, bq, nq, nkv;
+  float sl2;                 // log2(e) / sqrt(d)
+  const int32_t* crit_idx;   // per (bh, query block) row, list_stride apart: softmax blocks
+  const int32_t* negl_idx;   // same rows: blocks that only leave the linear sum (SLA); nullable
+  long long list_stride;     // elements between consecutive rows of both lists
+  int crit_max, negl_max;    // list capacities
+  const int32_t* counts;     // nullable: counts[2*row] = #crit, [2*row+1] = #negl; else crit_max, 0
+  const float* alpha;        // SLA2: [BH, nq]; null for SLA
+  const void* wproj;         // SLA: bf16 [d][d]; null for SLA2
+  const float* htot;         // [BH, 128, 128]
+  const float* ztot;         // [BH, 128]
+  void* out;
+  int out_bf16;
+  int phi;
+  int* status;
+};
+
+// 3-D tensor map over a [BH][N][128] 16-bit array: boxes of 64 channels x
+// box_rows tokens, 128-byte swizzle, rows past N read as zero.
+cudaError_t encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int N, int BH, int box_rows);
+
+cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
+                          const void* phik16, const void* v16, cudaStream_t st);
+
+}  // namespace sla

@@ -1,0 +1,138 @@
+"""libsla's C ABI on the host (no GPU): every symbol in include/sla.h is
+exported, and argument checks fail before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from oracle import sla_oracle
+from sparse_linear_attention_b200 import sla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "sla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sla\w+)\s*\(", src)))
+
+
+def test_header_matches_binding():
+    assert _header_functions() == sorted(sla.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = sla.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", sla.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (\w+)$", out, flags=re.M))
+    for name in _header_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_status_strings():
+    for code, name in sla.STATUS_NAMES.items():
+        assert sla.lib().sla_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("n_kv", [1, 7, 16, 512, 591, 1182, 2048])
+def test_keep_count_matches_oracle(n_kv):
+    for ratio in [0.0, 1e-6, 0.01, 0.03, 0.04, 0.05, 0.1, 0.25, 0.5, 0.97, 1.0, 1.5]:
+        assert sla.sla_keep_count(ratio, n_kv) == sla_oracle.keep_count(ratio, n_kv), (ratio, n_kv)
+
+
+def _shape(**kw):
+    base = dict(B=1, H=12, N=32760, d=128, bq=128, bkv=64, in_dtype=sla.SLA_BF16)
+    base.update(kw)
+    return sla.Shape(**base)
+
+
+def test_workspace_size():
+    good = _shape()
+    a = sla.sla_workspace_size(good, sla.SLA_MODE_SLA2_TOPK)
+    b = sla.sla_workspace_size(good, sla.SLA_MODE_SLA_3WAY)
+    assert 0 < a < b
+    assert a % 256 == 0
+    # phi(K) and V staged as fp16 [BH, N, 128] dominate
+    assert a >= 2 * 12 * 32760 * 128 * 2
+    for bad in [dict(d=100), dict(d=136), dict(bq=96), dict(bkv=128), dict(N=0), dict(N=131073),
+                dict(B=0), dict(in_dtype=7)]:
+        assert sla.sla_workspace_size(_shape(**bad), 0) == 0, bad
+    assert sla.sla_workspace_size(good, 5) == 0
+    # f32 inputs or d != 128 need the padded bf16 copies of Q and K
+    assert sla.sla_workspace_size(_shape(d=64), 0) > sla.sla_workspace_size(_shape(), 0) // 2
+
+
+FAKE = 0x7F0000000000  # never dereferenced: every call below fails its checks first
+
+
+def _route(shape, q=FAKE, k=FAKE, mode=0, k_keep=15, k_neg=0, kept=FAKE, ws=FAKE, ws_bytes=1 << 40):
+    return sla.lib().sla_route(ctypes.byref(shape), q, k, None, None, mode, k_keep, k_neg, kept, None, None,
+                               ws, ws_bytes, None)
+
+
+def test_route_rejects_bad_arguments_before_launch():
+    s = _shape()
+    assert _route(s, q=None) == 1
+    assert _route(s, q=FAKE + 2) == 3
+    assert _route(s, mode=3) == 1
+    assert _route(s, k_keep=513) == 1
+    assert _route(s, k_keep=-1) == 1
+    assert _route(s, k_neg=1) == 1            # SLA2 takes no negligible count
+    assert _route(s, mode=1, k_keep=300, k_neg=300) == 1
+    assert _route(s, kept=None) == 1
+    assert _route(s, ws=None) == 1
+    assert _route(s, ws=FAKE + 16) == 3       # workspace must be 256-byte aligned
+    assert _route(s, ws_bytes=1000) == 4
+    assert _route(_shape(N=131072 + 64)) == 2
+    assert _route(s, kept=None) == 1
+    assert "kept_idx" in sla.lib().sla_last_error_detail().decode()
+
+
+def test_attention_rejects_bad_arguments_before_launch():
+    s = _shape()
+    L = sla.lib()
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, kept=FAKE, k_keep=15, alpha=FAKE, phi=0, flags=0, out=FAKE, odt=1,
+                 ws=FAKE, wsb=1 << 40)
+        a.update(kw)
+        return L.sla2_attn_fwd(ctypes.byref(s), a["q"], a["k"], a["v"], a["kept"], a["k_keep"], a["alpha"],
+                               a["phi"], a["flags"], a["out"], a["odt"], a["ws"], a["wsb"], None)
+
+    assert call(v=None) == 1
+    assert call(k=FAKE + 8) == 3
+    assert call(k_keep=513) == 1
+    assert call(kept=None) == 1
+    assert call(alpha=None) == 1
+    assert call(phi=2) == 1
+    assert call(flags=8) == 1
+    assert call(flags=sla.SLA_FLAG_FP8) == 2
+    assert call(out=None) == 1
+    assert call(out=FAKE + 4) == 3
+    assert call(odt=9) == 1
+    assert call(wsb=10) == 4
+    assert "ws" in L.sla_last_error_detail().decode()
+
+    def call3(**kw):
+        a = dict(labels=FAKE, wp=FAKE, wsb=1 << 40)
+        a.update(kw)
+        return L.sla_attn_fwd(ctypes.byref(s), FAKE, FAKE, FAKE, a["labels"], a["wp"], 0, 0, FAKE, 1, FAKE,
+                              a["wsb"], None)
+
+    assert call3(labels=None) == 1
+    assert call3(wp=None) == 1
+    assert call3(wp=FAKE + 2) == 3
+    # the SLA workspace also holds the per-row block lists
+    need2 = sla.sla_workspace_size(s, 0)
+    assert call3(wsb=need2) == 4
+
+
+def test_prepare_rejects_bad_arguments_before_launch():
+    s = _shape()
+    L = sla.lib()
+    assert L.sla_prepare(ctypes.byref(s), None, FAKE, 0, FAKE, 1 << 40, None) == 1
+    assert L.sla_prepare(ctypes.byref(s), FAKE, FAKE, 5, FAKE, 1 << 40, None) == 1
+    assert L.sla_prepare(ctypes.byref(_shape(bkv=32)), FAKE, FAKE, 0, FAKE, 1 << 40, None) == 2

@@ -1,0 +1,220 @@
+"""libsla on a B200 against the CPU oracle, on the same seeded inputs.
+
+Masks and scores must match bit for bit; outputs within max-abs 2e-3 and
+relative L1 1e-2 of the fp64 oracle (bf16 tensor-core arithmetic)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import sla_oracle as orc
+from sparse_linear_attention_b200 import inputs, sla
+from tests.gpu_common import (TOL_BF16, as32, as64, compare, run_route, run_sla, run_sla2, sample_blocks)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("the gpu tests need a CUDA device")
+    sla.lib()
+
+
+_CACHE = {}
+
+
+def workload(name):
+    if name not in _CACHE:
+        w = inputs.WORKLOADS[name]
+        _CACHE[name] = (w, inputs.make_inputs(w))
+    return _CACHE[name]
+
+
+def k_of(w):
+    return w.keep_count if w.keep_count is not None else orc.keep_count(w.keep_ratio, w.n_kv)
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("name", ["tiny", "wan13", "wan14"])
+@pytest.mark.parametrize("proj", [True, False])
+def test_route_sla2_bitexact(name, proj):
+    w, x = workload(name)
+    kk = k_of(w)
+    wq, wk = (x["wq"], x["wk"]) if proj else (None, None)
+    kept, lab, sc = run_route(x["q"], x["k"], wq, wk, w.bq, w.bkv, sla.SLA_MODE_SLA2_TOPK, kk)
+    okept, olab, osc = orc.route(as32(x["q"]), as32(x["k"]), None if wq is None else wq.numpy(),
+                                 None if wk is None else wk.numpy(), w.bq, w.bkv, "sla2", kk)
+    assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32)), "scores differ"
+    assert np.array_equal(kept, okept), f"{int((kept != okept).sum())} kept indices differ"
+    assert np.array_equal(lab, olab)
+
+
+def test_route_sla_three_way_bitexact():
+    w, x = workload("sla13")
+    kh, kl = orc.keep_count(w.crit_ratio, w.n_kv), orc.keep_count(w.negl_ratio, w.n_kv)
+    kept, lab, sc = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, sla.SLA_MODE_SLA_3WAY, kh, kl)
+    okept, olab, osc = orc.route(as32(x["q"]), as32(x["k"]), x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv,
+                                 "sla", kh, kl)
+    assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32))
+    assert np.array_equal(kept, okept)
+    assert np.array_equal(lab, olab)
+    assert ((lab == 1).sum(-1) == kh).all() and ((lab == -1).sum(-1) == kl).all()
+
+
+def test_route_ties_break_to_lower_index():
+    # identical key blocks -> equal scores; the lower block index must win
+    B, H, N, d = 1, 1, 512, 64
+    q = torch.randn(B, H, N, d).to(torch.bfloat16)
+    k = torch.randn(B, H, 64, d).repeat(1, 1, N // 64, 1).to(torch.bfloat16)
+    kept, _, sc = run_route(q, k, None, None, 64, 64, 0, 3)
+    assert np.all(kept == np.arange(3))
+    assert np.all(sc == sc[..., :1])
+
+
+# ------------------------------------------------------------------ SLA2 attention
+
+def _sla2_check(w, x, kept, blocks=None, phi=sla.SLA_PHI_ELU1, out_dtype=torch.float32, tol=TOL_BF16):
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, phi, out_dtype)
+    kind = "elu1" if phi == sla.SLA_PHI_ELU1 else "softmax"
+    want = orc.sla2_forward(as64(x["q"]), as64(x["k"]), as64(x["v"]), kept, x["alpha"].numpy(), w.bq, w.bkv,
+                            kind, blocks=blocks)["o"]
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(w.n_q)]
+    return compare(got, want, blocks, w.bq, tol=tol)
+
+
+def test_sla2_tiny_all_rows():
+    w, x = workload("tiny")
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, k_of(w))
+    _sla2_check(w, x, kept)
+
+
+def test_sla2_wan13_sampled_blocks():
+    w, x = workload("wan13")
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, k_of(w))
+    _sla2_check(w, x, kept, blocks=sample_blocks(w.B, w.H, w.n_q, 4))
+
+
+def test_sla2_wan14_sampled_blocks():
+    """Full 14B-shape launch; the oracle checks 4 heads x 4 query blocks."""
+    w, x = workload("wan14")
+    kk = k_of(w)
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, kk)
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv)
+    hs = [0, 13, 26, 39]
+    sub = lambda t: t[:, hs]  # noqa: E731
+    blocks = sample_blocks(1, len(hs), w.n_q, 4, seed=1)
+    want = orc.sla2_forward(as64(sub(x["q"])), as64(sub(x["k"])), as64(sub(x["v"])), kept[:, hs],
+                            x["alpha"][:, hs].numpy(), w.bq, w.bkv, blocks=blocks)["o"]
+    compare(got[:, hs], want, blocks, w.bq)
+
+
+def _rand_case(N, d, dtype="bf16", B=1, H=2, bq=128, seed=3, scale=1.0):
+    w = inputs.Workload("case", B, H, (1, 1, N), d, bq, 64, dtype, keep_count=1)
+    x = inputs.random_inputs(B, H, N, d, dtype=dtype, seed=seed, scale=scale, n_q=w.n_q)
+    return w, x
+
+
+def _rand_kept(w, k, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.stack([np.sort(rng.choice(w.n_kv, k, replace=False)) for _ in range(w.B * w.H * w.n_q)]
+                    ).reshape(w.B, w.H, w.n_q, k).astype(np.int32)
+
+
+@pytest.mark.parametrize("N,d,bq", [(200, 128, 128), (1000, 64, 64), (777, 128, 64), (64, 128, 128),
+                                    (1, 128, 128), (4100, 96, 128)])
+def test_sla2_ragged_shapes(N, d, bq):
+    w, x = _rand_case(N, d, bq=bq, scale=1.5)
+    kk = max(1, min(3, w.n_kv - 1)) if w.n_kv > 1 else 1
+    _sla2_check(w, x, _rand_kept(w, kk))
+
+
+def test_sla2_no_block_kept_is_linear_attention():
+    w, x = _rand_case(1000, 128)
+    _sla2_check(w, x, np.zeros((1, 2, w.n_q, 0), np.int32))
+
+
+def test_sla2_every_block_kept():
+    w, x = _rand_case(1000, 128, scale=1.5)
+    kept = np.broadcast_to(np.arange(w.n_kv, dtype=np.int32), (1, 2, w.n_q, w.n_kv))
+    _sla2_check(w, x, kept)
+
+
+def test_sla2_softmax_feature_map():
+    w, x = workload("tiny")
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, k_of(w))
+    _sla2_check(w, x, kept, phi=sla.SLA_PHI_SOFTMAX)
+
+
+def test_sla2_bf16_output():
+    w, x = _rand_case(1500, 128, scale=1.5)
+    kept = _rand_kept(w, 4)
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, out_dtype=torch.bfloat16)
+    want = orc.sla2_forward(as64(x["q"]), as64(x["k"]), as64(x["v"]), kept, x["alpha"].numpy(), w.bq, w.bkv)["o"]
+    # bf16 output rounding adds up to half an ulp of |O|
+    assert np.all(np.abs(got - want) <= TOL_BF16 + np.abs(want) * 2.0 ** -8)
+
+
+def test_sla2_fp32_inputs_off_the_bf16_grid():
+    """f32 inputs are rounded to bf16 for the tensor-core stages; against the
+    oracle on the rounded values the usual bound holds."""
+    B, H, N, d = 1, 2, 900, 128
+    g = torch.Generator().manual_seed(11)
+    q, k, v = (torch.randn(B, H, N, d, generator=g) * 1.3 for _ in range(3))
+    w = inputs.Workload("f32", B, H, (1, 1, N), d, 128, 64, "f32", keep_count=3)
+    alpha = torch.rand(B, H, w.n_q, generator=g)
+    kept = _rand_kept(w, 3)
+    got = run_sla2(q, k, v, kept, alpha, 128, 64)
+    r = lambda t: t.to(torch.bfloat16).to(torch.float64).numpy()  # noqa: E731
+    want = orc.sla2_forward(r(q), r(k), v.to(torch.float64).numpy(), kept, alpha.numpy(), 128, 64)["o"]
+    compare(got, want, [(0, h, i) for h in range(H) for i in range(w.n_q)], 128)
+
+
+def test_sla2_prepared_flag_and_determinism():
+    w, x = _rand_case(3000, 128, scale=1.5)
+    kept = _rand_kept(w, 5)
+    dev = "cuda"
+    shape = sla.make_shape(x["q"].cuda(), w.bq, w.bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, 0), dtype=torch.uint8, device=dev)
+    a = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, ws=ws)
+    b = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, ws=ws, flags=sla.SLA_FLAG_PREPARED)
+    c = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert np.array_equal(a.view(np.uint32), c.view(np.uint32))
+
+
+# ------------------------------------------------------------------ SLA attention
+
+def _sla_check(w, x, labels, blocks=None):
+    got = run_sla(x["q"], x["k"], x["v"], labels, x["wproj"], w.bq, w.bkv)
+    want = orc.sla_forward(as64(x["q"]), as64(x["k"]), as64(x["v"]), labels, as64(x["wproj"]), w.bq, w.bkv,
+                           blocks=blocks)["o"]
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(w.n_q)]
+    return compare(got, want, blocks, w.bq)
+
+
+def test_sla_tiny_all_rows():
+    w, x = workload("tiny")
+    _, lab, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 1, 2, 3)
+    _sla_check(w, x, lab)
+
+
+def test_sla_wan13_sampled_blocks():
+    w, x = workload("sla13")
+    kh, kl = orc.keep_count(w.crit_ratio, w.n_kv), orc.keep_count(w.negl_ratio, w.n_kv)
+    _, lab, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 1, kh, kl)
+    _sla_check(w, x, lab, blocks=sample_blocks(w.B, w.H, w.n_q, 3, seed=2))
+
+
+def test_sla_label_edge_cases():
+    w, x = _rand_case(700, 128, scale=1.5)
+    rng = np.random.default_rng(5)
+    lab = rng.integers(-1, 2, (1, 2, w.n_q, w.n_kv)).astype(np.int8)
+    lab[0, 0, 0, :] = 1          # all critical: no linear term
+    lab[0, 0, 1, :] = 0          # all marginal: no softmax term
+    lab[0, 1, 0, :] = -1         # all negligible: output 0
+    lab[0, 1, 1, :] = 0
+    lab[0, 1, 1, 0] = -1         # marginal except one negligible block
+    _sla_check(w, x, lab)
