@@ -120,6 +120,29 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k,
                      float* scores_dbg, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* Router without a workspace.  The pages have no counterpart to this entry
+ * point: it exists for callers that cannot give the library device memory,
+ * for example code that runs under another framework's memory manager and
+ * may not allocate outside it, or that must not call cudaMalloc where it
+ * routes.  It computes exactly what sla_route computes (same kernels, same
+ * bit-exact results) with the same arguments minus ws / ws_bytes; its scratch
+ * is a 16 MiB array compiled into the library, held by every GPU that loads
+ * libsla until the process exits.
+ *   - Shapes whose scratch, 2*B*H*(n_q + n_kv)*d floats (each of the four
+ *     pieces rounded up to 256 bytes), exceeds 16 MiB are rejected with
+ *     SLA_ERR_WORKSPACE before any launch (sla_last_error_detail says how
+ *     much was needed).  The 1.3B-shape workload needs 9.4 MB.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race.  Nothing
+ *     in it needs to start at zero; each call overwrites what it reads.
+ *   - Nothing is allocated or freed. */
+sla_status sla_route_noalloc(const sla_shape* shape, const void* q, const void* k,
+                             const float* Wq, const float* Wk, int mode, int k_keep,
+                             int k_neg, int32_t* kept_idx, int8_t* labels,
+                             float* scores_dbg, void* stream);
+
 /* Linear-branch totals [SLA 关键设计 3, 4; SLA2-deep §08]: per (b,h)
  *   H_tot = sum_n phi(k_n)^T v_n  (d x d),  Z_tot = sum_n phi(k_n)  (d)
  * over all N tokens, plus the per-token phi(K) and V staged in ws for the

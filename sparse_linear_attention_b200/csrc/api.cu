@@ -34,11 +34,17 @@ cudaError_t encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType d
 
 }  // namespace sla
 
-using namespace sla;
-
 namespace {
 
 thread_local char g_detail[256] = "";
+
+}  // namespace
+
+void sla::set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+
+using namespace sla;
+
+namespace {
 
 sla_status cuda_fail(cudaError_t e, const char* where) {
   snprintf(g_detail, sizeof(g_detail), "%s: %s", where, cudaGetErrorString(e));

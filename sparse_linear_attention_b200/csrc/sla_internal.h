@@ -31,6 +31,9 @@ struct WsLayout {
   bool need_hat = false;
 };
 
+// Record the one-line detail that sla_last_error_detail() returns.
+void set_error_detail(const char* msg);
+
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
