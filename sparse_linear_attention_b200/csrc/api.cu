@@ -101,13 +101,15 @@ sla_status run_attention(const sla_shape* s, const void* q, const void* k, const
   a.nq = ceil_div(s->N, s->bq);
   a.nkv = ceil_div(s->N, s->bkv);
   a.sl2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s->d)));
-  a.htot = reinterpret_cast<const float*>(ws + L.htot);
+  a.sigma = reinterpret_cast<const float*>(ws + L.sigma);
+  a.zblk = reinterpret_cast<const float*>(ws + L.zblk);
   a.ztot = reinterpret_cast<const float*>(ws + L.ztot);
   a.phi = phi;
   a.status = reinterpret_cast<int*>(ws + L.status);
   const void* q128 = L.need_hat ? static_cast<const void*>(ws + L.qhat) : q;
   const void* k128 = L.need_hat ? static_cast<const void*>(ws + L.khat) : k;
-  if ((e = launch_sparse(a, q128, k128, ws + L.phik, ws + L.v16, st)) != cudaSuccess) return cuda_fail(e, "sparse");
+  if ((e = launch_sparse(a, q128, k128, ws + L.phik, ws + L.v16, ws + L.hs16, st)) != cudaSuccess)
+    return cuda_fail(e, "sparse");
   return SLA_OK;
 }
 

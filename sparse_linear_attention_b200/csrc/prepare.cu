@@ -14,8 +14,9 @@
 //   kernel, channels past d zero), and the partial sums
 //   H_part = phi(K)^T V (tcgen05, fp16 in / fp32 accumulate in TMEM) and
 //   Z_part = phi(K)^T 1 (same, against a column of ones).
-// reduce_kernel: H_tot, Z_tot = sum of the partials in split order (fixed, so
-//   deterministic).
+// zsum_kernel / hsum_kernel: Z_tot, H_tot = sum of the partials in split
+//   order (fixed, so deterministic); H_tot is stored as fp16 H_tot / sigma
+//   with sigma an exact per-head power of two (see hsum_kernel).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -28,7 +29,8 @@ namespace sla {
 
 namespace {
 
-constexpr int kPreThreads = 128;
+constexpr int kPreThreads = 256;
+constexpr int kUnits = 64 * 16 / kPreThreads;  // 16-byte channel units per thread per 64-token tile
 constexpr uint32_t kTileBytes = 64 * 128 * 2;  // 64 tokens x 128 channels x 2 B
 constexpr uint32_t kOffPhi0 = 0;
 constexpr uint32_t kOffV0 = kTileBytes;
@@ -36,19 +38,32 @@ constexpr uint32_t kBufBytes = 2 * kTileBytes;       // phi(K) + V for one buffe
 constexpr uint32_t kOffOnes = 2 * kBufBytes;          // 65536
 constexpr uint32_t kOffBar = kOffOnes + 2048;         // 2 mma barriers + done
 constexpr uint32_t kOffMisc = kOffBar + 64;           // tmem base, abort flag
-constexpr uint32_t kPreSmem = kOffMisc + 64 + 1024;   // + alignment slack
-constexpr uint32_t kPreTmemCols = 256;                // H: 0..127, Z: 128..143
+constexpr uint32_t kOffZred = kOffMisc + 64;          // [8 warps][128] column-sum partials
+constexpr uint32_t kPreSmem = kOffZred + 8 * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kPreTmemCols = 128;                // H: 0..127
 
-// 8 consecutive channels [8u, 8u+8) of token row `row` as fp32; zero past d.
+// Raw 16-byte words holding 8 consecutive channels of T.
 template <typename T>
-__device__ __forceinline__ void load8(const T* __restrict__ base, long long row, int d, int u, bool valid,
-                                      float* f) {
+struct Raw8 {
+  static constexpr int W = sizeof(T) * 8 / 16;  // 1 for bf16, 2 for f32
+  uint4 w[W];
+};
+
+template <typename T>
+__device__ __forceinline__ void load_raw8(const T* __restrict__ base, long long row, int d, int u, bool valid,
+                                          Raw8<T>& r) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+  for (int i = 0; i < Raw8<T>::W; ++i) r.w[i] = make_uint4(0, 0, 0, 0);
   if (!valid || 8 * u >= d) return;
+  const uint4* src = reinterpret_cast<const uint4*>(base + row * d + 8 * u);
+#pragma unroll
+  for (int i = 0; i < Raw8<T>::W; ++i) r.w[i] = __ldg(src + i);
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const Raw8<T>& r, float* f) {
   if constexpr (sizeof(T) == 2) {
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(base + row * d + 8 * u));
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const uint32_t w[4] = {r.w[0].x, r.w[0].y, r.w[0].z, r.w[0].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 p = unpack_bf162(w[i]);
@@ -56,24 +71,37 @@ __device__ __forceinline__ void load8(const T* __restrict__ base, long long row,
       f[2 * i + 1] = p.y;
     }
   } else {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(base + row * d + 8 * u));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(base + row * d + 8 * u + 4));
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      f[4 * i + 0] = __uint_as_float(r.w[i].x);
+      f[4 * i + 1] = __uint_as_float(r.w[i].y);
+      f[4 * i + 2] = __uint_as_float(r.w[i].z);
+      f[4 * i + 3] = __uint_as_float(r.w[i].w);
+    }
   }
 }
 
+// 8 consecutive channels [8u, 8u+8) of token row `row` as fp32; zero past d.
 template <typename T>
-__global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
+__device__ __forceinline__ void load8(const T* __restrict__ base, long long row, int d, int u, bool valid,
+                                      float* f) {
+  Raw8<T> r;
+  load_raw8<T>(base, row, d, u, valid, r);
+  unpack8<T>(r, f);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
     const T* __restrict__ k, const T* __restrict__ v, __half* __restrict__ phik, __half* __restrict__ v16,
-    __nv_bfloat16* __restrict__ khat, float* __restrict__ hpart, float* __restrict__ zpart, int N, int d,
-    int nkv, int nsplit, int phi_kind, int* status) {
+    __nv_bfloat16* __restrict__ khat, float* __restrict__ hpart, float* __restrict__ zpart,
+    float* __restrict__ zblk, int N, int d, int nkv, int nsplit, int phi_kind, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [0], [1]
   uint64_t* done_bar = mma_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+  float* zred = reinterpret_cast<float*>(sm + kOffZred);
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int split = blockIdx.x;
@@ -81,11 +109,6 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
   const int jb0 = static_cast<int>((static_cast<long long>(split) * nkv) / nsplit);
   const int jb1 = static_cast<int>((static_cast<long long>(split + 1) * nkv) / nsplit);
 
-  // ones column for Z: K-major 16 x 64 tile, row 0 = 1.0, rows 1..15 = 0
-  for (int i = tid; i < 2048 / 4; i += kPreThreads) {
-    const uint32_t one2 = 0x3C003C00u;  // two fp16 ones
-    reinterpret_cast<uint32_t*>(sm + kOffOnes)[i] = (i < 32) ? one2 : 0u;
-  }
   if (tid == 0) {
     mbar_init(&mma_bar[0], 1);
     mbar_init(&mma_bar[1], 1);
@@ -110,33 +133,43 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
   __nv_bfloat16* khb = khat ? khat + bh * static_cast<long long>(N) * kDPad : nullptr;
 
   const uint32_t idesc_h = idesc_f16(0, 1, 1, 128, 128);  // phi(K)^T (MN-major) x V (MN-major)
-  const uint32_t idesc_z = idesc_f16(0, 1, 0, 128, 16);   // phi(K)^T x ones (K-major)
   bool ok = true;
+
+  // this thread's units of a 64-token tile: row m = tid/16 + 16*i, channels [8u, 8u+8)
+  const int u = tid % 16;
+  Raw8<T> kr[kUnits], vr[kUnits];
+  auto fetch = [&](int jb) {
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i) {
+      const int tok = jb * 64 + tid / 16 + 16 * i;
+      load_raw8<T>(kb, tok, d, u, tok < N, kr[i]);
+      load_raw8<T>(vb, tok, d, u, tok < N, vr[i]);
+    }
+  };
+  if (jb0 < jb1) fetch(jb0);
 
   for (int jb = jb0; jb < jb1; ++jb) {
     const int it = jb - jb0;
     const int buf = it & 1;
     uint8_t* sphi = sm + buf * kBufBytes + kOffPhi0;
     uint8_t* sv = sm + buf * kBufBytes + kOffV0;
-    // this thread's 8 units: row m = tid/16 + 8*i, unit u = tid % 16
-    float kf[8][8], vf[8][8];
-    const int u = tid % 16;
+    float kf[kUnits][8], vf[kUnits][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int m = tid / 16 + 8 * i;
-      const int tok = jb * 64 + m;
-      load8<T>(kb, tok, d, u, tok < N, kf[i]);
-      load8<T>(vb, tok, d, u, tok < N, vf[i]);
+    for (int i = 0; i < kUnits; ++i) {
+      unpack8<T>(kr[i], kf[i]);
+      unpack8<T>(vr[i], vf[i]);
     }
+    if (jb + 1 < jb1) fetch(jb + 1);  // next tile's loads overlap this tile's work
     // buffer reuse: the MMA that read this buffer two tiles ago must be done
     if (it >= 2) {
       if (!mbar_wait(&mma_bar[buf], ((it - 2) >> 1) & 1, abort_flag, status)) ok = false;
     }
     ok = __syncthreads_and(ok) != 0;  // CTA-uniform verdict
     if (!ok) break;
+    float csum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // this thread's rows, rounded phi(K)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int m = tid / 16 + 8 * i;
+    for (int i = 0; i < kUnits; ++i) {
+      const int m = tid / 16 + 16 * i;
       const int tok = jb * 64 + m;
       const bool valid = tok < N;
       float ph[8];
@@ -168,6 +201,13 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
                         pack_half2(ph[6], ph[7]));
         vu = make_uint4(pack_half2(vf[i][0], vf[i][1]), pack_half2(vf[i][2], vf[i][3]),
                         pack_half2(vf[i][4], vf[i][5]), pack_half2(vf[i][6], vf[i][7]));
+        const uint32_t pw[4] = {pu.x, pu.y, pu.z, pu.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_half2(pw[e]);
+          csum[2 * e] += f.x;
+          csum[2 * e + 1] += f.y;
+        }
         const long long g = static_cast<long long>(tok) * kDPad + 8 * u;
         *reinterpret_cast<uint4*>(phib + g) = pu;
         *reinterpret_cast<uint4*>(v16b + g) = vu;
@@ -184,25 +224,36 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
       *reinterpret_cast<uint4*>(sphi + off) = pu;
       *reinterpret_cast<uint4*>(sv + off) = vu;
     }
+    // column sums of this key block: lanes u and u+16 hold the same channels
+#pragma unroll
+    for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], 16);
+    if ((tid & 31) < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) zred[warp * 128 + 8 * u + e] = csum[e];
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid < 128) {
+      float z = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kPreThreads / 32; ++w) z += zred[w * 128 + tid];
+      zblk[(bh * nkv + jb) * kDPad + tid] = z;
+    }
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t aphi = smem_u32(sphi), av = smem_u32(sv), aones = smem_u32(sm + kOffOnes);
+      const uint32_t aphi = smem_u32(sphi), av = smem_u32(sv);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t a = sdesc_sw128(aphi + kk * 2048, 8192, 1024);
         const uint64_t b = sdesc_sw128(av + kk * 2048, 8192, 1024);
-        const uint64_t bo = sdesc_sw128(aones + kk * 32, 16, 1024);
         const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
         mma_f16_ss(tmem + 0, a, b, idesc_h, acc);
-        mma_f16_ss(tmem + 128, a, bo, idesc_z, acc);
       }
       mma_commit(&mma_bar[buf]);
     }
   }
-  // all MMAs of this CTA done -> read the partial sums out of TMEM
+  // all MMAs of this CTA done -> read the partial sums out of TMEM (warps 0..3: one lane each)
   if (tid == 0) mma_commit(done_bar);
   __syncwarp();
   bool have = ok && (jb1 > jb0);
@@ -214,7 +265,7 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
     have = have && w_ok;
   }
   tc_fence_after();
-  if (have) {
+  if (have && warp < 4) {
     float* hp = hpart + ((bh * nsplit + split) * kDPad + tid) * kDPad;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
@@ -225,10 +276,6 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
       for (int i = 0; i < 32; i += 4)
         *reinterpret_cast<float4*>(hp + cc * 32 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
     }
-    float z[32];
-    tmem_ld32(tmem + ((warp * 32) << 16) + 128, z);
-    tmem_wait_ld();
-    zpart[(bh * nsplit + split) * kDPad + tid] = z[0];
   }
   tc_fence_before();
   __syncthreads();
@@ -238,23 +285,43 @@ __global__ void __launch_bounds__(kPreThreads) lin_prepass_kernel(
   }
 }
 
-// H_tot[bh] = sum over splits (ascending) of H_part; Z_tot likewise.
-__global__ void __launch_bounds__(256) reduce_kernel(const float* __restrict__ hpart,
-                                                     const float* __restrict__ zpart, float* __restrict__ htot,
-                                                     float* __restrict__ ztot, int BH, int nsplit) {
-  const long long per = kDPad * kDPad + kDPad;
+// Z_tot[bh][e] = sum over key blocks (ascending) of the per-block column sums,
+// and the per-head scale sigma = 2^ceil(log2(max_e Z_tot)) (one block of 128
+// threads per head).
+__global__ void __launch_bounds__(128) zsum_kernel(const float* __restrict__ zblk, float* __restrict__ ztot,
+                                                   float* __restrict__ sigma, int nkv) {
+  const long long bh = blockIdx.x;
+  const int e = threadIdx.x;
+  float z = 0.0f;
+  for (int j = 0; j < nkv; ++j) z += zblk[(bh * nkv + j) * kDPad + e];
+  ztot[bh * kDPad + e] = z;
+  __shared__ float red[4];
+  float m = z;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((e & 31) == 0) red[e >> 5] = m;
+  __syncthreads();
+  if (e == 0) {
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    int ex = 0;
+    if (m > 0.0f) frexpf(m, &ex);  // m < 2^ex
+    sigma[bh] = ldexpf(1.0f, ex);
+  }
+}
+
+// H_tot / sigma as fp16: sum of H_part over splits in ascending order, then one
+// exact power-of-two scaling and one rounding.  |H_tot / sigma| <= max |V|
+// because phi(K) >= 0 makes H_tot[e][c] a phi-weighted sum of v[c] with
+// total weight Z_tot[e] <= sigma.
+__global__ void __launch_bounds__(256) hsum_kernel(const float* __restrict__ hpart, const float* __restrict__ sigma,
+                                                   __half* __restrict__ hs16, int BH, int nsplit) {
+  const long long per = kDPad * kDPad;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= per * BH) return;
   const long long bh = idx / per, r = idx % per;
   float acc = 0.0f;
-  if (r < kDPad * kDPad) {
-    for (int s = 0; s < nsplit; ++s) acc += hpart[(bh * nsplit + s) * kDPad * kDPad + r];
-    htot[bh * kDPad * kDPad + r] = acc;
-  } else {
-    const long long e = r - kDPad * kDPad;
-    for (int s = 0; s < nsplit; ++s) acc += zpart[(bh * nsplit + s) * kDPad + e];
-    ztot[bh * kDPad + e] = acc;
-  }
+  for (int s = 0; s < nsplit; ++s) acc += hpart[(bh * nsplit + s) * per + r];
+  hs16[idx] = __float2half_rn(acc / sigma[bh]);
 }
 
 // Q as bf16 with the head dim padded to 128 (needed when d != 128 or the
@@ -289,22 +356,31 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
   if (s.in_dtype == SLA_BF16) {
     e = cudaFuncSetAttribute(lin_prepass_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kPreSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(lin_prepass_kernel<__nv_bfloat16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               100);
     if (e != cudaSuccess) return e;
     lin_prepass_kernel<__nv_bfloat16><<<grid, kPreThreads, kPreSmem, st>>>(
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), phik, v16, khat, hpart,
-        zpart, s.N, s.d, nkv, L.nsplit, phi, status);
+        zpart, reinterpret_cast<float*>(ws + L.zblk), s.N, s.d, nkv, L.nsplit, phi, status);
   } else {
     e = cudaFuncSetAttribute(lin_prepass_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(lin_prepass_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     lin_prepass_kernel<float><<<grid, kPreThreads, kPreSmem, st>>>(
-        static_cast<const float*>(k), static_cast<const float*>(v), phik, v16, khat, hpart, zpart, s.N, s.d,
-        nkv, L.nsplit, phi, status);
+        static_cast<const float*>(k), static_cast<const float*>(v), phik, v16, khat, hpart, zpart,
+        reinterpret_cast<float*>(ws + L.zblk), s.N, s.d, nkv, L.nsplit, phi, status);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long n = static_cast<long long>(BH) * (kDPad * kDPad + kDPad);
-  reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-      hpart, zpart, reinterpret_cast<float*>(ws + L.htot), reinterpret_cast<float*>(ws + L.ztot), BH, L.nsplit);
+  float* sig = reinterpret_cast<float*>(ws + L.sigma);
+  zsum_kernel<<<BH, 128, 0, st>>>(reinterpret_cast<const float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.ztot),
+                                  sig, nkv);
+  const long long n = static_cast<long long>(BH) * kDPad * kDPad;
+  hsum_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(hpart, sig,
+                                                                      reinterpret_cast<__half*>(ws + L.hs16), BH,
+                                                                      L.nsplit);
   return cudaGetLastError();
 }
 

@@ -23,7 +23,9 @@ struct WsLayout {
   size_t v16 = 0;             // fp16 [BH, N, 128]  V, zero past d
   size_t qhat = 0, khat = 0;  // bf16 [BH, N, 128]  Q, K (only when need_hat)
   size_t hpart = 0, zpart = 0;  // fp32 [BH, nsplit, 128, 128], [BH, nsplit, 128]
-  size_t htot = 0, ztot = 0;    // fp32 [BH, 128, 128], [BH, 128]
+  size_t hs16 = 0, ztot = 0;    // fp16 [BH, 128, 128] = H_tot / sigma, fp32 [BH, 128] = Z_tot
+  size_t sigma = 0;             // fp32 [BH]: per-head power of two >= max_e Z_tot[e]
+  size_t zblk = 0;              // fp32 [BH, n_kv, 128]: colsum of phi(K) per key block
   size_t lists = 0;             // SLA: int32 [BH, n_q, 2, n_kv] critical / negligible lists
   size_t counts = 0;            // SLA: int32 [BH, n_q, 2]
   size_t total = 0;
@@ -64,8 +66,10 @@ inline WsLayout ws_layout(const sla_shape& s, int mode) {
   }
   L.hpart = take(BH * L.nsplit * kDPad * kDPad * 4);
   L.zpart = take(BH * L.nsplit * kDPad * 4);
-  L.htot = take(BH * kDPad * kDPad * 4);
+  L.hs16 = take(BH * kDPad * kDPad * 2);
   L.ztot = take(BH * kDPad * 4);
+  L.sigma = take(BH * 4);
+  L.zblk = take(BH * static_cast<size_t>(nkv) * kDPad * 4);
   if (mode == SLA_MODE_SLA_3WAY) {
     L.lists = take(BH * nq * 2 * static_cast<size_t>(nkv) * 4);
     L.counts = take(BH * nq * 2 * 4);

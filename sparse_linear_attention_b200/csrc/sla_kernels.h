@@ -30,8 +30,9 @@ struct SparseArgs {
   const int32_t* counts;     // nullable: counts[2*row] = #crit, [2*row+1] = #negl; else crit_max, 0
   const float* alpha;        // SLA2: [BH, nq]; null for SLA
   const void* wproj;         // SLA: bf16 [d][d]; null for SLA2
-  const float* htot;         // [BH, 128, 128]
+  const float* sigma;        // [BH]: power of two >= max_e Z_tot[e]
   const float* ztot;         // [BH, 128]
+  const float* zblk;         // [BH, nkv, 128]: per-block column sums of phi(K)
   void* out;
   int out_bf16;
   int phi;
@@ -43,6 +44,6 @@ struct SparseArgs {
 cudaError_t encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int N, int BH, int box_rows);
 
 cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
-                          const void* phik16, const void* v16, cudaStream_t st);
+                          const void* phik16, const void* v16, const void* hs16, cudaStream_t st);
 
 }  // namespace sla
