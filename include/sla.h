@@ -99,8 +99,9 @@ sla_status sla_workspace_init(void* ws, size_t ws_bytes, void* stream);
 /* Router [SLA2-deep §05; SLA 关键设计 2; SLA2-sum §2.B]:
  *   Qbar = pool_bq(Q), Kbar = pool_bkv(K)          (block means, valid tokens)
  *   Qt = Qbar Wq, Kt = Kbar Wk                     (Wq, Wk: d x d row-major fp32,
- *                                                   shared by all heads; NULL =
- *                                                   identity = SLA heuristic)
+ *                                                   16-byte aligned, shared by
+ *                                                   all heads; NULL = identity
+ *                                                   = SLA heuristic)
  *   s[i,j] = Qt_i . Kt_j
  * then per query block i, with key blocks ordered by (s desc, index asc):
  *   SLA2: the first k_keep are kept;

@@ -161,6 +161,7 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k, const
   if (mode != SLA_MODE_SLA2_TOPK && mode != SLA_MODE_SLA_3WAY) return arg_fail(SLA_ERR_INVALID_ARG, "mode");
   if (q == nullptr || k == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Q or K is null");
   if (!aligned16(q) || !aligned16(k)) return arg_fail(SLA_ERR_ALIGNMENT, "Q, K must be 16-byte aligned");
+  if (!aligned16(Wq) || !aligned16(Wk)) return arg_fail(SLA_ERR_ALIGNMENT, "Wq, Wk must be 16-byte aligned");
   const int nkv = ceil_div(shape->N, shape->bkv);
   if (nkv > kMaxNKV) return arg_fail(SLA_ERR_UNSUPPORTED, "router needs n_kv <= 2048");
   if (k_keep < 0 || k_neg < 0 || k_keep + k_neg > nkv) return arg_fail(SLA_ERR_INVALID_ARG, "k_keep/k_neg");

@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
 
   const uint32_t idesc_h = idesc_f16(0, 1, 1, 128, 128);  // phi(K)^T (MN-major) x V (MN-major)
   bool ok = true;
+  float zacc = 0.0f;  // threads < 128: this split's Z for channel tid, blocks in ascending order
 
   // this thread's units of a 64-token tile: row m = tid/16 + 16*i, channels [8u, 8u+8)
   const int u = tid % 16;
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
         float sum = 0.0f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          ph[e] = (8 * u + e < d) ? expf(kf[i][e] - mx) : 0.0f;
+          ph[e] = (8 * u + e < d) ? ex2_approx((kf[i][e] - mx) * 1.4426950408889634f) : 0.0f;
           sum += ph[e];
         }
 #pragma unroll
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
 #pragma unroll
       for (int w = 0; w < kPreThreads / 32; ++w) z += zred[w * 128 + tid];
       zblk[(bh * nkv + jb) * kDPad + tid] = z;
+      zacc += z;
     }
     if (tid == 0) {
       tc_fence_after();
@@ -266,6 +268,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
   }
   tc_fence_after();
   if (have && warp < 4) {
+    zpart[(bh * nsplit + split) * kDPad + tid] = zacc;
     float* hp = hpart + ((bh * nsplit + split) * kDPad + tid) * kDPad;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
@@ -285,15 +288,15 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
   }
 }
 
-// Z_tot[bh][e] = sum over key blocks (ascending) of the per-block column sums,
-// and the per-head scale sigma = 2^ceil(log2(max_e Z_tot)) (one block of 128
-// threads per head).
-__global__ void __launch_bounds__(128) zsum_kernel(const float* __restrict__ zblk, float* __restrict__ ztot,
-                                                   float* __restrict__ sigma, int nkv) {
+// Z_tot[bh][e] = sum over splits (ascending) of each split's sum of per-block
+// column sums, and the per-head scale sigma = 2^ceil(log2(max_e Z_tot)) (one
+// block of 128 threads per head).
+__global__ void __launch_bounds__(128) zsum_kernel(const float* __restrict__ zpart, float* __restrict__ ztot,
+                                                   float* __restrict__ sigma, int nsplit) {
   const long long bh = blockIdx.x;
   const int e = threadIdx.x;
   float z = 0.0f;
-  for (int j = 0; j < nkv; ++j) z += zblk[(bh * nkv + j) * kDPad + e];
+  for (int s = 0; s < nsplit; ++s) z += zpart[(bh * nsplit + s) * kDPad + e];
   ztot[bh * kDPad + e] = z;
   __shared__ float red[4];
   float m = z;
@@ -375,8 +378,7 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   float* sig = reinterpret_cast<float*>(ws + L.sigma);
-  zsum_kernel<<<BH, 128, 0, st>>>(reinterpret_cast<const float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.ztot),
-                                  sig, nkv);
+  zsum_kernel<<<BH, 128, 0, st>>>(zpart, reinterpret_cast<float*>(ws + L.ztot), sig, L.nsplit);
   const long long n = static_cast<long long>(BH) * kDPad * kDPad;
   hsum_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(hpart, sig,
                                                                       reinterpret_cast<__half*>(ws + L.hs16), BH,

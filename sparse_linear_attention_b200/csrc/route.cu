@@ -74,10 +74,12 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
 // ---------------------------------------------------------------- projection
 // xt^T[bh][c][r] = sum_e fl(xbar[bh][r][e] * W[e][c]) (or xbar itself when W is
 // null), written channel-major so the score kernel reads it coalesced.
-// Block: 128 threads (one per output channel), 16 rows of one head.
-constexpr int kProjRows = 16;
+// Block: 256 threads, 64 rows of one head x all d output channels; thread
+// (ty, tx) owns rows 4ty..4ty+3 and channels 8tx..8tx+7.  The sum over e runs
+// in ascending order for every output, as specified.
+constexpr int kProjRows = 64;
 
-__global__ void __launch_bounds__(128) project_kernel(const float* __restrict__ qbar,
+__global__ void __launch_bounds__(256) project_kernel(const float* __restrict__ qbar,
                                                       const float* __restrict__ kbar,
                                                       const float* __restrict__ Wq,
                                                       const float* __restrict__ Wk, float* __restrict__ qtT,
@@ -90,31 +92,56 @@ __global__ void __launch_bounds__(128) project_kernel(const float* __restrict__ 
   const int r0 = blockIdx.x * kProjRows;
   if (r0 >= nrows) return;
   const long long bh = blockIdx.y;
-  __shared__ float xs[kProjRows][kDPad];
-  const int c = threadIdx.x;
-  for (int i = threadIdx.x; i < kProjRows * d; i += blockDim.x) {
-    const int r = i / d, e = i % d;
-    xs[r][e] = (r0 + r < nrows) ? xbar[(bh * nrows + r0 + r) * d + e] : 0.0f;
+  extern __shared__ __align__(16) float psm[];
+  float* xs = psm;                     // [d][64]: xs[e][r] = xbar[r0 + r][e]
+  float* ws = psm + kDPad * kProjRows; // [d][128]: W[e][c]
+  const int tid = threadIdx.x;
+  // rows: float4 along e, one row per thread in a group of 64 -> transposed store
+  for (int i = tid; i < kProjRows * (d / 4); i += 256) {
+    const int r = i % kProjRows, e4 = i / kProjRows;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < nrows) v = *reinterpret_cast<const float4*>(xbar + (bh * nrows + r0 + r) * d + 4 * e4);
+    xs[(4 * e4 + 0) * kProjRows + r] = v.x;
+    xs[(4 * e4 + 1) * kProjRows + r] = v.y;
+    xs[(4 * e4 + 2) * kProjRows + r] = v.z;
+    xs[(4 * e4 + 3) * kProjRows + r] = v.w;
   }
+  if (W != nullptr)
+    for (int i = tid; i < d * (d / 4); i += 256) cp_async16(ws + (i / (d / 4)) * kDPad + 4 * (i % (d / 4)), W + 4 * i);
+  cp_async_wait_all();
   __syncthreads();
-  if (c >= d) return;
-  float acc[kProjRows];
+  const int ty = tid / 16, tx = tid % 16;
+  if (8 * tx >= d) return;
+  float acc[4][8];
   if (W == nullptr) {
 #pragma unroll
-    for (int r = 0; r < kProjRows; ++r) acc[r] = xs[r][c];
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] = xs[(8 * tx + b) * kProjRows + 4 * ty + a];
   } else {
 #pragma unroll
-    for (int r = 0; r < kProjRows; ++r) acc[r] = 0.0f;
-    for (int e = 0; e < d; ++e) {
-      const float w = __ldg(W + e * d + c);
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int r = 0; r < kProjRows; ++r) acc[r] = __fadd_rn(acc[r], __fmul_rn(xs[r][e], w));
+      for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+    for (int e = 0; e < d; ++e) {
+      const float4 xv = *reinterpret_cast<const float4*>(xs + e * kProjRows + 4 * ty);
+      const float4 w0 = *reinterpret_cast<const float4*>(ws + e * kDPad + 8 * tx);
+      const float4 w1 = *reinterpret_cast<const float4*>(ws + e * kDPad + 8 * tx + 4);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float wb[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xa[a], wb[b]));
     }
   }
-  float* dst = xtT + (bh * d + c) * nrows + r0;
 #pragma unroll
-  for (int r = 0; r < kProjRows; ++r)
-    if (r0 + r < nrows) dst[r] = acc[r];
+  for (int b = 0; b < 8; ++b) {
+    float* dst = xtT + (bh * d + 8 * tx + b) * nrows + r0 + 4 * ty;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      if (r0 + 4 * ty + a < nrows) dst[a] = acc[a][b];
+  }
 }
 
 // ---------------------------------------------------------------- scores + selection
@@ -184,13 +211,23 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
     const int c = i / kScoreRows, r = i % kScoreRows;
     qs[i] = (r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
   }
+  const bool vec_ok = (nkv % 4) == 0;  // rows of ktT 16-byte aligned
   const int ty = tid / 32;  // rows 2*ty, 2*ty+1
   const int tx = tid % 32;  // key blocks 4*tx .. 4*tx+3 of the chunk
   for (int j0 = 0; j0 < nkv; j0 += kScoreKeys) {
     __syncthreads();  // previous chunk's ks reads done (and qs ready on the first pass)
-    for (int i = tid; i < d * kScoreKeys; i += 256) {
-      const int c = i / kScoreKeys, j = i % kScoreKeys;
-      ks[i] = (j0 + j < nkv) ? ktT[(bh * d + c) * nkv + j0 + j] : 0.0f;
+    if (vec_ok && j0 + kScoreKeys <= nkv) {
+      for (int i = tid; i < d * (kScoreKeys / 4); i += 256) {
+        const int c = i / (kScoreKeys / 4), j4 = i % (kScoreKeys / 4);
+        cp_async16(ks + c * kScoreKeys + 4 * j4, ktT + (bh * d + c) * nkv + j0 + 4 * j4);
+      }
+      cp_async_wait_all();
+    } else {
+#pragma unroll 8
+      for (int i = tid; i < d * kScoreKeys; i += 256) {
+        const int c = i / kScoreKeys, j = i % kScoreKeys;
+        ks[i] = (j0 + j < nkv) ? ktT[(bh * d + c) * nkv + j0 + j] : 0.0f;
+      }
     }
     __syncthreads();
     float acc[2][4];
@@ -286,8 +323,12 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                                                 qbar, kbar, BH, s.N, s.d, s.bq, s.bkv);
   }
   {
+    const size_t psmem = static_cast<size_t>(kDPad) * (kProjRows + kDPad) * 4;
+    cudaError_t e = cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(psmem));
+    if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(nkv > nq ? nkv : nq, kProjRows), BH, 2);
-    project_kernel<<<grid, 128, 0, st>>>(qbar, kbar, Wq, Wk, qtT, ktT, nq, nkv, s.d);
+    project_kernel<<<grid, 256, psmem, st>>>(qbar, kbar, Wq, Wk, qtT, ktT, nq, nkv, s.d);
   }
   {
     const size_t smem = (kDPad * kScoreRows + kDPad * kScoreKeys + static_cast<size_t>(kScoreRows) * nkv) * 4;

@@ -94,7 +94,9 @@ extern "C" sla_status sla_route_noalloc(const sla_shape* shape, const void* q, c
     return SLA_ERR_UNSUPPORTED;
   if (mode != SLA_MODE_SLA2_TOPK && mode != SLA_MODE_SLA_3WAY) return SLA_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr) return SLA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(k) & 15u)) return SLA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(k) & 15u) ||
+      (reinterpret_cast<uintptr_t>(Wq) & 15u) || (reinterpret_cast<uintptr_t>(Wk) & 15u))
+    return SLA_ERR_ALIGNMENT;
   const int nkv = ceil_div(s.N, s.bkv);
   if (nkv > kMaxNKV) return SLA_ERR_UNSUPPORTED;
   if (k_keep < 0 || k_neg < 0 || k_keep + k_neg > nkv) return SLA_ERR_INVALID_ARG;

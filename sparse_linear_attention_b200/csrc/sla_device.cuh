@@ -123,6 +123,18 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- cp.async
+
+// 16-byte asynchronous copy global -> shared (L2 only), completed by
+// cp_async_wait_all().
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -253,6 +265,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float elu1(float x) {
+  return x > 0.f ? x + 1.0f : ex2_approx(x * 1.4426950408889634f);
+}
+
 // ---------------------------------------------------------------- descriptors
 //
 // All MMA operands live in shared memory in the 128-byte-swizzled layout that
@@ -312,7 +328,8 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
   return __half22float2(h);
 }
 
-// phi(x) = ELU(x) + 1
-__device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.0f : expf(x); }
+// phi(x) = ELU(x) + 1.  Its results are rounded to fp16 or bf16 right after,
+// so the hardware exp2 (relative error near 2^-22) is ample.
+__device__ __forceinline__ float elu1(float x);
 
 }  // namespace sla

@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float sum = 0.0f;
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            x[c] = (c0 + c < a.d) ? expf(x[c] - mx) : 0.0f;
+            x[c] = (c0 + c < a.d) ? ex2_approx((x[c] - mx) * 1.4426950408889634f) : 0.0f;
             sum += x[c];
           }
           RED(1, half)[r] = sum;
@@ -563,10 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) x[c] *= inv;
         } else {
-          // ELU(x)+1 with the hardware exp2 (fp16 result, far coarser than its error)
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            x[c] = (c0 + c < a.d) ? (x[c] > 0.0f ? x[c] + 1.0f : ex2_approx(x[c] * 1.4426950408889634f)) : 0.0f;
+          for (int c = 0; c < 64; ++c) x[c] = (c0 + c < a.d) ? elu1(x[c]) : 0.0f;
         }
         uint32_t pk[32];
 #pragma unroll

@@ -68,8 +68,8 @@ def test_workspace_size():
 FAKE = 0x7F0000000000  # never dereferenced: every call below fails its checks first
 
 
-def _route(shape, q=FAKE, k=FAKE, mode=0, k_keep=15, k_neg=0, kept=FAKE, ws=FAKE, ws_bytes=1 << 40):
-    return sla.lib().sla_route(ctypes.byref(shape), q, k, None, None, mode, k_keep, k_neg, kept, None, None,
+def _route(shape, q=FAKE, k=FAKE, mode=0, k_keep=15, k_neg=0, kept=FAKE, ws=FAKE, ws_bytes=1 << 40, wq=None):
+    return sla.lib().sla_route(ctypes.byref(shape), q, k, wq, None, mode, k_keep, k_neg, kept, None, None,
                                ws, ws_bytes, None)
 
 
@@ -77,6 +77,7 @@ def test_route_rejects_bad_arguments_before_launch():
     s = _shape()
     assert _route(s, q=None) == 1
     assert _route(s, q=FAKE + 2) == 3
+    assert _route(s, wq=FAKE + 4) == 3       # projections are read 16 bytes at a time
     assert _route(s, mode=3) == 1
     assert _route(s, k_keep=513) == 1
     assert _route(s, k_keep=-1) == 1
