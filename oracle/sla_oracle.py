@@ -310,3 +310,95 @@ def e4m3_decode(code: np.ndarray) -> np.ndarray:
 def e4m3_round(x32: np.ndarray) -> np.ndarray:
     """Value of x after an e4m3 round trip, float64."""
     return e4m3_decode(e4m3_encode(x32))
+
+
+# ----------------------------------------------------------------------------
+# Low-bit (FP8 e4m3) sparse branch  [SLA2-deep §07]
+#
+# The page quantises Q and K, computes the low-bit Q K^T, dequantises and takes
+# the softmax; quantises P and V, computes the low-bit P V and dequantises;
+# before that K is smoothed by subtracting its column mean.  It does not fix
+# the format or the scale granularity; the readings taken here:
+#   - format e4m3 (OCP), round to nearest even, saturating;
+#   - K smoothing: mu = mean of K over the valid tokens of (b,h), K' = K - mu
+#     rounded to fp32 (a constant shift of every score in a row, which the
+#     softmax ignores);
+#   - Q and K': one scale per (b,h) and 128-token block: amax over the block,
+#     inv = 448 / amax in fp32 (1 if amax = 0), x8 = e4m3(fp32(x * inv)),
+#     scale = amax / 448 in fp32;
+#   - V: one scale per (b,h) and channel over all valid tokens, same rule;
+#   - P: online softmax over the kept blocks in ascending order; after each
+#     block p = exp(S - m) with m the running row max including that block,
+#     p8 = e4m3(fp32(p * 448)); the row sum uses the unquantised p.
+# ----------------------------------------------------------------------------
+
+def _e4m3_q(x32, codec):
+    return codec(np.asarray(x32, dtype=F32))
+
+
+def _quant_blocks(x32, blk, codec):
+    """Per block of `blk` tokens (rows of x32 [n, d]): (decoded values, scales)."""
+    n = x32.shape[0]
+    vals = np.empty(x32.shape, dtype=F64)
+    scales = []
+    for t0 in range(0, n, blk):
+        xb = x32[t0:t0 + blk]
+        amax = F32(np.abs(xb).max()) if xb.size else F32(0.0)
+        inv = F32(448.0) / amax if amax > 0 else F32(1.0)
+        vals[t0:t0 + blk] = _e4m3_q(xb * inv, codec)
+        scales.append(F64(F32(amax / F32(448.0))) if amax > 0 else F64(F32(1.0) / F32(448.0)))
+    return vals, np.array(scales, dtype=F64)
+
+
+def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, codec=None, qblk=128):
+    """SLA2 output with the low-bit sparse branch described above; the linear
+    branch and the combine are the fp64 ones of sla2_forward.  q, k, v: exact
+    values of the inputs as float64 [B,H,N,d].  codec(x32) -> float64 values
+    after the e4m3 round trip (e4m3_round by default; an identity codec turns
+    the quantisation off, which pins the bookkeeping to sla2_forward)."""
+    codec = e4m3_round if codec is None else codec
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    n_kv = -(-N // bkv)
+    out = {n: np.full(v.shape, np.nan) for n in ("o", "o_s", "o_l")}
+    todo = _blocks_to_do(B, H, nq, blocks)
+    heads = sorted({(b, h) for (b, h, _) in todo})
+    for (b, h) in heads:
+        qs, ks, vs = q[b, h], k[b, h], v[b, h]
+        mu = ks.mean(axis=0)
+        kp32 = (ks - mu).astype(F32)
+        q8, sq = _quant_blocks(qs.astype(F32), qblk, codec)
+        k8, sk = _quant_blocks(kp32, qblk, codec)
+        v32 = vs.astype(F32)
+        vamax = np.abs(v32).max(axis=0)
+        vinv = np.where(vamax > 0, F32(448.0) / np.where(vamax > 0, vamax, F32(1.0)), F32(1.0)).astype(F32)
+        v8 = _e4m3_q(v32 * vinv[None, :], codec)
+        sv = np.where(vamax > 0, (vamax / F32(448.0)).astype(F32), F32(1.0) / F32(448.0)).astype(F64)
+        vdq = v8 * sv[None, :]
+        tok_q = np.arange(N) // qblk
+        for (_, _, i) in [t for t in todo if (t[0], t[1]) == (b, h)]:
+            rows = _rows(i, bq, N)
+            sel = sorted(int(j) for j in kept[b, h, i])
+            uns = [j for j in range(n_kv) if j not in set(sel)]
+            m = np.full(len(rows), -np.inf)
+            l = np.zeros(len(rows))
+            acc = np.zeros((len(rows), v.shape[-1]))
+            qdq = q8[rows] * sq[tok_q[rows]][:, None]
+            for j in sel:
+                keys = _rows(j, bkv, N)
+                kdq = k8[keys] * sk[tok_q[keys]][:, None]
+                s = (qdq @ kdq.T) / math.sqrt(d)
+                m_new = np.maximum(m, s.max(axis=1))
+                corr = np.exp(m - m_new)
+                p = np.exp(s - m_new[:, None])
+                l = l * corr + p.sum(axis=1)
+                p8 = _e4m3_q((p * 448.0).astype(F32), codec) / 448.0
+                acc = acc * corr[:, None] + p8 @ vdq[keys]
+                m = m_new
+            o_s = acc / l[:, None] if sel else np.zeros((len(rows), v.shape[-1]))
+            o_l = linear_branch(qs, ks, vs, rows, _tokens_of(uns, bkv, N), phi_kind)
+            a = float(alpha[b, h, i])
+            out["o_s"][b, h, rows] = o_s
+            out["o_l"][b, h, rows] = o_l
+            out["o"][b, h, rows] = a * o_s + (1.0 - a) * o_l
+    return out

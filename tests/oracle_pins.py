@@ -402,7 +402,61 @@ def pin_hand_example(orc):
     assert np.allclose(o, want, atol=1e-14, rtol=0)
 
 
-ALL_PINS = [pin_hand_example, 
+# ---------------------------------------------------------------- fp8 branch
+
+def _fp8_case(seed, N=300, d=16, offset=0.0):
+    q, k, v = _rand((1, 1, N, d), seed), _rand((1, 1, N, d), seed + 1) + offset, _rand((1, 1, N, d), seed + 2)
+    kept = np.array([[[[0, 2], [1, 3], [0, 4]]]])
+    alpha = np.array([[[0.3, 0.6, 0.9]]])
+    return q, k, v, kept, alpha
+
+
+def pin_fp8_identity_codec_is_fp64(orc):
+    """With the e4m3 round trip replaced by the identity, the low-bit branch's
+    bookkeeping (smoothing, per-block and per-channel scales, online softmax,
+    P scaling) must give the fp64 SLA2 output up to fp32 rounding of K' and of
+    the scaled values."""
+    q, k, v, kept, alpha = _fp8_case(90)
+    ident = lambda x: np.asarray(x, np.float64)  # noqa: E731
+    a = orc.sla2_forward(q, k, v, kept, alpha, 128, 64)["o"]
+    b = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64, codec=ident)["o"]
+    assert np.abs(a - b).max() < 1e-6
+
+
+def pin_fp8_quantisation_error_bounded(orc):
+    """e4m3 keeps 3 mantissa bits: the output moves, but by a bounded amount."""
+    q, k, v, kept, alpha = _fp8_case(91)
+    a = orc.sla2_forward(q, k, v, kept, alpha, 128, 64)["o"]
+    c = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64)["o"]
+    err = np.abs(a - c).max()
+    assert 1e-4 < err < 0.2, err
+
+
+def pin_fp8_k_smoothing(orc):
+    """A constant offset on every key row does not change softmax attention;
+    after K smoothing it does not change the quantised branch either (the mean
+    is removed before quantising).  Without smoothing the offset would swamp
+    the e4m3 scale."""
+    q, k, v, kept, alpha = _fp8_case(92)
+    k_off = k + 40.0
+    # the linear branch does see the offset: compare the sparse part only
+    a = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64)["o_s"]
+    b = orc.sla2_forward_fp8(q, k_off, v, kept, alpha, 128, 64)["o_s"]
+    assert np.abs(a - b).max() < 0.02
+
+
+def pin_fp8_block_scales(orc):
+    """Per-block scale = amax/448 and codes of x*448/amax: a block whose amax
+    is 448 quantises representable values exactly."""
+    x = np.array([[448.0, -2.0], [0.5, 3.0], [1.0, 0.0]], dtype=np.float32)
+    vals, scales = orc._quant_blocks(x, 2, orc.e4m3_round)
+    assert np.allclose(scales, [1.0, 1.0 / 448.0])
+    assert np.array_equal(vals[:2], np.array([[448.0, -2.0], [0.5, 3.0]]))
+    assert np.array_equal(vals[2], [448.0, 0.0]) and np.allclose(vals[2] * scales[1], [1.0, 0.0])
+
+
+ALL_PINS = [pin_hand_example, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
+            pin_fp8_k_smoothing, pin_fp8_block_scales, 
     pin_pool_bruteforce, pin_project_bruteforce, pin_scores_bruteforce, pin_topk_sort,
     pin_labels, pin_keep_count, pin_router_identity_and_permutation,
     pin_all_kept_is_full_attention, pin_masked_mass_identity, pin_nothing_kept_is_linear_attention,

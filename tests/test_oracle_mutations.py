@@ -31,11 +31,16 @@ MUTATIONS = {
     "e4m3_truncates": ("q = np.rint((f - 1.0) * 8.0)", "q = np.floor((f - 1.0) * 8.0)"),
     "unselected_uses_kept": ("uns = [j for j in range(n_kv) if j not in set(sel)]",
                              "uns = [j for j in range(n_kv)]"),
+    "fp8_no_k_smoothing": ("kp32 = (ks - mu).astype(F32)", "kp32 = ks.astype(F32)"),
+    "fp8_p_not_rescaled": ("p8 = _e4m3_q((p * 448.0).astype(F32), codec) / 448.0",
+                           "p8 = _e4m3_q((p * 448.0).astype(F32), codec)"),
+    "fp8_key_scale_of_row_block": ("kdq = k8[keys] * sk[tok_q[keys]][:, None]",
+                                   "kdq = k8[keys] * sk[tok_q[rows[0]]]"),
 }
 
 
 def _mutant(old, new):
-    assert SRC.count(old) == 1, old
+    assert SRC.count(old) >= 1, old  # applied wherever the line occurs
     mod = types.ModuleType("sla_oracle_mutant")
     exec(compile(SRC.replace(old, new), "sla_oracle_mutant", "exec"), mod.__dict__)
     return mod
