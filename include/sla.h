@@ -66,7 +66,11 @@ typedef enum { SLA_MODE_SLA2_TOPK = 0, SLA_MODE_SLA_3WAY = 1 } sla_route_mode;
 
 /* flags for the attention entry points */
 #define SLA_FLAG_PREPARED 1u  /* ws already holds sla_prepare's results for these K, V */
-#define SLA_FLAG_FP8 2u       /* low-bit (e4m3) sparse branch [SLA2-deep §07]; reserved */
+#define SLA_FLAG_FP8 2u       /* low-bit (e4m3) sparse branch [SLA2-deep §07], SLA2 only */
+
+/* OR into the mode of sla_workspace_size to include the buffers of the
+ * low-bit sparse branch (e4m3 copies of Q, K - mean(K), V and their scales). */
+#define SLA_WS_FP8 0x100
 
 typedef struct {
   int B, H, N, d;   /* batch, heads, tokens, head dim */
@@ -86,8 +90,8 @@ const char* sla_last_error_detail(void);
  * [0, n_kv].  (The pages give only the percentage.) */
 int sla_keep_count(double ratio, int n_kv);
 
-/* Bytes of device workspace the calls below need for this shape and mode.
- * Returns 0 for an invalid shape.  One workspace serves sla_route,
+/* Bytes of device workspace the calls below need for this shape and mode
+ * (optionally | SLA_WS_FP8).  Returns 0 for an invalid shape.  One workspace serves sla_route,
  * sla_prepare and the attention calls; calls that share it must be ordered
  * on one stream. */
 size_t sla_workspace_size(const sla_shape* shape, int mode);

@@ -32,6 +32,26 @@ cudaError_t encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType d
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_map8(CUtensorMap* map, const void* base, int N, int BH, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDPad), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDPad), static_cast<cuuint64_t>(N) * kDPad};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace sla
 
 namespace {
@@ -94,6 +114,14 @@ sla_status run_attention(const sla_shape* s, const void* q, const void* k, const
   if (L.need_hat) {
     if ((e = launch_qhat(*s, q, L, ws, st)) != cudaSuccess) return cuda_fail(e, "qhat");
   }
+  a.fp8 = (flags & SLA_FLAG_FP8) ? 1 : 0;
+  a.nb128 = ceil_div(s->N, 128);
+  if (a.fp8) {
+    if ((e = launch_fp8_quant(*s, q, k, v, L, ws, st)) != cudaSuccess) return cuda_fail(e, "fp8 quantisation");
+    a.sq = reinterpret_cast<const float*>(ws + L.sq);
+    a.sk = reinterpret_cast<const float*>(ws + L.sk);
+    a.vamax = reinterpret_cast<const float*>(ws + L.sv);
+  }
   a.BH = s->B * s->H;
   a.N = s->N;
   a.d = s->d;
@@ -108,7 +136,9 @@ sla_status run_attention(const sla_shape* s, const void* q, const void* k, const
   a.status = reinterpret_cast<int*>(ws + L.status);
   const void* q128 = L.need_hat ? static_cast<const void*>(ws + L.qhat) : q;
   const void* k128 = L.need_hat ? static_cast<const void*>(ws + L.khat) : k;
-  if ((e = launch_sparse(a, q128, k128, ws + L.phik, ws + L.v16, ws + L.hs16, st)) != cudaSuccess)
+  a.qsrc = q128;
+  if ((e = launch_sparse(a, q128, k128, ws + L.phik, ws + L.v16, ws + L.hs16, ws + L.q8, ws + L.k8, ws + L.v8,
+                         st)) != cudaSuccess)
     return cuda_fail(e, "sparse");
   return SLA_OK;
 }
@@ -143,7 +173,8 @@ int sla_keep_count(double ratio, int n_kv) {
 
 size_t sla_workspace_size(const sla_shape* shape, int mode) {
   if (check_shape(shape) != SLA_OK) return 0;
-  if (mode != SLA_MODE_SLA2_TOPK && mode != SLA_MODE_SLA_3WAY) return 0;
+  const int m = mode & ~SLA_WS_FP8;
+  if (m != SLA_MODE_SLA2_TOPK && m != SLA_MODE_SLA_3WAY) return 0;
   return ws_layout(*shape, mode).total;
 }
 
@@ -199,12 +230,12 @@ sla_status sla2_attn_fwd(const sla_shape* shape, const void* q, const void* k, c
   if (alpha == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "alpha is null");
   if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
   if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8)) return arg_fail(SLA_ERR_INVALID_ARG, "flags");
-  if (flags & SLA_FLAG_FP8) return arg_fail(SLA_ERR_UNSUPPORTED, "fp8 sparse branch not built");
   if (out == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "out is null");
   if (!aligned16(out)) return arg_fail(SLA_ERR_ALIGNMENT, "out must be 16-byte aligned");
   if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return arg_fail(SLA_ERR_INVALID_ARG, "out_dtype");
-  if ((s = check_ws(shape, SLA_MODE_SLA2_TOPK, ws, ws_bytes)) != SLA_OK) return s;
-  const WsLayout L = ws_layout(*shape, SLA_MODE_SLA2_TOPK);
+  const int wsmode = SLA_MODE_SLA2_TOPK | ((flags & SLA_FLAG_FP8) ? SLA_WS_FP8 : 0);
+  if ((s = check_ws(shape, wsmode, ws, ws_bytes)) != SLA_OK) return s;
+  const WsLayout L = ws_layout(*shape, wsmode);
   SparseArgs a{};
   static const int32_t kNoBlocks = 0;
   a.crit_idx = kept_idx ? kept_idx : &kNoBlocks;  // never read when k_keep == 0
@@ -231,7 +262,7 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k, co
   if (!aligned16(Wproj)) return arg_fail(SLA_ERR_ALIGNMENT, "Wproj must be 16-byte aligned");
   if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
   if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8)) return arg_fail(SLA_ERR_INVALID_ARG, "flags");
-  if (flags & SLA_FLAG_FP8) return arg_fail(SLA_ERR_UNSUPPORTED, "fp8 sparse branch not built");
+  if (flags & SLA_FLAG_FP8) return arg_fail(SLA_ERR_UNSUPPORTED, "the e4m3 sparse branch is built for SLA2 only");
   if (out == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "out is null");
   if (!aligned16(out)) return arg_fail(SLA_ERR_ALIGNMENT, "out must be 16-byte aligned");
   if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return arg_fail(SLA_ERR_INVALID_ARG, "out_dtype");

@@ -19,6 +19,7 @@
 //   with sigma an exact per-head power of two (see hsum_kernel).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "sla_device.cuh"
@@ -38,8 +39,8 @@ constexpr uint32_t kBufBytes = 2 * kTileBytes;       // phi(K) + V for one buffe
 constexpr uint32_t kOffOnes = 2 * kBufBytes;          // 65536
 constexpr uint32_t kOffBar = kOffOnes + 2048;         // 2 mma barriers + done
 constexpr uint32_t kOffMisc = kOffBar + 64;           // tmem base, abort flag
-constexpr uint32_t kOffZred = kOffMisc + 64;          // [8 warps][128] column-sum partials
-constexpr uint32_t kPreSmem = kOffZred + 8 * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kOffZred = kOffMisc + 64;          // [2][8 warps][128] column partials
+constexpr uint32_t kPreSmem = kOffZred + 2 * 8 * 128 * 4 + 1024;  // + alignment slack
 constexpr uint32_t kPreTmemCols = 128;                // H: 0..127
 
 // Raw 16-byte words holding 8 consecutive channels of T.
@@ -94,7 +95,8 @@ template <typename T>
 __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
     const T* __restrict__ k, const T* __restrict__ v, __half* __restrict__ phik, __half* __restrict__ v16,
     __nv_bfloat16* __restrict__ khat, float* __restrict__ hpart, float* __restrict__ zpart,
-    float* __restrict__ zblk, int N, int d, int nkv, int nsplit, int phi_kind, int* status) {
+    float* __restrict__ zblk, float* __restrict__ kstat, float* __restrict__ vstat, int N, int d, int nkv,
+    int nsplit, int phi_kind, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [0], [1]
@@ -135,6 +137,12 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
   const uint32_t idesc_h = idesc_f16(0, 1, 1, 128, 128);  // phi(K)^T (MN-major) x V (MN-major)
   bool ok = true;
   float zacc = 0.0f;  // threads < 128: this split's Z for channel tid, blocks in ascending order
+  float ksum[8], vmax[8];  // this thread's channels [8u, 8u+8): sum of K, absmax of V over its rows
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ksum[e] = 0.0f;
+    vmax[e] = 0.0f;
+  }
 
   // this thread's units of a 64-token tile: row m = tid/16 + 16*i, channels [8u, 8u+8)
   const int u = tid % 16;
@@ -159,6 +167,11 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
     for (int i = 0; i < kUnits; ++i) {
       unpack8<T>(kr[i], kf[i]);
       unpack8<T>(vr[i], vf[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {  // rows past N hold zeros
+        ksum[e] += kf[i][e];
+        vmax[e] = fmaxf(vmax[e], fabsf(vf[i][e]));
+      }
     }
     if (jb + 1 < jb1) fetch(jb + 1);  // next tile's loads overlap this tile's work
     // buffer reuse: the MMA that read this buffer two tiles ago must be done
@@ -267,6 +280,33 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
     have = have && w_ok;
   }
   tc_fence_after();
+  // per-split K column sums and V column absmax (used by the low-bit branch)
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ksum[e] += __shfl_xor_sync(0xffffffffu, ksum[e], 16);
+    vmax[e] = fmaxf(vmax[e], __shfl_xor_sync(0xffffffffu, vmax[e], 16));
+  }
+  __syncthreads();  // zred free
+  float* kred = reinterpret_cast<float*>(sm + kOffZred);
+  float* vred = kred + 8 * 128;
+  if ((tid & 31) < 16) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      kred[warp * 128 + 8 * u + e] = ksum[e];
+      vred[warp * 128 + 8 * u + e] = vmax[e];
+    }
+  }
+  __syncthreads();
+  if (tid < 128) {
+    float ks = 0.0f, vm = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kPreThreads / 32; ++w) {
+      ks += kred[w * 128 + tid];
+      vm = fmaxf(vm, vred[w * 128 + tid]);
+    }
+    kstat[(bh * nsplit + split) * kDPad + tid] = ks;
+    vstat[(bh * nsplit + split) * kDPad + tid] = vm;
+  }
   if (have && warp < 4) {
     zpart[(bh * nsplit + split) * kDPad + tid] = zacc;
     float* hp = hpart + ((bh * nsplit + split) * kDPad + tid) * kDPad;
@@ -342,7 +382,139 @@ __global__ void __launch_bounds__(256) qhat_kernel(const T* __restrict__ q, __nv
       make_uint4(pack_bf162(f[0], f[1]), pack_bf162(f[2], f[3]), pack_bf162(f[4], f[5]), pack_bf162(f[6], f[7]));
 }
 
+// ---------------------------------------------------------------- low-bit branch
+// "SLA2 深度解读 …" (jefxiong.cn) §07: Q, K, P, V quantised for the sparse
+// branch, K smoothed by its column mean first.  Readings (the page fixes
+// neither format nor granularity): e4m3, round to nearest even, saturating;
+// Q and K - mean(K) with one scale per 128-token block, V one per channel;
+// a block or channel with absmax a is multiplied by 448/a before rounding
+// and carries the scale a/448.
+
+// mean(K) and absmax(V) per (b,h) channel from the prepass's per-split partials.
+__global__ void __launch_bounds__(128) fp8_stats_kernel(const float* __restrict__ kstat,
+                                                        const float* __restrict__ vstat, float* __restrict__ mu,
+                                                        float* __restrict__ vamax, int nsplit, int N) {
+  const long long bh = blockIdx.x;
+  const int c = threadIdx.x;
+  float ks = 0.0f, vm = 0.0f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    ks += kstat[(bh * nsplit + sp) * kDPad + c];
+    vm = fmaxf(vm, vstat[(bh * nsplit + sp) * kDPad + c]);
+  }
+  mu[bh * kDPad + c] = ks / static_cast<float>(N);
+  vamax[bh * kDPad + c] = vm;
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+__device__ __forceinline__ float block_absmax(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = 0.0f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+// One 128-token block of one head per CTA (256 threads, 8 channel units each):
+// e4m3 copies of Q and K - mean(K) with the block's scale, and of V with the
+// per-channel scale.  Channels past d and rows past N stay zero.
+template <typename T>
+__global__ void __launch_bounds__(256) fp8_quant_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                        const T* __restrict__ v, const float* __restrict__ mu,
+                                                        const float* __restrict__ vamax, uint8_t* __restrict__ q8,
+                                                        uint8_t* __restrict__ k8, uint8_t* __restrict__ v8,
+                                                        float* __restrict__ sq, float* __restrict__ sk, int N, int d,
+                                                        int nb128) {
+  __shared__ float red[8];
+  const int blk = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const int tid = threadIdx.x, u = tid % 16;
+  const long long base = bh * static_cast<long long>(N);
+  float mc[8], vinv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int c = 8 * u + e;
+    mc[e] = c < d ? mu[bh * kDPad + c] : 0.0f;
+    const float a = c < d ? vamax[bh * kDPad + c] : 0.0f;
+    vinv[e] = a > 0.0f ? __fdiv_rn(448.0f, a) : 1.0f;
+  }
+  for (int which = 0; which < 3; ++which) {
+    const T* src = which == 0 ? q : (which == 1 ? k : v);
+    uint8_t* dst = which == 0 ? q8 : (which == 1 ? k8 : v8);
+    float x[8][8];
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int tok = blk * 128 + tid / 16 + 16 * i;
+      load8<T>(src + base * d, tok, d, u, tok < N, x[i]);
+      if (which == 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] = (tok < N && 8 * u + e < d) ? __fsub_rn(x[i][e], mc[e]) : 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[i][e]));
+    }
+    float inv[8];
+    if (which < 2) {
+      const float amax = block_absmax(am, red);
+      const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : __fdiv_rn(1.0f, 448.0f);
+      const float iv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+      if (tid == 0) (which == 0 ? sq : sk)[bh * nb128 + blk] = sc;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) inv[e] = iv;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) inv[e] = vinv[e];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int tok = blk * 128 + tid / 16 + 16 * i;
+      if (tok < N) {
+        const float* y = x[i];
+        const uint2 w = make_uint2(e4m3x4(__fmul_rn(y[0], inv[0]), __fmul_rn(y[1], inv[1]), __fmul_rn(y[2], inv[2]),
+                                          __fmul_rn(y[3], inv[3])),
+                                   e4m3x4(__fmul_rn(y[4], inv[4]), __fmul_rn(y[5], inv[5]), __fmul_rn(y[6], inv[6]),
+                                          __fmul_rn(y[7], inv[7])));
+        *reinterpret_cast<uint2*>(dst + (base + tok) * kDPad + 8 * u) = w;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_fp8_quant(const sla_shape& s, const void* q, const void* k, const void* v, const WsLayout& L,
+                             char* ws, cudaStream_t st) {
+  const int BH = s.B * s.H;
+  const int nb128 = ceil_div(s.N, 128);
+  float* mu = reinterpret_cast<float*>(ws + L.mu);
+  float* vam = reinterpret_cast<float*>(ws + L.sv);
+  fp8_stats_kernel<<<BH, 128, 0, st>>>(reinterpret_cast<const float*>(ws + L.kstat),
+                                       reinterpret_cast<const float*>(ws + L.vstat), mu, vam, L.nsplit, s.N);
+  dim3 grid(nb128, BH);
+  auto* q8 = reinterpret_cast<uint8_t*>(ws + L.q8);
+  auto* k8 = reinterpret_cast<uint8_t*>(ws + L.k8);
+  auto* v8 = reinterpret_cast<uint8_t*>(ws + L.v8);
+  auto* sq = reinterpret_cast<float*>(ws + L.sq);
+  auto* sk = reinterpret_cast<float*>(ws + L.sk);
+  if (s.in_dtype == SLA_BF16)
+    fp8_quant_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), mu, vam, q8, k8, v8, sq, sk, s.N, s.d, nb128);
+  else
+    fp8_quant_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                   static_cast<const float*>(v), mu, vam, q8, k8, v8, sq, sk, s.N,
+                                                   s.d, nb128);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
                            char* ws, cudaStream_t st) {
@@ -365,7 +537,8 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
     if (e != cudaSuccess) return e;
     lin_prepass_kernel<__nv_bfloat16><<<grid, kPreThreads, kPreSmem, st>>>(
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), phik, v16, khat, hpart,
-        zpart, reinterpret_cast<float*>(ws + L.zblk), s.N, s.d, nkv, L.nsplit, phi, status);
+        zpart, reinterpret_cast<float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.kstat),
+        reinterpret_cast<float*>(ws + L.vstat), s.N, s.d, nkv, L.nsplit, phi, status);
   } else {
     e = cudaFuncSetAttribute(lin_prepass_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmem);
     if (e == cudaSuccess)
@@ -373,7 +546,8 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
     if (e != cudaSuccess) return e;
     lin_prepass_kernel<float><<<grid, kPreThreads, kPreSmem, st>>>(
         static_cast<const float*>(k), static_cast<const float*>(v), phik, v16, khat, hpart, zpart,
-        reinterpret_cast<float*>(ws + L.zblk), s.N, s.d, nkv, L.nsplit, phi, status);
+        reinterpret_cast<float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.kstat),
+        reinterpret_cast<float*>(ws + L.vstat), s.N, s.d, nkv, L.nsplit, phi, status);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

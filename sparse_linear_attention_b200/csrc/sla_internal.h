@@ -26,6 +26,12 @@ struct WsLayout {
   size_t hs16 = 0, ztot = 0;    // fp16 [BH, 128, 128] = H_tot / sigma, fp32 [BH, 128] = Z_tot
   size_t sigma = 0;             // fp32 [BH]: per-head power of two >= max_e Z_tot[e]
   size_t zblk = 0;              // fp32 [BH, n_kv, 128]: colsum of phi(K) per key block
+  size_t kstat = 0, vstat = 0;  // fp32 [BH, nsplit, 128]: per-split column sum of K, column absmax of V
+  // low-bit sparse branch (only with SLA_WS_FP8)
+  size_t q8 = 0, k8 = 0, v8 = 0;  // e4m3 [BH, N, 128]: Q, K - mean(K), V
+  size_t sq = 0, sk = 0;          // fp32 [BH, ceil(N/128)]: per-block scales of Q and K - mean(K)
+  size_t mu = 0, sv = 0;          // fp32 [BH, 128]: column mean of K, column absmax of V
+  bool fp8 = false;
   size_t lists = 0;             // SLA: int32 [BH, n_q, 2, n_kv] critical / negligible lists
   size_t counts = 0;            // SLA: int32 [BH, n_q, 2]
   size_t total = 0;
@@ -40,8 +46,10 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-inline WsLayout ws_layout(const sla_shape& s, int mode) {
+inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
+  const int mode = mode_flags & 0xFF;
   WsLayout L;
+  L.fp8 = (mode_flags & SLA_WS_FP8) != 0;
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
   L.need_hat = (s.d != kDPad) || (s.in_dtype == SLA_F32);
@@ -70,6 +78,18 @@ inline WsLayout ws_layout(const sla_shape& s, int mode) {
   L.ztot = take(BH * kDPad * 4);
   L.sigma = take(BH * 4);
   L.zblk = take(BH * static_cast<size_t>(nkv) * kDPad * 4);
+  L.kstat = take(BH * L.nsplit * kDPad * 4);
+  L.vstat = take(BH * L.nsplit * kDPad * 4);
+  if (L.fp8) {
+    const size_t nb128 = static_cast<size_t>(ceil_div(s.N, 128));
+    L.q8 = take(BH * s.N * kDPad);
+    L.k8 = take(BH * s.N * kDPad);
+    L.v8 = take(BH * s.N * kDPad);
+    L.sq = take(BH * nb128 * 4);
+    L.sk = take(BH * nb128 * 4);
+    L.mu = take(BH * kDPad * 4);
+    L.sv = take(BH * kDPad * 4);
+  }
   if (mode == SLA_MODE_SLA_3WAY) {
     L.lists = take(BH * nq * 2 * static_cast<size_t>(nkv) * 4);
     L.counts = take(BH * nq * 2 * 4);

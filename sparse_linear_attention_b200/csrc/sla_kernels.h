@@ -15,6 +15,10 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
 cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
                            char* ws, cudaStream_t st);
 
+// e4m3 copies of Q, K - mean(K), V and their scales (needs sla_prepare's statistics).
+cudaError_t launch_fp8_quant(const sla_shape& s, const void* q, const void* k, const void* v, const WsLayout& L,
+                             char* ws, cudaStream_t st);
+
 cudaError_t launch_qhat(const sla_shape& s, const void* q, const WsLayout& L, char* ws, cudaStream_t st);
 
 cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, const WsLayout& L, char* ws,
@@ -37,13 +41,23 @@ struct SparseArgs {
   int out_bf16;
   int phi;
   int* status;
+  // e4m3 sparse branch
+  int fp8;
+  int nb128;                 // ceil(N / 128)
+  const float* sq;           // [BH, nb128] per-block scale of Q
+  const float* sk;           // [BH, nb128] per-block scale of K - mean(K)
+  const float* vamax;        // [BH, 128] column absmax of V
+  const void* qsrc;          // bf16 [BH, N, 128] Q (for phi(Q) when the smem tile holds e4m3)
 };
 
 // 3-D tensor map over a [BH][N][128] 16-bit array: boxes of 64 channels x
 // box_rows tokens, 128-byte swizzle, rows past N read as zero.
 cudaError_t encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int N, int BH, int box_rows);
+// Same over a [BH][N][128] byte array (e4m3), boxes of 128 bytes x box_rows.
+cudaError_t encode_map8(CUtensorMap* map, const void* base, int N, int BH, int box_rows);
 
 cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
-                          const void* phik16, const void* v16, const void* hs16, cudaStream_t st);
+                          const void* phik16, const void* v16, const void* hs16, const void* q8, const void* k8,
+                          const void* v8, cudaStream_t st);
 
 }  // namespace sla

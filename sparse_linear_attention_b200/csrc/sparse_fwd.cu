@@ -40,6 +40,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "sla_device.cuh"
@@ -52,19 +53,30 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kCompute = 256;
-constexpr int kStages = 3;                                   // slots of each ring
-constexpr uint32_t OFF_Q = 0;                                // Q tile (bf16): 2 x [128 rows][128 B]
-constexpr uint32_t KSLOT = 16384;                            // K tile: 2 x [64 rows][128 B]
-constexpr uint32_t VSLOT = 32768;                            // phi(K) | V tiles, each 2 x [64 rows][128 B]
-constexpr uint32_t OFF_K = 32768;
-constexpr uint32_t OFF_V = OFF_K + kStages * KSLOT;          // 81920
-constexpr uint32_t OFF_H = OFF_V + kStages * VSLOT;          // 180224: H_i (fp16) / W_proj (bf16), MN-major
-constexpr uint32_t OFF_BAR = OFF_H + 32768;                  // 212992
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;                 // tmem base, abort flag
-constexpr uint32_t OFF_RED = OFF_MISC + 64;                  // [4 slots][2 halves][128 rows] floats
-constexpr uint32_t OFF_Z = OFF_RED + 4096;                   // Z_i [128] + Z_ex halves [2][128] floats
-constexpr uint32_t SMEM_BYTES = OFF_Z + 1536 + 1024;         // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int kStages = 3;  // slots of each ring
+
+// Shared-memory layout.  bf16 branch: Q tile 2 x [128 rows][128 B], K tile
+// 2 x [64 rows][128 B], V slot = phi(K) | V (fp16, each 2 x [64 rows][128 B]).
+// e4m3 branch: Q8 [128 rows][128 B], K8 [64 rows][128 B], V slot = phi(K) |
+// V (fp16) | V8 [64 rows][128 B].  Then H_i / W_proj (MN-major, 32 KB),
+// barriers, flags, exchange buffers.
+template <bool kFP8>
+struct Lay {
+  static constexpr uint32_t QBYTES = kFP8 ? 16384 : 32768;
+  static constexpr uint32_t KSLOT = kFP8 ? 8192 : 16384;
+  static constexpr uint32_t VSLOT = kFP8 ? 40960 : 32768;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = QBYTES;
+  static constexpr uint32_t OFF_V = OFF_K + kStages * KSLOT;
+  static constexpr uint32_t OFF_H = OFF_V + kStages * VSLOT;
+  static constexpr uint32_t OFF_BAR = OFF_H + 32768;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + 256;  // tmem base, abort flag
+  static constexpr uint32_t OFF_RED = OFF_MISC + 64;   // [4 slots][2 halves][128 rows] floats
+  static constexpr uint32_t OFF_Z = OFF_RED + 4096;    // Z_i [128] + Z_ex halves [2][128] floats
+  static constexpr uint32_t SMEM_BYTES = OFF_Z + 1536 + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_H % 1024 == 0, "1 KB aligned tiles");
+};
 
 // TMEM columns (512 allocated; one CTA per SM)
 constexpr uint32_t T_S0 = 0, T_S1 = 64, T_P0 = 128, T_P1 = 160, T_O = 192, T_HK = 320;
@@ -146,10 +158,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok) != 0;
 }
 
+template <bool kFP8>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmV,
-                      const __grid_constant__ CUtensorMap tmH, const SparseArgs a) {
+                      const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmV8,
+                      const SparseArgs a) {
+  using L = Lay<kFP8>;
+  constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, OFF_H = L::OFF_H;
+  constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_RED = L::OFF_RED, OFF_Z = L::OFF_Z;
+  constexpr uint32_t KSLOT = L::KSLOT, VSLOT = L::VSLOT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
@@ -205,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmPhi);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmH);
+      if constexpr (kFP8) tma_prefetch_desc(&tmV8);
       int gk = 0, gv = 0, q_issued = 0, h_issued = 0;
       bool ok = true;
       auto load_block = [&](const Tile& T, int it) -> bool {
@@ -217,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t* fb = &bars[B_KFULL + sl];
           mbar_arrive_expect_tx(fb, KSLOT);
           tma_load_3d(sm + OFF_K + sl * KSLOT, &tmK, fb, 0, krow, T.bh);
-          tma_load_3d(sm + OFF_K + sl * KSLOT + 8192, &tmK, fb, 64, krow, T.bh);
+          if constexpr (!kFP8) tma_load_3d(sm + OFF_K + sl * KSLOT + 8192, &tmK, fb, 64, krow, T.bh);
           ++gk;
         }
         const int sl = gv % kStages;
@@ -230,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(vb + 8192, &tmPhi, fb, 64, krow, T.bh);
         tma_load_3d(vb + 16384, &tmV, fb, 0, krow, T.bh);
         tma_load_3d(vb + 16384 + 8192, &tmV, fb, 64, krow, T.bh);
+        if constexpr (kFP8) tma_load_3d(vb + 32768, &tmV8, fb, 0, krow, T.bh);
         ++gv;
         return true;
       };
@@ -241,9 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (; ok && it < pre; ++it) ok = load_block(T, it);  // key blocks first: they only need ring slots
         if (!ok) break;
         if (ti > 0 && !mbar_wait(&bars[B_QFREE], (ti - 1) & 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(&bars[B_QFULL], 32768);
+        mbar_arrive_expect_tx(&bars[B_QFULL], L::QBYTES);
         tma_load_3d(sm + OFF_Q, &tmQ, &bars[B_QFULL], 0, T.qb * a.bq, T.bh);
-        tma_load_3d(sm + OFF_Q + 16384, &tmQ, &bars[B_QFULL], 64, T.qb * a.bq, T.bh);
+        if constexpr (!kFP8) tma_load_3d(sm + OFF_Q + 16384, &tmQ, &bars[B_QFULL], 64, T.qb * a.bq, T.bh);
         q_issued = ti + 1;
         if (T.has_lin) {
           // H_tot / sigma of this head into the H buffer once the previous tile is done with it
@@ -277,14 +297,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dPhi = sdesc_sw128(smem_u32(sm + OFF_V), 8192, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sm + OFF_V) + 16384, 8192, 1024);
       const uint64_t dH = sdesc_sw128(smem_u32(sm + OFF_H), 16384, 1024);
+      const uint64_t dV8 = sdesc_sw128(smem_u32(sm + OFF_V) + 32768, 16, 1024);  // MN-major, N fits one atom
+      const uint32_t id_qk8 = idesc_f8(0, 0, 128, 64);   // Q8 (K-major) x K8 (K-major), e4m3
+      const uint32_t id_pv8 = idesc_f8(0, 1, 128, 128);  // P8 (TMEM) x V8 (MN-major), e4m3
       auto issue_qk = [&](int sl, int b) {
         const uint64_t kb = dK + ((sl * KSLOT) >> 4);
         const uint32_t d = tmem + (b ? T_S1 : T_S0);
+        if constexpr (kFP8) {
+          // e4m3 x e4m3: 4 MMAs of K = 32 inside the single 128-byte-wide tile
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t qo = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-          const uint32_t ko = ((kk >> 2) * 8192u + (kk & 3) * 32u) >> 4;
-          mma_f16_ss(d, dQ + qo, kb + ko, id_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + kk * 2u, kb + kk * 2u, id_qk8, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t qo = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+            const uint32_t ko = ((kk >> 2) * 8192u + (kk & 3) * 32u) >> 4;
+            mma_f16_ss(d, dQ + qo, kb + ko, id_qk, kk > 0 ? 1u : 0u);
+          }
         }
       };
       auto issue_h = [&](int sl, bool first) {
@@ -294,11 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16_ss(tmem + T_HK, pb + kk * 128u, vb + kk * 128u, id_h, (first && kk == 0) ? 0u : 1u);
       };
       auto issue_pv = [&](int sl, int b, bool first) {
-        const uint64_t vb = dV + ((sl * VSLOT) >> 4);
         const uint32_t pa = tmem + (b ? T_P1 : T_P0);
+        if constexpr (kFP8) {
+          // P8 (TMEM, 4 keys per column) x V8 (MN-major, one 128-byte atom wide): K = 32 per MMA
+          const uint64_t vb = dV8 + ((sl * VSLOT) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16_ts(tmem + T_O, pa + kk * 8u, vb + kk * 128u, id_pv, (first && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < 2; ++kk)
+            mma_f8_ts(tmem + T_O, pa + kk * 8u, vb + kk * 256u, id_pv8, (first && kk == 0) ? 0u : 1u);
+        } else {
+          const uint64_t vb = dV + ((sl * VSLOT) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ts(tmem + T_O, pa + kk * 8u, vb + kk * 128u, id_pv, (first && kk == 0) ? 0u : 1u);
+        }
       };
       // D[col] = A (TMEM, 64 columns of 16-bit pairs) x B (smem MN-major [128 K rows] x 2 chunks of 64 N)
       auto issue_ts128 = [&](uint32_t a_col, uint32_t col, uint32_t idesc, bool first) {
@@ -401,6 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
       const float sigma_t = T.has_lin ? a.sigma[T.bh] : 1.0f;
       const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
+      float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
+      if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
       float m_run = -INFINITY, l_part = 0.0f;
       for (int i = 0; i < T.n_crit; ++i) {
         const int b = (gs + i) & 1;
@@ -413,6 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) s[c] = 0.0f;
+        }
+        float sc = a.sl2;
+        if constexpr (kFP8) {
+          const int j = block_at(T, i, a.nkv, nullptr);
+          sc = sl2_q * a.sk[static_cast<long long>(T.bh) * a.nb128 + (j >> 1)];  // 128-token key scale block
         }
         if (tail) {
           const int j = block_at(T, i, a.nkv, nullptr);
@@ -428,10 +472,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) m8[c] = fmaxf(fmaxf(s[4 * c], s[4 * c + 1]), fmaxf(s[4 * c + 2], s[4 * c + 3]));
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        RED(i & 1, half)[r] = mx * a.sl2;
+        RED(i & 1, half)[r] = mx * sc;
         named_bar_sync(pair_bar, 64);
         const float mt = fmaxf(RED(i & 1, 0)[r], RED(i & 1, 1)[r]);
-        const bool need = mt > m_run + 15.0f;
+        // bf16: refresh the max only when it grows by more than 15 (p <= 2^15 fits
+        // fp16); e4m3: p * 448 must stay within e4m3, so the exact running max
+        const bool need = kFP8 ? (mt > m_run) : (mt > m_run + 15.0f);
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mt : m_run;
           const float f = need ? ex2_approx(m_run - m_new) : 1.0f;
@@ -460,16 +506,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
         const float nm = -m_run;
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if constexpr (kFP8) {
+          // p in (0, 1] against the running max; the row sum uses the unquantised p,
+          // the PV MMA p * 448 rounded to e4m3 (four keys per TMEM column)
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2_approx(fmaf(s[2 * c], a.sl2, nm));
-          const float p1 = ex2_approx(fmaf(s[2 * c + 1], a.sl2, nm));
-          l4[c & 3] += p0 + p1;
-          pk[c] = pack_half2(p0, p1);
+          for (int c = 0; c < 8; ++c) {
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(s[4 * c + e], sc, nm));
+            l4[c & 3] += (p[0] + p[1]) + (p[2] + p[3]);
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0] * 448.0f, p[1] * 448.0f), __NV_SATFINITE,
+                                                         __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2] * 448.0f, p[3] * 448.0f), __NV_SATFINITE,
+                                                         __NV_E4M3);
+            pk[c] = lo | (hi << 16);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2_approx(fmaf(s[2 * c], sc, nm));
+            const float p1 = ex2_approx(fmaf(s[2 * c + 1], sc, nm));
+            l4[c & 3] += p0 + p1;
+            pk[c] = pack_half2(p0, p1);
+          }
         }
         l_part += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         if (ok) {
-          tmem_st16(tmem + lrow + (b ? T_P1 : T_P0) + 16 * half, pk);
+          if constexpr (kFP8)
+            tmem_st8(tmem + lrow + (b ? T_P1 : T_P0) + 8 * half, pk);
+          else
+            tmem_st16(tmem + lrow + (b ? T_P1 : T_P0) + 16 * half, pk);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&bars[B_PFULL + b]);
@@ -532,7 +598,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[64];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 16384u + sw128_off(r, u));
+          uint4 w;
+          if constexpr (kFP8) {  // the smem tile holds e4m3 Q: read the bf16 row (L2-resident)
+            w = make_uint4(0, 0, 0, 0);
+            if (tok < a.N)
+              w = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
+                                                  (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
+          } else {
+            w = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 16384u + sw128_off(r, u));
+          }
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -660,6 +734,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && T.n_crit > 0) tmem_ld32(tmem + lrow + T_O + 64 * half + 32 * cc, o);
         if (ok && T.has_lin) tmem_ld32(tmem + lrow + lin_col + 64 * half + 32 * cc, nmv);
         tmem_wait_ld();
+        if constexpr (kFP8) {  // O accumulates e4m3 codes: times (absmax_c / 448) / 448 per channel
+          const float* va = a.vamax + static_cast<long long>(T.bh) * kDPad + 64 * half + 32 * cc;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
+        }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float os = (T.n_crit > 0) ? o[c] * w_s : 0.0f;
@@ -703,23 +782,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
-                          const void* phik16, const void* v16, const void* hs16, cudaStream_t st) {
-  CUtensorMap mq, mk, mp, mv, mh;
-  cudaError_t e;
-  if ((e = encode_map(&mq, q_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
-  if ((e = encode_map(&mk, k_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
-  if ((e = encode_map(&mp, phik16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
-  if ((e = encode_map(&mv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
-  if ((e = encode_map(&mh, hs16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kDPad, a.BH, 128)) != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(sparse_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+template <bool kFP8>
+static cudaError_t launch_sparse_t(const SparseArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
+                                   const CUtensorMap& mp, const CUtensorMap& mv, const CUtensorMap& mh,
+                                   const CUtensorMap& mv8, cudaStream_t st) {
+  constexpr uint32_t smem = Lay<kFP8>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(sparse_fwd_kernel<kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long ntiles = static_cast<long long>(a.BH) * a.nq;
   const unsigned grid = static_cast<unsigned>(ntiles < sms ? ntiles : sms);
-  sparse_fwd_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mp, mv, mh, a);
+  sparse_fwd_kernel<kFP8><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
+                          const void* phik16, const void* v16, const void* hs16, const void* q8, const void* k8,
+                          const void* v8, cudaStream_t st) {
+  CUtensorMap mq, mk, mp, mv, mh, mv8;
+  cudaError_t e;
+  if ((e = encode_map(&mp, phik16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mh, hs16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kDPad, a.BH, 128)) != cudaSuccess) return e;
+  if (a.fp8) {
+    if ((e = encode_map8(&mq, q8, a.N, a.BH, 128)) != cudaSuccess) return e;
+    if ((e = encode_map8(&mk, k8, a.N, a.BH, 64)) != cudaSuccess) return e;
+    if ((e = encode_map8(&mv8, v8, a.N, a.BH, 64)) != cudaSuccess) return e;
+    return launch_sparse_t<true>(a, mq, mk, mp, mv, mh, mv8, st);
+  }
+  if ((e = encode_map(&mq, q_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mk, k_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
+  return launch_sparse_t<false>(a, mq, mk, mp, mv, mh, mv, st);
 }
 
 }  // namespace sla

@@ -20,6 +20,7 @@ SLA_F32, SLA_BF16 = 0, 1
 SLA_PHI_ELU1, SLA_PHI_SOFTMAX = 0, 1
 SLA_MODE_SLA2_TOPK, SLA_MODE_SLA_3WAY = 0, 1
 SLA_FLAG_PREPARED, SLA_FLAG_FP8 = 1, 2
+SLA_WS_FP8 = 0x100
 
 STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_ALIGNMENT",
                 4: "SLA_ERR_WORKSPACE", 5: "SLA_ERR_CUDA", 6: "SLA_ERR_TIMEOUT", 7: "SLA_ERR_DEVICE_INDEX"}

@@ -110,7 +110,9 @@ def test_attention_rejects_bad_arguments_before_launch():
     assert call(alpha=None) == 1
     assert call(phi=2) == 1
     assert call(flags=8) == 1
-    assert call(flags=sla.SLA_FLAG_FP8) == 2
+    # the e4m3 branch needs the larger workspace (sla_workspace_size with SLA_WS_FP8)
+    need = sla.sla_workspace_size(s, 0)
+    assert call(flags=sla.SLA_FLAG_FP8, wsb=need) == 4
     assert call(out=None) == 1
     assert call(out=FAKE + 4) == 3
     assert call(odt=9) == 1
@@ -126,6 +128,8 @@ def test_attention_rejects_bad_arguments_before_launch():
     assert call3(labels=None) == 1
     assert call3(wp=None) == 1
     assert call3(wp=FAKE + 2) == 3
+    assert L.sla_attn_fwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, 0, sla.SLA_FLAG_FP8, FAKE, 1, FAKE,
+                          1 << 40, None) == 2  # e4m3 branch: SLA2 only
     # the SLA workspace also holds the per-row block lists
     need2 = sla.sla_workspace_size(s, 0)
     assert call3(wsb=need2) == 4

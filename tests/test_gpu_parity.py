@@ -218,3 +218,45 @@ def test_sla_label_edge_cases():
     lab[0, 1, 1, :] = 0
     lab[0, 1, 1, 0] = -1         # marginal except one negligible block
     _sla_check(w, x, lab)
+
+
+# ------------------------------------------------------------------ e4m3 sparse branch
+
+def _fp8_check(w, x, kept, blocks=None, heads=None):
+    from tests.gpu_common import TOL_FP8
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, flags=sla.SLA_FLAG_FP8)
+    hs = list(range(w.H)) if heads is None else heads
+    sub = lambda t: t[:, hs]  # noqa: E731
+    want = orc.sla2_forward_fp8(as64(sub(x["q"])), as64(sub(x["k"])), as64(sub(x["v"])), kept[:, hs],
+                                x["alpha"][:, hs].numpy(), w.bq, w.bkv, blocks=blocks)["o"]
+    if blocks is None:
+        blocks = [(0, h, i) for h in range(len(hs)) for i in range(w.n_q)]
+    return compare(got[:, hs], want, blocks, w.bq, tol=TOL_FP8)
+
+
+def test_fp8_tiny_all_rows():
+    w, x = workload("tiny")
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, k_of(w))
+    _fp8_check(w, x, kept)
+
+
+@pytest.mark.parametrize("ratio", [0.03, 0.05, 0.10])
+def test_fp8_wan13_keep_sweep(ratio):
+    w, x = workload("wan13")
+    kk = orc.keep_count(ratio, w.n_kv)
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, kk)
+    _fp8_check(w, x, kept, blocks=sample_blocks(1, 3, w.n_q, 3, seed=4), heads=[0, 5, 11])
+
+
+def test_fp8_wan14_sampled_blocks():
+    _, x = workload("wan14")  # same seeded inputs as the e4m3 14B workload
+    w = inputs.WORKLOADS["fp8_14"]
+    kk = k_of(w)
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, kk)
+    _fp8_check(w, x, kept, blocks=sample_blocks(1, 3, w.n_q, 3, seed=5), heads=[0, 21, 39])
+
+
+@pytest.mark.parametrize("N,d,bq", [(777, 128, 64), (300, 64, 128)])
+def test_fp8_ragged_shapes(N, d, bq):
+    w, x = _rand_case(N, d, bq=bq, scale=1.5)
+    _fp8_check(w, x, _rand_kept(w, min(3, w.n_kv)))
