@@ -327,9 +327,13 @@ def e4m3_round(x32: np.ndarray) -> np.ndarray:
 #     inv = 448 / amax in fp32 (1 if amax = 0), x8 = e4m3(fp32(x * inv)),
 #     scale = amax / 448 in fp32;
 #   - V: one scale per (b,h) and channel over all valid tokens, same rule;
-#   - P: online softmax over the kept blocks in ascending order; after each
-#     block p = exp(S - m) with m the running row max including that block,
-#     p8 = e4m3(fp32(p * 448)); the row sum uses the unquantised p.
+#   - P: online softmax over the kept blocks in ascending order, taken a tile
+#     of kv_tile consecutive kept blocks at a time (the page leaves the tile
+#     width open; 2 blocks = 128 keys by default, the width of the attention
+#     kernel's softmax step); after each tile p = exp(S - m) with m the
+#     running row max including that tile, p8 = e4m3(fp32(p * 448)); the row
+#     sum uses the unquantised p.  Without quantisation the tile width does
+#     not change the result (online softmax is exact for any grouping).
 # ----------------------------------------------------------------------------
 
 def _e4m3_q(x32, codec):
@@ -350,7 +354,8 @@ def _quant_blocks(x32, blk, codec):
     return vals, np.array(scales, dtype=F64)
 
 
-def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, codec=None, qblk=128):
+def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, codec=None, qblk=128,
+                     kv_tile=2):
     """SLA2 output with the low-bit sparse branch described above; the linear
     branch and the combine are the fp64 ones of sla2_forward.  q, k, v: exact
     values of the inputs as float64 [B,H,N,d].  codec(x32) -> float64 values
@@ -384,8 +389,8 @@ def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None
             l = np.zeros(len(rows))
             acc = np.zeros((len(rows), v.shape[-1]))
             qdq = q8[rows] * sq[tok_q[rows]][:, None]
-            for j in sel:
-                keys = _rows(j, bkv, N)
+            for g0 in range(0, len(sel), kv_tile):
+                keys = np.concatenate([_rows(j, bkv, N) for j in sel[g0:g0 + kv_tile]])
                 kdq = k8[keys] * sk[tok_q[keys]][:, None]
                 s = (qdq @ kdq.T) / math.sqrt(d)
                 m_new = np.maximum(m, s.max(axis=1))

@@ -455,8 +455,37 @@ def pin_fp8_block_scales(orc):
     assert np.array_equal(vals[2], [448.0, 0.0]) and np.allclose(vals[2] * scales[1], [1.0, 0.0])
 
 
+def pin_fp8_tile_width_exact_without_quantisation(orc):
+    """Online softmax is exact for any grouping of the kept blocks into tiles:
+    with the identity codec, tiles of 1, 2 or 3 kept blocks (3 kept per row,
+    so the grouping 2 + 1 occurs) agree up to the fp32 rounding of p * 448,
+    and match the fp64 SLA2 output."""
+    q, k, v, _, alpha = _fp8_case(93)
+    kept = np.array([[[[0, 2, 4], [1, 3, 4], [0, 1, 2]]]])
+    ident = lambda x: np.asarray(x, np.float64)  # noqa: E731
+    outs = [orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64, codec=ident, kv_tile=t)["o"] for t in (1, 2, 3)]
+    # the values reaching the codec are still rounded to fp32 against each tile's max
+    assert max(np.abs(outs[0] - o).max() for o in outs[1:]) < 1e-6
+    ref = orc.sla2_forward(q, k, v, kept, alpha, 128, 64)["o"]
+    assert np.abs(outs[1] - ref).max() < 1e-6
+
+
+def pin_fp8_tile_width_moves_quantisation(orc):
+    """With e4m3 on, P is quantised against the running max of its tile, so
+    the tile width changes the rounding (and only the rounding): the outputs
+    for 1 and 3 blocks per tile differ, by no more than the quantisation
+    error itself."""
+    q, k, v, _, alpha = _fp8_case(94)
+    kept = np.array([[[[0, 2, 4], [1, 3, 4], [0, 1, 2]]]])
+    a = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64, kv_tile=1)["o_s"]
+    b = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64, kv_tile=3)["o_s"]
+    d = np.abs(a - b).max()
+    assert 0.0 < d < 0.1, d
+
+
 ALL_PINS = [pin_hand_example, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
-            pin_fp8_k_smoothing, pin_fp8_block_scales, 
+            pin_fp8_k_smoothing, pin_fp8_block_scales, pin_fp8_tile_width_exact_without_quantisation,
+            pin_fp8_tile_width_moves_quantisation,
     pin_pool_bruteforce, pin_project_bruteforce, pin_scores_bruteforce, pin_topk_sort,
     pin_labels, pin_keep_count, pin_router_identity_and_permutation,
     pin_all_kept_is_full_attention, pin_masked_mass_identity, pin_nothing_kept_is_linear_attention,

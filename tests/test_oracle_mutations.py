@@ -34,6 +34,8 @@ MUTATIONS = {
     "fp8_no_k_smoothing": ("kp32 = (ks - mu).astype(F32)", "kp32 = ks.astype(F32)"),
     "fp8_p_not_rescaled": ("p8 = _e4m3_q((p * 448.0).astype(F32), codec) / 448.0",
                            "p8 = _e4m3_q((p * 448.0).astype(F32), codec)"),
+    "fp8_tile_drops_blocks": ("sel[g0:g0 + kv_tile]", "sel[g0:g0 + 1]"),
+    "fp8_tile_width_ignored": ("for g0 in range(0, len(sel), kv_tile):", "for g0 in range(0, len(sel), kv_tile):\n                kv_tile = 1"),
     "fp8_key_scale_of_row_block": ("kdq = k8[keys] * sk[tok_q[keys]][:, None]",
                                    "kdq = k8[keys] * sk[tok_q[rows[0]]]"),
 }
