@@ -10,33 +10,43 @@
 // and 关键设计 4 (sparse and linear parts in one kernel; h_j added per block).
 //
 // B200 design: persistent CTAs (one per SM), each walking 128-row query tiles
-// (b, h, query block) in head-major order; 320 threads:
-//   warp 8      TMA producer, running ahead across tiles: per listed key
-//               block its K tile (bf16) into a 3-slot ring that frees as soon
-//               as the S MMA has read it, and its phi(K), V tiles (fp16) into a
-//               3-slot ring that frees after PV; per tile the Q tile and the
-//               fp16 H_tot / sigma tile of its head.
+// (b, h, query block) in head-major order.  The listed key blocks of a tile
+// are taken two at a time ("steps" of 128 keys): one N = 128 tensor-core
+// product per step for S, and one max exchange per 128 keys.  320 threads:
+//   warp 8      TMA producer, running ahead across tiles: per step the two
+//               key tiles side by side in one 128-row slot of a 2-slot ring
+//               (freed once S has read it); per listed block its phi(K), V
+//               tiles (fp16) in a 4-slot ring (freed after PV); per tile the
+//               Q tile (as soon as the previous tile's S products are done)
+//               and, in the next ring slot after its blocks, the fp16
+//               H_tot / sigma tile of its head.
 //   warp 9      tcgen05 issuer (one thread), fp32 accumulators in TMEM:
-//                 S_j   = Q K_j^T                    (bf16 operands from smem)
+//                 S     = Q [K_a | K_b]^T               (bf16 operands in smem)
 //                 H_ex += phi(K_j)^T V_j                (fp16)
-//                 O    += P_j V_j                    (fp16 P read from TMEM)
-//               and per tile phi(Q) H_i (fp16, phi(Q) in TMEM), for SLA also
-//               O_l W_proj (bf16 hi + lo split, O_l in TMEM).
+//                 O    += [P_a | P_b] [V_a ; V_b]       (fp16 P read from TMEM)
+//               in the order S_{i+1}, H_i, PV_i so S runs ahead of the
+//               softmax; per tile phi(Q) H_i / sigma (phi(Q) in TMEM), for SLA
+//               also O_l W_proj (bf16 hi + lo split).  It starts the next
+//               tile's first S product before the previous tile's epilogue
+//               products.
 //   warps 0..7  softmax and epilogue: warp w owns query rows 32(w%4)..+31
-//               (its TMEM lane quarter) and key / channel half w/4, so two
-//               warps share each row and every sub-partition runs two.
-//               Online softmax in log2 units with the running max refreshed
-//               only when a block's max exceeds it by more than 15 (exact:
-//               the stale max scales numerator and denominator alike, and
-//               p <= 2^15 still fits fp16); P is rounded to fp16 and stored
-//               to TMEM for the PV MMA.
+//               (its TMEM lane quarter) and key / channel half w/4 (one of
+//               the two key blocks of a step), so two warps share each row.
+//               Online softmax in log2 units; the running max is refreshed
+//               only when a step's max exceeds it by more than 15 (exact: the
+//               stale max scales numerator and denominator alike, and
+//               p <= 2^15 still fits fp16).  P is rounded to fp16 and written
+//               over the step's S columns in TMEM for the PV product.
+//               The epilogue re-reads the tile's Q rows (bf16, L2-resident)
+//               for phi(Q), so the Q tile in smem is replaced as soon as the
+//               tile's S products are done.
+// TMEM (512 columns): S0 | S1 (128 each, P over their first 64) | O (128) |
+// H_ex (128, then phi(Q) H_i or the SLA projection in the epilogue).
 // The linear branch uses H_i = H_tot - sum over the listed blocks of
-// phi(K_j)^T V_j (H_tot from sla_prepare): one extra 128x128x64 MMA per
-// listed block instead of a sum over every unselected block; Z_ex sums the
-// per-block column sums of phi(K) that sla_prepare stores.  H_i enters the
-// MMA as fp16 scaled by an exact power of two sigma >= max_e Z_tot[e], which
-// bounds |H_i / sigma| by max|V|; H_tot / sigma arrives by TMA and the
-// epilogue subtracts H_ex / sigma in place.
+// phi(K_j)^T V_j (H_tot from sla_prepare) and Z_i = Z_tot - the listed
+// blocks' column sums of phi(K), summed during the steps.  H_i enters the
+// product as fp16 scaled by an exact power of two sigma >= max_e Z_tot[e],
+// which bounds |H_i / sigma| by max|V|.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -53,66 +63,65 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kCompute = 256;
-constexpr int kStages = 3;  // slots of each ring
+constexpr int kKSlots = 2;  // key-pair slots
+constexpr int kVSlots = 4;  // phi(K) | V block slots (one also carries the H tile)
 
-// Shared-memory layout.  bf16 branch: Q tile 2 x [128 rows][128 B], K tile
-// 2 x [64 rows][128 B], V slot = phi(K) | V (fp16, each 2 x [64 rows][128 B]).
-// e4m3 branch: Q8 [128 rows][128 B], K8 [64 rows][128 B], V slot = phi(K) |
-// V (fp16) | V8 [64 rows][128 B].  Then H_i / W_proj (MN-major, 32 KB),
-// barriers, flags, exchange buffers.
+// Shared-memory layout (the dynamic shared window is 1024-byte aligned).
+//   bf16 branch: Q tile 2 x [128 rows][128 B]; key-pair slot
+//     [chunk 0: A rows | B rows][chunk 1: A rows | B rows] (128 rows per
+//     chunk); V slot = phi(K) | V (fp16, each 2 x [64 rows][128 B]).
+//   e4m3 branch: Q8 [128 rows][128 B]; key-pair slot [A rows | B rows] x
+//     128 B; V slot = phi(K) | V (fp16) | V8 [64 rows][128 B].
+// then barriers, flags, the row-pair exchange buffer and Z_i.
 template <bool kFP8>
 struct Lay {
   static constexpr uint32_t QBYTES = kFP8 ? 16384 : 32768;
-  static constexpr uint32_t KSLOT = kFP8 ? 8192 : 16384;
+  static constexpr uint32_t KBLK = kFP8 ? 8192 : 16384;  // bytes of one key block
+  static constexpr uint32_t KSLOT = 2 * KBLK;
   static constexpr uint32_t VSLOT = kFP8 ? 40960 : 32768;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = QBYTES;
-  static constexpr uint32_t OFF_V = OFF_K + kStages * KSLOT;
-  static constexpr uint32_t OFF_H = OFF_V + kStages * VSLOT;
-  static constexpr uint32_t OFF_BAR = OFF_H + 32768;
+  static constexpr uint32_t OFF_V = OFF_K + kKSlots * KSLOT;
+  static constexpr uint32_t OFF_BAR = OFF_V + kVSlots * VSLOT;
   static constexpr uint32_t OFF_MISC = OFF_BAR + 256;  // tmem base, abort flag
-  static constexpr uint32_t OFF_RED = OFF_MISC + 64;   // [4 slots][2 halves][128 rows] floats
-  static constexpr uint32_t OFF_Z = OFF_RED + 4096;    // Z_i [128] + Z_ex halves [2][128] floats
-  static constexpr uint32_t SMEM_BYTES = OFF_Z + 1536 + 1024;  // + alignment slack
+  static constexpr uint32_t OFF_RED = OFF_MISC + 64;   // [2 slots][2 halves][128 rows] floats
+  static constexpr uint32_t OFF_Z = OFF_RED + 2048;    // Z_i [128] floats
+  static constexpr uint32_t SMEM_BYTES = OFF_Z + 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_H % 1024 == 0, "1 KB aligned tiles");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && VSLOT % 1024 == 0, "1 KB aligned tiles");
 };
 
 // TMEM columns (512 allocated; one CTA per SM)
-constexpr uint32_t T_S0 = 0, T_S1 = 64, T_P0 = 128, T_P1 = 160, T_O = 192, T_HK = 320;
-constexpr uint32_t T_PHIQ = 0;    // epilogue: phi(Q) as the A operand (fp16 pairs), 64 columns
-constexpr uint32_t T_NUM = 64;    // epilogue: phi(Q) H_i, 128 columns
-constexpr uint32_t T_OLHI = 64;   // SLA epilogue: O_l hi / lo (bf16 pairs), 64 columns each
-constexpr uint32_t T_OLLO = 128;
-constexpr uint32_t T_PROJ = 320;  // SLA epilogue: O_l W_proj
+constexpr uint32_t T_S0 = 0;     // S buffer b at T_S0 + 128 b; P_b over its first 64 (bf16) / 32 (e4m3)
+constexpr uint32_t T_O = 256;    // O accumulator
+constexpr uint32_t T_HK = 384;   // H_ex accumulator; epilogue: phi(Q) H_i, then O_l W_proj
 constexpr uint32_t TMEM_COLS = 512;
 
 enum {
   B_QFULL = 0,
-  B_QFREE = 1,
+  B_QFREE = 1,    // MMA commit after the tile's last S product
   B_KFULL = 2,    // +slot
-  B_KEMPTY = 5,   // +slot
-  B_VFULL = 8,    // +slot
-  B_VEMPTY = 11,  // +slot
+  B_KEMPTY = 4,   // +slot
+  B_VFULL = 6,    // +slot
+  B_VEMPTY = 10,  // +slot
   B_SFULL = 14,   // +buffer
   B_PFULL = 16,   // +buffer
   B_PEMPTY = 18,  // +buffer
-  B_HFULL = 20,
-  B_OFINAL = 21,
-  B_EPI = 22,
-  B_NUM = 23,
-  B_EPIDONE = 24,
-  B_PROJR = 25,
-  B_PROJF = 26,
-  B_DRAIN = 27,
-  NBAR = 28
+  B_OFINAL = 20,
+  B_EPI = 21,
+  B_NUM = 22,
+  B_EPIDONE = 23,
+  B_PROJR = 24,
+  B_PROJF = 25,
+  B_DRAIN = 26,
+  NBAR = 27
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
 struct Tile {
   int bh, qb;
   long long row;
-  int n_crit, n_negl, n_total;
+  int n_crit, n_negl, n_total, nsteps;
   const int32_t* crit;
   const int32_t* negl;
   bool has_lin;
@@ -136,16 +145,19 @@ __device__ __forceinline__ Tile tile_at(const SparseArgs& a, int t, bool report)
     T.n_negl = 0;
   }
   T.n_total = T.n_crit + T.n_negl;
+  T.nsteps = (T.n_crit + 1) >> 1;
   T.crit = a.crit_idx + T.row * a.list_stride;
   T.negl = a.negl_idx ? a.negl_idx + T.row * a.list_stride : T.crit;
   T.has_lin = (a.nkv - T.n_total) > 0;
   return T;
 }
 
+// Key block at list position it (critical blocks first, then negligible ones);
+// an index outside [0, n_kv) is reported and replaced by 0.
 __device__ __forceinline__ int block_at(const Tile& T, int it, int nkv, int* status) {
   int j = it < T.n_crit ? T.crit[it] : T.negl[it - T.n_crit];
   if (j < 0 || j >= nkv) {
-    report_error(status, SLA_ERR_DEVICE_INDEX);
+    if (status) report_error(status, SLA_ERR_DEVICE_INDEX);
     j = 0;
   }
   return j;
@@ -165,11 +177,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmV8,
                       const SparseArgs a) {
   using L = Lay<kFP8>;
-  constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, OFF_H = L::OFF_H;
+  constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V;
   constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_RED = L::OFF_RED, OFF_Z = L::OFF_Z;
-  constexpr uint32_t KSLOT = L::KSLOT, VSLOT = L::VSLOT;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t KBLK = L::KBLK, KSLOT = L::KSLOT, VSLOT = L::VSLOT;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  // The swizzled tiles need a 1024-byte aligned window; the runtime gives one
+  // when the kernel has no static shared memory.  Check rather than assume.
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(a.status, SLA_ERR_UNSUPPORTED);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
@@ -182,14 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     mbar_init(&bars[B_QFULL], 1);
-    mbar_init(&bars[B_QFREE], kCompute);
-    for (int s = 0; s < kStages; ++s) {
+    mbar_init(&bars[B_QFREE], 1);
+    for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
       mbar_init(&bars[B_KEMPTY + s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bars[B_VFULL + s], 1);
       mbar_init(&bars[B_VEMPTY + s], 1);
     }
-    mbar_init(&bars[B_HFULL], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[B_SFULL + b], 1);
       mbar_init(&bars[B_PFULL + b], kCompute);
@@ -224,97 +242,141 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmH);
       if constexpr (kFP8) tma_prefetch_desc(&tmV8);
-      int gk = 0, gv = 0, q_issued = 0, h_issued = 0;
+      int gk = 0, gv = 0, q_issued = 0;
       bool ok = true;
-      auto load_block = [&](const Tile& T, int it) -> bool {
-        const int j = block_at(T, it, a.nkv, a.status);
-        const int krow = j * kBlockKV;
-        if (it < T.n_crit) {
-          const int sl = gk % kStages;
-          if (gk >= kStages && !mbar_wait(&bars[B_KEMPTY + sl], ((gk / kStages) - 1) & 1, abort_flag, a.status))
-            return false;
-          uint64_t* fb = &bars[B_KFULL + sl];
-          mbar_arrive_expect_tx(fb, KSLOT);
-          tma_load_3d(sm + OFF_K + sl * KSLOT, &tmK, fb, 0, krow, T.bh);
-          if constexpr (!kFP8) tma_load_3d(sm + OFF_K + sl * KSLOT + 8192, &tmK, fb, 64, krow, T.bh);
-          ++gk;
-        }
-        const int sl = gv % kStages;
-        if (gv >= kStages && !mbar_wait(&bars[B_VEMPTY + sl], ((gv / kStages) - 1) & 1, abort_flag, a.status))
+      // the key tiles of step s (list positions 2s, 2s+1) into the next pair slot
+      auto load_k = [&](const Tile& T, int s) -> bool {
+        const int sl = gk % kKSlots;
+        if (gk >= kKSlots && !mbar_wait(&bars[B_KEMPTY + sl], ((gk / kKSlots) - 1) & 1, abort_flag, a.status))
           return false;
-        uint8_t* vb = sm + OFF_V + sl * VSLOT;
-        uint64_t* fb = &bars[B_VFULL + sl];
+        const bool two = 2 * s + 1 < T.n_crit;
+        const int ra = block_at(T, 2 * s, a.nkv, a.status) * kBlockKV;
+        const int rb = two ? block_at(T, 2 * s + 1, a.nkv, a.status) * kBlockKV : 0;
+        uint64_t* fb = &bars[B_KFULL + sl];
+        uint8_t* kb = sm + OFF_K + sl * KSLOT;
+        mbar_arrive_expect_tx(fb, two ? 2 * KBLK : KBLK);
+        if constexpr (kFP8) {
+          tma_load_3d(kb, &tmK, fb, 0, ra, T.bh);
+          if (two) tma_load_3d(kb + 8192, &tmK, fb, 0, rb, T.bh);
+        } else {
+          tma_load_3d(kb, &tmK, fb, 0, ra, T.bh);
+          tma_load_3d(kb + 16384, &tmK, fb, 64, ra, T.bh);
+          if (two) {
+            tma_load_3d(kb + 8192, &tmK, fb, 0, rb, T.bh);
+            tma_load_3d(kb + 16384 + 8192, &tmK, fb, 64, rb, T.bh);
+          }
+        }
+        ++gk;
+        return true;
+      };
+      auto v_slot = [&](uint64_t*& fb) -> uint8_t* {
+        const int sl = gv % kVSlots;
+        if (gv >= kVSlots && !mbar_wait(&bars[B_VEMPTY + sl], ((gv / kVSlots) - 1) & 1, abort_flag, a.status))
+          return nullptr;
+        fb = &bars[B_VFULL + sl];
+        ++gv;
+        return sm + OFF_V + sl * VSLOT;
+      };
+      // phi(K), V (and V8) tiles of the block at list position it
+      auto load_v = [&](const Tile& T, int it) -> bool {
+        const int krow = block_at(T, it, a.nkv, a.status) * kBlockKV;
+        uint64_t* fb = nullptr;
+        uint8_t* vb = v_slot(fb);
+        if (vb == nullptr) return false;
         mbar_arrive_expect_tx(fb, VSLOT);
         tma_load_3d(vb, &tmPhi, fb, 0, krow, T.bh);
         tma_load_3d(vb + 8192, &tmPhi, fb, 64, krow, T.bh);
         tma_load_3d(vb + 16384, &tmV, fb, 0, krow, T.bh);
         tma_load_3d(vb + 16384 + 8192, &tmV, fb, 64, krow, T.bh);
         if constexpr (kFP8) tma_load_3d(vb + 32768, &tmV8, fb, 0, krow, T.bh);
-        ++gv;
+        return true;
+      };
+      auto load_h = [&](const Tile& T) -> bool {
+        uint64_t* fb = nullptr;
+        uint8_t* hb = v_slot(fb);
+        if (hb == nullptr) return false;
+        mbar_arrive_expect_tx(fb, 32768);
+        tma_load_3d(hb, &tmH, fb, 0, 0, T.bh);
+        tma_load_3d(hb + 16384, &tmH, fb, 64, 0, T.bh);
         return true;
       };
       int ti = 0;
       for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++ti) {
         const Tile T = tile_at(a, t, true);
-        const int pre = T.n_total < kStages ? T.n_total : kStages;
-        int it = 0;
-        for (; ok && it < pre; ++it) ok = load_block(T, it);  // key blocks first: they only need ring slots
-        if (!ok) break;
         if (ti > 0 && !mbar_wait(&bars[B_QFREE], (ti - 1) & 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(&bars[B_QFULL], L::QBYTES);
         tma_load_3d(sm + OFF_Q, &tmQ, &bars[B_QFULL], 0, T.qb * a.bq, T.bh);
         if constexpr (!kFP8) tma_load_3d(sm + OFF_Q + 16384, &tmQ, &bars[B_QFULL], 64, T.qb * a.bq, T.bh);
         q_issued = ti + 1;
-        if (T.has_lin) {
-          // H_tot / sigma of this head into the H buffer once the previous tile is done with it
-          if (ti > 0 && !mbar_wait(&bars[B_EPIDONE], (ti - 1) & 1, abort_flag, a.status)) break;
-          mbar_arrive_expect_tx(&bars[B_HFULL], 32768);
-          tma_load_3d(sm + OFF_H, &tmH, &bars[B_HFULL], 0, 0, T.bh);
-          tma_load_3d(sm + OFF_H + 16384, &tmH, &bars[B_HFULL], 64, 0, T.bh);
-          ++h_issued;
+        // key pairs run one step ahead of the value blocks
+        if (T.nsteps > 0) ok = load_k(T, 0);
+        if (ok && T.nsteps > 1) ok = load_k(T, 1);
+        for (int s = 0; ok && s < T.nsteps; ++s) {
+          ok = load_v(T, 2 * s);
+          if (ok && 2 * s + 1 < T.n_crit) ok = load_v(T, 2 * s + 1);
+          if (ok && s + 2 < T.nsteps) ok = load_k(T, s + 2);
         }
-        for (; ok && it < T.n_total; ++it) ok = load_block(T, it);
+        for (int it = T.n_crit; ok && it < T.n_total; ++it) ok = load_v(T, it);
+        if (ok && T.has_lin) ok = load_h(T);
       }
       // every issued copy must land before the CTA may exit
       if (q_issued > 0) mbar_wait_drain(&bars[B_QFULL], (q_issued - 1) & 1);
-      if (h_issued > 0) mbar_wait_drain(&bars[B_HFULL], (h_issued - 1) & 1);
-      for (int g = gk > kStages ? gk - kStages : 0; g < gk; ++g)
-        mbar_wait_drain(&bars[B_KFULL + g % kStages], (g / kStages) & 1);
-      for (int g = gv > kStages ? gv - kStages : 0; g < gv; ++g)
-        mbar_wait_drain(&bars[B_VFULL + g % kStages], (g / kStages) & 1);
+      for (int g = gk > kKSlots ? gk - kKSlots : 0; g < gk; ++g)
+        mbar_wait_drain(&bars[B_KFULL + g % kKSlots], (g / kKSlots) & 1);
+      for (int g = gv > kVSlots ? gv - kVSlots : 0; g < gv; ++g)
+        mbar_wait_drain(&bars[B_VFULL + g % kVSlots], (g / kVSlots) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_qk = idesc_f16(1, 0, 0, 128, 64);   // Q (K-major) x K_j (K-major), bf16
+      const uint32_t id_qk = idesc_f16(1, 0, 0, 128, 128);  // Q (K-major) x [K_a|K_b] (K-major), bf16
+      const uint32_t id_qk1 = idesc_f16(1, 0, 0, 128, 64);  // one key block
       const uint32_t id_h = idesc_f16(0, 1, 1, 128, 128);   // phi(K)^T (MN-major) x V (MN-major), f16
-      const uint32_t id_pv = idesc_f16(0, 0, 1, 128, 128);  // P (TMEM) x V (MN-major), f16
-      const uint32_t id_bf = idesc_f16(1, 0, 1, 128, 128);  // TMEM A x MN-major B, bf16
-      // Descriptors built once; a byte offset d inside a tile adds d >> 4 to the
-      // start-address field (addresses stay below 2^18, so the field cannot carry).
+      const uint32_t id_pv = idesc_f16(0, 0, 1, 128, 128);  // TMEM A (f16) x MN-major B
+      const uint32_t id_bf = idesc_f16(1, 0, 1, 128, 128);  // TMEM A (bf16) x MN-major B
+      const uint32_t id_qk8 = idesc_f8(0, 0, 128, 128);     // Q8 x [K8_a|K8_b], e4m3
+      const uint32_t id_qk81 = idesc_f8(0, 0, 128, 64);
+      const uint32_t id_pv8 = idesc_f8(0, 1, 128, 128);     // P8 (TMEM) x V8 (MN-major), e4m3
+      // Descriptors built once; a byte offset d inside the window adds d >> 4 to
+      // the start-address field (addresses stay below 2^18, so it cannot carry).
       const uint64_t dQ = sdesc_sw128(smem_u32(sm + OFF_Q), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(sm + OFF_K), 16, 1024);
       const uint64_t dPhi = sdesc_sw128(smem_u32(sm + OFF_V), 8192, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sm + OFF_V) + 16384, 8192, 1024);
-      const uint64_t dH = sdesc_sw128(smem_u32(sm + OFF_H), 16384, 1024);
       const uint64_t dV8 = sdesc_sw128(smem_u32(sm + OFF_V) + 32768, 16, 1024);  // MN-major, N fits one atom
-      const uint32_t id_qk8 = idesc_f8(0, 0, 128, 64);   // Q8 (K-major) x K8 (K-major), e4m3
-      const uint32_t id_pv8 = idesc_f8(0, 1, 128, 128);  // P8 (TMEM) x V8 (MN-major), e4m3
-      auto issue_qk = [&](int sl, int b) {
+      const uint64_t dH = sdesc_sw128(smem_u32(sm + OFF_V), 16384, 1024);       // H tile / W_proj in a V slot
+      int gk = 0, gv = 0, gs = 0, ti = 0;
+      bool ok = true;
+      // S for step s of T into buffer g & 1; frees the key slot when done
+      auto issue_s = [&](const Tile& T, int s, int g, bool last_s) -> bool {
+        const int sl = gk % kKSlots;
+        if (!mbar_wait(&bars[B_KFULL + sl], (gk / kKSlots) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const bool two = 2 * s + 1 < T.n_crit;
         const uint64_t kb = dK + ((sl * KSLOT) >> 4);
-        const uint32_t d = tmem + (b ? T_S1 : T_S0);
+        const uint32_t d = tmem + T_S0 + (g & 1) * 128;
         if constexpr (kFP8) {
-          // e4m3 x e4m3: 4 MMAs of K = 32 inside the single 128-byte-wide tile
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + kk * 2u, kb + kk * 2u, id_qk8, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + kk * 2u, kb + kk * 2u, two ? id_qk8 : id_qk81, kk > 0 ? 1u : 0u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t qo = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-            const uint32_t ko = ((kk >> 2) * 8192u + (kk & 3) * 32u) >> 4;
-            mma_f16_ss(d, dQ + qo, kb + ko, id_qk, kk > 0 ? 1u : 0u);
+            const uint32_t o = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;  // same offsets in Q and the pair slot
+            mma_f16_ss(d, dQ + o, kb + o, two ? id_qk : id_qk1, kk > 0 ? 1u : 0u);
           }
         }
+        mma_commit(&bars[B_SFULL + (g & 1)]);
+        mma_commit(&bars[B_KEMPTY + sl]);
+        if (last_s) mma_commit(&bars[B_QFREE]);
+        ++gk;
+        return true;
+      };
+      auto take_v = [&]() -> int {  // next V-ring entry, once it has landed
+        const int sl = gv % kVSlots;
+        if (!mbar_wait(&bars[B_VFULL + sl], (gv / kVSlots) & 1, abort_flag, a.status)) return -1;
+        tc_fence_after();
+        ++gv;
+        return sl;
       };
       auto issue_h = [&](int sl, bool first) {
         const uint64_t pb = dPhi + ((sl * VSLOT) >> 4), vb = dV + ((sl * VSLOT) >> 4);
@@ -322,101 +384,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 4; ++kk)
           mma_f16_ss(tmem + T_HK, pb + kk * 128u, vb + kk * 128u, id_h, (first && kk == 0) ? 0u : 1u);
       };
-      auto issue_pv = [&](int sl, int b, bool first) {
-        const uint32_t pa = tmem + (b ? T_P1 : T_P0);
+      // O (+)= P V for one key block: P columns from pcol, V from slot sl
+      auto issue_pv = [&](int sl, uint32_t pcol, bool first) {
         if constexpr (kFP8) {
           // P8 (TMEM, 4 keys per column) x V8 (MN-major, one 128-byte atom wide): K = 32 per MMA
           const uint64_t vb = dV8 + ((sl * VSLOT) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_f8_ts(tmem + T_O, pa + kk * 8u, vb + kk * 256u, id_pv8, (first && kk == 0) ? 0u : 1u);
+            mma_f8_ts(tmem + T_O, tmem + pcol + kk * 8u, vb + kk * 256u, id_pv8, (first && kk == 0) ? 0u : 1u);
         } else {
           const uint64_t vb = dV + ((sl * VSLOT) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ts(tmem + T_O, pa + kk * 8u, vb + kk * 128u, id_pv, (first && kk == 0) ? 0u : 1u);
+            mma_f16_ts(tmem + T_O, tmem + pcol + kk * 8u, vb + kk * 128u, id_pv, (first && kk == 0) ? 0u : 1u);
         }
       };
       // D[col] = A (TMEM, 64 columns of 16-bit pairs) x B (smem MN-major [128 K rows] x 2 chunks of 64 N)
-      auto issue_ts128 = [&](uint32_t a_col, uint32_t col, uint32_t idesc, bool first) {
+      auto issue_ts128 = [&](uint32_t a_col, uint32_t col, uint64_t b, uint32_t idesc, bool first) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ts(tmem + col, tmem + a_col + kk * 8u, dH + kk * 128u, idesc, (first && kk == 0) ? 0u : 1u);
+          mma_f16_ts(tmem + col, tmem + a_col + kk * 8u, b + kk * 128u, idesc, (first && kk == 0) ? 0u : 1u);
       };
 
-      // Issue order per block i: S_{i+1} (overlaps the softmax of block i), H_i,
-      // then PV_i once P_i is in TMEM.  MMA issue is blocking on this hardware
-      // (about one instruction per 48-64 cycles), so the issuer waits in
-      // suspending barrier tests rather than polling.
-      int gk = 0, gv = 0, gs = 0, ti = 0;
-      bool ok = true;
-      auto issue_s = [&](int b) -> bool {  // S = Q K^T for the next K slot; the slot frees when S is done
-        const int sl = gk % kStages;
-        if (!mbar_wait(&bars[B_KFULL + sl], (gk / kStages) & 1, abort_flag, a.status)) return false;
+      // the previous tile's epilogue products, run after the next tile's first S
+      bool pend = false, pend_lin = false;
+      int pend_ti = 0, pend_sl = 0, pend_par = 0;
+      uint32_t pend_col = 0;
+      auto finish_epi = [&]() -> bool {
+        pend = false;
+        if (!mbar_wait(&bars[B_EPI], pend_ti & 1, abort_flag, a.status)) return false;
         tc_fence_after();
-        issue_qk(sl, b);
-        mma_commit(&bars[B_SFULL + b]);
-        mma_commit(&bars[B_KEMPTY + sl]);
-        ++gk;
+        const uint64_t hb = dH + ((pend_sl * VSLOT) >> 4);
+        if (pend_lin) {
+          if (!mbar_wait(&bars[B_VFULL + pend_sl], pend_par, abort_flag, a.status)) return false;
+          tc_fence_after();
+          issue_ts128(pend_col, T_HK, hb, id_pv, true);  // phi(Q) H_i / sigma
+        }
+        mma_commit(&bars[B_NUM]);
+        if (a.wproj != nullptr) {
+          if (!mbar_wait(&bars[B_PROJR], pend_ti & 1, abort_flag, a.status)) return false;
+          tc_fence_after();
+          if (pend_lin) {
+            issue_ts128(pend_col, T_HK, hb, id_bf, true);        // O_l hi x W_proj
+            issue_ts128(pend_col + 64, T_HK, hb, id_bf, false);  // O_l lo x W_proj
+          }
+          mma_commit(&bars[B_PROJF]);
+        }
+        if (pend_lin) mma_commit(&bars[B_VEMPTY + pend_sl]);
+        if (!mbar_wait(&bars[B_EPIDONE], pend_ti & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
         return true;
       };
+
       for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++ti) {
         const Tile T = tile_at(a, t, false);
         if (!mbar_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status)) break;
-        if (ti > 0 && !mbar_wait(&bars[B_EPIDONE], (ti - 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const int n = T.n_crit;
-        if (n > 0 && !issue_s(gs & 1)) break;
-        for (int i = 0; ok && i < n; ++i) {
-          const int b = (gs + i) & 1, sl = gv % kStages;
-          if (i + 1 < n && !issue_s((gs + i + 1) & 1)) {
+        const int ns = T.nsteps;
+        if (ns > 0 && !issue_s(T, 0, gs, ns == 1)) break;
+        if (pend && !finish_epi()) break;
+        if (ns == 0) mma_commit(&bars[B_QFREE]);
+        for (int i = 0; ok && i < ns; ++i) {
+          const int g = gs + i, b = g & 1;
+          if (i + 1 < ns && !issue_s(T, i + 1, g + 1, i + 1 == ns - 1)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&bars[B_VFULL + sl], (gv / kStages) & 1, abort_flag, a.status)) {
+          const bool two = 2 * i + 1 < T.n_crit;
+          const int sa = take_v();
+          if (sa < 0) {
+            ok = false;
+            break;
+          }
+          issue_h(sa, i == 0);
+          int sb = -1;
+          if (two) {
+            sb = take_v();
+            if (sb < 0) {
+              ok = false;
+              break;
+            }
+            issue_h(sb, false);
+          }
+          if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_h(sl, i == 0);
-          if (!mbar_wait(&bars[B_PFULL + b], ((gs + i) >> 1) & 1, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(sl, b, i == 0);
+          const uint32_t pcol = T_S0 + b * 128;
+          issue_pv(sa, pcol, i == 0);
+          if (two) issue_pv(sb, pcol + (kFP8 ? 16u : 32u), false);
           mma_commit(&bars[B_PEMPTY + b]);
-          mma_commit(&bars[B_VEMPTY + sl]);
-          ++gv;
+          mma_commit(&bars[B_VEMPTY + sa]);
+          if (two) mma_commit(&bars[B_VEMPTY + sb]);
         }
-        for (int i = n; ok && i < T.n_total; ++i) {
-          const int sl = gv % kStages;
-          if (!mbar_wait(&bars[B_VFULL + sl], (gv / kStages) & 1, abort_flag, a.status)) {
+        for (int it = T.n_crit; ok && it < T.n_total; ++it) {
+          const int sl = take_v();
+          if (sl < 0) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_h(sl, i == 0);
+          issue_h(sl, it == 0);
           mma_commit(&bars[B_VEMPTY + sl]);
-          ++gv;
         }
         if (!ok) break;
         mma_commit(&bars[B_OFINAL]);
-        gs += n;
-        if (T.has_lin) {
-          if (!mbar_wait(&bars[B_EPI], ti & 1, abort_flag, a.status)) break;
-          tc_fence_after();
-          issue_ts128(T_PHIQ, T_NUM, idesc_f16(0, 0, 1, 128, 128), true);
-          mma_commit(&bars[B_NUM]);
-          if (a.wproj != nullptr) {
-            if (!mbar_wait(&bars[B_PROJR], ti & 1, abort_flag, a.status)) break;
-            tc_fence_after();
-            issue_ts128(T_OLHI, T_PROJ, id_bf, true);
-            issue_ts128(T_OLLO, T_PROJ, id_bf, false);
-            mma_commit(&bars[B_PROJF]);
-          }
+        gs += ns;
+        pend = true;
+        pend_ti = ti;
+        pend_lin = T.has_lin;
+        pend_col = T_S0 + ((gs - 1) & 1) * 128;  // the tile's last S buffer: phi(Q), SLA O_l
+        if (T.has_lin) {  // the H tile follows the tile's blocks in the V ring
+          pend_sl = gv % kVSlots;
+          pend_par = (gv / kVSlots) & 1;
+          ++gv;
         }
       }
+      if (ok && pend) finish_epi();
       // all MMAs must finish before the CTA releases TMEM
       mma_commit(&bars[B_DRAIN]);
       mbar_wait_drain(&bars[B_DRAIN], 0);
@@ -427,54 +511,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;  // tile row = TMEM lane
     const uint32_t lrow = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t pair_bar = 1 + quarter;  // the two warps that share these rows
-    auto RED = [&](int slot, int h) -> float* { return red + (slot * 2 + h) * 128; };
     const bool tail = (a.N & (kBlockKV - 1)) != 0;
-    int gs = 0, ti = 0, hc = 0;
+    int gs = 0, ti = 0, gv = 0, xc = 0;
     bool ok = true;
+    // value exchange with the other warp of the row pair (two alternating slots)
+    auto xchg = [&](float v) -> float {
+      float* base = red + (xc & 1) * 256;
+      base[half * 128 + r] = v;
+      named_bar_sync(pair_bar, 64);
+      const float o = base[(1 - half) * 128 + r];
+      ++xc;
+      return o;
+    };
+    auto list_at = [&](const Tile& T, int p) -> int {  // critical block at position p, or -1
+      if (p >= T.n_crit) return -1;
+      const int j = T.crit[p];
+      return (j < 0 || j >= a.nkv) ? 0 : j;
+    };
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
       const Tile T = tile_at(a, t, false);
       const int tok = T.qb * a.bq + r;
       const bool row_valid = (r < a.bq) && (tok < a.N);
-      const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
-      const float sigma_t = T.has_lin ? a.sigma[T.bh] : 1.0f;
-      const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
       float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
       if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
-      float m_run = -INFINITY, l_part = 0.0f;
-      for (int i = 0; i < T.n_crit; ++i) {
-        const int b = (gs + i) & 1;
-        ok = ok && warp_wait(&bars[B_SFULL + b], ((gs + i) >> 1) & 1, abort_flag, a.status);
-        float s[32];
-        if (ok) {
+      int j_cur = list_at(T, half);
+
+      // ---------------------------------------------------------- steps of two key blocks
+      float m_run = -INFINITY, l_part = 0.0f, zex = 0.0f;
+      const float* zb = a.zblk + static_cast<long long>(T.bh) * a.nkv * kDPad + r;
+      for (int i = 0; i < T.nsteps; ++i) {
+        const int g = gs + i, b = g & 1;
+        const int j_next = list_at(T, 2 * (i + 1) + half);
+        const float zv = (T.has_lin && j_cur >= 0) ? zb[static_cast<long long>(j_cur) * kDPad] : 0.0f;
+        ok = ok && warp_wait(&bars[B_SFULL + b], (g >> 1) & 1, abort_flag, a.status);
+        float s[64];
+        if (ok && j_cur >= 0) {
           tc_fence_after();
-          tmem_ld32(tmem + lrow + (b ? T_S1 : T_S0) + 32 * half, s);
+          tmem_ld32(tmem + lrow + T_S0 + b * 128 + 64 * half, s);
+          tmem_ld32(tmem + lrow + T_S0 + b * 128 + 64 * half + 32, s + 32);
           tmem_wait_ld();
-        } else {
+          if (tail && j_cur == a.nkv - 1) {
+            const int nvalid = a.N - j_cur * kBlockKV;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = 0.0f;
+            for (int c = 0; c < 64; ++c)
+              if (c >= nvalid) s[c] = -INFINITY;
+          }
+        } else {
+          const float fill = ok ? -INFINITY : 0.0f;  // no second block in this step
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = fill;
         }
         float sc = a.sl2;
         if constexpr (kFP8) {
-          const int j = block_at(T, i, a.nkv, nullptr);
-          sc = sl2_q * a.sk[static_cast<long long>(T.bh) * a.nb128 + (j >> 1)];  // 128-token key scale block
-        }
-        if (tail) {
-          const int j = block_at(T, i, a.nkv, nullptr);
-          if (j == a.nkv - 1) {
-            const int nvalid = a.N - j * kBlockKV - 32 * half;
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (c >= nvalid) s[c] = -INFINITY;
-          }
+          if (j_cur >= 0) sc = sl2_q * a.sk[static_cast<long long>(T.bh) * a.nb128 + (j_cur >> 1)];  // 128-token key block
         }
         float m8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(fmaxf(s[4 * c], s[4 * c + 1]), fmaxf(s[4 * c + 2], s[4 * c + 3]));
+        for (int c = 0; c < 8; ++c) {
+          m8[c] = fmaxf(fmaxf(fmaxf(s[8 * c], s[8 * c + 1]), fmaxf(s[8 * c + 2], s[8 * c + 3])),
+                        fmaxf(fmaxf(s[8 * c + 4], s[8 * c + 5]), fmaxf(s[8 * c + 6], s[8 * c + 7])));
+        }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        RED(i & 1, half)[r] = mx * sc;
-        named_bar_sync(pair_bar, 64);
-        const float mt = fmaxf(RED(i & 1, 0)[r], RED(i & 1, 1)[r]);
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                         sc;
+        const float mt = fmaxf(mx, xchg(mx));
         // bf16: refresh the max only when it grows by more than 15 (p <= 2^15 fits
         // fp16); e4m3: p * 448 must stay within e4m3, so the exact running max
         const bool need = kFP8 ? (mt > m_run) : (mt > m_run + 15.0f);
@@ -482,19 +582,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float m_new = need ? mt : m_run;
           const float f = need ? ex2_approx(m_run - m_new) : 1.0f;
           if (i > 0) {
-            // O holds P V of the previous blocks: wait for the last PV, rescale
-            ok = ok && warp_wait(&bars[B_PEMPTY + ((gs + i - 1) & 1)], ((gs + i - 1) >> 1) & 1, abort_flag,
-                                 a.status);
+            // O holds P V of the previous steps: wait for the last PV, rescale
+            ok = ok && warp_wait(&bars[B_PEMPTY + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag, a.status);
             if (ok) {
               tc_fence_after();
-#pragma unroll
-              for (int cc = 0; cc < 2; ++cc) {
-                float o[32];
-                tmem_ld32(tmem + lrow + T_O + 64 * half + 32 * cc, o);
+#pragma unroll 1
+              for (int cc = 0; cc < 4; ++cc) {  // 16 columns at a time: few registers next to s[]
+                float o[16];
+                tmem_ld16(tmem + lrow + T_O + 64 * half + 16 * cc, o);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) o[c] *= f;
-                tmem_st32(tmem + lrow + T_O + 64 * half + 32 * cc, o);
+                for (int c = 0; c < 16; ++c) o[c] *= f;
+                tmem_st16f(tmem + lrow + T_O + 64 * half + 16 * cc, o);
               }
               tmem_wait_st();
             }
@@ -502,15 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_part *= f;
           m_run = m_new;
         }
-        if (i >= 2) ok = ok && warp_wait(&bars[B_PEMPTY + b], ((gs + i - 2) >> 1) & 1, abort_flag, a.status);
-        uint32_t pk[16];
         const float nm = -m_run;
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if constexpr (kFP8) {
           // p in (0, 1] against the running max; the row sum uses the unquantised p,
-          // the PV MMA p * 448 rounded to e4m3 (four keys per TMEM column)
+          // the PV product p * 448 rounded to e4m3 (four keys per TMEM column)
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 16; ++c) {
             float p[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(s[4 * c + e], sc, nm));
@@ -521,41 +619,70 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          __NV_E4M3);
             pk[c] = lo | (hi << 16);
           }
+          if (ok) tmem_st16(tmem + lrow + T_S0 + b * 128 + 16 * half, pk);
         } else {
+          uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 32; ++c) {
             const float p0 = ex2_approx(fmaf(s[2 * c], sc, nm));
             const float p1 = ex2_approx(fmaf(s[2 * c + 1], sc, nm));
             l4[c & 3] += p0 + p1;
             pk[c] = pack_half2(p0, p1);
           }
+          if (ok) {
+            tmem_st16(tmem + lrow + T_S0 + b * 128 + 32 * half, pk);
+            tmem_st16(tmem + lrow + T_S0 + b * 128 + 32 * half + 16, pk + 16);
+          }
         }
         l_part += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         if (ok) {
-          if constexpr (kFP8)
-            tmem_st8(tmem + lrow + (b ? T_P1 : T_P0) + 8 * half, pk);
-          else
-            tmem_st16(tmem + lrow + (b ? T_P1 : T_P0) + 16 * half, pk);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&bars[B_PFULL + b]);
         }
+        zex += zv;
+        j_cur = j_next;
       }
-      gs += T.n_crit;
+      gs += T.nsteps;
+      // SLA: the negligible blocks only leave the linear sum
+      if (T.has_lin) {
+        float z4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int it = T.n_crit + half; it < T.n_total; it += 8) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i2 = it + 2 * u;
+            if (i2 < T.n_total) z4[u] += zb[static_cast<long long>(block_at(T, i2, a.nkv, nullptr)) * kDPad];
+          }
+        }
+        zex += (z4[0] + z4[1]) + (z4[2] + z4[3]);
+      }
 
       // ---------------------------------------------------------- epilogue
+      // this row's 64 channels of Q (bf16, from L2: the tile was read moments ago)
+      uint4 qw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        qw[u] = make_uint4(0, 0, 0, 0);
+        if (T.has_lin && tok < a.N)
+          qw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
+                                                  (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
+      }
+      const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
+      const float sigma = T.has_lin ? a.sigma[T.bh] : 1.0f;
+      const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
       ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
       if (ok) tc_fence_after();
-      RED(2, half)[r] = l_part;
-      named_bar_sync(pair_bar, 64);
-      const float l_run = RED(2, 0)[r] + RED(2, 1)[r];
-      const float sigma = sigma_t;
+      const float l_run = l_part + xchg(l_part);
+      const uint32_t pcol = T_S0 + ((gs - 1) & 1) * 128;  // the tile's last S buffer
+      const int hidx = gv + T.n_total;                     // V-ring entry of the H tile
+      const int hsl = hidx % kVSlots;
+      uint8_t* hbuf = sm + OFF_V + hsl * VSLOT;
+      gv += T.n_total + (T.has_lin ? 1 : 0);
       float den = 0.0f;
       if (T.has_lin) {
         // H_i / sigma = H_tot / sigma (fp16 tile from TMA) - H_ex / sigma, row e = r,
-        // channels 64*half.., in place in the MN-major H buffer
-        ok = ok && warp_wait(&bars[B_HFULL], hc & 1, abort_flag, a.status);
-        ++hc;
+        // channels 64*half.., in place in the MN-major H tile
+        ok = ok && warp_wait(&bars[B_VFULL + hsl], (hidx / kVSlots) & 1, abort_flag, a.status);
         const float inv_sigma = 1.0f / sigma;  // exact: sigma is a power of two
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -569,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            uint4* hp = reinterpret_cast<uint4*>(sm + OFF_H + half * 16384u + sw128_off(r, 4 * cc + q4));
+            uint4* hp = reinterpret_cast<uint4*>(hbuf + half * 16384u + sw128_off(r, 4 * cc + q4));
             const uint4 h8 = *hp;
             const uint32_t hw[4] = {h8.x, h8.y, h8.z, h8.w};
             uint32_t o4[4];
@@ -581,33 +708,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             *hp = make_uint4(o4[0], o4[1], o4[2], o4[3]);
           }
         }
-        // Z_ex[e] for e = r: this half sums every other listed block's column sums
-        {
-          const float* zb = a.zblk + static_cast<long long>(T.bh) * a.nkv * kDPad + r;
-          float z4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          for (int it = half; it < T.n_total; it += 8) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int i2 = it + 2 * u;
-              if (i2 < T.n_total) z4[u] += zb[static_cast<long long>(block_at(T, i2, a.nkv, nullptr)) * kDPad];
-            }
-          }
-          zsh[128 + 128 * half + r] = (z4[0] + z4[1]) + (z4[2] + z4[3]);
-        }
-        // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), fp16 into TMEM
+        // Z_i[e] for e = r, shared with every row for the denominator
+        const float zi = zt_r - (zex + xchg(zex));
+        if (half == 0) zsh[r] = zi;
+        // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), fp16 pairs
+        const int c0 = 64 * half;
         float x[64];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          uint4 w;
-          if constexpr (kFP8) {  // the smem tile holds e4m3 Q: read the bf16 row (L2-resident)
-            w = make_uint4(0, 0, 0, 0);
-            if (tok < a.N)
-              w = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
-                                                  (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
-          } else {
-            w = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 16384u + sw128_off(r, u));
-          }
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f2 = unpack_bf162(ww[e]);
@@ -615,146 +724,136 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[8 * u + 2 * e + 1] = f2.y;
           }
         }
-        mbar_arrive(&bars[B_QFREE]);  // Q tile no longer read: the next one may load
-        const int c0 = 64 * half;
         if (a.phi == SLA_PHI_SOFTMAX) {
           float mx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if (c0 + c < a.d) mx = fmaxf(mx, x[c]);
-          RED(0, half)[r] = mx;
-          named_bar_sync(pair_bar, 64);
-          mx = fmaxf(RED(0, 0)[r], RED(0, 1)[r]);
+          mx = fmaxf(mx, xchg(mx));
           float sum = 0.0f;
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             x[c] = (c0 + c < a.d) ? ex2_approx((x[c] - mx) * 1.4426950408889634f) : 0.0f;
             sum += x[c];
           }
-          RED(1, half)[r] = sum;
-          named_bar_sync(pair_bar, 64);
-          const float inv = 1.0f / (RED(1, 0)[r] + RED(1, 1)[r]);
+          const float inv = 1.0f / (sum + xchg(sum));
 #pragma unroll
           for (int c = 0; c < 64; ++c) x[c] *= inv;
         } else {
 #pragma unroll
           for (int c = 0; c < 64; ++c) x[c] = (c0 + c < a.d) ? elu1(x[c]) : 0.0f;
         }
-        uint32_t pk[32];
+        uint32_t phq[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          pk[c] = pack_half2(x[2 * c], x[2 * c + 1]);
-          const float2 back = unpack_half2(pk[c]);  // the denominator uses the rounded phi(Q)
-          x[2 * c] = back.x;
-          x[2 * c + 1] = back.y;
-        }
-        if (ok) {
-          tmem_st16(tmem + lrow + T_PHIQ + 32 * half, pk);
-          tmem_st16(tmem + lrow + T_PHIQ + 32 * half + 16, pk + 16);
-        }
-        named_bar_sync(5, kCompute);  // Z_ex halves complete
-        if (half == 0) zsh[r] = zt_r - (zsh[128 + r] + zsh[256 + r]);
+        for (int c = 0; c < 32; ++c) phq[c] = pack_half2(x[2 * c], x[2 * c + 1]);
         named_bar_sync(5, kCompute);  // Z_i complete
         float dp = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) dp = fmaf(x[c], zsh[c0 + c], dp);
-        RED(3, half)[r] = dp;
-        named_bar_sync(pair_bar, 64);
-        den = RED(3, 0)[r] + RED(3, 1)[r];
-        if (ok) {
-          tmem_wait_st();
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&bars[B_EPI]);
+        for (int c = 0; c < 32; ++c) {
+          const float2 f = unpack_half2(phq[c]);  // the denominator uses the rounded phi(Q)
+          dp = fmaf(f.x, zsh[c0 + 2 * c], dp);
+          dp = fmaf(f.y, zsh[c0 + 2 * c + 1], dp);
         }
-        ok = ok && warp_wait(&bars[B_NUM], ti & 1, abort_flag, a.status);
-        if (ok) tc_fence_after();
-      } else {
-        mbar_arrive(&bars[B_QFREE]);
+        den = dp + xchg(dp);
+        if (ok) {
+          tmem_st16(tmem + lrow + pcol + 32 * half, phq);
+          tmem_st16(tmem + lrow + pcol + 32 * half + 16, phq + 16);
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
       }
+      if (ok) {
+        tc_fence_before();
+        mbar_arrive(&bars[B_EPI]);
+      }
+      ok = ok && warp_wait(&bars[B_NUM], ti & 1, abort_flag, a.status);
+      if (ok) tc_fence_after();
 
       const float inv_l = (T.n_crit > 0 && l_run > 0.0f) ? 1.0f / l_run : 0.0f;
       const float lin_scale = (T.has_lin && den > 0.0f) ? sigma / den : 0.0f;
-      const long long obase = (static_cast<long long>(T.bh) * a.N + tok) * a.d;
-      uint32_t lin_col = T_NUM;
       float w_s, lin_w;
       if (a.wproj != nullptr) {
         w_s = inv_l;
         lin_w = 1.0f;
         if (T.has_lin) {
-          // SLA: O_l -> bf16 hi + lo into TMEM (A operand), W_proj -> smem (MN-major), MMA
-          lin_col = T_PROJ;
-          float ol[64];
-          if (ok) {
-            tmem_ld32(tmem + lrow + T_NUM + 64 * half, ol);
-            tmem_ld32(tmem + lrow + T_NUM + 64 * half + 32, ol + 32);
-            tmem_wait_ld();
-          } else {
+          // SLA: O_l -> bf16 hi + lo into TMEM (A operand), W_proj -> the H tile's slot (MN-major)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) ol[c] = 0.0f;
-          }
-          named_bar_sync(pair_bar, 64);  // both halves have read NUM before it is overwritten
-          uint32_t hi[32], lo[32];
+          for (int cc = 0; cc < 2; ++cc) {
+            float ol[32];
+            if (ok) {
+              tmem_ld32(tmem + lrow + T_HK + 64 * half + 32 * cc, ol);
+              tmem_wait_ld();
+            } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v0 = ol[2 * c] * lin_scale, v1 = ol[2 * c + 1] * lin_scale;
-            hi[c] = pack_bf162(v0, v1);
-            const float2 hb = unpack_bf162(hi[c]);
-            lo[c] = pack_bf162(v0 - hb.x, v1 - hb.y);
-          }
-          if (ok) {
-            tmem_st16(tmem + lrow + T_OLHI + 32 * half, hi);
-            tmem_st16(tmem + lrow + T_OLHI + 32 * half + 16, hi + 16);
-            tmem_st16(tmem + lrow + T_OLLO + 32 * half, lo);
-            tmem_st16(tmem + lrow + T_OLLO + 32 * half + 16, lo + 16);
+              for (int c = 0; c < 32; ++c) ol[c] = 0.0f;
+            }
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float v0 = ol[2 * c] * lin_scale, v1 = ol[2 * c + 1] * lin_scale;
+              hi[c] = pack_bf162(v0, v1);
+              const float2 hb = unpack_bf162(hi[c]);
+              lo[c] = pack_bf162(v0 - hb.x, v1 - hb.y);
+            }
+            if (ok) {
+              tmem_st16(tmem + lrow + pcol + 32 * half + 16 * cc, hi);
+              tmem_st16(tmem + lrow + pcol + 64 + 32 * half + 16 * cc, lo);
+            }
           }
           const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(a.wproj);
           for (int idx = tid; idx < 128 * 16; idx += kCompute) {
             const int e = idx >> 4, u = idx & 15;
             uint4 w = make_uint4(0, 0, 0, 0);
             if (e < a.d && 8 * u < a.d) w = *reinterpret_cast<const uint4*>(wp + e * a.d + 8 * u);
-            *reinterpret_cast<uint4*>(sm + OFF_H + (u >> 3) * 16384u + sw128_off(e, u & 7)) = w;
+            *reinterpret_cast<uint4*>(hbuf + (u >> 3) * 16384u + sw128_off(e, u & 7)) = w;
           }
-          if (ok) {
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[B_PROJR]);
-          }
-          ok = ok && warp_wait(&bars[B_PROJF], ti & 1, abort_flag, a.status);
-          if (ok) tc_fence_after();
+          if (ok) tmem_wait_st();
+          fence_proxy_async_smem();
         }
+        if (ok) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_PROJR]);
+        }
+        ok = ok && warp_wait(&bars[B_PROJF], ti & 1, abort_flag, a.status);
+        if (ok) tc_fence_after();
       } else {
         w_s = alpha_t * inv_l;
         lin_w = (1.0f - alpha_t) * lin_scale;
       }
+      // combine 32 channels at a time; TMEM goes back after the last read
+      const long long obase = (static_cast<long long>(T.bh) * a.N + tok) * a.d;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
+        const int ch0 = 64 * half + 32 * cc;
         float o[32], nmv[32];
-        if (ok && T.n_crit > 0) tmem_ld32(tmem + lrow + T_O + 64 * half + 32 * cc, o);
-        if (ok && T.has_lin) tmem_ld32(tmem + lrow + lin_col + 64 * half + 32 * cc, nmv);
+        if (ok && T.n_crit > 0) tmem_ld32(tmem + lrow + T_O + ch0, o);
+        if (ok && T.has_lin) tmem_ld32(tmem + lrow + T_HK + ch0, nmv);
         tmem_wait_ld();
+        if (cc == 1 && ok) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_EPIDONE]);
+        }
         if constexpr (kFP8) {  // O accumulates e4m3 codes: times (absmax_c / 448) / 448 per channel
-          const float* va = a.vamax + static_cast<long long>(T.bh) * kDPad + 64 * half + 32 * cc;
+          const float* va = a.vamax + static_cast<long long>(T.bh) * kDPad + ch0;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
+          for (int c = 0; c < 32; ++c)
+            o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
         }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float os = (T.n_crit > 0) ? o[c] * w_s : 0.0f;
-          const float olv = T.has_lin ? nmv[c] * lin_w : 0.0f;
+          const float os = (ok && T.n_crit > 0) ? o[c] * w_s : 0.0f;
+          const float olv = (ok && T.has_lin) ? nmv[c] * lin_w : 0.0f;
           o[c] = os + olv;
         }
-        const int ch0 = 64 * half + 32 * cc;
         if (ok && row_valid) {
           if (a.out_bf16) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + obase;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              if (ch0 + 8 * q4 < a.d)
-                *reinterpret_cast<uint4*>(dst + ch0 + 8 * q4) =
-                    make_uint4(pack_bf162(o[8 * q4], o[8 * q4 + 1]), pack_bf162(o[8 * q4 + 2], o[8 * q4 + 3]),
-                               pack_bf162(o[8 * q4 + 4], o[8 * q4 + 5]), pack_bf162(o[8 * q4 + 6], o[8 * q4 + 7]));
+            for (int q8 = 0; q8 < 4; ++q8)
+              if (ch0 + 8 * q8 < a.d)
+                *reinterpret_cast<uint4*>(dst + ch0 + 8 * q8) =
+                    make_uint4(pack_bf162(o[8 * q8], o[8 * q8 + 1]), pack_bf162(o[8 * q8 + 2], o[8 * q8 + 3]),
+                               pack_bf162(o[8 * q8 + 4], o[8 * q8 + 5]), pack_bf162(o[8 * q8 + 6], o[8 * q8 + 7]));
           } else {
             float* dst = static_cast<float*>(a.out) + obase;
 #pragma unroll
@@ -764,10 +863,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
           }
         }
-      }
-      if (ok) {
-        tc_fence_before();
-        mbar_arrive(&bars[B_EPIDONE]);
       }
     }
   }
