@@ -12,23 +12,23 @@
 // B200 design: persistent CTAs (one per SM), each walking 128-row query tiles
 // (b, h, query block) in head-major order.  The listed key blocks of a tile
 // are taken two at a time ("steps" of 128 keys): one N = 128 tensor-core
-// product per step for S, and one max exchange per 128 keys.  320 threads:
+// product per step for S, and one max exchange per 128 keys.  352 threads:
 //   warp 8      TMA producer, running ahead across tiles: per step the two
 //               key tiles side by side in one 128-row slot of a 2-slot ring
 //               (freed once S has read it); per listed block its phi(K), V
-//               tiles (fp16) in a 4-slot ring (freed after PV); per tile the
-//               Q tile (as soon as the previous tile's S products are done)
-//               and, in the next ring slot after its blocks, the fp16
+//               tiles (fp16) in a 4-slot ring (freed after PV and H); per tile
+//               the Q tile (as soon as the previous tile's S products are
+//               done) and, in the next ring slot after its blocks, the fp16
 //               H_tot / sigma tile of its head.
-//   warp 9      tcgen05 issuer (one thread), fp32 accumulators in TMEM:
-//                 S     = Q [K_a | K_b]^T               (bf16 operands in smem)
-//                 H_ex += phi(K_j)^T V_j                (fp16)
-//                 O    += [P_a | P_b] [V_a ; V_b]       (fp16 P read from TMEM)
-//               in the order S_{i+1}, H_i, PV_i so S runs ahead of the
-//               softmax; per tile phi(Q) H_i / sigma (phi(Q) in TMEM), for SLA
-//               also O_l W_proj (bf16 hi + lo split).  It starts the next
-//               tile's first S product before the previous tile's epilogue
-//               products.
+//   warps 9, 10 tcgen05 issuers (one thread each), fp32 accumulators in TMEM.
+//               Warp 9:   S = Q [K_a | K_b]^T  (bf16 operands in smem) and
+//                         O += [P_a | P_b] [V_a ; V_b] (fp16 P from TMEM), in
+//                         the order S_{i+1}, PV_i so S runs ahead of the softmax.
+//               Warp 10:  H_ex += phi(K_j)^T V_j (fp16), and per tile
+//                         phi(Q) H_i / sigma (phi(Q) in TMEM), for SLA also
+//                         O_l W_proj (bf16 hi + lo split).
+//               Two issuers keep the tensor pipe fed with H work while warp 9
+//               waits for P.
 //   warps 0..7  softmax and epilogue: warp w owns query rows 32(w%4)..+31
 //               (its TMEM lane quarter) and key / channel half w/4 (one of
 //               the two key blocks of a step), so two warps share each row.
@@ -40,7 +40,7 @@
 //               The epilogue re-reads the tile's Q rows (bf16, L2-resident)
 //               for phi(Q), so the Q tile in smem is replaced as soon as the
 //               tile's S products are done.
-// TMEM (512 columns): S0 | S1 (128 each, P over their first 64) | O (128) |
+// TMEM (512 columns): S0 | S1 (128 each, P over part of them) | O (128) |
 // H_ex (128, then phi(Q) H_i or the SLA projection in the epilogue).
 // The linear branch uses H_i = H_tot - sum over the listed blocks of
 // phi(K_j)^T V_j (H_tot from sla_prepare) and Z_i = Z_tot - the listed
@@ -61,7 +61,7 @@ namespace sla {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // 8 softmax warps, producer, two MMA issuers
 constexpr int kCompute = 256;
 constexpr int kKSlots = 2;  // key-pair slots
 constexpr int kVSlots = 4;  // phi(K) | V block slots (one also carries the H tile)
@@ -92,7 +92,8 @@ struct Lay {
 };
 
 // TMEM columns (512 allocated; one CTA per SM)
-constexpr uint32_t T_S0 = 0;     // S buffer b at T_S0 + 128 b; P_b over its first 64 (bf16) / 32 (e4m3)
+constexpr uint32_t T_S0 = 0;     // S buffer b at T_S0 + 128 b; each key block's P over the first 32 (bf16) /
+                                 // 16 (e4m3) columns of its 64
 constexpr uint32_t T_O = 256;    // O accumulator
 constexpr uint32_t T_HK = 384;   // H_ex accumulator; epilogue: phi(Q) H_i, then O_l W_proj
 constexpr uint32_t TMEM_COLS = 512;
@@ -113,8 +114,8 @@ enum {
   B_EPIDONE = 23,
   B_PROJR = 24,
   B_PROJF = 25,
-  B_DRAIN = 26,
-  NBAR = 27
+  B_DRAIN = 26,   // +issuer (2)
+  NBAR = 28
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
@@ -206,20 +207,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bars[B_VFULL + s], 1);
-      mbar_init(&bars[B_VEMPTY + s], 1);
+      mbar_init(&bars[B_VEMPTY + s], 2);  // released by both issuers
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[B_SFULL + b], 1);
       mbar_init(&bars[B_PFULL + b], kCompute);
       mbar_init(&bars[B_PEMPTY + b], 1);
     }
-    mbar_init(&bars[B_OFINAL], 1);
+    mbar_init(&bars[B_OFINAL], 2);  // both issuers' products of the tile are done
     mbar_init(&bars[B_EPI], kCompute);
     mbar_init(&bars[B_NUM], 1);
     mbar_init(&bars[B_EPIDONE], kCompute);
     mbar_init(&bars[B_PROJR], kCompute);
     mbar_init(&bars[B_PROJF], 1);
     mbar_init(&bars[B_DRAIN], 1);
+    mbar_init(&bars[B_DRAIN + 1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -326,9 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = gv > kVSlots ? gv - kVSlots : 0; g < gv; ++g)
         mbar_wait_drain(&bars[B_VFULL + g % kVSlots], (g / kVSlots) & 1);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 9 issues S and PV (the chain through the softmax), warp 10 the
+    // phi(K)^T V products and the epilogue products, so the tensor pipe gets
+    // H work while warp 9 waits for P.  Both walk the V ring and release each
+    // entry once its data has landed and their products on it are done.
     if (lane == 0) {
+      const bool sp = warp == 9;
       const uint32_t id_qk = idesc_f16(1, 0, 0, 128, 128);  // Q (K-major) x [K_a|K_b] (K-major), bf16
       const uint32_t id_qk1 = idesc_f16(1, 0, 0, 128, 64);  // one key block
       const uint32_t id_h = idesc_f16(0, 1, 1, 128, 128);   // phi(K)^T (MN-major) x V (MN-major), f16
@@ -347,11 +354,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dH = sdesc_sw128(smem_u32(sm + OFF_V), 16384, 1024);       // H tile / W_proj in a V slot
       int gk = 0, gv = 0, gs = 0, ti = 0;
       bool ok = true;
-      // S for step s of T into buffer g & 1; frees the key slot when done
-      auto issue_s = [&](const Tile& T, int s, int g, bool last_s) -> bool {
+      // The first barrier test after products that read both operands from
+      // smem stalls until their reads drain (~300 cycles); after products
+      // with A in TMEM it costs little.  So warp 9 waits for all of a step's
+      // data right after the previous PV.
+      auto wait_k = [&]() -> bool {  // the next key pair has landed (TMA data: no tcgen05 fence needed)
         const int sl = gk % kKSlots;
-        if (!mbar_wait(&bars[B_KFULL + sl], (gk / kKSlots) & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
+        return mbar_wait(&bars[B_KFULL + sl], (gk / kKSlots) & 1, abort_flag, a.status);
+      };
+      // S for step s of T into buffer g & 1 (key pair already waited for); frees the slot when done
+      auto issue_s = [&](const Tile& T, int s, int g, bool last_s) {
+        const int sl = gk % kKSlots;
         const bool two = 2 * s + 1 < T.n_crit;
         const uint64_t kb = dK + ((sl * KSLOT) >> 4);
         const uint32_t d = tmem + T_S0 + (g & 1) * 128;
@@ -369,12 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[B_KEMPTY + sl]);
         if (last_s) mma_commit(&bars[B_QFREE]);
         ++gk;
-        return true;
       };
       auto take_v = [&]() -> int {  // next V-ring entry, once it has landed
         const int sl = gv % kVSlots;
         if (!mbar_wait(&bars[B_VFULL + sl], (gv / kVSlots) & 1, abort_flag, a.status)) return -1;
-        tc_fence_after();
         ++gv;
         return sl;
       };
@@ -405,32 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_f16_ts(tmem + col, tmem + a_col + kk * 8u, b + kk * 128u, idesc, (first && kk == 0) ? 0u : 1u);
       };
-
-      // the previous tile's epilogue products, run after the next tile's first S
-      bool pend = false, pend_lin = false;
-      int pend_ti = 0, pend_sl = 0, pend_par = 0;
-      uint32_t pend_col = 0;
-      auto finish_epi = [&]() -> bool {
+      bool pend = false;  // the previous tile's epilogue is outstanding
+      int pend_ti = 0;
+      auto wait_epidone = [&]() -> bool {
         pend = false;
-        if (!mbar_wait(&bars[B_EPI], pend_ti & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const uint64_t hb = dH + ((pend_sl * VSLOT) >> 4);
-        if (pend_lin) {
-          if (!mbar_wait(&bars[B_VFULL + pend_sl], pend_par, abort_flag, a.status)) return false;
-          tc_fence_after();
-          issue_ts128(pend_col, T_HK, hb, id_pv, true);  // phi(Q) H_i / sigma
-        }
-        mma_commit(&bars[B_NUM]);
-        if (a.wproj != nullptr) {
-          if (!mbar_wait(&bars[B_PROJR], pend_ti & 1, abort_flag, a.status)) return false;
-          tc_fence_after();
-          if (pend_lin) {
-            issue_ts128(pend_col, T_HK, hb, id_bf, true);        // O_l hi x W_proj
-            issue_ts128(pend_col + 64, T_HK, hb, id_bf, false);  // O_l lo x W_proj
-          }
-          mma_commit(&bars[B_PROJF]);
-        }
-        if (pend_lin) mma_commit(&bars[B_VEMPTY + pend_sl]);
         if (!mbar_wait(&bars[B_EPIDONE], pend_ti & 1, abort_flag, a.status)) return false;
         tc_fence_after();
         return true;
@@ -438,72 +427,99 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++ti) {
         const Tile T = tile_at(a, t, false);
-        if (!mbar_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status)) break;
-        tc_fence_after();
-        const int ns = T.nsteps;
-        if (ns > 0 && !issue_s(T, 0, gs, ns == 1)) break;
-        if (pend && !finish_epi()) break;
-        if (ns == 0) mma_commit(&bars[B_QFREE]);
-        for (int i = 0; ok && i < ns; ++i) {
-          const int g = gs + i, b = g & 1;
-          if (i + 1 < ns && !issue_s(T, i + 1, g + 1, i + 1 == ns - 1)) {
-            ok = false;
-            break;
+        if (sp) {
+          // ---------------------------------------------- warp 9: S, PV
+          if (!mbar_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          const int ns = T.nsteps;
+          if (ns > 0) {
+            if (!wait_k()) break;
+            issue_s(T, 0, gs, ns == 1);
           }
-          const bool two = 2 * i + 1 < T.n_crit;
-          const int sa = take_v();
-          if (sa < 0) {
-            ok = false;
-            break;
-          }
-          issue_h(sa, i == 0);
-          int sb = -1;
-          if (two) {
-            sb = take_v();
-            if (sb < 0) {
+          if (ns == 0) mma_commit(&bars[B_QFREE]);
+          if (pend && !wait_epidone()) break;  // O is free again
+          for (int i = 0; ok && i < ns; ++i) {
+            const int g = gs + i, b = g & 1;
+            const bool two = 2 * i + 1 < T.n_crit;
+            if (i + 1 < ns && !wait_k()) {
               ok = false;
               break;
             }
-            issue_h(sb, false);
+            const int sa = take_v();
+            const int sb = (sa >= 0 && two) ? take_v() : -1;
+            if (sa < 0 || (two && sb < 0)) {
+              ok = false;
+              break;
+            }
+            if (i + 1 < ns) issue_s(T, i + 1, g + 1, i + 1 == ns - 1);
+            if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pcol = T_S0 + b * 128;
+            issue_pv(sa, pcol, i == 0);
+            if (two) issue_pv(sb, pcol + 64u, false);  // block B's P over the first columns of its S half
+            mma_commit(&bars[B_PEMPTY + b]);
+            mma_commit(&bars[B_VEMPTY + sa]);
+            if (two) mma_commit(&bars[B_VEMPTY + sb]);
           }
-          if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status)) {
-            ok = false;
-            break;
+          // the tile's other V-ring entries (negligible blocks, H tile) are warp 10's
+          for (int it = T.n_crit; ok && it < T.n_total + (T.has_lin ? 1 : 0); ++it) {
+            const int sl = take_v();
+            if (sl < 0) {
+              ok = false;
+              break;
+            }
+            mma_commit(&bars[B_VEMPTY + sl]);
           }
+          if (!ok) break;
+          mma_commit(&bars[B_OFINAL]);
+          gs += ns;
+        } else {
+          // ---------------------------------------------- warp 10: H, epilogue products
+          if (pend && !wait_epidone()) break;  // H_ex, phi(Q) H_i of the previous tile have been read
+          for (int it = 0; ok && it < T.n_total; ++it) {
+            const int sl = take_v();
+            if (sl < 0) {
+              ok = false;
+              break;
+            }
+            issue_h(sl, it == 0);  // (TMA data: no tcgen05 fence needed)
+            mma_commit(&bars[B_VEMPTY + sl]);
+          }
+          if (!ok) break;
+          mma_commit(&bars[B_OFINAL]);
+          // epilogue: phi(Q) (TMEM, the tile's last S buffer) x H_i / sigma (smem, the H tile's slot)
+          if (!mbar_wait(&bars[B_EPI], ti & 1, abort_flag, a.status)) break;
           tc_fence_after();
-          const uint32_t pcol = T_S0 + b * 128;
-          issue_pv(sa, pcol, i == 0);
-          if (two) issue_pv(sb, pcol + (kFP8 ? 16u : 32u), false);
-          mma_commit(&bars[B_PEMPTY + b]);
-          mma_commit(&bars[B_VEMPTY + sa]);
-          if (two) mma_commit(&bars[B_VEMPTY + sb]);
-        }
-        for (int it = T.n_crit; ok && it < T.n_total; ++it) {
-          const int sl = take_v();
-          if (sl < 0) {
-            ok = false;
-            break;
+          const uint32_t ecol = T_S0 + ((gs + T.nsteps - 1) & 1) * 128;
+          gs += T.nsteps;
+          int hs = 0;
+          if (T.has_lin) {
+            hs = take_v();
+            if (hs < 0) break;
+            issue_ts128(ecol, T_HK, dH + ((hs * VSLOT) >> 4), id_pv, true);
           }
-          issue_h(sl, it == 0);
-          mma_commit(&bars[B_VEMPTY + sl]);
+          mma_commit(&bars[B_NUM]);
+          if (a.wproj != nullptr) {
+            if (!mbar_wait(&bars[B_PROJR], ti & 1, abort_flag, a.status)) break;
+            tc_fence_after();
+            if (T.has_lin) {
+              const uint64_t hb = dH + ((hs * VSLOT) >> 4);
+              issue_ts128(ecol, T_HK, hb, id_bf, true);        // O_l hi x W_proj
+              issue_ts128(ecol + 64, T_HK, hb, id_bf, false);  // O_l lo x W_proj
+            }
+            mma_commit(&bars[B_PROJF]);
+          }
+          if (T.has_lin) mma_commit(&bars[B_VEMPTY + hs]);
         }
-        if (!ok) break;
-        mma_commit(&bars[B_OFINAL]);
-        gs += ns;
         pend = true;
         pend_ti = ti;
-        pend_lin = T.has_lin;
-        pend_col = T_S0 + ((gs - 1) & 1) * 128;  // the tile's last S buffer: phi(Q), SLA O_l
-        if (T.has_lin) {  // the H tile follows the tile's blocks in the V ring
-          pend_sl = gv % kVSlots;
-          pend_par = (gv / kVSlots) & 1;
-          ++gv;
-        }
       }
-      if (ok && pend) finish_epi();
       // all MMAs must finish before the CTA releases TMEM
-      mma_commit(&bars[B_DRAIN]);
-      mbar_wait_drain(&bars[B_DRAIN], 0);
+      mma_commit(&bars[B_DRAIN + (sp ? 0 : 1)]);
+      mbar_wait_drain(&bars[B_DRAIN + (sp ? 0 : 1)], 0);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 0..7)
@@ -523,7 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++xc;
       return o;
     };
-    auto list_at = [&](const Tile& T, int p) -> int {  // critical block at position p, or -1
+    // Lane l holds the block of this half at step 32 c + l of the current
+    // chunk c (one coalesced load per 32 steps); steps read it by shuffle.
+    auto list_chunk = [&](const Tile& T, int c) -> int {
+      const int p = 2 * (32 * c + lane) + half;
       if (p >= T.n_crit) return -1;
       const int j = T.crit[p];
       return (j < 0 || j >= a.nkv) ? 0 : j;
@@ -534,46 +553,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_valid = (r < a.bq) && (tok < a.N);
       float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
       if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
-      int j_cur = list_at(T, half);
+      int jl = list_chunk(T, 0);
+      const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
+      const float sigma = T.has_lin ? a.sigma[T.bh] : 1.0f;
+      const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
 
       // ---------------------------------------------------------- steps of two key blocks
       float m_run = -INFINITY, l_part = 0.0f, zex = 0.0f;
       const float* zb = a.zblk + static_cast<long long>(T.bh) * a.nkv * kDPad + r;
       for (int i = 0; i < T.nsteps; ++i) {
         const int g = gs + i, b = g & 1;
-        const int j_next = list_at(T, 2 * (i + 1) + half);
+        if (i > 0 && (i & 31) == 0) jl = list_chunk(T, i >> 5);
+        const int j_cur = __shfl_sync(0xffffffffu, jl, i & 31);
+        if (i == T.nsteps - 1 && T.has_lin && tok < a.N) {
+          // the epilogue re-reads this row of Q: bring it back into L2 now
+          asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(static_cast<const __nv_bfloat16*>(a.qsrc) +
+                                                                   (static_cast<long long>(T.bh) * a.N + tok) * kDPad +
+                                                                   64 * half));
+        }
         const float zv = (T.has_lin && j_cur >= 0) ? zb[static_cast<long long>(j_cur) * kDPad] : 0.0f;
         ok = ok && warp_wait(&bars[B_SFULL + b], (g >> 1) & 1, abort_flag, a.status);
-        float s[64];
-        if (ok && j_cur >= 0) {
-          tc_fence_after();
-          tmem_ld32(tmem + lrow + T_S0 + b * 128 + 64 * half, s);
-          tmem_ld32(tmem + lrow + T_S0 + b * 128 + 64 * half + 32, s + 32);
-          tmem_wait_ld();
-          if (tail && j_cur == a.nkv - 1) {
-            const int nvalid = a.N - j_cur * kBlockKV;
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c >= nvalid) s[c] = -INFINITY;
-          }
-        } else {
-          const float fill = ok ? -INFINITY : 0.0f;  // no second block in this step
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = fill;
-        }
+        const bool live = ok && j_cur >= 0;  // this half has a key block in this step
+        const uint32_t scol = tmem + lrow + T_S0 + b * 128 + 64 * half;  // this half's 64 S columns
+        const int nvalid = (tail && j_cur == a.nkv - 1) ? a.N - j_cur * kBlockKV : kBlockKV;
         float sc = a.sl2;
         if constexpr (kFP8) {
           if (j_cur >= 0) sc = sl2_q * a.sk[static_cast<long long>(T.bh) * a.nb128 + (j_cur >> 1)];  // 128-token key block
         }
-        float m8[8];
+        // pass 1: the block's row max (keys past N masked)
+        float mx = -INFINITY;
+        if (live) {
+          tc_fence_after();
+          float s[64];
+          tmem_ld32(scol, s);
+          tmem_ld32(scol + 32, s + 32);
+          tmem_wait_ld();
+          if (nvalid < kBlockKV) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          m8[c] = fmaxf(fmaxf(fmaxf(s[8 * c], s[8 * c + 1]), fmaxf(s[8 * c + 2], s[8 * c + 3])),
-                        fmaxf(fmaxf(s[8 * c + 4], s[8 * c + 5]), fmaxf(s[8 * c + 6], s[8 * c + 7])));
+            for (int c = 0; c < 64; ++c)
+              if (c >= nvalid) s[c] = -INFINITY;
+          }
+          float m8[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            m8[c] = fmaxf(fmaxf(fmaxf(s[8 * c], s[8 * c + 1]), fmaxf(s[8 * c + 2], s[8 * c + 3])),
+                          fmaxf(fmaxf(s[8 * c + 4], s[8 * c + 5]), fmaxf(s[8 * c + 6], s[8 * c + 7])));
+          }
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sc;
         }
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
-                         sc;
         const float mt = fmaxf(mx, xchg(mx));
         // bf16: refresh the max only when it grows by more than 15 (p <= 2^15 fits
         // fp16); e4m3: p * 448 must stay within e4m3, so the exact running max
@@ -587,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
               tc_fence_after();
 #pragma unroll 1
-              for (int cc = 0; cc < 4; ++cc) {  // 16 columns at a time: few registers next to s[]
+              for (int cc = 0; cc < 4; ++cc) {  // 16 columns at a time
                 float o[16];
                 tmem_ld16(tmem + lrow + T_O + 64 * half + 16 * cc, o);
                 tmem_wait_ld();
@@ -601,37 +628,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_part *= f;
           m_run = m_new;
         }
+        // pass 2: p = 2^(s*sc - m), 32 keys at a time; P goes over the first 32
+        // (bf16) / 16 (e4m3) columns of this half's S, which pass 1 has read
         const float nm = -m_run;
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if constexpr (kFP8) {
-          // p in (0, 1] against the running max; the row sum uses the unquantised p,
-          // the PV product p * 448 rounded to e4m3 (four keys per TMEM column)
-          uint32_t pk[16];
+        if (live) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float p[4];
+          for (int cc = 0; cc < 2; ++cc) {
+            float s[32];
+            tmem_ld32(scol + 32 * cc, s);
+            tmem_wait_ld();
+            if (nvalid < kBlockKV) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(s[4 * c + e], sc, nm));
-            l4[c & 3] += (p[0] + p[1]) + (p[2] + p[3]);
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0] * 448.0f, p[1] * 448.0f), __NV_SATFINITE,
-                                                         __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2] * 448.0f, p[3] * 448.0f), __NV_SATFINITE,
-                                                         __NV_E4M3);
-            pk[c] = lo | (hi << 16);
-          }
-          if (ok) tmem_st16(tmem + lrow + T_S0 + b * 128 + 16 * half, pk);
-        } else {
-          uint32_t pk[32];
+              for (int c = 0; c < 32; ++c)
+                if (32 * cc + c >= nvalid) s[c] = -INFINITY;
+            }
+            if constexpr (kFP8) {
+              // the row sum uses the unquantised p; the PV product p * 448 rounded
+              // to e4m3 (four keys per TMEM column)
+              uint32_t pk[8];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(s[2 * c], sc, nm));
-            const float p1 = ex2_approx(fmaf(s[2 * c + 1], sc, nm));
-            l4[c & 3] += p0 + p1;
-            pk[c] = pack_half2(p0, p1);
-          }
-          if (ok) {
-            tmem_st16(tmem + lrow + T_S0 + b * 128 + 32 * half, pk);
-            tmem_st16(tmem + lrow + T_S0 + b * 128 + 32 * half + 16, pk + 16);
+              for (int c = 0; c < 8; ++c) {
+                float p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(s[4 * c + e], sc, nm));
+                l4[c & 3] += (p[0] + p[1]) + (p[2] + p[3]);
+                const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0] * 448.0f, p[1] * 448.0f),
+                                                             __NV_SATFINITE, __NV_E4M3);
+                const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p[2] * 448.0f, p[3] * 448.0f),
+                                                             __NV_SATFINITE, __NV_E4M3);
+                pk[c] = lo | (hi << 16);
+              }
+              tmem_st8(scol + 8 * cc, pk);
+            } else {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const float p0 = ex2_approx(fmaf(s[2 * c], sc, nm));
+                const float p1 = ex2_approx(fmaf(s[2 * c + 1], sc, nm));
+                l4[c & 3] += p0 + p1;
+                pk[c] = pack_half2(p0, p1);
+              }
+              tmem_st16(scol + 16 * cc, pk);
+            }
           }
         }
         l_part += (l4[0] + l4[1]) + (l4[2] + l4[3]);
@@ -641,7 +680,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bars[B_PFULL + b]);
         }
         zex += zv;
-        j_cur = j_next;
       }
       gs += T.nsteps;
       // SLA: the negligible blocks only leave the linear sum
@@ -667,9 +705,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           qw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
                                                   (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
       }
-      const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
-      const float sigma = T.has_lin ? a.sigma[T.bh] : 1.0f;
-      const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
       ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
       if (ok) tc_fence_after();
       const float l_run = l_part + xchg(l_part);
@@ -687,13 +722,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           float hk[32];
-          if (ok && T.n_total > 0) {
-            tmem_ld32(tmem + lrow + T_HK + 64 * half + 32 * cc, hk);
-            tmem_wait_ld();
-          } else {
+          tmem_ld32(tmem + lrow + T_HK + 64 * half + 32 * cc, hk);  // stale without listed blocks: dropped below
+          tmem_wait_ld();
+          const bool use_h = ok && T.n_total > 0;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) hk[c] = 0.0f;
-          }
+          for (int c = 0; c < 32; ++c) hk[c] = use_h ? hk[c] : 0.0f;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint4* hp = reinterpret_cast<uint4*>(hbuf + half * 16384u + sw128_off(r, 4 * cc + q4));
@@ -713,39 +746,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (half == 0) zsh[r] = zi;
         // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), fp16 pairs
         const int c0 = 64 * half;
-        float x[64];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f2 = unpack_bf162(ww[e]);
-            x[8 * u + 2 * e] = f2.x;
-            x[8 * u + 2 * e + 1] = f2.y;
-          }
-        }
+        uint32_t phq[32];
         if (a.phi == SLA_PHI_SOFTMAX) {
           float mx = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c0 + c < a.d) mx = fmaxf(mx, x[c]);
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              if (c0 + 8 * u + 2 * e < a.d) mx = fmaxf(mx, f2.x);
+              if (c0 + 8 * u + 2 * e + 1 < a.d) mx = fmaxf(mx, f2.y);
+            }
+          }
           mx = fmaxf(mx, xchg(mx));
           float sum = 0.0f;
+          float y[64];
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            x[c] = (c0 + c < a.d) ? ex2_approx((x[c] - mx) * 1.4426950408889634f) : 0.0f;
-            sum += x[c];
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              const int c = 8 * u + 2 * e;
+              y[c] = (c0 + c < a.d) ? ex2_approx((f2.x - mx) * 1.4426950408889634f) : 0.0f;
+              y[c + 1] = (c0 + c + 1 < a.d) ? ex2_approx((f2.y - mx) * 1.4426950408889634f) : 0.0f;
+              sum += y[c] + y[c + 1];
+            }
           }
           const float inv = 1.0f / (sum + xchg(sum));
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] *= inv;
+          for (int c = 0; c < 32; ++c) phq[c] = pack_half2(y[2 * c] * inv, y[2 * c + 1] * inv);
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = (c0 + c < a.d) ? elu1(x[c]) : 0.0f;
-        }
-        uint32_t phq[32];
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) phq[c] = pack_half2(x[2 * c], x[2 * c + 1]);
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              const int c = 8 * u + 2 * e;
+              phq[4 * u + e] = pack_half2((c0 + c < a.d) ? elu1(f2.x) : 0.0f, (c0 + c + 1 < a.d) ? elu1(f2.y) : 0.0f);
+            }
+          }
+        }
         named_bar_sync(5, kCompute);  // Z_i complete
         float dp = 0.0f;
 #pragma unroll
@@ -822,12 +865,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // combine 32 channels at a time; TMEM goes back after the last read
       const long long obase = (static_cast<long long>(T.bh) * a.N + tok) * a.d;
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int ch0 = 64 * half + 32 * cc;
+        // both accumulators are read unconditionally (a stale column is dropped by the select below)
         float o[32], nmv[32];
-        if (ok && T.n_crit > 0) tmem_ld32(tmem + lrow + T_O + ch0, o);
-        if (ok && T.has_lin) tmem_ld32(tmem + lrow + T_HK + ch0, nmv);
+        tmem_ld32(tmem + lrow + T_O + ch0, o);
+        tmem_ld32(tmem + lrow + T_HK + ch0, nmv);
         tmem_wait_ld();
         if (cc == 1 && ok) {
           tc_fence_before();
@@ -839,10 +883,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c)
             o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
         }
+        const bool use_s = ok && T.n_crit > 0, use_l = ok && T.has_lin;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float os = (ok && T.n_crit > 0) ? o[c] * w_s : 0.0f;
-          const float olv = (ok && T.has_lin) ? nmv[c] * lin_w : 0.0f;
+          const float os = use_s ? o[c] * w_s : 0.0f;
+          const float olv = use_l ? nmv[c] * lin_w : 0.0f;
           o[c] = os + olv;
         }
         if (ok && row_valid) {
