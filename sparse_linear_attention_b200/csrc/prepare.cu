@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
         float sum = 0.0f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          ph[e] = (8 * u + e < d) ? ex2_approx((kf[i][e] - mx) * 1.4426950408889634f) : 0.0f;
+          const float v = ex2_approx((kf[i][e] - mx) * 1.4426950408889634f);  // evaluated, then selected
+          ph[e] = (8 * u + e < d) ? v : 0.0f;
           sum += ph[e];
         }
 #pragma unroll
@@ -207,7 +208,10 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
         for (int e = 0; e < 8; ++e) ph[e] *= inv;
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ph[e] = (8 * u + e < d) ? elu1(kf[i][e]) : 0.0f;
+        for (int e = 0; e < 8; ++e) {
+          const float v = elu1(kf[i][e]);  // evaluated, then selected: no branch
+          ph[e] = (8 * u + e < d) ? v : 0.0f;
+        }
       }
       uint4 pu, vu;
       if (valid) {

@@ -150,6 +150,20 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Tile store smem -> global through a tensor map (elements past the map's
+// extent are not written); completion is tracked per thread by bulk groups.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until the committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
@@ -313,8 +327,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Branch-free: the exponential is always evaluated (on min(x, 0), so it
+// cannot overflow) and then selected; an asm call under a data-dependent
+// ternary becomes a divergent branch per element.
 __device__ __forceinline__ float elu1(float x) {
-  return x > 0.f ? x + 1.0f : ex2_approx(x * 1.4426950408889634f);
+  const float e = ex2_approx(fminf(x, 0.0f) * 1.4426950408889634f);
+  return x > 0.f ? x + 1.0f : e;
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -380,9 +398,5 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
   __half2 h = *reinterpret_cast<__half2*>(&u);
   return __half22float2(h);
 }
-
-// phi(x) = ELU(x) + 1.  Its results are rounded to fp16 or bf16 right after,
-// so the hardware exp2 (relative error near 2^-22) is ample.
-__device__ __forceinline__ float elu1(float x);
 
 }  // namespace sla

@@ -39,6 +39,7 @@ struct SparseArgs {
   const float* zblk;         // [BH, nkv, 128]: per-block column sums of phi(K)
   void* out;
   int out_bf16;
+  int tma_out;               // bf16 output, d = 128, bq = 128: 128-row tiles leave through a TMA store
   int phi;
   int* status;
   // e4m3 sparse branch

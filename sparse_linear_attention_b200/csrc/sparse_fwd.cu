@@ -37,8 +37,8 @@
 //               stale max scales numerator and denominator alike, and
 //               p <= 2^15 still fits fp16).  P is rounded to fp16 and written
 //               over the step's S columns in TMEM for the PV product.
-//               The epilogue re-reads the tile's Q rows (bf16, L2-resident)
-//               for phi(Q), so the Q tile in smem is replaced as soon as the
+//               phi(Q) is formed when the tile's Q lands and kept packed in
+//               registers, so the Q tile in smem is replaced as soon as the
 //               tile's S products are done.
 // TMEM (512 columns): S0 | S1 (128 each, P over part of them) | O (128) |
 // H_ex (128, then phi(Q) H_i or the SLA projection in the epilogue).
@@ -100,7 +100,7 @@ constexpr uint32_t TMEM_COLS = 512;
 
 enum {
   B_QFULL = 0,
-  B_QFREE = 1,    // MMA commit after the tile's last S product
+  B_QFREE = 1,    // the 256 softmax threads have read the Q tile + MMA commit after its last S
   B_KFULL = 2,    // +slot
   B_KEMPTY = 4,   // +slot
   B_VFULL = 6,    // +slot
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmV8,
-                      const SparseArgs a) {
+                      const __grid_constant__ CUtensorMap tmO, const SparseArgs a) {
   using L = Lay<kFP8>;
   constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V;
   constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_RED = L::OFF_RED, OFF_Z = L::OFF_Z;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     mbar_init(&bars[B_QFULL], 1);
-    mbar_init(&bars[B_QFREE], 1);
+    mbar_init(&bars[B_QFREE], kCompute + 1);
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
       mbar_init(&bars[B_KEMPTY + s], 1);
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(&bars[B_PROJF]);
           }
-          if (T.has_lin) mma_commit(&bars[B_VEMPTY + hs]);
+          if (T.has_lin && !a.tma_out) mma_commit(&bars[B_VEMPTY + hs]);  // else released after the output store
         }
         pend = true;
         pend_ti = ti;
@@ -554,6 +554,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
       if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
       int jl = list_chunk(T, 0);
+      // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), packed fp16,
+      // formed as soon as the tile's Q lands so the Q tile can be replaced early
+      uint32_t phq[32];
+      ok = ok && warp_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status);
+      {
+        uint4 qw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          qw[u] = make_uint4(0, 0, 0, 0);
+          if (T.has_lin) {
+            if constexpr (kFP8) {  // the smem tile holds e4m3 Q: read the bf16 row
+              if (tok < a.N)
+                qw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
+                                                        (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
+            } else {
+              qw[u] = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 16384u + sw128_off(r, u));
+            }
+          }
+        }
+        mbar_arrive(&bars[B_QFREE]);  // this thread no longer reads the Q tile
+        const int c0 = 64 * half;
+        if (a.phi == SLA_PHI_SOFTMAX) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              if (c0 + 8 * u + 2 * e < a.d) mx = fmaxf(mx, f2.x);
+              if (c0 + 8 * u + 2 * e + 1 < a.d) mx = fmaxf(mx, f2.y);
+            }
+          }
+          mx = fmaxf(mx, xchg(mx));
+          float sum = 0.0f;
+          float y[64];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              const int c = 8 * u + 2 * e;
+              const float e0 = ex2_approx((f2.x - mx) * 1.4426950408889634f);  // evaluated, then selected
+              const float e1 = ex2_approx((f2.y - mx) * 1.4426950408889634f);
+              y[c] = (c0 + c < a.d) ? e0 : 0.0f;
+              y[c + 1] = (c0 + c + 1 < a.d) ? e1 : 0.0f;
+              sum += y[c] + y[c + 1];
+            }
+          }
+          const float inv = 1.0f / (sum + xchg(sum));
+#pragma unroll
+          for (int c = 0; c < 32; ++c) phq[c] = pack_half2(y[2 * c] * inv, y[2 * c + 1] * inv);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf162(ww[e]);
+              const int c = 8 * u + 2 * e;
+              const float e0 = elu1(f2.x), e1 = elu1(f2.y);  // evaluated, then selected: no branch
+              phq[4 * u + e] = pack_half2((c0 + c < a.d) ? e0 : 0.0f, (c0 + c + 1 < a.d) ? e1 : 0.0f);
+            }
+          }
+        }
+      }
       const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
       const float sigma = T.has_lin ? a.sigma[T.bh] : 1.0f;
       const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
@@ -565,12 +632,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = gs + i, b = g & 1;
         if (i > 0 && (i & 31) == 0) jl = list_chunk(T, i >> 5);
         const int j_cur = __shfl_sync(0xffffffffu, jl, i & 31);
-        if (i == T.nsteps - 1 && T.has_lin && tok < a.N) {
-          // the epilogue re-reads this row of Q: bring it back into L2 now
-          asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(static_cast<const __nv_bfloat16*>(a.qsrc) +
-                                                                   (static_cast<long long>(T.bh) * a.N + tok) * kDPad +
-                                                                   64 * half));
-        }
         const float zv = (T.has_lin && j_cur >= 0) ? zb[static_cast<long long>(j_cur) * kDPad] : 0.0f;
         ok = ok && warp_wait(&bars[B_SFULL + b], (g >> 1) & 1, abort_flag, a.status);
         const bool live = ok && j_cur >= 0;  // this half has a key block in this step
@@ -696,15 +757,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ---------------------------------------------------------- epilogue
-      // this row's 64 channels of Q (bf16, from L2: the tile was read moments ago)
-      uint4 qw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        qw[u] = make_uint4(0, 0, 0, 0);
-        if (T.has_lin && tok < a.N)
-          qw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
-                                                  (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
-      }
       ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
       if (ok) tc_fence_after();
       const float l_run = l_part + xchg(l_part);
@@ -744,51 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Z_i[e] for e = r, shared with every row for the denominator
         const float zi = zt_r - (zex + xchg(zex));
         if (half == 0) zsh[r] = zi;
-        // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), fp16 pairs
         const int c0 = 64 * half;
-        uint32_t phq[32];
-        if (a.phi == SLA_PHI_SOFTMAX) {
-          float mx = -INFINITY;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f2 = unpack_bf162(ww[e]);
-              if (c0 + 8 * u + 2 * e < a.d) mx = fmaxf(mx, f2.x);
-              if (c0 + 8 * u + 2 * e + 1 < a.d) mx = fmaxf(mx, f2.y);
-            }
-          }
-          mx = fmaxf(mx, xchg(mx));
-          float sum = 0.0f;
-          float y[64];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f2 = unpack_bf162(ww[e]);
-              const int c = 8 * u + 2 * e;
-              y[c] = (c0 + c < a.d) ? ex2_approx((f2.x - mx) * 1.4426950408889634f) : 0.0f;
-              y[c + 1] = (c0 + c + 1 < a.d) ? ex2_approx((f2.y - mx) * 1.4426950408889634f) : 0.0f;
-              sum += y[c] + y[c + 1];
-            }
-          }
-          const float inv = 1.0f / (sum + xchg(sum));
-#pragma unroll
-          for (int c = 0; c < 32; ++c) phq[c] = pack_half2(y[2 * c] * inv, y[2 * c + 1] * inv);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f2 = unpack_bf162(ww[e]);
-              const int c = 8 * u + 2 * e;
-              phq[4 * u + e] = pack_half2((c0 + c < a.d) ? elu1(f2.x) : 0.0f, (c0 + c + 1 < a.d) ? elu1(f2.y) : 0.0f);
-            }
-          }
-        }
         named_bar_sync(5, kCompute);  // Z_i complete
         float dp = 0.0f;
 #pragma unroll
@@ -863,7 +871,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         w_s = alpha_t * inv_l;
         lin_w = (1.0f - alpha_t) * lin_scale;
       }
-      // combine 32 channels at a time; TMEM goes back after the last read
+      // combine 32 channels at a time; TMEM goes back after the last read.  With
+      // a TMA store the bf16 rows are staged in the H tile's slot (its products
+      // are done) and leave as two 64-channel boxes.
+      const bool tma_o = a.tma_out && T.has_lin;
       const long long obase = (static_cast<long long>(T.bh) * a.N + tok) * a.d;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
@@ -890,7 +901,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float olv = use_l ? nmv[c] * lin_w : 0.0f;
           o[c] = os + olv;
         }
-        if (ok && row_valid) {
+        if (tma_o) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8)
+            *reinterpret_cast<uint4*>(hbuf + half * 16384u + sw128_off(r, 4 * cc + q8)) =
+                make_uint4(pack_bf162(o[8 * q8], o[8 * q8 + 1]), pack_bf162(o[8 * q8 + 2], o[8 * q8 + 3]),
+                           pack_bf162(o[8 * q8 + 4], o[8 * q8 + 5]), pack_bf162(o[8 * q8 + 6], o[8 * q8 + 7]));
+        } else if (ok && row_valid) {
           if (a.out_bf16) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + obase;
 #pragma unroll
@@ -909,7 +926,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (tma_o) {
+        fence_proxy_async_smem();      // the staged rows are visible to the TMA engine
+        named_bar_sync(5, kCompute);   // ... from every thread
+        if (tid == 0) {
+          if (ok) {
+            tma_store_3d(&tmO, hbuf, 0, T.qb * 128, T.bh);
+            tma_store_3d(&tmO, hbuf + 16384, 64, T.qb * 128, T.bh);
+            bulk_commit_group();
+            bulk_wait_read_all();      // the slot may be refilled once the store has read it
+          }
+          mbar_arrive(&bars[B_VEMPTY + hsl]);
+        }
+      }
     }
+    if (tid == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -925,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <bool kFP8>
 static cudaError_t launch_sparse_t(const SparseArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
                                    const CUtensorMap& mp, const CUtensorMap& mv, const CUtensorMap& mh,
-                                   const CUtensorMap& mv8, cudaStream_t st) {
+                                   const CUtensorMap& mv8, const CUtensorMap& mo, cudaStream_t st) {
   constexpr uint32_t smem = Lay<kFP8>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(sparse_fwd_kernel<kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -933,15 +964,23 @@ static cudaError_t launch_sparse_t(const SparseArgs& a, const CUtensorMap& mq, c
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long ntiles = static_cast<long long>(a.BH) * a.nq;
   const unsigned grid = static_cast<unsigned>(ntiles < sms ? ntiles : sms);
-  sparse_fwd_kernel<kFP8><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, a);
+  sparse_fwd_kernel<kFP8><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, mo, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const void* k_bf16_128,
+cudaError_t launch_sparse(const SparseArgs& a_in, const void* q_bf16_128, const void* k_bf16_128,
                           const void* phik16, const void* v16, const void* hs16, const void* q8, const void* k8,
                           const void* v8, cudaStream_t st) {
-  CUtensorMap mq, mk, mp, mv, mh, mv8;
+  CUtensorMap mq, mk, mp, mv, mh, mv8, mo;
   cudaError_t e;
+  SparseArgs a = a_in;
+  // bf16 output of 128-row query blocks at d = 128 leaves through TMA tile stores
+  a.tma_out = (a.out_bf16 && a.d == kDPad && a.bq == 128) ? 1 : 0;
+  if (a.tma_out) {
+    if ((e = encode_map(&mo, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
+  } else {
+    mo = {};
+  }
   if ((e = encode_map(&mp, phik16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
   if ((e = encode_map(&mv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
   if ((e = encode_map(&mh, hs16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kDPad, a.BH, 128)) != cudaSuccess) return e;
@@ -949,11 +988,11 @@ cudaError_t launch_sparse(const SparseArgs& a, const void* q_bf16_128, const voi
     if ((e = encode_map8(&mq, q8, a.N, a.BH, 128)) != cudaSuccess) return e;
     if ((e = encode_map8(&mk, k8, a.N, a.BH, 64)) != cudaSuccess) return e;
     if ((e = encode_map8(&mv8, v8, a.N, a.BH, 64)) != cudaSuccess) return e;
-    return launch_sparse_t<true>(a, mq, mk, mp, mv, mh, mv8, st);
+    return launch_sparse_t<true>(a, mq, mk, mp, mv, mh, mv8, mo, st);
   }
   if ((e = encode_map(&mq, q_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
   if ((e = encode_map(&mk, k_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
-  return launch_sparse_t<false>(a, mq, mk, mp, mv, mh, mv, st);
+  return launch_sparse_t<false>(a, mq, mk, mp, mv, mh, mv, mo, st);
 }
 
 }  // namespace sla
