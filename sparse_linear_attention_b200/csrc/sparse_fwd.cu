@@ -64,7 +64,7 @@ namespace {
 constexpr int kThreads = 352;  // 8 softmax warps, producer, two MMA issuers
 constexpr int kCompute = 256;
 constexpr int kKSlots = 2;  // key-pair slots
-constexpr int kVSlots = 4;  // phi(K) | V block slots (one also carries the H tile)
+constexpr int kVSlots = 2;  // value entries: the phi(K) | V tiles of a step's two blocks, or the H tile
 
 // Shared-memory layout (the dynamic shared window is 1024-byte aligned).
 //   bf16 branch: Q tile 2 x [128 rows][128 B]; key-pair slot
@@ -78,7 +78,8 @@ struct Lay {
   static constexpr uint32_t QBYTES = kFP8 ? 16384 : 32768;
   static constexpr uint32_t KBLK = kFP8 ? 8192 : 16384;  // bytes of one key block
   static constexpr uint32_t KSLOT = 2 * KBLK;
-  static constexpr uint32_t VSLOT = kFP8 ? 40960 : 32768;
+  static constexpr uint32_t VBLK = kFP8 ? 40960 : 32768;  // one key block's phi(K) | V (| V8)
+  static constexpr uint32_t VSLOT = 2 * VBLK;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = QBYTES;
   static constexpr uint32_t OFF_V = OFF_K + kKSlots * KSLOT;
@@ -88,7 +89,7 @@ struct Lay {
   static constexpr uint32_t OFF_Z = OFF_RED + 2048;    // Z_i [128] floats
   static constexpr uint32_t SMEM_BYTES = OFF_Z + 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && VSLOT % 1024 == 0, "1 KB aligned tiles");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && VBLK % 1024 == 0, "1 KB aligned tiles");
 };
 
 // TMEM columns (512 allocated; one CTA per SM)
@@ -101,28 +102,27 @@ constexpr uint32_t TMEM_COLS = 512;
 enum {
   B_QFULL = 0,
   B_QFREE = 1,    // the 256 softmax threads have read the Q tile + MMA commit after its last S
-  B_KFULL = 2,    // +slot
-  B_KEMPTY = 4,   // +slot
-  B_VFULL = 6,    // +slot
-  B_VEMPTY = 10,  // +slot
-  B_SFULL = 14,   // +buffer
-  B_PFULL = 16,   // +buffer
-  B_PEMPTY = 18,  // +buffer
-  B_OFINAL = 20,
-  B_EPI = 21,
-  B_NUM = 22,
-  B_EPIDONE = 23,
-  B_PROJR = 24,
-  B_PROJF = 25,
-  B_DRAIN = 26,   // +issuer (2)
-  NBAR = 28
+  B_KFULL = 2,    // +slot; a key-pair slot is free again once S of its step is done (B_SFULL)
+  B_VFULL = 4,    // +slot
+  B_VEMPTY = 6,   // +slot
+  B_SFULL = 8,    // +buffer (= key-pair slot)
+  B_PFULL = 10,   // +buffer
+  B_PEMPTY = 12,  // +buffer
+  B_OFINAL = 14,
+  B_EPI = 15,
+  B_NUM = 16,
+  B_EPIDONE = 17,
+  B_PROJR = 18,
+  B_PROJF = 19,
+  B_DRAIN = 20,   // +issuer (2)
+  NBAR = 22
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
 struct Tile {
   int bh, qb;
   long long row;
-  int n_crit, n_negl, n_total, nsteps;
+  int n_crit, n_negl, n_total, nsteps, nnegl_e;  // nnegl_e: value entries of negligible blocks (two per entry)
   const int32_t* crit;
   const int32_t* negl;
   bool has_lin;
@@ -147,6 +147,7 @@ __device__ __forceinline__ Tile tile_at(const SparseArgs& a, int t, bool report)
   }
   T.n_total = T.n_crit + T.n_negl;
   T.nsteps = (T.n_crit + 1) >> 1;
+  T.nnegl_e = (T.n_negl + 1) >> 1;
   T.crit = a.crit_idx + T.row * a.list_stride;
   T.negl = a.negl_idx ? a.negl_idx + T.row * a.list_stride : T.crit;
   T.has_lin = (a.nkv - T.n_total) > 0;
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = Lay<kFP8>;
   constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V;
   constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_RED = L::OFF_RED, OFF_Z = L::OFF_Z;
-  constexpr uint32_t KBLK = L::KBLK, KSLOT = L::KSLOT, VSLOT = L::VSLOT;
+  constexpr uint32_t KBLK = L::KBLK, KSLOT = L::KSLOT, VBLK = L::VBLK, VSLOT = L::VSLOT;
   extern __shared__ __align__(1024) uint8_t sm[];
   // The swizzled tiles need a 1024-byte aligned window; the runtime gives one
   // when the kernel has no static shared memory.  Check rather than assume.
@@ -201,10 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&bars[B_QFULL], 1);
     mbar_init(&bars[B_QFREE], kCompute + 1);
-    for (int s = 0; s < kKSlots; ++s) {
-      mbar_init(&bars[B_KFULL + s], 1);
-      mbar_init(&bars[B_KEMPTY + s], 1);
-    }
+    for (int s = 0; s < kKSlots; ++s) mbar_init(&bars[B_KFULL + s], 1);
     for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bars[B_VFULL + s], 1);
       mbar_init(&bars[B_VEMPTY + s], 2);  // released by both issuers
@@ -249,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the key tiles of step s (list positions 2s, 2s+1) into the next pair slot
       auto load_k = [&](const Tile& T, int s) -> bool {
         const int sl = gk % kKSlots;
-        if (gk >= kKSlots && !mbar_wait(&bars[B_KEMPTY + sl], ((gk / kKSlots) - 1) & 1, abort_flag, a.status))
-          return false;
+        if (gk >= kKSlots && !mbar_wait(&bars[B_SFULL + sl], ((gk / kKSlots) - 1) & 1, abort_flag, a.status))
+          return false;  // S of the step two back has read this slot
         const bool two = 2 * s + 1 < T.n_crit;
         const int ra = block_at(T, 2 * s, a.nkv, a.status) * kBlockKV;
         const int rb = two ? block_at(T, 2 * s + 1, a.nkv, a.status) * kBlockKV : 0;
@@ -279,18 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++gv;
         return sm + OFF_V + sl * VSLOT;
       };
-      // phi(K), V (and V8) tiles of the block at list position it
-      auto load_v = [&](const Tile& T, int it) -> bool {
-        const int krow = block_at(T, it, a.nkv, a.status) * kBlockKV;
+      // phi(K), V (and V8) tiles of the blocks at list positions p0 and p0 + 1 (if below p_end)
+      auto load_pair = [&](const Tile& T, int p0, int p_end) -> bool {
         uint64_t* fb = nullptr;
         uint8_t* vb = v_slot(fb);
         if (vb == nullptr) return false;
-        mbar_arrive_expect_tx(fb, VSLOT);
-        tma_load_3d(vb, &tmPhi, fb, 0, krow, T.bh);
-        tma_load_3d(vb + 8192, &tmPhi, fb, 64, krow, T.bh);
-        tma_load_3d(vb + 16384, &tmV, fb, 0, krow, T.bh);
-        tma_load_3d(vb + 16384 + 8192, &tmV, fb, 64, krow, T.bh);
-        if constexpr (kFP8) tma_load_3d(vb + 32768, &tmV8, fb, 0, krow, T.bh);
+        const int nb = p0 + 1 < p_end ? 2 : 1;
+        mbar_arrive_expect_tx(fb, nb * VBLK);
+        for (int b = 0; b < nb; ++b) {
+          const int krow = block_at(T, p0 + b, a.nkv, a.status) * kBlockKV;
+          uint8_t* bb = vb + b * VBLK;
+          tma_load_3d(bb, &tmPhi, fb, 0, krow, T.bh);
+          tma_load_3d(bb + 8192, &tmPhi, fb, 64, krow, T.bh);
+          tma_load_3d(bb + 16384, &tmV, fb, 0, krow, T.bh);
+          tma_load_3d(bb + 16384 + 8192, &tmV, fb, 64, krow, T.bh);
+          if constexpr (kFP8) tma_load_3d(bb + 32768, &tmV8, fb, 0, krow, T.bh);
+        }
         return true;
       };
       auto load_h = [&](const Tile& T) -> bool {
@@ -314,11 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (T.nsteps > 0) ok = load_k(T, 0);
         if (ok && T.nsteps > 1) ok = load_k(T, 1);
         for (int s = 0; ok && s < T.nsteps; ++s) {
-          ok = load_v(T, 2 * s);
-          if (ok && 2 * s + 1 < T.n_crit) ok = load_v(T, 2 * s + 1);
+          ok = load_pair(T, 2 * s, T.n_crit);
           if (ok && s + 2 < T.nsteps) ok = load_k(T, s + 2);
         }
-        for (int it = T.n_crit; ok && it < T.n_total; ++it) ok = load_v(T, it);
+        for (int it = T.n_crit; ok && it < T.n_total; it += 2) ok = load_pair(T, it, T.n_total);
         if (ok && T.has_lin) ok = load_h(T);
       }
       // every issued copy must land before the CTA may exit
@@ -378,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ss(d, dQ + o, kb + o, two ? id_qk : id_qk1, kk > 0 ? 1u : 0u);
           }
         }
-        mma_commit(&bars[B_SFULL + (g & 1)]);
-        mma_commit(&bars[B_KEMPTY + sl]);
+        mma_commit(&bars[B_SFULL + (g & 1)]);  // also frees key-pair slot g & 1 (== sl)
         if (last_s) mma_commit(&bars[B_QFREE]);
         ++gk;
       };
@@ -389,22 +389,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++gv;
         return sl;
       };
-      auto issue_h = [&](int sl, bool first) {
-        const uint64_t pb = dPhi + ((sl * VSLOT) >> 4), vb = dV + ((sl * VSLOT) >> 4);
+      auto issue_h = [&](int sl, int blk, bool first) {
+        const uint32_t off = (sl * VSLOT + blk * VBLK) >> 4;
+        const uint64_t pb = dPhi + off, vb = dV + off;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16_ss(tmem + T_HK, pb + kk * 128u, vb + kk * 128u, id_h, (first && kk == 0) ? 0u : 1u);
       };
-      // O (+)= P V for one key block: P columns from pcol, V from slot sl
-      auto issue_pv = [&](int sl, uint32_t pcol, bool first) {
+      // O (+)= P V for one key block: P columns from pcol, V of block blk of entry sl
+      auto issue_pv = [&](int sl, int blk, uint32_t pcol, bool first) {
+        const uint32_t off = (sl * VSLOT + blk * VBLK) >> 4;
         if constexpr (kFP8) {
           // P8 (TMEM, 4 keys per column) x V8 (MN-major, one 128-byte atom wide): K = 32 per MMA
-          const uint64_t vb = dV8 + ((sl * VSLOT) >> 4);
+          const uint64_t vb = dV8 + off;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
             mma_f8_ts(tmem + T_O, tmem + pcol + kk * 8u, vb + kk * 256u, id_pv8, (first && kk == 0) ? 0u : 1u);
         } else {
-          const uint64_t vb = dV + ((sl * VSLOT) >> 4);
+          const uint64_t vb = dV + off;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_f16_ts(tmem + T_O, tmem + pcol + kk * 8u, vb + kk * 128u, id_pv, (first && kk == 0) ? 0u : 1u);
@@ -441,31 +443,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; ok && i < ns; ++i) {
             const int g = gs + i, b = g & 1;
             const bool two = 2 * i + 1 < T.n_crit;
-            if (i + 1 < ns && !wait_k()) {
-              ok = false;
-              break;
+            if (i + 1 < ns) {  // right after the previous PV: a cheap place to wait
+              if (!wait_k()) {
+                ok = false;
+                break;
+              }
+              issue_s(T, i + 1, g + 1, i + 1 == ns - 1);
             }
-            const int sa = take_v();
-            const int sb = (sa >= 0 && two) ? take_v() : -1;
-            if (sa < 0 || (two && sb < 0)) {
-              ok = false;
-              break;
-            }
-            if (i + 1 < ns) issue_s(T, i + 1, g + 1, i + 1 == ns - 1);
             if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            const int ve = take_v();  // (this step's blocks: long landed)
+            if (ve < 0) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t pcol = T_S0 + b * 128;
-            issue_pv(sa, pcol, i == 0);
-            if (two) issue_pv(sb, pcol + 64u, false);  // block B's P over the first columns of its S half
+            issue_pv(ve, 0, pcol, i == 0);
+            if (two) issue_pv(ve, 1, pcol + 64u, false);  // block B's P over the first columns of its S half
             mma_commit(&bars[B_PEMPTY + b]);
-            mma_commit(&bars[B_VEMPTY + sa]);
-            if (two) mma_commit(&bars[B_VEMPTY + sb]);
+            mma_commit(&bars[B_VEMPTY + ve]);
           }
-          // the tile's other V-ring entries (negligible blocks, H tile) are warp 10's
-          for (int it = T.n_crit; ok && it < T.n_total + (T.has_lin ? 1 : 0); ++it) {
+          // the tile's other value entries (negligible blocks, H tile) are warp 10's
+          for (int it = 0; ok && it < T.nnegl_e + (T.has_lin ? 1 : 0); ++it) {
             const int sl = take_v();
             if (sl < 0) {
               ok = false;
@@ -479,13 +481,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // ---------------------------------------------- warp 10: H, epilogue products
           if (pend && !wait_epidone()) break;  // H_ex, phi(Q) H_i of the previous tile have been read
-          for (int it = 0; ok && it < T.n_total; ++it) {
+          for (int e = 0; ok && e < T.nsteps + T.nnegl_e; ++e) {
             const int sl = take_v();
             if (sl < 0) {
               ok = false;
               break;
             }
-            issue_h(sl, it == 0);  // (TMA data: no tcgen05 fence needed)
+            const int p0 = e < T.nsteps ? 2 * e : T.n_crit + 2 * (e - T.nsteps);
+            const int p_end = e < T.nsteps ? T.n_crit : T.n_total;
+            issue_h(sl, 0, e == 0);  // (TMA data: no tcgen05 fence needed)
+            if (p0 + 1 < p_end) issue_h(sl, 1, false);
             mma_commit(&bars[B_VEMPTY + sl]);
           }
           if (!ok) break;
@@ -761,10 +766,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) tc_fence_after();
       const float l_run = l_part + xchg(l_part);
       const uint32_t pcol = T_S0 + ((gs - 1) & 1) * 128;  // the tile's last S buffer
-      const int hidx = gv + T.n_total;                     // V-ring entry of the H tile
+      const int hidx = gv + T.nsteps + T.nnegl_e;          // value entry of the H tile
       const int hsl = hidx % kVSlots;
       uint8_t* hbuf = sm + OFF_V + hsl * VSLOT;
-      gv += T.n_total + (T.has_lin ? 1 : 0);
+      gv += T.nsteps + T.nnegl_e + (T.has_lin ? 1 : 0);
       float den = 0.0f;
       if (T.has_lin) {
         // H_i / sigma = H_tot / sigma (fp16 tile from TMA) - H_ex / sigma, row e = r,
