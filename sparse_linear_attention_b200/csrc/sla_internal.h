@@ -53,7 +53,9 @@ inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
   L.need_hat = (s.d != kDPad) || (s.in_dtype == SLA_F32);
-  int ns = ceil_div(2 * kNumSMs, static_cast<int>(BH > 0 ? BH : 1));
+  // prepass splits per head: one wave of two CTAs per SM (rounding up would leave a
+  // few CTAs for a second wave and double the prepass time)
+  int ns = (2 * kNumSMs) / static_cast<int>(BH > 0 ? BH : 1);
   L.nsplit = ns < 1 ? 1 : (ns > nkv ? nkv : ns);
   size_t off = 0;
   auto take = [&](size_t bytes) {
