@@ -74,12 +74,12 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
 // ---------------------------------------------------------------- projection
 // xt^T[bh][c][r] = sum_e fl(xbar[bh][r][e] * W[e][c]) (or xbar itself when W is
 // null), written channel-major so the score kernel reads it coalesced.
-// Block: 256 threads, 64 rows of one head x all d output channels; thread
-// (ty, tx) owns rows 4ty..4ty+3 and channels 8tx..8tx+7.  The sum over e runs
-// in ascending order for every output, as specified.
-constexpr int kProjRows = 64;
+// Block: 128 threads = output channels, kProjRows pooled rows of one head;
+// every output sums over e in ascending order, as specified.  W (d x d fp32,
+// shared by all heads) is read in coalesced rows through the L1 cache.
+constexpr int kProjRows = 8;
 
-__global__ void __launch_bounds__(256) project_kernel(const float* __restrict__ qbar,
+__global__ void __launch_bounds__(128) project_kernel(const float* __restrict__ qbar,
                                                       const float* __restrict__ kbar,
                                                       const float* __restrict__ Wq,
                                                       const float* __restrict__ Wk, float* __restrict__ qtT,
@@ -92,107 +92,50 @@ __global__ void __launch_bounds__(256) project_kernel(const float* __restrict__ 
   const int r0 = blockIdx.x * kProjRows;
   if (r0 >= nrows) return;
   const long long bh = blockIdx.y;
-  extern __shared__ __align__(16) float psm[];
-  float* xs = psm;                     // [d][64]: xs[e][r] = xbar[r0 + r][e]
-  float* ws = psm + kDPad * kProjRows; // [d][128]: W[e][c]
-  const int tid = threadIdx.x;
-  // rows: float4 along e, one row per thread in a group of 64 -> transposed store
-  for (int i = tid; i < kProjRows * (d / 4); i += 256) {
-    const int r = i % kProjRows, e4 = i / kProjRows;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r0 + r < nrows) v = *reinterpret_cast<const float4*>(xbar + (bh * nrows + r0 + r) * d + 4 * e4);
-    xs[(4 * e4 + 0) * kProjRows + r] = v.x;
-    xs[(4 * e4 + 1) * kProjRows + r] = v.y;
-    xs[(4 * e4 + 2) * kProjRows + r] = v.z;
-    xs[(4 * e4 + 3) * kProjRows + r] = v.w;
+  __shared__ __align__(16) float xs[kProjRows][kDPad];
+  const int c = threadIdx.x;
+  for (int i = c; i < kProjRows * d; i += 128) {
+    const int r = i / d, e = i % d;
+    xs[r][e] = (r0 + r < nrows) ? xbar[(bh * nrows + r0 + r) * d + e] : 0.0f;
   }
-  if (W != nullptr)
-    for (int i = tid; i < d * (d / 4); i += 256) cp_async16(ws + (i / (d / 4)) * kDPad + 4 * (i % (d / 4)), W + 4 * i);
-  cp_async_wait_all();
   __syncthreads();
-  const int ty = tid / 16, tx = tid % 16;
-  if (8 * tx >= d) return;
-  float acc[4][8];
+  if (c >= d) return;
+  float acc[kProjRows];
   if (W == nullptr) {
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = xs[(8 * tx + b) * kProjRows + 4 * ty + a];
+    for (int r = 0; r < kProjRows; ++r) acc[r] = xs[r][c];
   } else {
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int r = 0; r < kProjRows; ++r) acc[r] = 0.0f;
+    for (int e = 0; e < d; e += 4) {  // d % 4 == 0: 4 channels of the 8 rows per vector read
+      float4 x4[kProjRows];
 #pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
-    for (int e = 0; e < d; ++e) {
-      const float4 xv = *reinterpret_cast<const float4*>(xs + e * kProjRows + 4 * ty);
-      const float4 w0 = *reinterpret_cast<const float4*>(ws + e * kDPad + 8 * tx);
-      const float4 w1 = *reinterpret_cast<const float4*>(ws + e * kDPad + 8 * tx + 4);
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wb[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      for (int r = 0; r < kProjRows; ++r) x4[r] = *reinterpret_cast<const float4*>(&xs[r][e]);
+      float w[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int u = 0; u < 4; ++u) w[u] = __ldg(W + (e + u) * d + c);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xa[a], wb[b]));
+      for (int r = 0; r < kProjRows; ++r) {
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].x, w[0]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].y, w[1]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].z, w[2]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].w, w[3]));
+      }
     }
   }
+  float* dst = xtT + (bh * d + c) * nrows + r0;
 #pragma unroll
-  for (int b = 0; b < 8; ++b) {
-    float* dst = xtT + (bh * d + 8 * tx + b) * nrows + r0 + 4 * ty;
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-      if (r0 + 4 * ty + a < nrows) dst[a] = acc[a][b];
-  }
+  for (int r = 0; r < kProjRows; ++r)
+    if (r0 + r < nrows) dst[r] = acc[r];
 }
 
 // ---------------------------------------------------------------- scores + selection
-// Block: 256 threads, 16 query blocks of one head.  Scores for the 16 rows
-// are built in shared memory chunk by chunk (128 key blocks per chunk, each
-// thread 2 rows x 4 key blocks), then each warp selects for 2 rows.
-constexpr int kScoreRows = 16;
-constexpr int kScoreKeys = 128;
-
-struct Cand {
-  float s;
-  int j;
-};
-
-// a ranks before b in (score desc, index asc)
-__device__ __forceinline__ bool ranks_before(float sa, int ja, float sb, int jb) {
-  return sa > sb || (sa == sb && ja < jb);
-}
-
-__device__ __forceinline__ Cand warp_best(Cand c, bool top) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float s2 = __shfl_xor_sync(0xffffffffu, c.s, o);
-    const int j2 = __shfl_xor_sync(0xffffffffu, c.j, o);
-    const bool take = top ? ranks_before(s2, j2, c.s, c.j) : ranks_before(c.s, c.j, s2, j2);
-    if (take) {
-      c.s = s2;
-      c.j = j2;
-    }
-  }
-  return c;
-}
-
-// Best unmarked element of this lane (j = lane + 32 t); `top` picks the
-// first in rank order, otherwise the last.
-__device__ __forceinline__ Cand lane_best(const float* row, int nkv, int lane, uint64_t excl, bool top) {
-  Cand c;
-  c.s = top ? -CUDART_INF_F : CUDART_INF_F;
-  c.j = top ? INT32_MAX : -1;
-  for (int t = 0; lane + 32 * t < nkv; ++t) {
-    if ((excl >> t) & 1ull) continue;
-    const int j = lane + 32 * t;
-    const float s = row[j];
-    const bool take = top ? ranks_before(s, j, c.s, c.j) : ranks_before(c.s, c.j, s, j);
-    if (take) {
-      c.s = s;
-      c.j = j;
-    }
-  }
-  return c;
-}
+// Block: 256 threads, kScoreRows query blocks of one head.  Each thread forms
+// the scores of all rows for key blocks tid, tid + 256, ...: the projected
+// query rows sit in shared memory (broadcast reads), the projected key blocks
+// stream from L2, coalesced across the threads (channel-major layout).  Then
+// warp w selects for row w.
+constexpr int kScoreRows = 8;
 
 __global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ qtT,
                                                            const float* __restrict__ ktT, int nq, int nkv,
@@ -201,84 +144,105 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
                                                            int8_t* __restrict__ labels,
                                                            float* __restrict__ scores_dbg) {
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                            // [d][16]
-  float* ks = qs + kDPad * kScoreRows;       // [d][128]
-  float* sc = ks + kDPad * kScoreKeys;       // [16][nkv]
+  float* qs = sm;                      // [kScoreRows][128]
+  float* sc = qs + kScoreRows * kDPad; // [kScoreRows][nkv]
   const long long bh = blockIdx.y;
   const int r0 = blockIdx.x * kScoreRows;
   const int tid = threadIdx.x;
-  for (int i = tid; i < d * kScoreRows; i += 256) {
-    const int c = i / kScoreRows, r = i % kScoreRows;
-    qs[i] = (r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
+  for (int i = tid; i < kScoreRows * d; i += 256) {
+    const int r = i % kScoreRows, c = i / kScoreRows;
+    qs[r * kDPad + c] = (r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
   }
-  const bool vec_ok = (nkv % 4) == 0;  // rows of ktT 16-byte aligned
-  const int ty = tid / 32;  // rows 2*ty, 2*ty+1
-  const int tx = tid % 32;  // key blocks 4*tx .. 4*tx+3 of the chunk
-  for (int j0 = 0; j0 < nkv; j0 += kScoreKeys) {
-    __syncthreads();  // previous chunk's ks reads done (and qs ready on the first pass)
-    if (vec_ok && j0 + kScoreKeys <= nkv) {
-      for (int i = tid; i < d * (kScoreKeys / 4); i += 256) {
-        const int c = i / (kScoreKeys / 4), j4 = i % (kScoreKeys / 4);
-        cp_async16(ks + c * kScoreKeys + 4 * j4, ktT + (bh * d + c) * nkv + j0 + 4 * j4);
-      }
-      cp_async_wait_all();
-    } else {
-#pragma unroll 8
-      for (int i = tid; i < d * kScoreKeys; i += 256) {
-        const int c = i / kScoreKeys, j = i % kScoreKeys;
-        ks[i] = (j0 + j < nkv) ? ktT[(bh * d + c) * nkv + j0 + j] : 0.0f;
+  __syncthreads();
+  // key blocks tid, tid + 256, ... (coalesced loads); one vector read of a
+  // query row brings four channels
+  const float* kcol = ktT + bh * d * static_cast<long long>(nkv);
+#pragma unroll 1
+  for (int j = tid; j < nkv; j += 256) {
+    float acc[kScoreRows];
+#pragma unroll
+    for (int r = 0; r < kScoreRows; ++r) acc[r] = 0.0f;
+    for (int c = 0; c < d; c += 4) {  // d % 4 == 0
+      float kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kv[u] = __ldg(kcol + static_cast<long long>(c + u) * nkv + j);
+#pragma unroll
+      for (int r = 0; r < kScoreRows; ++r) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qs + r * kDPad + c);
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.x, kv[0]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.y, kv[1]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.z, kv[2]));
+        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.w, kv[3]));
       }
     }
-    __syncthreads();
-    float acc[2][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-    for (int c = 0; c < d; ++c) {
-      const float2 qv = *reinterpret_cast<const float2*>(qs + c * kScoreRows + 2 * ty);
-      const float4 kv = *reinterpret_cast<const float4*>(ks + c * kScoreKeys + 4 * tx);
-      const float qa[2] = {qv.x, qv.y};
-      const float kb[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qa[a], kb[b]));
-    }
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int j = j0 + 4 * tx + b;
-        if (j < nkv) sc[(2 * ty + a) * nkv + j] = acc[a][b];
-      }
+    for (int r = 0; r < kScoreRows; ++r) sc[r * nkv + j] = acc[r];
   }
   __syncthreads();
 
   const int lane = tid % 32, warp = tid / 32;
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = warp * 2 + rr;
+  {
+    const int r = warp;
     const int row = r0 + r;
-    if (row >= nq) break;
+    if (row >= nq) return;
     const float* srow = sc + r * nkv;
     const long long grow = bh * nq + row;
-    uint64_t top = 0, bot = 0;
-    Cand mine = lane_best(srow, nkv, lane, top, true);
-    for (int it = 0; it < k_keep; ++it) {
-      const Cand w = warp_best(mine, true);
-      if ((w.j & 31) == lane) {
-        top |= 1ull << (w.j >> 5);
-        mine = lane_best(srow, nkv, lane, top, true);
+    // Rank keys: the scores mapped to unsigned integers in the same order
+    // (-0 taken as +0, as the comparison does); the k-th largest is found bit
+    // by bit with warp-wide counts, ties at it go by block index.
+    uint32_t* orow = reinterpret_cast<uint32_t*>(sc + r * nkv);
+    for (int j = lane; j < nkv; j += 32) {
+      const float sv = srow[j];
+      if (scores_dbg) scores_dbg[grow * nkv + j] = sv;
+      uint32_t u = __float_as_uint(sv);
+      if (u == 0x80000000u) u = 0u;
+      orow[j] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    }
+    __syncwarp();
+    auto count_ge = [&](uint32_t cand, uint32_t flip) -> int {
+      int c = 0;
+      for (int j = lane; j < nkv; j += 32) c += ((orow[j] ^ flip) >= cand) ? 1 : 0;
+      return __reduce_add_sync(0xffffffffu, c);
+    };
+    // largest T with at least k keys >= T (flip = ~0: keys of the worst blocks)
+    auto kth_key = [&](int k, uint32_t flip) -> uint32_t {
+      uint32_t T = 0;
+      for (int b = 31; b >= 0; --b) {
+        const uint32_t cand = T | (1u << b);
+        if (count_ge(cand, flip) >= k) T = cand;
+      }
+      return T;
+    };
+    const int nt = (nkv + 31) / 32;
+    uint64_t top = 0, bot = 0;  // bit t <-> block lane + 32 t
+    if (k_keep > 0) {
+      // the first k_keep in (score desc, index asc)
+      const uint32_t T = kth_key(k_keep, 0u);
+      const int need = k_keep - (T == 0xFFFFFFFFu ? 0 : count_ge(T + 1u, 0u));  // from the ties at T
+      int seen = 0;
+      for (int t = 0; t < nt; ++t) {  // ascending index: the lower indices win the ties
+        const int j = lane + 32 * t;
+        const uint32_t o = j < nkv ? orow[j] : 0u;
+        const bool eq = j < nkv && o == T;
+        const uint32_t m = __ballot_sync(0xffffffffu, eq);
+        const int rank = seen + __popc(m & ((1u << lane) - 1u));
+        if (j < nkv && (o > T || (eq && rank < need))) top |= 1ull << t;
+        seen += __popc(m);
       }
     }
     if (mode == SLA_MODE_SLA_3WAY && k_neg > 0) {
-      mine = lane_best(srow, nkv, lane, top, false);
-      for (int it = 0; it < k_neg; ++it) {
-        const Cand w = warp_best(mine, false);
-        if ((w.j & 31) == lane) {
-          bot |= 1ull << (w.j >> 5);
-          mine = lane_best(srow, nkv, lane, top | bot, false);
-        }
+      // the last k_neg in (score desc, index asc): lowest scores, higher index first
+      const uint32_t T = kth_key(k_neg, 0xFFFFFFFFu);
+      const int need = k_neg - (T == 0xFFFFFFFFu ? 0 : count_ge(T + 1u, 0xFFFFFFFFu));
+      int seen = 0;
+      for (int t = nt - 1; t >= 0; --t) {  // descending index: the higher indices go first
+        const int j = lane + 32 * t;
+        const uint32_t o = j < nkv ? ~orow[j] : 0u;
+        const bool eq = j < nkv && o == T;
+        const uint32_t m = __ballot_sync(0xffffffffu, eq);
+        const int rank = seen + __popc(m & ~((2u << lane) - 1u));  // equal keys on higher lanes
+        if (j < nkv && (o > T || (eq && rank < need))) bot |= 1ull << t;
+        seen += __popc(m);
       }
     }
     // kept indices in ascending order
@@ -289,10 +253,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
       const uint32_t m = __ballot_sync(0xffffffffu, s);
       if (s) kept_idx[grow * k_keep + base + __popc(m & ((1u << lane) - 1u))] = j;
       base += __popc(m);
-      if (j < nkv) {
-        if (labels) labels[grow * nkv + j] = s ? 1 : (((bot >> t) & 1ull) ? -1 : 0);
-        if (scores_dbg) scores_dbg[grow * nkv + j] = srow[j];
-      }
+      if (j < nkv && labels) labels[grow * nkv + j] = s ? 1 : (((bot >> t) & 1ull) ? -1 : 0);
     }
   }
 }
@@ -323,15 +284,11 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                                                 qbar, kbar, BH, s.N, s.d, s.bq, s.bkv);
   }
   {
-    const size_t psmem = static_cast<size_t>(kDPad) * (kProjRows + kDPad) * 4;
-    cudaError_t e = cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(psmem));
-    if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(nkv > nq ? nkv : nq, kProjRows), BH, 2);
-    project_kernel<<<grid, 256, psmem, st>>>(qbar, kbar, Wq, Wk, qtT, ktT, nq, nkv, s.d);
+    project_kernel<<<grid, 128, 0, st>>>(qbar, kbar, Wq, Wk, qtT, ktT, nq, nkv, s.d);
   }
   {
-    const size_t smem = (kDPad * kScoreRows + kDPad * kScoreKeys + static_cast<size_t>(kScoreRows) * nkv) * 4;
+    const size_t smem = (static_cast<size_t>(kScoreRows) * kDPad + static_cast<size_t>(kScoreRows) * nkv) * 4;
     cudaError_t e = cudaFuncSetAttribute(score_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
