@@ -332,6 +332,273 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_kernel(
   }
 }
 
+// lin_prepass_tma_kernel: the same results for bf16 inputs with d = 128 (the
+// video shapes), built for HBM throughput.  K and V tiles (64 tokens) arrive
+// by TMA in a kStagesP-deep ring; the threads turn them into phi(K) and V as
+// fp16 in place (the 128-byte swizzled layout of the load is the layout the
+// tensor core reads); a TMA tile store writes them to the workspace and the
+// same tiles feed H_part += phi(K)^T V.  A stage is refilled once its product
+// is done and its store has read it.  Thread 0 issues every TMA operation and
+// product; all waits are bounded.
+constexpr int kStagesP = 3;
+constexpr uint32_t kStageBytes = 2 * kTileBytes;  // K (-> phi(K)) | V (-> fp16)
+constexpr uint32_t kTOffBar = kStagesP * kStageBytes;            // full[kStagesP], mma[kStagesP], done
+constexpr uint32_t kTOffMisc = kTOffBar + 128;                   // tmem base, abort flag
+constexpr uint32_t kTOffZred = kTOffMisc + 64;                   // [8 warps][128] column partials
+constexpr uint32_t kTPreSmem = kTOffZred + 8 * 128 * 4;
+static_assert(2 * kStagesP + 1 <= 16, "barrier area");
+
+__global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_tma_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const __grid_constant__ CUtensorMap tmPhiOut, const __grid_constant__ CUtensorMap tmVOut,
+    float* __restrict__ hpart, float* __restrict__ zpart, float* __restrict__ zblk, float* __restrict__ kstat,
+    float* __restrict__ vstat, int N, int nkv, int nsplit, int phi_kind, int* status) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  if ((smem_u32(sm) & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned window
+    if (threadIdx.x == 0) report_error(status, SLA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kTOffBar);
+  uint64_t* mmad = full + kStagesP;
+  uint64_t* done_bar = mmad + kStagesP;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kTOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kTOffMisc + 4);
+  float* zred = reinterpret_cast<float*>(sm + kTOffZred);
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int split = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int jb0 = static_cast<int>((static_cast<long long>(split) * nkv) / nsplit);
+  const int jb1 = static_cast<int>((static_cast<long long>(split + 1) * nkv) / nsplit);
+  const int nt = jb1 - jb0;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStagesP; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&mmad[i], 1);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kPreTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int issued = 0;  // thread 0: tiles whose loads were issued
+  auto load_tile = [&](int it) {  // thread 0: tile it of this split into stage it % kStagesP
+    issued = it + 1;
+    uint8_t* st = sm + (it % kStagesP) * kStageBytes;
+    uint64_t* fb = &full[it % kStagesP];
+    const int row = (jb0 + it) * 64;
+    mbar_arrive_expect_tx(fb, kStageBytes);
+    tma_load_3d(st, &tmK, fb, 0, row, bh);
+    tma_load_3d(st + 8192, &tmK, fb, 64, row, bh);
+    tma_load_3d(st + kTileBytes, &tmV, fb, 0, row, bh);
+    tma_load_3d(st + kTileBytes + 8192, &tmV, fb, 64, row, bh);
+  };
+  if (tid == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    for (int it = 0; it < kStagesP - 1 && it < nt; ++it) load_tile(it);
+  }
+
+  const uint32_t idesc_h = idesc_f16(0, 1, 1, 128, 128);  // phi(K)^T (MN-major) x V (MN-major)
+  bool ok = true;
+  float zacc = 0.0f;  // threads < 128: this split's Z for channel tid, blocks in ascending order
+  float ksum[8], vmax[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ksum[e] = 0.0f;
+    vmax[e] = 0.0f;
+  }
+  const int u = tid % 16;  // this thread's 16-byte unit (channels 8u .. 8u+7) of rows tid/16 + 16 i
+  for (int it = 0; it < nt; ++it) {
+    const int jb = jb0 + it;
+    const int stg = it % kStagesP;
+    uint8_t* sk = sm + stg * kStageBytes;
+    uint8_t* sv = sk + kTileBytes;
+    ok = ok && mbar_wait(&full[stg], (it / kStagesP) & 1, abort_flag, status);
+    ok = __syncthreads_and(ok) != 0;  // CTA-uniform verdict
+    if (!ok) break;
+    float csum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // this thread's rows, rounded phi(K)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = tid / 16 + 16 * i;
+      const bool valid = jb * 64 + m < N;
+      const uint32_t off = (u >> 3) * 8192u + sw128_off(m, u & 7);
+      uint4* kp = reinterpret_cast<uint4*>(sk + off);
+      uint4* vp = reinterpret_cast<uint4*>(sv + off);
+      const uint4 kw = *kp, vw = *vp;  // rows past N were zero-filled by the load
+      float kf[8], vf[8];
+      {
+        const uint32_t a[4] = {kw.x, kw.y, kw.z, kw.w}, b[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 p = unpack_bf162(a[e]), q = unpack_bf162(b[e]);
+          kf[2 * e] = p.x;
+          kf[2 * e + 1] = p.y;
+          vf[2 * e] = q.x;
+          vf[2 * e + 1] = q.y;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ksum[e] += kf[e];
+        vmax[e] = fmaxf(vmax[e], fabsf(vf[e]));
+      }
+      float ph[8];
+      if (phi_kind == SLA_PHI_SOFTMAX) {
+        float mx = kf[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e) mx = fmaxf(mx, kf[e]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ph[e] = ex2_approx((kf[e] - mx) * 1.4426950408889634f);
+          sum += ph[e];
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ph[e] *= inv;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ph[e] = elu1(kf[e]);
+      }
+      uint4 pu = make_uint4(pack_half2(ph[0], ph[1]), pack_half2(ph[2], ph[3]), pack_half2(ph[4], ph[5]),
+                            pack_half2(ph[6], ph[7]));
+      const uint4 vu = make_uint4(pack_half2(vf[0], vf[1]), pack_half2(vf[2], vf[3]), pack_half2(vf[4], vf[5]),
+                                  pack_half2(vf[6], vf[7]));
+      if (!valid) pu = make_uint4(0, 0, 0, 0);  // keys past N leave the sums (V is zero there)
+      const uint32_t pw[4] = {pu.x, pu.y, pu.z, pu.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_half2(pw[e]);
+        csum[2 * e] += f.x;
+        csum[2 * e + 1] += f.y;
+      }
+      *kp = pu;
+      *vp = vu;
+    }
+    // column sums of this key block: lanes u and u+16 hold the same channels
+#pragma unroll
+    for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], 16);
+    if ((tid & 31) < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) zred[warp * 128 + 8 * u + e] = csum[e];
+    }
+    fence_proxy_async_smem();  // the fp16 tiles are visible to the TMA store and the tensor core
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 128) {
+      float z = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kPreThreads / 32; ++w) z += zred[w * 128 + tid];
+      zblk[(static_cast<long long>(bh) * nkv + jb) * kDPad + tid] = z;
+      zacc += z;
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      // phi(K), V (fp16) to the workspace (rows past N are not written)
+      tma_store_3d(&tmPhiOut, sk, 0, jb * 64, bh);
+      tma_store_3d(&tmPhiOut, sk + 8192, 64, jb * 64, bh);
+      tma_store_3d(&tmVOut, sv, 0, jb * 64, bh);
+      tma_store_3d(&tmVOut, sv + 8192, 64, jb * 64, bh);
+      bulk_commit_group();
+      const uint32_t aphi = smem_u32(sk), av = smem_u32(sv);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = sdesc_sw128(aphi + kk * 2048, 8192, 1024);
+        const uint64_t b = sdesc_sw128(av + kk * 2048, 8192, 1024);
+        mma_f16_ss(tmem + 0, a, b, idesc_h, (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&mmad[stg]);
+      // refill the stage of the previous tile: its product and its store must be done with it
+      const int nx = it + kStagesP - 1;
+      if (nx < nt) {
+        if (it >= 1) {
+          if (!mbar_wait(&mmad[(it - 1) % kStagesP], ((it - 1) / kStagesP) & 1, abort_flag, status)) ok = false;
+          bulk_wait_read_one();  // all but the latest store group have read their tiles
+        }
+        if (ok) load_tile(nx);
+      }
+    }
+    __syncthreads();  // zred is rewritten by the next tile
+  }
+  // all products done -> read the partial sums out of TMEM (warps 0..3: one lane each)
+  if (tid == 0) {
+    mma_commit(done_bar);
+    bulk_wait_all();  // the stores are complete before the CTA exits
+    // loads still in flight after an early exit must land before shared memory is reused
+    for (int t = issued > kStagesP ? issued - kStagesP : 0; t < issued; ++t)
+      mbar_wait_drain(&full[t % kStagesP], (t / kStagesP) & 1);
+  }
+  __syncwarp();
+  bool have = ok && (nt > 0);
+  {
+    int w_ok = 0;
+    if ((tid & 31) == 0) w_ok = mbar_wait(done_bar, 0, abort_flag, status) ? 1 : 0;
+    w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+    have = have && w_ok;
+  }
+  tc_fence_after();
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ksum[e] += __shfl_xor_sync(0xffffffffu, ksum[e], 16);
+    vmax[e] = fmaxf(vmax[e], __shfl_xor_sync(0xffffffffu, vmax[e], 16));
+  }
+  __syncthreads();
+  float* kred = zred;
+  float* vred = reinterpret_cast<float*>(sm);  // stage 0 is idle now: 4 KB for the V partials
+  if ((tid & 31) < 16) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      kred[warp * 128 + 8 * u + e] = ksum[e];
+      vred[warp * 128 + 8 * u + e] = vmax[e];
+    }
+  }
+  __syncthreads();
+  if (tid < 128) {
+    float ks = 0.0f, vm = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kPreThreads / 32; ++w) {
+      ks += kred[w * 128 + tid];
+      vm = fmaxf(vm, vred[w * 128 + tid]);
+    }
+    kstat[(static_cast<long long>(bh) * nsplit + split) * kDPad + tid] = ks;
+    vstat[(static_cast<long long>(bh) * nsplit + split) * kDPad + tid] = vm;
+  }
+  if (have && warp < 4) {
+    zpart[(static_cast<long long>(bh) * nsplit + split) * kDPad + tid] = zacc;
+    float* hp = hpart + ((static_cast<long long>(bh) * nsplit + split) * kDPad + tid) * kDPad;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      float x[32];
+      tmem_ld32(tmem + ((warp * 32) << 16) + cc * 32, x);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(hp + cc * 32 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kPreTmemCols);
+  }
+}
+
 // Z_tot[bh][e] = sum over splits (ascending) of each split's sum of per-block
 // column sums, and the per-head scale sigma = 2^ceil(log2(max_e Z_tot)) (one
 // block of 128 threads per head).
@@ -532,7 +799,20 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
   int* status = reinterpret_cast<int*>(ws + L.status);
   dim3 grid(L.nsplit, BH);
   cudaError_t e;
-  if (s.in_dtype == SLA_BF16) {
+  if (s.in_dtype == SLA_BF16 && s.d == kDPad) {
+    CUtensorMap mk, mv, mpo, mvo;
+    if ((e = encode_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.N, BH, 64)) != cudaSuccess) return e;
+    if ((e = encode_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.N, BH, 64)) != cudaSuccess) return e;
+    if ((e = encode_map(&mpo, phik, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s.N, BH, 64)) != cudaSuccess) return e;
+    if ((e = encode_map(&mvo, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s.N, BH, 64)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(lin_prepass_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTPreSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(lin_prepass_tma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    lin_prepass_tma_kernel<<<grid, kPreThreads, kTPreSmem, st>>>(
+        mk, mv, mpo, mvo, hpart, zpart, reinterpret_cast<float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.kstat),
+        reinterpret_cast<float*>(ws + L.vstat), s.N, nkv, L.nsplit, phi, status);
+  } else if (s.in_dtype == SLA_BF16) {
     e = cudaFuncSetAttribute(lin_prepass_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kPreSmem);
     if (e == cudaSuccess)
