@@ -133,10 +133,11 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k,
  * bit-exact results) with the same arguments minus ws / ws_bytes; its scratch
  * is a 16 MiB array compiled into the library, held by every GPU that loads
  * libsla until the process exits.
- *   - Shapes whose scratch, 2*B*H*(n_q + n_kv)*d floats (each of the four
- *     pieces rounded up to 256 bytes), exceeds 16 MiB are rejected with
- *     SLA_ERR_WORKSPACE before any launch (sla_last_error_detail says how
- *     much was needed).  The 1.3B-shape workload needs 9.4 MB.
+ *   - Shapes whose scratch, B*H*(n_q + n_kv)*d floats (the projected block
+ *     means of Q and K, each piece rounded up to 256 bytes), exceeds 16 MiB
+ *     are rejected with SLA_ERR_WORKSPACE before any launch
+ *     (sla_last_error_detail says how much was needed).  The 1.3B-shape
+ *     workload needs 4.7 MB.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.

@@ -9,7 +9,8 @@
 // Every floating-point step is a single IEEE round-to-nearest operation in a
 // fixed order (__fadd_rn / __fmul_rn / __fdiv_rn never contract into FMA), so
 // the selected blocks are reproducible bit for bit on any implementation that
-// follows the same order:
+// follows the same order (pooling and projection run in one kernel, the means
+// staying in shared memory):
 //   pooled mean : tokens ascending from +0.0, then divide by the count
 //   projection  : y[c] = sum_e fl(x[e] * W[e][c]), e ascending, from +0.0
 //   score       : s[i][j] = sum_c fl(qt[i][c] * kt[j][c]), c ascending, from +0.0
@@ -24,109 +25,93 @@
 
 namespace sla {
 
-// ---------------------------------------------------------------- pooling
-// One thread per (head, block, 16-byte channel unit); tokens summed in
-// ascending order.  The grid's y index selects Q (0) or K (1).
+// ---------------------------------------------------------------- pooling + projection
+// One block per kPPRows blocks (rows) of one head and one of Q (grid z = 0) or
+// K (z = 1): the block means go to shared memory (tokens ascending from +0.0,
+// then one division, as in pool_kernel) and are projected at once (e
+// ascending, no FMA, as in project_kernel), so the projection's arithmetic
+// runs under the pooling's HBM traffic and the means never leave the chip.
+constexpr int kPPRows = 16;
+
 template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                   float* __restrict__ qbar, float* __restrict__ kbar,
-                                                   int BH, int N, int d, int bq, int bkv) {
+__global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                           const float* __restrict__ Wq,
+                                                           const float* __restrict__ Wk,
+                                                           float* __restrict__ qtT, float* __restrict__ ktT,
+                                                           int N, int d, int bq, int bkv) {
   constexpr int VPU = 16 / sizeof(T);  // channels per 16-byte unit
-  const bool isK = blockIdx.y == 1;
-  const T* x = isK ? k : q;
-  float* xbar = isK ? kbar : qbar;
-  const int b = isK ? bkv : bq;
-  const int nb = (N + b - 1) / b;
-  const int upr = d / VPU;
-  const long long total = static_cast<long long>(BH) * nb * upr;
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const int u = static_cast<int>(idx % upr);
-  const int blk = static_cast<int>((idx / upr) % nb);
-  const long long bh = idx / (static_cast<long long>(upr) * nb);
-  const int start = blk * b;
-  const int cnt = min(b, N - start);
-  const uint4* src = reinterpret_cast<const uint4*>(x + (bh * N + start) * d) + u;
-  const int stride = d / VPU;  // uint4 per token row
-  float acc[VPU];
-#pragma unroll
-  for (int c = 0; c < VPU; ++c) acc[c] = 0.0f;
-  for (int t0 = 0; t0 < cnt; t0 += 8) {
-    uint4 buf[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (t0 + i < cnt) buf[i] = __ldg(src + static_cast<long long>(t0 + i) * stride);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (t0 + i < cnt) {
-        const T* e = reinterpret_cast<const T*>(&buf[i]);
-#pragma unroll
-        for (int c = 0; c < VPU; ++c) acc[c] = __fadd_rn(acc[c], static_cast<float>(e[c]));
-      }
-    }
-  }
-  const float fc = static_cast<float>(cnt);
-  float* dst = xbar + (bh * nb + blk) * d + u * VPU;
-#pragma unroll
-  for (int c = 0; c < VPU; ++c) dst[c] = __fdiv_rn(acc[c], fc);
-}
-
-// ---------------------------------------------------------------- projection
-// xt^T[bh][c][r] = sum_e fl(xbar[bh][r][e] * W[e][c]) (or xbar itself when W is
-// null), written channel-major so the score kernel reads it coalesced.
-// Block: 128 threads = output channels, kProjRows pooled rows of one head;
-// every output sums over e in ascending order, as specified.  W (d x d fp32,
-// shared by all heads) is read in coalesced rows through the L1 cache.
-constexpr int kProjRows = 8;
-
-__global__ void __launch_bounds__(128) project_kernel(const float* __restrict__ qbar,
-                                                      const float* __restrict__ kbar,
-                                                      const float* __restrict__ Wq,
-                                                      const float* __restrict__ Wk, float* __restrict__ qtT,
-                                                      float* __restrict__ ktT, int nq, int nkv, int d) {
   const bool isK = blockIdx.z == 1;
-  const float* xbar = isK ? kbar : qbar;
+  const T* x = isK ? k : q;
   const float* W = isK ? Wk : Wq;
   float* xtT = isK ? ktT : qtT;
-  const int nrows = isK ? nkv : nq;
-  const int r0 = blockIdx.x * kProjRows;
+  const int b = isK ? bkv : bq;
+  const int nrows = (N + b - 1) / b;
+  const int r0 = blockIdx.x * kPPRows;
   if (r0 >= nrows) return;
   const long long bh = blockIdx.y;
-  __shared__ __align__(16) float xs[kProjRows][kDPad];
-  const int c = threadIdx.x;
-  for (int i = c; i < kProjRows * d; i += 128) {
-    const int r = i / d, e = i % d;
-    xs[r][e] = (r0 + r < nrows) ? xbar[(bh * nrows + r0 + r) * d + e] : 0.0f;
+  __shared__ __align__(16) float xs[kPPRows][kDPad];
+  const int tid = threadIdx.x;
+  const int upr = d / VPU;
+  for (int i = tid; i < kPPRows * upr; i += 256) {
+    const int r = i / upr, u = i % upr;
+    const int blk = r0 + r;
+    float acc[VPU];
+#pragma unroll
+    for (int c = 0; c < VPU; ++c) acc[c] = 0.0f;
+    if (blk < nrows) {
+      const int start = blk * b;
+      const int cnt = min(b, N - start);
+      const uint4* src = reinterpret_cast<const uint4*>(x + (bh * N + start) * d) + u;
+      for (int t0 = 0; t0 < cnt; t0 += 8) {
+        uint4 buf[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (t0 + j < cnt) buf[j] = __ldg(src + static_cast<long long>(t0 + j) * upr);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (t0 + j < cnt) {
+            const T* e = reinterpret_cast<const T*>(&buf[j]);
+#pragma unroll
+            for (int c = 0; c < VPU; ++c) acc[c] = __fadd_rn(acc[c], static_cast<float>(e[c]));
+          }
+        }
+      }
+      const float fc = static_cast<float>(cnt);
+#pragma unroll
+      for (int c = 0; c < VPU; ++c) acc[c] = __fdiv_rn(acc[c], fc);
+    }
+#pragma unroll
+    for (int c = 0; c < VPU; ++c) xs[r][u * VPU + c] = acc[c];
   }
   __syncthreads();
+  // projection: thread = output channel c of rows rh*8 .. rh*8+7
+  const int c = tid % kDPad, rh = tid / kDPad;
   if (c >= d) return;
-  float acc[kProjRows];
+  float out[8];
   if (W == nullptr) {
 #pragma unroll
-    for (int r = 0; r < kProjRows; ++r) acc[r] = xs[r][c];
+    for (int r = 0; r < 8; ++r) out[r] = xs[rh * 8 + r][c];
   } else {
 #pragma unroll
-    for (int r = 0; r < kProjRows; ++r) acc[r] = 0.0f;
-    for (int e = 0; e < d; e += 4) {  // d % 4 == 0: 4 channels of the 8 rows per vector read
-      float4 x4[kProjRows];
-#pragma unroll
-      for (int r = 0; r < kProjRows; ++r) x4[r] = *reinterpret_cast<const float4*>(&xs[r][e]);
+    for (int r = 0; r < 8; ++r) out[r] = 0.0f;
+    for (int e = 0; e < d; e += 4) {  // d % 4 == 0
       float w[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) w[u] = __ldg(W + (e + u) * d + c);
+      for (int uu = 0; uu < 4; ++uu) w[uu] = __ldg(W + (e + uu) * d + c);
 #pragma unroll
-      for (int r = 0; r < kProjRows; ++r) {
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].x, w[0]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].y, w[1]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].z, w[2]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(x4[r].w, w[3]));
+      for (int r = 0; r < 8; ++r) {
+        const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e]);
+        out[r] = __fadd_rn(out[r], __fmul_rn(x4.x, w[0]));
+        out[r] = __fadd_rn(out[r], __fmul_rn(x4.y, w[1]));
+        out[r] = __fadd_rn(out[r], __fmul_rn(x4.z, w[2]));
+        out[r] = __fadd_rn(out[r], __fmul_rn(x4.w, w[3]));
       }
     }
   }
-  float* dst = xtT + (bh * d + c) * nrows + r0;
+  float* dst = xtT + (bh * d + c) * nrows + r0 + rh * 8;
 #pragma unroll
-  for (int r = 0; r < kProjRows; ++r)
-    if (r0 + r < nrows) dst[r] = acc[r];
+  for (int r = 0; r < 8; ++r)
+    if (r0 + rh * 8 + r < nrows) dst[r] = out[r];
 }
 
 // ---------------------------------------------------------------- scores + selection
@@ -265,27 +250,17 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                          float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st) {
   const int BH = s.B * s.H;
   const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
-  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
   float* qtT = reinterpret_cast<float*>(ws + L.qt);
   float* ktT = reinterpret_cast<float*>(ws + L.kt);
   {
-    const int vpu = s.in_dtype == SLA_BF16 ? 8 : 4;
-    const long long nthr = static_cast<long long>(BH) * nq * (s.d / vpu);
-    const long long nthr_k = static_cast<long long>(BH) * nkv * (s.d / vpu);
-    const long long mx = nthr > nthr_k ? nthr : nthr_k;
-    dim3 grid(static_cast<unsigned>((mx + 255) / 256), 2);
+    dim3 grid(ceil_div(nkv > nq ? nkv : nq, kPPRows), BH, 2);
     if (s.in_dtype == SLA_BF16)
-      pool_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                        static_cast<const __nv_bfloat16*>(k), qbar, kbar, BH,
-                                                        s.N, s.d, s.bq, s.bkv);
+      pool_project_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                                                static_cast<const __nv_bfloat16*>(k), Wq, Wk,
+                                                                qtT, ktT, s.N, s.d, s.bq, s.bkv);
     else
-      pool_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                qbar, kbar, BH, s.N, s.d, s.bq, s.bkv);
-  }
-  {
-    dim3 grid(ceil_div(nkv > nq ? nkv : nq, kProjRows), BH, 2);
-    project_kernel<<<grid, 128, 0, st>>>(qbar, kbar, Wq, Wk, qtT, ktT, nq, nkv, s.d);
+      pool_project_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                        Wq, Wk, qtT, ktT, s.N, s.d, s.bq, s.bkv);
   }
   {
     const size_t smem = (static_cast<size_t>(kScoreRows) * kDPad + static_cast<size_t>(kScoreRows) * nkv) * 4;

@@ -28,8 +28,8 @@
 
 namespace sla {
 
-// 16 MiB: pooled + projected means of Q and K, 2 * B*H*(n_q + n_kv)*d floats
-// plus alignment (the 1.3B-shape workload needs 9.4 MB).
+// 16 MiB: projected block means of Q and K, B*H*(n_q + n_kv)*d floats plus
+// alignment (the 1.3B-shape workload needs 4.7 MB).
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 
 static __device__ __align__(256) char g_route_scratch[kNoAllocScratchBytes];
@@ -63,10 +63,6 @@ WsLayout route_scratch_layout(const sla_shape& s, size_t* bytes) {
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const size_t nq = static_cast<size_t>(ceil_div(s.N, s.bq)), nkv = static_cast<size_t>(ceil_div(s.N, s.bkv));
   size_t off = 0;
-  L.qbar = off;
-  off = align256(off + BH * nq * s.d * 4);
-  L.kbar = off;
-  off = align256(off + BH * nkv * s.d * 4);
   L.qt = off;
   off = align256(off + BH * nq * s.d * 4);
   L.kt = off;

@@ -17,8 +17,7 @@ constexpr int kNumSMs = 148;
 // Device workspace layout.  All offsets are 256-byte aligned.
 struct WsLayout {
   size_t status = 0;  // int32 status word (+ padding)
-  size_t qbar = 0, kbar = 0;  // fp32 [BH, n_q, d], [BH, n_kv, d]   pooled means
-  size_t qt = 0, kt = 0;      // fp32, same shapes                  projected
+  size_t qt = 0, kt = 0;      // fp32 [d][rows] per head: projected block means of Q, K
   size_t phik = 0;            // fp16 [BH, N, 128]  phi(K), zero past d
   size_t v16 = 0;             // fp16 [BH, N, 128]  V, zero past d
   size_t qhat = 0, khat = 0;  // bf16 [BH, N, 128]  Q, K (only when need_hat)
@@ -64,8 +63,6 @@ inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
     return o;
   };
   L.status = take(256);
-  L.qbar = take(BH * nq * s.d * 4);
-  L.kbar = take(BH * nkv * s.d * 4);
   L.qt = take(BH * nq * s.d * 4);
   L.kt = take(BH * nkv * s.d * 4);
   L.phik = take(BH * s.N * kDPad * 2);
