@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
                                                            const float* __restrict__ Wq,
                                                            const float* __restrict__ Wk,
                                                            float* __restrict__ qtT, float* __restrict__ ktT,
-                                                           int N, int d, int bq, int bkv) {
+                                                           int N, int d, int bq, int bkv, int kstride) {
   constexpr int VPU = 16 / sizeof(T);  // channels per 16-byte unit
   const bool isK = blockIdx.z == 1;
   const T* x = isK ? k : q;
@@ -108,60 +108,95 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
       }
     }
   }
-  float* dst = xtT + (bh * d + c) * nrows + r0 + rh * 8;
+  const int stride = isK ? kstride : nrows;  // key rows padded to a multiple of 4 floats
+  float* dst = xtT + (bh * d + c) * stride + r0 + rh * 8;
 #pragma unroll
   for (int r = 0; r < 8; ++r)
     if (r0 + rh * 8 + r < nrows) dst[r] = out[r];
 }
 
 // ---------------------------------------------------------------- scores + selection
-// Block: 256 threads, kScoreRows query blocks of one head.  Each thread forms
-// the scores of all rows for key blocks tid, tid + 256, ...: the projected
-// query rows sit in shared memory (broadcast reads), the projected key blocks
-// stream from L2, coalesced across the threads (channel-major layout).  Then
-// warp w selects for row w.
+// Block: 256 threads, kScoreRows = 8 query blocks of one head.  The scores are
+// a small fp32 GEMM: per 256-key pass, thread (ry, kx) forms rows 2ry, 2ry+1 x
+// keys 4kx .. 4kx+3 (two shared-memory reads per eight products), the
+// projected keys streaming through a double-buffered cp.async ring of
+// kScoreC-channel slices.  Every score sums c ascending, one rounding per
+// product and per sum.  Then warp w selects for row w.
 constexpr int kScoreRows = 8;
+constexpr int kScoreKeys = 256;
+constexpr int kScoreC = 16;
 
 __global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ qtT,
                                                            const float* __restrict__ ktT, int nq, int nkv,
-                                                           int d, int mode, int k_keep, int k_neg,
+                                                           int kstride, int d, int mode, int k_keep, int k_neg,
                                                            int32_t* __restrict__ kept_idx,
                                                            int8_t* __restrict__ labels,
                                                            float* __restrict__ scores_dbg) {
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                      // [kScoreRows][128]
-  float* sc = qs + kScoreRows * kDPad; // [kScoreRows][nkv]
+  float* qsT = sm;                              // [128 channels][8 rows]
+  float* kbuf = qsT + kDPad * kScoreRows;       // 2 x [kScoreC][kScoreKeys]
+  float* sc = kbuf + 2 * kScoreC * kScoreKeys;  // [kScoreRows][nkv]
   const long long bh = blockIdx.y;
   const int r0 = blockIdx.x * kScoreRows;
   const int tid = threadIdx.x;
-  for (int i = tid; i < kScoreRows * d; i += 256) {
+  for (int i = tid; i < kScoreRows * kDPad; i += 256) {
     const int r = i % kScoreRows, c = i / kScoreRows;
-    qs[r * kDPad + c] = (r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
+    qsT[i] = (c < d && r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
   }
-  __syncthreads();
-  // key blocks tid, tid + 256, ... (coalesced loads); one vector read of a
-  // query row brings four channels
-  const float* kcol = ktT + bh * d * static_cast<long long>(nkv);
-#pragma unroll 1
-  for (int j = tid; j < nkv; j += 256) {
-    float acc[kScoreRows];
-#pragma unroll
-    for (int r = 0; r < kScoreRows; ++r) acc[r] = 0.0f;
-    for (int c = 0; c < d; c += 4) {  // d % 4 == 0
-      float kv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) kv[u] = __ldg(kcol + static_cast<long long>(c + u) * nkv + j);
-#pragma unroll
-      for (int r = 0; r < kScoreRows; ++r) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qs + r * kDPad + c);
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.x, kv[0]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.y, kv[1]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.z, kv[2]));
-        acc[r] = __fadd_rn(acc[r], __fmul_rn(q4.w, kv[3]));
+  const float* kbase = ktT + bh * d * static_cast<long long>(kstride);
+  const int ry = tid / 64, kx = tid % 64;
+  const int nslices = (d + kScoreC - 1) / kScoreC;  // channels past d (d % 16 == 8) are zero-filled
+  for (int k0 = 0; k0 < nkv; k0 += kScoreKeys) {
+    const int kend = min(kScoreKeys, kstride - k0);  // keys of this pass inside the padded rows
+    // slice s of this pass into buffer s & 1: kScoreC rows of kend floats, 16 bytes per copy
+    auto load_slice = [&](int sl) {
+      float* dstb = kbuf + (sl & 1) * kScoreC * kScoreKeys;
+      for (int i = tid; i < kScoreC * (kScoreKeys / 4); i += 256) {
+        const int cc = i / (kScoreKeys / 4), k4 = 4 * (i % (kScoreKeys / 4));
+        if (sl * kScoreC + cc >= d)
+          *reinterpret_cast<float4*>(dstb + cc * kScoreKeys + k4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        else if (k4 < kend)
+          cp_async16(dstb + cc * kScoreKeys + k4, kbase + static_cast<long long>(sl * kScoreC + cc) * kstride + k0 + k4);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    __syncthreads();  // the previous pass is done with both buffers (and qsT is ready on the first)
+    load_slice(0);
+    float acc[2][4];
+#pragma unroll
+    for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+      for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = 0.0f;
+    for (int sl = 0; sl < nslices; ++sl) {
+      if (sl + 1 < nslices) {
+        load_slice(sl + 1);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      __syncthreads();  // slice sl visible to every thread
+      const float* kb = kbuf + (sl & 1) * kScoreC * kScoreKeys;
+#pragma unroll
+      for (int cc = 0; cc < kScoreC; ++cc) {
+        const int c = sl * kScoreC + cc;
+        const float2 q2 = *reinterpret_cast<const float2*>(qsT + c * kScoreRows + 2 * ry);
+        const float4 k4 = *reinterpret_cast<const float4*>(kb + cc * kScoreKeys + 4 * kx);
+        const float qa[2] = {q2.x, q2.y};
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+          for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = __fadd_rn(acc[a2][b4], __fmul_rn(qa[a2], kv[b4]));
+      }
+      __syncthreads();  // buffer sl & 1 may be refilled
     }
 #pragma unroll
-    for (int r = 0; r < kScoreRows; ++r) sc[r * nkv + j] = acc[r];
+    for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+      for (int b4 = 0; b4 < 4; ++b4) {
+        const int j = k0 + 4 * kx + b4;
+        if (j < nkv) sc[(2 * ry + a2) * nkv + j] = acc[a2][b4];
+      }
   }
   __syncthreads();
 
@@ -257,19 +292,20 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
     if (s.in_dtype == SLA_BF16)
       pool_project_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                                 static_cast<const __nv_bfloat16*>(k), Wq, Wk,
-                                                                qtT, ktT, s.N, s.d, s.bq, s.bkv);
+                                                                qtT, ktT, s.N, s.d, s.bq, s.bkv, kt_stride(nkv));
     else
       pool_project_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                        Wq, Wk, qtT, ktT, s.N, s.d, s.bq, s.bkv);
+                                                        Wq, Wk, qtT, ktT, s.N, s.d, s.bq, s.bkv, kt_stride(nkv));
   }
   {
-    const size_t smem = (static_cast<size_t>(kScoreRows) * kDPad + static_cast<size_t>(kScoreRows) * nkv) * 4;
+    const size_t smem =
+        (static_cast<size_t>(kDPad) * kScoreRows + 2 * kScoreC * kScoreKeys + static_cast<size_t>(kScoreRows) * nkv) * 4;
     cudaError_t e = cudaFuncSetAttribute(score_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(nq, kScoreRows), BH);
-    score_select_kernel<<<grid, 256, smem, st>>>(qtT, ktT, nq, nkv, s.d, mode, k_keep, k_neg, kept_idx, labels,
-                                                 scores_dbg);
+    score_select_kernel<<<grid, 256, smem, st>>>(qtT, ktT, nq, nkv, kt_stride(nkv), s.d, mode, k_keep, k_neg,
+                                                 kept_idx, labels, scores_dbg);
   }
   return cudaGetLastError();
 }

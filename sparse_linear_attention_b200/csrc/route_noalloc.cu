@@ -66,7 +66,7 @@ WsLayout route_scratch_layout(const sla_shape& s, size_t* bytes) {
   L.qt = off;
   off = align256(off + BH * nq * s.d * 4);
   L.kt = off;
-  off = align256(off + BH * nkv * s.d * 4);
+  off = align256(off + BH * static_cast<size_t>(kt_stride(static_cast<int>(nkv))) * s.d * 4);
   *bytes = off;
   return L;
 }

@@ -17,7 +17,7 @@ constexpr int kNumSMs = 148;
 // Device workspace layout.  All offsets are 256-byte aligned.
 struct WsLayout {
   size_t status = 0;  // int32 status word (+ padding)
-  size_t qt = 0, kt = 0;      // fp32 [d][rows] per head: projected block means of Q, K
+  size_t qt = 0, kt = 0;      // fp32 [d][rows] per head: projected block means of Q, K (K rows kt_stride long)
   size_t phik = 0;            // fp16 [BH, N, 128]  phi(K), zero past d
   size_t v16 = 0;             // fp16 [BH, N, 128]  V, zero past d
   size_t qhat = 0, khat = 0;  // bf16 [BH, N, 128]  Q, K (only when need_hat)
@@ -45,6 +45,10 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Row stride (floats) of the projected key means: n_kv rounded up to 4, so
+// every row starts on 16 bytes for the score kernel's async copies.
+inline int kt_stride(int nkv) { return (nkv + 3) & ~3; }
+
 inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
   const int mode = mode_flags & 0xFF;
   WsLayout L;
@@ -64,7 +68,7 @@ inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
   };
   L.status = take(256);
   L.qt = take(BH * nq * s.d * 4);
-  L.kt = take(BH * nkv * s.d * 4);
+  L.kt = take(BH * static_cast<size_t>(kt_stride(nkv)) * s.d * 4);
   L.phik = take(BH * s.N * kDPad * 2);
   L.v16 = take(BH * s.N * kDPad * 2);
   if (L.need_hat) {

@@ -62,6 +62,25 @@ def test_route_sla_three_way_bitexact():
     assert ((lab == 1).sum(-1) == kh).all() and ((lab == -1).sum(-1) == kl).all()
 
 
+@pytest.mark.parametrize("N,d,mode", [(1000, 40, 0), (777, 24, 1), (300, 128, 1)])
+def test_route_bitexact_odd_shapes(N, d, mode):
+    """Head dims that are not a multiple of 16 (the score kernel feeds 16-channel
+    slices), n_kv not a multiple of 4 (padded key rows), ragged tails, both modes."""
+    g = torch.Generator().manual_seed(N + d)
+    B, H = 1, 3
+    q = (torch.randn(B, H, N, d, generator=g) * 1.5).to(torch.bfloat16)
+    k = (torch.randn(B, H, N, d, generator=g) * 1.5).to(torch.bfloat16)
+    wq = torch.randn(d, d, generator=g) / d ** 0.5
+    wk = torch.randn(d, d, generator=g) / d ** 0.5
+    nkv = -(-N // 64)
+    kh, kl = min(3, nkv), (min(2, nkv - 3) if mode == 1 else 0)
+    kept, lab, sc = run_route(q, k, wq, wk, 128, 64, mode, kh, kl)
+    okept, olab, osc = orc.route(as32(q), as32(k), wq.numpy(), wk.numpy(), 128, 64, "sla" if mode else "sla2", kh, kl)
+    assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32)), "scores differ"
+    assert np.array_equal(kept, okept)
+    assert np.array_equal(lab, olab)
+
+
 def test_route_ties_break_to_lower_index():
     # identical key blocks -> equal scores; the lower block index must win
     B, H, N, d = 1, 1, 512, 64
