@@ -20,9 +20,9 @@ Precision.  Attention arithmetic is fp64 on the exact values of the input bytes.
 The router is fixed-order fp32 (below) because a hard top-k must be reproduced
 bit for bit; every fp32 step is one IEEE round-to-nearest-even operation:
   pooled mean : sum tokens in ascending order from +0.0, then divide by count;
-  projection  : y[c] = sum_e fl(xbar[e] * W[e,c]), e ascending, from +0.0
-                (product rounded, then sum rounded: no fused multiply-add);
-  score       : s[i,j] = sum_c fl(qt[i,c] * kt[j,c]), c ascending, from +0.0.
+  projection  : y[c] = fma(xbar[e], W[e,c], y[c]) for e ascending, from +0.0
+                (each multiply-add rounded once);
+  score       : s[i,j] = fma(qt[i,c], kt[j,c], s[i,j]) for c ascending, from +0.0.
 Neither 1/sqrt(d) nor the softmax of the SLA compressed map is applied before
 ranking: both are strictly increasing per row, so they cannot change a top-k.
 
@@ -73,9 +73,29 @@ def pool_blocks(x32: np.ndarray, b: int) -> np.ndarray:
     return acc / counts.astype(F32)[None, None, :, None]
 
 
+def fma32(a, b, c) -> np.ndarray:
+    """fl32(a * b + c) with a single rounding, elementwise, for fp32 a, b, c.
+    a * b is exact in fp64 (24 + 24 bits); the fp64 sum is then rounded to
+    odd (when it is inexact, of the two fp64 neighbours of the exact value the
+    one with an odd last bit), and rounding that to fp32 (53 >= 24 + 2 bits)
+    gives the correctly rounded result (Boldo and Melquiond, rounding to odd)."""
+    a = np.asarray(a, dtype=F32).astype(F64)
+    b = np.asarray(b, dtype=F32).astype(F64)
+    c = np.asarray(c, dtype=F32).astype(F64)
+    p = a * b
+    s = p + c
+    bb = s - p
+    e = (p - (s - bb)) + (c - bb)                 # exact error of the fp64 sum
+    even = (np.asarray(s).view(np.uint64) & np.uint64(1)) == 0
+    step = np.nextafter(s, np.where(e > 0, np.inf, -np.inf))
+    s = np.where((e != 0) & even, step, s)
+    return np.asarray(s, dtype=F64).astype(F32)
+
+
 def project(xbar32: np.ndarray, w32) -> np.ndarray:
     """Learnable projection proj(X) = X W (no bias) [SLA2-deep §05]; W = None is
-    the identity, which turns the router into SLA's pooled heuristic."""
+    the identity, which turns the router into SLA's pooled heuristic.  Each
+    output is a chain of fused multiply-adds over e ascending from +0.0."""
     if w32 is None:
         return np.array(xbar32, dtype=F32, copy=True)
     xbar32 = np.asarray(xbar32, dtype=F32)
@@ -83,20 +103,21 @@ def project(xbar32: np.ndarray, w32) -> np.ndarray:
     d = xbar32.shape[-1]
     acc = np.zeros(xbar32.shape[:-1] + (w32.shape[1],), dtype=F32)
     for e in range(d):
-        acc = acc + xbar32[..., e:e + 1] * w32[e, :]
+        acc = fma32(xbar32[..., e:e + 1], w32[e, :], acc)
     return acc
 
 
 def block_scores(qt32: np.ndarray, kt32: np.ndarray) -> np.ndarray:
     """Compressed score map P_c = proj_q(Qbar) proj_k(Kbar)^T [SLA2-deep §05],
-    fixed-order fp32, without the monotone 1/sqrt(d) and softmax of
-    [SLA 关键设计 2].  qt32 [B,H,nq,d], kt32 [B,H,nkv,d] -> [B,H,nq,nkv]."""
+    a chain of fused multiply-adds over c ascending from +0.0, without the
+    monotone 1/sqrt(d) and softmax of [SLA 关键设计 2].
+    qt32 [B,H,nq,d], kt32 [B,H,nkv,d] -> [B,H,nq,nkv]."""
     qt32 = np.asarray(qt32, dtype=F32)
     kt32 = np.asarray(kt32, dtype=F32)
     d = qt32.shape[-1]
     acc = np.zeros(qt32.shape[:-1] + (kt32.shape[-2],), dtype=F32)
     for c in range(d):
-        acc = acc + qt32[..., :, c, None] * kt32[..., None, :, c]
+        acc = fma32(qt32[..., :, c, None], kt32[..., None, :, c], acc)
     return acc
 
 

@@ -12,6 +12,8 @@ from __future__ import annotations
 
 import math
 
+from fractions import Fraction
+
 import numpy as np
 import torch
 
@@ -44,18 +46,68 @@ def pin_pool_bruteforce(orc):
     assert np.array_equal(gi[0, 0], np.array([[4, 5], [14, 15], [21, 22]], dtype=np.float32))
 
 
+def _rn32(v: Fraction) -> np.float32:
+    """The fp32 nearest to the exact rational v (ties to even), by exact
+    comparison with the fp32 neighbours of a first guess."""
+    f = np.float32(float(v))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    return min(cands, key=lambda c: (abs(Fraction(float(c)) - v), int(np.float32(c).view(np.uint32)) & 1))
+
+
+def _fma_chain(xs, ys) -> np.float32:
+    """acc = rn32(x * y + acc) over the pairs in order, from +0.0, in exact
+    rational arithmetic: each multiply-add rounded once."""
+    acc = np.float32(0.0)
+    for x, y in zip(xs, ys):
+        acc = _rn32(Fraction(float(x)) * Fraction(float(y)) + Fraction(float(acc)))
+    return acc
+
+
+def pin_fma32_exact(orc):
+    """The vectorised single-rounding multiply-add equals the exact rational
+    result rounded once, on random values and on cancelling ones."""
+    g = np.random.default_rng(41)
+    a = (g.standard_normal(400) * np.exp2(g.integers(-20, 20, 400))).astype(np.float32)
+    b = (g.standard_normal(400) * np.exp2(g.integers(-20, 20, 400))).astype(np.float32)
+    c = (g.standard_normal(400) * np.exp2(g.integers(-20, 20, 400))).astype(np.float32)
+    c[:100] = -(a[:100].astype(np.float64) * b[:100]).astype(np.float32)  # near-cancelling sums
+    got = orc.fma32(a, b, c)
+    for i in range(400):
+        want = _rn32(Fraction(float(a[i])) * Fraction(float(b[i])) + Fraction(float(c[i])))
+        assert got[i] == want, (i, a[i], b[i], c[i], got[i], want)
+
+
+def pin_fma32_double_rounding_case(orc):
+    """A multiply-add where rounding the fp64 sum to fp32 rounds twice and
+    goes wrong: a * b = 2^-24 (1 + eta), 0 < eta < 2^-29, plus c = 1.  The fp64
+    sum lands exactly on the fp32 midpoint 1 + 2^-24 and ties-to-even would
+    give 1; the exact value is above the midpoint, so the answer is 1 + 2^-23."""
+    g = np.random.default_rng(7)
+    for _ in range(20000):
+        a = np.float32(g.uniform(2.0 ** -12, 2.0 ** -11))
+        b = np.float32(2.0 ** -24 / float(a))
+        eta = Fraction(float(a)) * Fraction(float(b)) / Fraction(1, 2 ** 24) - 1
+        if 0 < eta < Fraction(1, 2 ** 29):
+            break
+    else:
+        raise AssertionError("no case found")
+    c = np.float32(1.0)
+    naive = np.float32(np.float64(a) * np.float64(b) + np.float64(c))
+    want = _rn32(Fraction(float(a)) * Fraction(float(b)) + 1)
+    assert naive != want and want == np.float32(1.0 + 2.0 ** -23)
+    assert orc.fma32(np.array([a]), np.array([b]), np.array([c]))[0] == want
+
+
 def pin_project_bruteforce(orc):
-    """Projection is x W (row vector times matrix) in ascending fp32 order;
+    """Projection is x W (row vector times matrix), a chain of single-rounding
+    multiply-adds in ascending order (checked in exact rational arithmetic);
     W = None and W = I are both the identity; a permutation matrix permutes."""
     x = _rand((1, 1, 3, 4), 2).astype(np.float32)
     w = _rand((4, 4), 3).astype(np.float32)
     got = orc.project(x, w)
     for r in range(3):
         for c in range(4):
-            acc = np.float32(0.0)
-            for e in range(4):
-                acc = np.float32(acc + np.float32(x[0, 0, r, e] * w[e, c]))
-            assert got[0, 0, r, c] == acc
+            assert got[0, 0, r, c] == _fma_chain(x[0, 0, r, :], w[:, c])
     assert np.array_equal(orc.project(x, None), x)
     assert np.array_equal(orc.project(x, np.eye(4, dtype=np.float32)), x)
     perm = np.eye(4, dtype=np.float32)[[2, 0, 3, 1]]   # x @ perm picks columns
@@ -70,10 +122,7 @@ def pin_scores_bruteforce(orc):
     assert got.shape == (1, 1, 3, 4)
     for i in range(3):
         for j in range(4):
-            acc = np.float32(0.0)
-            for c in range(5):
-                acc = np.float32(acc + np.float32(qt[0, 0, i, c] * kt[0, 0, j, c]))
-            assert got[0, 0, i, j] == acc
+            assert got[0, 0, i, j] == _fma_chain(qt[0, 0, i, :], kt[0, 0, j, :])
     ref = qt[0, 0].astype(np.float64) @ kt[0, 0].astype(np.float64).T
     assert np.allclose(got[0, 0], ref, rtol=1e-5, atol=1e-6)
 
@@ -483,7 +532,7 @@ def pin_fp8_tile_width_moves_quantisation(orc):
     assert 0.0 < d < 0.1, d
 
 
-ALL_PINS = [pin_hand_example, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
+ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
             pin_fp8_k_smoothing, pin_fp8_block_scales, pin_fp8_tile_width_exact_without_quantisation,
             pin_fp8_tile_width_moves_quantisation,
     pin_pool_bruteforce, pin_project_bruteforce, pin_scores_bruteforce, pin_topk_sort,

@@ -21,7 +21,10 @@ MUTATIONS = {
     "alpha_swapped": ("a * o_s + (1.0 - a) * o_l", "(1.0 - a) * o_s + a * o_l"),
     "pool_divides_by_block_size": ("return acc / counts.astype(F32)[None, None, :, None]",
                                    "return acc / F32(b)"),
-    "project_uses_W_transpose": ("xbar32[..., e:e + 1] * w32[e, :]", "xbar32[..., e:e + 1] * w32[:, e]"),
+    "project_uses_W_transpose": ("fma32(xbar32[..., e:e + 1], w32[e, :], acc)", "fma32(xbar32[..., e:e + 1], w32[:, e], acc)"),
+    "fma_rounds_twice": ("    s = np.where((e != 0) & even, step, s)\n", ""),
+    "score_mul_then_add": ("acc = fma32(qt32[..., :, c, None], kt32[..., None, :, c], acc)",
+                           "acc = (acc + qt32[..., :, c, None] * kt32[..., None, :, c]).astype(F32)"),
     "ties_prefer_higher_index": ('return np.argsort(-scores, axis=-1, kind="stable")',
                                  'return scores.shape[-1] - 1 - np.argsort(-scores[..., ::-1], axis=-1, kind="stable")'),
     "negligible_taken_from_top": ("order[..., n_kv - k_l:]", "order[..., k_h:k_h + k_l]"),
