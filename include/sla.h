@@ -110,9 +110,10 @@ sla_status sla_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * then per query block i, with key blocks ordered by (s desc, index asc):
  *   SLA2: the first k_keep are kept;
  *   SLA : the first k_keep are critical (+1), the last k_neg negligible (-1).
- * All of this is fixed-order fp32 (sums in ascending index order from +0.0,
- * each multiply and add rounded separately, no fused multiply-add), so the
- * selection is reproducible bit for bit.  The 1/sqrt(d) and softmax of SLA's
+ * All of this is fixed-order fp32 (sums in ascending index order from +0.0;
+ * the means by one division; the projections and scores as chains of
+ * multiply-adds, each rounded once), so the selection is reproducible bit
+ * for bit.  The 1/sqrt(d) and softmax of SLA's
  * compressed map are not applied: both are monotone per row.
  * Outputs (device):
  *   kept_idx   int32 [B,H,n_q,k_keep], ascending per row (k_keep may be 0)

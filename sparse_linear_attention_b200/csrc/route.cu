@@ -7,13 +7,13 @@
 // labels: top k_h critical, bottom k_l negligible, rest marginal).
 //
 // Every floating-point step is a single IEEE round-to-nearest operation in a
-// fixed order (__fadd_rn / __fmul_rn / __fdiv_rn never contract into FMA), so
-// the selected blocks are reproducible bit for bit on any implementation that
-// follows the same order (pooling and projection run in one kernel, the means
-// staying in shared memory):
+// fixed order (__fadd_rn / __fdiv_rn / __fmaf_rn), so the selected blocks are
+// reproducible bit for bit on any implementation that follows the same order
+// (pooling and projection run in one kernel, the means staying in shared
+// memory):
 //   pooled mean : tokens ascending from +0.0, then divide by the count
-//   projection  : y[c] = sum_e fl(x[e] * W[e][c]), e ascending, from +0.0
-//   score       : s[i][j] = sum_c fl(qt[i][c] * kt[j][c]), c ascending, from +0.0
+//   projection  : y[c] = fma(x[e], W[e][c], y[c]), e ascending, from +0.0
+//   score       : s[i][j] = fma(qt[i][c], kt[j][c], s[i][j]), c ascending, from +0.0
 // The ranking is (score descending, block index ascending).
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -28,8 +28,8 @@ namespace sla {
 // ---------------------------------------------------------------- pooling + projection
 // One block per kPPRows blocks (rows) of one head and one of Q (grid z = 0) or
 // K (z = 1): the block means go to shared memory (tokens ascending from +0.0,
-// then one division, as in pool_kernel) and are projected at once (e
-// ascending, no FMA, as in project_kernel), so the projection's arithmetic
+// then one division) and are projected at once (e ascending, one rounding
+// per multiply-add), so the projection's arithmetic
 // runs under the pooling's HBM traffic and the means never leave the chip.
 constexpr int kPPRows = 16;
 
@@ -101,10 +101,10 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e]);
-        out[r] = __fadd_rn(out[r], __fmul_rn(x4.x, w[0]));
-        out[r] = __fadd_rn(out[r], __fmul_rn(x4.y, w[1]));
-        out[r] = __fadd_rn(out[r], __fmul_rn(x4.z, w[2]));
-        out[r] = __fadd_rn(out[r], __fmul_rn(x4.w, w[3]));
+        out[r] = __fmaf_rn(x4.x, w[0], out[r]);
+        out[r] = __fmaf_rn(x4.y, w[1], out[r]);
+        out[r] = __fmaf_rn(x4.z, w[2], out[r]);
+        out[r] = __fmaf_rn(x4.w, w[3], out[r]);
       }
     }
   }
@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
 // a small fp32 GEMM: per 256-key pass, thread (ry, kx) forms rows 2ry, 2ry+1 x
 // keys 4kx .. 4kx+3 (two shared-memory reads per eight products), the
 // projected keys streaming through a double-buffered cp.async ring of
-// kScoreC-channel slices.  Every score sums c ascending, one rounding per
-// product and per sum.  Then warp w selects for row w.
+// kScoreC-channel slices.  Every score is a multiply-add chain over c
+// ascending, one rounding each.  Then warp w selects for row w.
 constexpr int kScoreRows = 8;
 constexpr int kScoreKeys = 256;
 constexpr int kScoreC = 16;
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
 #pragma unroll
         for (int a2 = 0; a2 < 2; ++a2)
 #pragma unroll
-          for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = __fadd_rn(acc[a2][b4], __fmul_rn(qa[a2], kv[b4]));
+          for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = __fmaf_rn(qa[a2], kv[b4], acc[a2][b4]);
       }
       __syncthreads();  // buffer sl & 1 may be refilled
     }
