@@ -15,11 +15,11 @@
 // product per step for S, and one max exchange per 128 keys.  352 threads:
 //   warp 8      TMA producer, running ahead across tiles: per step the two
 //               key tiles side by side in one 128-row slot of a 2-slot ring
-//               (freed once S has read it); per listed block its phi(K), V
-//               tiles (fp16) in a 4-slot ring (freed after PV and H); per tile
-//               the Q tile (as soon as the previous tile's S products are
-//               done) and, in the next ring slot after its blocks, the fp16
-//               H_tot / sigma tile of its head.
+//               (freed once S has read it); per step the phi(K), V tiles
+//               (fp16) of its two blocks in one entry of a 2-entry ring (freed
+//               after PV and H); per tile the Q tile (as soon as the previous
+//               tile's S products are done) and, in the ring entry after its
+//               blocks, the fp16 H_tot / sigma tile of its head.
 //   warps 9, 10 tcgen05 issuers (one thread each), fp32 accumulators in TMEM.
 //               Warp 9:   S = Q [K_a | K_b]^T  (bf16 operands in smem) and
 //                         O += [P_a | P_b] [V_a ; V_b] (fp16 P from TMEM), in
@@ -37,9 +37,13 @@
 //               stale max scales numerator and denominator alike, and
 //               p <= 2^15 still fits fp16).  P is rounded to fp16 and written
 //               over the step's S columns in TMEM for the PV product.
-//               phi(Q) is formed when the tile's Q lands and kept packed in
-//               registers, so the Q tile in smem is replaced as soon as the
-//               tile's S products are done.
+//               phi(Q) of a tile is formed (packed in registers) during the
+//               previous tile's epilogue, while phi(Q) H_i runs, so the Q tile
+//               in smem is replaced early.  The epilogue does the work that
+//               needs no product (row sums, Z_i, the denominator) and H_i
+//               (once warp 10's products are done) before it waits for the
+//               last PV; the output store's smem read is waited for only
+//               after the next tile's first step.
 // TMEM (512 columns): S0 | S1 (128 each, P over part of them) | O (128) |
 // H_ex (128, then phi(Q) H_i or the SLA projection in the epilogue).
 // The linear branch uses H_i = H_tot - sum over the listed blocks of
@@ -108,14 +112,15 @@ enum {
   B_SFULL = 8,    // +buffer (= key-pair slot)
   B_PFULL = 10,   // +buffer
   B_PEMPTY = 12,  // +buffer
-  B_OFINAL = 14,
+  B_OFINAL = 14,  // warp 9's products of the tile (its last PV) are done
   B_EPI = 15,
   B_NUM = 16,
   B_EPIDONE = 17,
   B_PROJR = 18,
   B_PROJF = 19,
   B_DRAIN = 20,   // +issuer (2)
-  NBAR = 22
+  B_HFIN = 22,    // warp 10's products of the tile (H_ex) are done
+  NBAR = 23
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
@@ -212,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_PFULL + b], kCompute);
       mbar_init(&bars[B_PEMPTY + b], 1);
     }
-    mbar_init(&bars[B_OFINAL], 2);  // both issuers' products of the tile are done
+    mbar_init(&bars[B_OFINAL], 1);
+    mbar_init(&bars[B_HFIN], 1);
     mbar_init(&bars[B_EPI], kCompute);
     mbar_init(&bars[B_NUM], 1);
     mbar_init(&bars[B_EPIDONE], kCompute);
@@ -494,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bars[B_VEMPTY + sl]);
           }
           if (!ok) break;
-          mma_commit(&bars[B_OFINAL]);
+          mma_commit(&bars[B_HFIN]);
           // epilogue: phi(Q) (TMEM, the tile's last S buffer) x H_i / sigma (smem, the H tile's slot)
           if (!mbar_wait(&bars[B_EPI], ti & 1, abort_flag, a.status)) break;
           tc_fence_after();
@@ -552,27 +558,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = T.crit[p];
       return (j < 0 || j >= a.nkv) ? 0 : j;
     };
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
-      const Tile T = tile_at(a, t, false);
-      const int tok = T.qb * a.bq + r;
-      const bool row_valid = (r < a.bq) && (tok < a.N);
-      float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
-      if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
-      int jl = list_chunk(T, 0);
-      // phi(Q) for row r, channels 64*half .. 64*half+63 (zero past d), packed fp16,
-      // formed as soon as the tile's Q lands so the Q tile can be replaced early
-      uint32_t phq[32];
-      ok = ok && warp_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status);
+    // phi(Q) of tile Tq for row r, channels 64*half .. 64*half+63 (zero past d),
+    // packed fp16 into phq.  Formed as soon as the tile's Q lands (for every tile
+    // after the first, while the previous tile's epilogue products run), so the
+    // Q tile can be replaced early.
+    uint32_t phq[32];
+    auto form_phi_q = [&](const Tile& Tq, int tiq) {
+      ok = ok && warp_wait(&bars[B_QFULL], tiq & 1, abort_flag, a.status);
+      const int tokq = Tq.qb * a.bq + r;
       {
         uint4 qw[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           qw[u] = make_uint4(0, 0, 0, 0);
-          if (T.has_lin) {
+          if (Tq.has_lin) {
             if constexpr (kFP8) {  // the smem tile holds e4m3 Q: read the bf16 row
-              if (tok < a.N)
+              if (tokq < a.N)
                 qw[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qsrc) +
-                                                        (static_cast<long long>(T.bh) * a.N + tok) * kDPad + 64 * half + 8 * u);
+                                                        (static_cast<long long>(Tq.bh) * a.N + tokq) * kDPad + 64 * half + 8 * u);
             } else {
               qw[u] = *reinterpret_cast<const uint4*>(sm + OFF_Q + half * 16384u + sw128_off(r, u));
             }
@@ -626,6 +629,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    };
+    if (blockIdx.x < ntiles) form_phi_q(tile_at(a, blockIdx.x, false), 0);
+    // The previous tile's output store may still read its smem slot: thread 0
+    // waits for that read and frees the slot after the next tile's first step.
+    bool pend_store = false;
+    int pend_hsl = 0;
+    auto release_store = [&]() {
+      if (pend_store) {
+        if (tid == 0) {
+          bulk_wait_read_all();
+          mbar_arrive(&bars[B_VEMPTY + pend_hsl]);
+        }
+        pend_store = false;
+      }
+    };
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
+      const Tile T = tile_at(a, t, false);
+      const int tok = T.qb * a.bq + r;
+      const bool row_valid = (r < a.bq) && (tok < a.N);
+      float sl2_q = a.sl2;  // e4m3 branch: times the query block's scale
+      if constexpr (kFP8) sl2_q *= a.sq[static_cast<long long>(T.bh) * a.nb128 + (T.qb * a.bq) / 128];
+      int jl = list_chunk(T, 0);
       const float alpha_t = a.alpha ? a.alpha[T.row] : 0.0f;
       const float sigma = T.has_lin ? a.sigma[T.bh] : 1.0f;
       const float zt_r = T.has_lin ? a.ztot[static_cast<long long>(T.bh) * kDPad + r] : 0.0f;
@@ -699,15 +724,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float nm = -m_run;
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (live) {
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < 2; ++cc) {
-            float s[32];
-            tmem_ld32(scol + 32 * cc, s);
+            float sk[32];
+            tmem_ld32(scol + 32 * cc, sk);
             tmem_wait_ld();
             if (nvalid < kBlockKV) {
 #pragma unroll
               for (int c = 0; c < 32; ++c)
-                if (32 * cc + c >= nvalid) s[c] = -INFINITY;
+                if (32 * cc + c >= nvalid) sk[c] = -INFINITY;
             }
             if constexpr (kFP8) {
               // the row sum uses the unquantised p; the PV product p * 448 rounded
@@ -717,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int c = 0; c < 8; ++c) {
                 float p[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(s[4 * c + e], sc, nm));
+                for (int e = 0; e < 4; ++e) p[e] = ex2_approx(fmaf(sk[4 * c + e], sc, nm));
                 l4[c & 3] += (p[0] + p[1]) + (p[2] + p[3]);
                 const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p[0] * 448.0f, p[1] * 448.0f),
                                                              __NV_SATFINITE, __NV_E4M3);
@@ -730,8 +755,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t pk[16];
 #pragma unroll
               for (int c = 0; c < 16; ++c) {
-                const float p0 = ex2_approx(fmaf(s[2 * c], sc, nm));
-                const float p1 = ex2_approx(fmaf(s[2 * c + 1], sc, nm));
+                const float p0 = ex2_approx(fmaf(sk[2 * c], sc, nm));
+                const float p1 = ex2_approx(fmaf(sk[2 * c + 1], sc, nm));
                 l4[c & 3] += p0 + p1;
                 pk[c] = pack_half2(p0, p1);
               }
@@ -745,6 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&bars[B_PFULL + b]);
         }
+        if (i == 0) release_store();
         zex += zv;
       }
       gs += T.nsteps;
@@ -762,8 +788,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ---------------------------------------------------------- epilogue
-      ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
-      if (ok) tc_fence_after();
+      // Work that needs no product first (l, Z_i and the denominator), then H_i
+      // once warp 10's products are done, then phi(Q) over the last S buffer once
+      // the last PV has read it.
+      release_store();  // (a tile without steps)
       const float l_run = l_part + xchg(l_part);
       const uint32_t pcol = T_S0 + ((gs - 1) & 1) * 128;  // the tile's last S buffer
       const int hidx = gv + T.nsteps + T.nnegl_e;          // value entry of the H tile
@@ -772,6 +800,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       gv += T.nsteps + T.nnegl_e + (T.has_lin ? 1 : 0);
       float den = 0.0f;
       if (T.has_lin) {
+        // Z_i[e] for e = r, shared with every row for the denominator
+        const float zi = zt_r - (zex + xchg(zex));
+        if (half == 0) zsh[r] = zi;
+        const int c0 = 64 * half;
+        named_bar_sync(5, kCompute);  // Z_i complete
+        float dp = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float2 f = unpack_half2(phq[c]);  // the denominator uses the rounded phi(Q)
+          dp = fmaf(f.x, zsh[c0 + 2 * c], dp);
+          dp = fmaf(f.y, zsh[c0 + 2 * c + 1], dp);
+        }
+        den = dp + xchg(dp);
+        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status);
+        if (ok) tc_fence_after();
         // H_i / sigma = H_tot / sigma (fp16 tile from TMA) - H_ex / sigma, row e = r,
         // channels 64*half.., in place in the MN-major H tile
         ok = ok && warp_wait(&bars[B_VFULL + hsl], (hidx / kVSlots) & 1, abort_flag, a.status);
@@ -798,30 +841,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             *hp = make_uint4(o4[0], o4[1], o4[2], o4[3]);
           }
         }
-        // Z_i[e] for e = r, shared with every row for the denominator
-        const float zi = zt_r - (zex + xchg(zex));
-        if (half == 0) zsh[r] = zi;
-        const int c0 = 64 * half;
-        named_bar_sync(5, kCompute);  // Z_i complete
-        float dp = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float2 f = unpack_half2(phq[c]);  // the denominator uses the rounded phi(Q)
-          dp = fmaf(f.x, zsh[c0 + 2 * c], dp);
-          dp = fmaf(f.y, zsh[c0 + 2 * c + 1], dp);
-        }
-        den = dp + xchg(dp);
+      } else {
+        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status);  // (every tile: phases stay aligned)
+      }
+      ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
+      if (ok) tc_fence_after();
+      if (T.has_lin) {
         if (ok) {
           tmem_st16(tmem + lrow + pcol + 32 * half, phq);
           tmem_st16(tmem + lrow + pcol + 32 * half + 16, phq + 16);
           tmem_wait_st();
         }
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // the H_i tile is visible to the tensor core
       }
       if (ok) {
         tc_fence_before();
         mbar_arrive(&bars[B_EPI]);
       }
+      // the next tile's phi(Q) while phi(Q) H_i runs
+      if (t + static_cast<int>(gridDim.x) < ntiles) form_phi_q(tile_at(a, t + gridDim.x, false), ti + 1);
       ok = ok && warp_wait(&bars[B_NUM], ti & 1, abort_flag, a.status);
       if (ok) tc_fence_after();
 
@@ -934,15 +972,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tma_o) {
         fence_proxy_async_smem();      // the staged rows are visible to the TMA engine
         named_bar_sync(5, kCompute);   // ... from every thread
-        if (tid == 0) {
-          if (ok) {
-            tma_store_3d(&tmO, hbuf, 0, T.qb * 128, T.bh);
-            tma_store_3d(&tmO, hbuf + 16384, 64, T.qb * 128, T.bh);
-            bulk_commit_group();
-            bulk_wait_read_all();      // the slot may be refilled once the store has read it
-          }
-          mbar_arrive(&bars[B_VEMPTY + hsl]);
+        if (tid == 0 && ok) {
+          tma_store_3d(&tmO, hbuf, 0, T.qb * 128, T.bh);
+          tma_store_3d(&tmO, hbuf + 16384, 64, T.qb * 128, T.bh);
+          bulk_commit_group();
         }
+        pend_store = true;  // the slot is refilled once the store has read it (release_store)
+        pend_hsl = hsl;
       }
     }
     if (tid == 0) bulk_wait_all();
