@@ -94,18 +94,30 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
   } else {
 #pragma unroll
     for (int r = 0; r < 8; ++r) out[r] = 0.0f;
-    for (int e = 0; e < d; e += 4) {  // d % 4 == 0
-      float w[4];
+    // 16 rows of W per batch, the next batch loading while this one is used:
+    // every CTA projects at the same time, so the loads must not wait in turn
+    float w[16];
 #pragma unroll
-      for (int uu = 0; uu < 4; ++uu) w[uu] = __ldg(W + (e + uu) * d + c);
+    for (int j = 0; j < 16; ++j) w[j] = j < d ? __ldg(W + j * d + c) : 0.0f;
+    for (int e0 = 0; e0 < d; e0 += 16) {  // d % 8 == 0: a batch is 8 or 16 rows
+      float wn[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) wn[j] = e0 + 16 + j < d ? __ldg(W + (e0 + 16 + j) * d + c) : 0.0f;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e]);
-        out[r] = __fmaf_rn(x4.x, w[0], out[r]);
-        out[r] = __fmaf_rn(x4.y, w[1], out[r]);
-        out[r] = __fmaf_rn(x4.z, w[2], out[r]);
-        out[r] = __fmaf_rn(x4.w, w[3], out[r]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (e0 + 4 * q < d) {
+            const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e0 + 4 * q]);
+            out[r] = __fmaf_rn(x4.x, w[4 * q], out[r]);
+            out[r] = __fmaf_rn(x4.y, w[4 * q + 1], out[r]);
+            out[r] = __fmaf_rn(x4.z, w[4 * q + 2], out[r]);
+            out[r] = __fmaf_rn(x4.w, w[4 * q + 3], out[r]);
+          }
+        }
       }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = wn[j];
     }
   }
   const int stride = isK ? kstride : nrows;  // key rows padded to a multiple of 4 floats
@@ -116,120 +128,146 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
 }
 
 // ---------------------------------------------------------------- scores + selection
-// Block: 256 threads, kScoreRows = 8 query blocks of one head.  The scores are
-// a small fp32 GEMM: per 256-key pass, thread (ry, kx) forms rows 2ry, 2ry+1 x
-// keys 4kx .. 4kx+3 (two shared-memory reads per eight products), the
-// projected keys streaming through a double-buffered cp.async ring of
-// kScoreC-channel slices.  Every score is a multiply-add chain over c
-// ascending, one rounding each.  Then warp w selects for row w.
+// Block: 128 threads, kScoreRows = 8 query blocks of one head (three blocks fit
+// an SM, so a head-major grid runs in one wave with at most 24 rows per SM).
+// The scores are a small fp32 GEMM, taken 512 keys per pass: warp w forms rows
+// 4 (w % 2) .. +3 against keys 256 (w / 2) + 4 lane .. +3 and 256 (w / 2) +
+// 128 + 4 lane .. +3 of the pass, so each channel costs a thread one broadcast
+// read of its four query values and two conflict-free reads of its eight keys
+// for 32 products.  The projected keys stream through a kScoreStages-deep
+// cp.async ring of kScoreC-channel slices.  Every score is a multiply-add chain
+// over c ascending, one rounding each.  Then each warp selects for two rows.
 constexpr int kScoreRows = 8;
-constexpr int kScoreKeys = 256;
-constexpr int kScoreC = 16;
+constexpr int kScoreThreads = 128;
+constexpr int kScoreKeys = 512;
+constexpr int kScoreC = 8;
+constexpr int kScoreStages = 3;
 
-__global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ qtT,
+__host__ __device__ constexpr size_t score_smem_bytes(int kstride) {
+  return (static_cast<size_t>(kDPad) * kScoreRows + static_cast<size_t>(kScoreStages) * kScoreC * kScoreKeys +
+          static_cast<size_t>(kScoreRows) * kstride) * 4;
+}
+
+template <int kKPL>  // keys per lane held in registers by the selection: n_kv <= 32 kKPL
+__global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const float* __restrict__ qtT,
                                                            const float* __restrict__ ktT, int nq, int nkv,
                                                            int kstride, int d, int mode, int k_keep, int k_neg,
                                                            int32_t* __restrict__ kept_idx,
                                                            int8_t* __restrict__ labels,
                                                            float* __restrict__ scores_dbg) {
   extern __shared__ __align__(16) float sm[];
-  float* qsT = sm;                              // [128 channels][8 rows]
-  float* kbuf = qsT + kDPad * kScoreRows;       // 2 x [kScoreC][kScoreKeys]
-  float* sc = kbuf + 2 * kScoreC * kScoreKeys;  // [kScoreRows][nkv]
+  float* qsT = sm;                                         // [128 channels][8 rows]
+  float* kbuf = qsT + kDPad * kScoreRows;                  // kScoreStages x [kScoreC][kScoreKeys]
+  float* sc = kbuf + kScoreStages * kScoreC * kScoreKeys;  // [kScoreRows][kstride]
   const long long bh = blockIdx.y;
   const int r0 = blockIdx.x * kScoreRows;
   const int tid = threadIdx.x;
-  for (int i = tid; i < kScoreRows * kDPad; i += 256) {
+  for (int i = tid; i < kScoreRows * kDPad; i += kScoreThreads) {
     const int r = i % kScoreRows, c = i / kScoreRows;
     qsT[i] = (c < d && r0 + r < nq) ? qtT[(bh * d + c) * nq + r0 + r] : 0.0f;
   }
   const float* kbase = ktT + bh * d * static_cast<long long>(kstride);
-  const int ry = tid / 64, kx = tid % 64;
-  const int nslices = (d + kScoreC - 1) / kScoreC;  // channels past d (d % 16 == 8) are zero-filled
+  const int wq = tid / 32;
+  const int rq = wq & 1;                                // rows 4 rq .. 4 rq + 3
+  const int kc = 256 * (wq >> 1) + 4 * (tid & 31);      // keys kc .. kc + 3, kc + 128 .. kc + 131 of the pass
+  const int nslices = d / kScoreC;                      // d % 8 == 0
   for (int k0 = 0; k0 < nkv; k0 += kScoreKeys) {
-    const int kend = min(kScoreKeys, kstride - k0);  // keys of this pass inside the padded rows
-    // slice s of this pass into buffer s & 1: kScoreC rows of kend floats, 16 bytes per copy
+    const int kend = min(kScoreKeys, kstride - k0);     // keys of this pass inside the padded rows
+    // slice sl (channels kScoreC sl ..) into stage sl % kScoreStages, 16 bytes per copy; a
+    // group is committed even when empty so the wait counts stay aligned
     auto load_slice = [&](int sl) {
-      float* dstb = kbuf + (sl & 1) * kScoreC * kScoreKeys;
-      for (int i = tid; i < kScoreC * (kScoreKeys / 4); i += 256) {
-        const int cc = i / (kScoreKeys / 4), k4 = 4 * (i % (kScoreKeys / 4));
-        if (sl * kScoreC + cc >= d)
-          *reinterpret_cast<float4*>(dstb + cc * kScoreKeys + k4) = make_float4(0.f, 0.f, 0.f, 0.f);
-        else if (k4 < kend)
-          cp_async16(dstb + cc * kScoreKeys + k4, kbase + static_cast<long long>(sl * kScoreC + cc) * kstride + k0 + k4);
+      if (sl < nslices) {
+        float* dstb = kbuf + (sl % kScoreStages) * kScoreC * kScoreKeys;
+        for (int i = tid; i < kScoreC * (kScoreKeys / 4); i += kScoreThreads) {
+          const int cc = i / (kScoreKeys / 4), k4 = 4 * (i % (kScoreKeys / 4));
+          if (k4 < kend)
+            cp_async16(dstb + cc * kScoreKeys + k4, kbase + static_cast<long long>(sl * kScoreC + cc) * kstride + k0 + k4);
+        }
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    __syncthreads();  // the previous pass is done with both buffers (and qsT is ready on the first)
-    load_slice(0);
-    float acc[2][4];
+    __syncthreads();  // the previous pass is done with every stage (and qsT is ready on the first)
 #pragma unroll
-    for (int a2 = 0; a2 < 2; ++a2)
+    for (int sl = 0; sl < kScoreStages - 1; ++sl) load_slice(sl);
+    float acc[4][8];
 #pragma unroll
-      for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = 0.0f;
+    for (int a4 = 0; a4 < 4; ++a4)
+#pragma unroll
+      for (int b8 = 0; b8 < 8; ++b8) acc[a4][b8] = 0.0f;
     for (int sl = 0; sl < nslices; ++sl) {
-      if (sl + 1 < nslices) {
-        load_slice(sl + 1);
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      }
-      __syncthreads();  // slice sl visible to every thread
-      const float* kb = kbuf + (sl & 1) * kScoreC * kScoreKeys;
+      asm volatile("cp.async.wait_group %0;" ::"n"(kScoreStages - 2) : "memory");
+      __syncthreads();  // slice sl visible to every thread; stage (sl - 1) % kScoreStages free again
+      load_slice(sl + kScoreStages - 1);
+      const float* kb = kbuf + (sl % kScoreStages) * kScoreC * kScoreKeys + kc;
 #pragma unroll
       for (int cc = 0; cc < kScoreC; ++cc) {
         const int c = sl * kScoreC + cc;
-        const float2 q2 = *reinterpret_cast<const float2*>(qsT + c * kScoreRows + 2 * ry);
-        const float4 k4 = *reinterpret_cast<const float4*>(kb + cc * kScoreKeys + 4 * kx);
-        const float qa[2] = {q2.x, q2.y};
-        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        const float4 q4 = *reinterpret_cast<const float4*>(qsT + c * kScoreRows + 4 * rq);
+        const float4 ka = *reinterpret_cast<const float4*>(kb + cc * kScoreKeys);
+        const float4 kb4 = *reinterpret_cast<const float4*>(kb + cc * kScoreKeys + 128);
+        const float qa[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb4.x, kb4.y, kb4.z, kb4.w};
 #pragma unroll
-        for (int a2 = 0; a2 < 2; ++a2)
+        for (int a4 = 0; a4 < 4; ++a4)
 #pragma unroll
-          for (int b4 = 0; b4 < 4; ++b4) acc[a2][b4] = __fmaf_rn(qa[a2], kv[b4], acc[a2][b4]);
+          for (int b8 = 0; b8 < 8; ++b8) acc[a4][b8] = __fmaf_rn(qa[a4], kv[b8], acc[a4][b8]);
       }
-      __syncthreads();  // buffer sl & 1 may be refilled
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
-    for (int a2 = 0; a2 < 2; ++a2)
+    for (int a4 = 0; a4 < 4; ++a4)
 #pragma unroll
-      for (int b4 = 0; b4 < 4; ++b4) {
-        const int j = k0 + 4 * kx + b4;
-        if (j < nkv) sc[(2 * ry + a2) * nkv + j] = acc[a2][b4];
+      for (int b8 = 0; b8 < 8; ++b8) {
+        const int j = k0 + kc + (b8 & 3) + 128 * (b8 >> 2);
+        if (j < nkv) sc[(4 * rq + a4) * kstride + j] = acc[a4][b8];
       }
   }
   __syncthreads();
 
   const int lane = tid % 32, warp = tid / 32;
-  {
-    const int r = warp;
+  for (int r = warp; r < kScoreRows; r += kScoreThreads / 32) {
     const int row = r0 + r;
-    if (row >= nq) return;
-    const float* srow = sc + r * nkv;
+    if (row >= nq) break;
+    const float* srow = sc + r * kstride;
     const long long grow = bh * nq + row;
     // Rank keys: the scores mapped to unsigned integers in the same order
-    // (-0 taken as +0, as the comparison does); the k-th largest is found bit
-    // by bit with warp-wide counts, ties at it go by block index.
-    uint32_t* orow = reinterpret_cast<uint32_t*>(sc + r * nkv);
-    for (int j = lane; j < nkv; j += 32) {
-      const float sv = srow[j];
-      if (scores_dbg) scores_dbg[grow * nkv + j] = sv;
-      uint32_t u = __float_as_uint(sv);
-      if (u == 0x80000000u) u = 0u;
-      orow[j] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    // (-0 taken as +0, as the comparison does), held in registers: lane l has
+    // the keys of blocks l + 32 t, t < nvl.  The k-th largest is found bit by
+    // bit with warp-wide counts, ties at it go by block index.
+    const int nvl = nkv > lane ? (nkv - lane + 31) / 32 : 0;  // this lane's blocks
+    uint32_t key[kKPL];
+#pragma unroll
+    for (int t = 0; t < kKPL; ++t) {
+      const int j = lane + 32 * t;
+      uint32_t u = 0u;
+      if (t < nvl) {
+        const float sv = srow[j];
+        if (scores_dbg) scores_dbg[grow * nkv + j] = sv;
+        u = __float_as_uint(sv);
+        if (u == 0x80000000u) u = 0u;
+        u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      }
+      key[t] = u;
     }
-    __syncwarp();
+    // keys >= cand over the warp: a ballot per register slot (no reduction step)
     auto count_ge = [&](uint32_t cand, uint32_t flip) -> int {
       int c = 0;
-      for (int j = lane; j < nkv; j += 32) c += ((orow[j] ^ flip) >= cand) ? 1 : 0;
-      return __reduce_add_sync(0xffffffffu, c);
+#pragma unroll
+      for (int t = 0; t < kKPL; ++t) c += __popc(__ballot_sync(0xffffffffu, t < nvl && (key[t] ^ flip) >= cand));
+      return c;
     };
-    // largest T with at least k keys >= T (flip = ~0: keys of the worst blocks)
+    // A threshold T that selects the k best blocks: the largest T with at least
+    // k keys >= T (flip = ~0: keys of the worst blocks), found bit by bit.  The
+    // search stops early at a candidate with exactly k keys >= it: the keys >= it
+    // are then the k largest, and the selection below (keys > T, then keys == T
+    // by index up to k) takes exactly those.
     auto kth_key = [&](int k, uint32_t flip) -> uint32_t {
       uint32_t T = 0;
       for (int b = 31; b >= 0; --b) {
         const uint32_t cand = T | (1u << b);
-        if (count_ge(cand, flip) >= k) T = cand;
+        const int cnt = count_ge(cand, flip);
+        if (cnt >= k) T = cand;
+        if (cnt == k) break;
       }
       return T;
     };
@@ -240,14 +278,17 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
       const uint32_t T = kth_key(k_keep, 0u);
       const int need = k_keep - (T == 0xFFFFFFFFu ? 0 : count_ge(T + 1u, 0u));  // from the ties at T
       int seen = 0;
-      for (int t = 0; t < nt; ++t) {  // ascending index: the lower indices win the ties
-        const int j = lane + 32 * t;
-        const uint32_t o = j < nkv ? orow[j] : 0u;
-        const bool eq = j < nkv && o == T;
-        const uint32_t m = __ballot_sync(0xffffffffu, eq);
-        const int rank = seen + __popc(m & ((1u << lane) - 1u));
-        if (j < nkv && (o > T || (eq && rank < need))) top |= 1ull << t;
-        seen += __popc(m);
+#pragma unroll
+      for (int t = 0; t < kKPL; ++t) {  // ascending index: the lower indices win the ties
+        if (t < nt) {
+          const bool v = t < nvl;
+          const uint32_t o = key[t];
+          const bool eq = v && o == T;
+          const uint32_t m = __ballot_sync(0xffffffffu, eq);
+          const int rank = seen + __popc(m & ((1u << lane) - 1u));
+          if (v && (o > T || (eq && rank < need))) top |= 1ull << t;
+          seen += __popc(m);
+        }
       }
     }
     if (mode == SLA_MODE_SLA_3WAY && k_neg > 0) {
@@ -255,14 +296,17 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
       const uint32_t T = kth_key(k_neg, 0xFFFFFFFFu);
       const int need = k_neg - (T == 0xFFFFFFFFu ? 0 : count_ge(T + 1u, 0xFFFFFFFFu));
       int seen = 0;
-      for (int t = nt - 1; t >= 0; --t) {  // descending index: the higher indices go first
-        const int j = lane + 32 * t;
-        const uint32_t o = j < nkv ? ~orow[j] : 0u;
-        const bool eq = j < nkv && o == T;
-        const uint32_t m = __ballot_sync(0xffffffffu, eq);
-        const int rank = seen + __popc(m & ~((2u << lane) - 1u));  // equal keys on higher lanes
-        if (j < nkv && (o > T || (eq && rank < need))) bot |= 1ull << t;
-        seen += __popc(m);
+#pragma unroll
+      for (int t = kKPL - 1; t >= 0; --t) {  // descending index: the higher indices go first
+        if (t < nt) {
+          const bool v = t < nvl;
+          const uint32_t o = ~key[t];
+          const bool eq = v && o == T;
+          const uint32_t m = __ballot_sync(0xffffffffu, eq);
+          const int rank = seen + __popc(m & ~((2u << lane) - 1u));  // equal keys on higher lanes
+          if (v && (o > T || (eq && rank < need))) bot |= 1ull << t;
+          seen += __popc(m);
+        }
       }
     }
     // kept indices in ascending order
@@ -298,14 +342,19 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                                                         Wq, Wk, qtT, ktT, s.N, s.d, s.bq, s.bkv, kt_stride(nkv));
   }
   {
-    const size_t smem =
-        (static_cast<size_t>(kDPad) * kScoreRows + 2 * kScoreC * kScoreKeys + static_cast<size_t>(kScoreRows) * nkv) * 4;
-    cudaError_t e = cudaFuncSetAttribute(score_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const size_t smem = score_smem_bytes(kt_stride(nkv));
+    const dim3 grid(ceil_div(nq, kScoreRows), BH);
+    auto run = [&](auto kernel) -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      kernel<<<grid, kScoreThreads, smem, st>>>(qtT, ktT, nq, nkv, kt_stride(nkv), s.d, mode, k_keep, k_neg, kept_idx, labels,
+                                      scores_dbg);
+      return cudaSuccess;
+    };
+    static_assert(kMaxNKV <= 32 * 64, "selection keys per lane");
+    const cudaError_t e = nkv <= 512 ? run(score_select_kernel<16>)
+                          : nkv <= 1024 ? run(score_select_kernel<32>) : run(score_select_kernel<64>);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(nq, kScoreRows), BH);
-    score_select_kernel<<<grid, 256, smem, st>>>(qtT, ktT, nq, nkv, kt_stride(nkv), s.d, mode, k_keep, k_neg,
-                                                 kept_idx, labels, scores_dbg);
   }
   return cudaGetLastError();
 }
