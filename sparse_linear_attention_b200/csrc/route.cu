@@ -94,30 +94,18 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
   } else {
 #pragma unroll
     for (int r = 0; r < 8; ++r) out[r] = 0.0f;
-    // 16 rows of W per batch, the next batch loading while this one is used:
-    // every CTA projects at the same time, so the loads must not wait in turn
-    float w[16];
+    for (int e = 0; e < d; e += 4) {  // d % 4 == 0
+      float w[4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) w[j] = j < d ? __ldg(W + j * d + c) : 0.0f;
-    for (int e0 = 0; e0 < d; e0 += 16) {  // d % 8 == 0: a batch is 8 or 16 rows
-      float wn[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) wn[j] = e0 + 16 + j < d ? __ldg(W + (e0 + 16 + j) * d + c) : 0.0f;
+      for (int uu = 0; uu < 4; ++uu) w[uu] = __ldg(W + (e + uu) * d + c);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (e0 + 4 * q < d) {
-            const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e0 + 4 * q]);
-            out[r] = __fmaf_rn(x4.x, w[4 * q], out[r]);
-            out[r] = __fmaf_rn(x4.y, w[4 * q + 1], out[r]);
-            out[r] = __fmaf_rn(x4.z, w[4 * q + 2], out[r]);
-            out[r] = __fmaf_rn(x4.w, w[4 * q + 3], out[r]);
-          }
-        }
+        const float4 x4 = *reinterpret_cast<const float4*>(&xs[rh * 8 + r][e]);
+        out[r] = __fmaf_rn(x4.x, w[0], out[r]);
+        out[r] = __fmaf_rn(x4.y, w[1], out[r]);
+        out[r] = __fmaf_rn(x4.z, w[2], out[r]);
+        out[r] = __fmaf_rn(x4.w, w[3], out[r]);
       }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) w[j] = wn[j];
     }
   }
   const int stride = isK ? kstride : nrows;  // key rows padded to a multiple of 4 floats
