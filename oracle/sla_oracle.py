@@ -10,7 +10,8 @@ Plain, slow and written to be checked by eye against the pages:
               (gist.science summary), section 2 "Methodology: SLA2".
   [SLA2-deep] "SLA2 深度解读：97% 稀疏、18.7 倍注意力加速，它和 DeepSeek DSA 的可学习
               Indexer 到底差在哪" (jefxiong.cn), sections 04 (formulation),
-              05 (learnable router), 07 (QAT), 08 (inference kernel).
+              05 (learnable router), 06 (two-stage training: SoftTop-k),
+              07 (QAT), 08 (inference kernel).
   [SLA]       "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
               Sparse-Linear Attention" (papernotes.org), 方法详解 / 关键设计 2
               (compressed map and three labels), 3 (linear branch and Proj),
@@ -146,6 +147,50 @@ def three_way_labels(scores: np.ndarray, k_h: int, k_l: int) -> np.ndarray:
     if k_l > 0:
         np.put_along_axis(lab, order[..., n_kv - k_l:], np.int8(-1), axis=-1)
     return lab
+
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """Logistic function 1 / (1 + e^-z) in fp64, written per sign so that
+    neither branch overflows."""
+    z = np.asarray(z, dtype=np.float64)
+    out = np.empty_like(z)
+    pos = z >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-z[pos]))
+    ez = np.exp(z[~pos])
+    out[~pos] = ez / (1.0 + ez)
+    return out
+
+
+def soft_topk(scores: np.ndarray, k: int, tau: float = 0.1, iters: int = 200):
+    """SoftTop-k of the router map, the differentiable stand-in for the hard
+    Top-k during the router's first training stage [SLA2-deep §06]:
+    M[i, j] = sigmoid(P_c[i, j] / tau + lambda_i), with tau = 0.1 on the pages
+    and lambda_i found by bisection so that each row's soft selections sum to
+    the budget k.
+
+    The row sum is strictly increasing in lambda, from 0 to n, so for
+    0 < k < n the root is unique.  The bracket starts at
+    [-max(s)/tau - 40, -min(s)/tau + 40], where the sum is below n * e^-40
+    and above n - n * e^-40, and the interval is halved `iters` times (fp64).
+    k <= 0 gives M = 0 (lambda = -inf), k >= n gives M = 1 (lambda = +inf).
+    scores: [..., n]; returns (M float64 [..., n], lambda float64 [...])."""
+    x = np.asarray(scores, dtype=np.float64) / tau
+    n = x.shape[-1]
+    lead = x.shape[:-1]
+    if k <= 0:
+        return np.zeros(x.shape), np.full(lead, -np.inf)
+    if k >= n:
+        return np.ones(x.shape), np.full(lead, np.inf)
+    lo = -x.max(axis=-1) - 40.0
+    hi = -x.min(axis=-1) + 40.0
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        f = sigmoid(x + mid[..., None]).sum(axis=-1)
+        below = f < k
+        lo = np.where(below, mid, lo)
+        hi = np.where(below, hi, mid)
+    lam = 0.5 * (lo + hi)
+    return sigmoid(x + lam[..., None]), lam
 
 
 def route(q, k, wq, wk, bq, bkv, mode="sla2", k_keep=0, k_neg=0):

@@ -532,6 +532,76 @@ def pin_fp8_tile_width_moves_quantisation(orc):
     assert 0.0 < d < 0.1, d
 
 
+# ---------------------------------------------------------------- SoftTop-k pins
+# "SLA2 深度解读 …" (jefxiong.cn) §06 Stage 1: SoftTop-k(P_c)_ij = sigmoid(P_c_ij / tau
+# + lambda_i), tau = 0.1, lambda_i by bisection so the row's soft selections sum to
+# the budget.
+
+def pin_soft_topk_two_blocks_closed_form(orc):
+    """n = 2, k = 1: sigmoid(a + l) + sigmoid(b + l) = 1 has the root
+    l = -(a + b) / 2 (as sigmoid(u) + sigmoid(-u) = 1), so the mask is
+    [1 / (1 + e^{-(a-b)/2}), 1 / (1 + e^{(a-b)/2})] with a, b = s / tau."""
+    for s0, s1, tau in ((0.3, -0.2, 0.1), (1.5, 1.4, 0.1), (-2.0, 0.7, 0.5)):
+        m, lam = orc.soft_topk(np.array([[s0, s1]]), 1, tau=tau)
+        a, b = s0 / tau, s1 / tau
+        want = [1.0 / (1.0 + math.exp(-(a - b) / 2)), 1.0 / (1.0 + math.exp((a - b) / 2))]
+        assert np.allclose(m[0], want, rtol=0, atol=1e-12), (m, want)
+        assert abs(lam[0] + (a + b) / 2) < 1e-9, (lam, a, b)
+
+
+def pin_soft_topk_equal_scores(orc):
+    """All scores equal: by symmetry every block gets k / n, and
+    lambda = log(k / (n - k)) - s / tau."""
+    for n, k, sv in ((512, 15, 0.37), (16, 4, -1.2), (7, 6, 0.0)):
+        m, lam = orc.soft_topk(np.full((2, n), sv), k)
+        assert np.allclose(m, k / n, rtol=0, atol=1e-12), m[0, :3]
+        assert np.allclose(lam, math.log(k / (n - k)) - sv / 0.1, rtol=0, atol=1e-9), lam
+
+
+def pin_soft_topk_budget_and_order(orc):
+    """Random rows: the soft selections sum to k, lie in (0, 1) and keep the
+    order of the scores."""
+    s = _rand((6, 200), 301, scale=0.4)
+    for k in (1, 6, 50, 199):
+        m, _ = orc.soft_topk(s, k)
+        assert np.allclose(m.sum(axis=-1), k, rtol=0, atol=1e-9), m.sum(axis=-1)
+        assert (m > 0).all() and (m < 1).all()
+        for r in range(s.shape[0]):
+            o = np.argsort(s[r])
+            assert (np.diff(m[r][o]) >= 0).all()
+
+
+def pin_soft_topk_hard_limit(orc):
+    """As tau -> 0 the soft mask becomes the hard Top-k: rows whose k best
+    scores are >= 1 and the rest <= 0 give ~1 on the hard Top-k set and ~0
+    elsewhere at tau = 1e-3."""
+    g = np.random.default_rng(302)
+    n, k = 40, 7
+    s = np.empty((5, n))
+    for r in range(5):
+        idx = g.permutation(n)
+        s[r, idx[:k]] = 1.0 + g.random(k)
+        s[r, idx[k:]] = -g.random(n - k)
+    m, _ = orc.soft_topk(s, k, tau=1e-3)
+    hard = np.zeros((5, n))
+    np.put_along_axis(hard, orc.topk_blocks(s, k).astype(np.int64), 1.0, axis=-1)
+    assert np.abs(m - hard).max() < 1e-6, np.abs(m - hard).max()
+
+
+def pin_soft_topk_edges_and_shift(orc):
+    """k = 0 selects nothing, k = n everything; adding c to a row leaves the
+    mask unchanged and moves lambda by -c / tau."""
+    s = _rand((3, 30), 303)
+    m0, l0 = orc.soft_topk(s, 0)
+    mn, ln = orc.soft_topk(s, 30)
+    assert (m0 == 0).all() and np.isneginf(l0).all()
+    assert (mn == 1).all() and np.isposinf(ln).all()
+    m, lam = orc.soft_topk(s, 9)
+    m2, lam2 = orc.soft_topk(s + 2.5, 9)
+    assert np.allclose(m, m2, rtol=0, atol=1e-10)
+    assert np.allclose(lam2, lam - 25.0, rtol=0, atol=1e-8)
+
+
 ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
             pin_fp8_k_smoothing, pin_fp8_block_scales, pin_fp8_tile_width_exact_without_quantisation,
             pin_fp8_tile_width_moves_quantisation,
@@ -540,4 +610,6 @@ ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, p
     pin_all_kept_is_full_attention, pin_masked_mass_identity, pin_nothing_kept_is_linear_attention,
     pin_bruteforce_sla2, pin_bruteforce_sla, pin_total_minus_kept, pin_closed_forms,
     pin_sla_special_cases, pin_e4m3_codec,
+    pin_soft_topk_two_blocks_closed_form, pin_soft_topk_equal_scores, pin_soft_topk_budget_and_order,
+    pin_soft_topk_hard_limit, pin_soft_topk_edges_and_shift,
 ]

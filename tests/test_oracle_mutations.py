@@ -41,6 +41,11 @@ MUTATIONS = {
     "fp8_tile_width_ignored": ("for g0 in range(0, len(sel), kv_tile):", "for g0 in range(0, len(sel), kv_tile):\n                kv_tile = 1"),
     "fp8_key_scale_of_row_block": ("kdq = k8[keys] * sk[tok_q[keys]][:, None]",
                                    "kdq = k8[keys] * sk[tok_q[rows[0]]]"),
+    "soft_topk_tau_ignored": ("x = np.asarray(scores, dtype=np.float64) / tau",
+                              "x = np.asarray(scores, dtype=np.float64)"),
+    "soft_topk_bisection_backwards": ("lo = np.where(below, mid, lo)\n        hi = np.where(below, hi, mid)",
+                                      "lo = np.where(below, lo, mid)\n        hi = np.where(below, mid, hi)"),
+    "sigmoid_sign_flipped": ("out[pos] = 1.0 / (1.0 + np.exp(-z[pos]))", "out[pos] = 1.0 / (1.0 + np.exp(z[pos]))"),
 }
 
 
