@@ -178,6 +178,68 @@ class OracleTimer:
         return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
 
 
+def soft_topk_leg(args, w, dev, stream):
+    """SoftTop-k router forward [SLA2-deep §06] through sla_route_soft at the
+    same workload: ms per call with Q, K resident, and its roofline.  The
+    sigmoids run on the special-function unit (an exponential and a
+    reciprocal each), so the bound is that unit: 16 operations per SM per clock
+    = 8 sigmoids, times 148 SMs and the sampled SM clock.  Work per row =
+    (bisection iterations + 1) x n_kv sigmoids; the fp32 bisection halves the
+    bracket [-max(s/tau) - 40, -min(s/tau) + 40] until its midpoint stops
+    moving, i.e. about log2(bracket / ulp(lambda)) times, counted from the
+    scores and lambda the library returns."""
+    import numpy as np
+    x = inputs.make_inputs(w)
+    q, kk = x["q"].to(dev), x["k"].to(dev)
+    wq, wk = x["wq"].to(dev), x["wk"].to(dev)
+    k, tau = keep_of(w), 0.1
+    shape = sla.make_shape(q, w.bq, w.bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, sla.SLA_MODE_SLA2_TOPK), dtype=torch.uint8, device=dev)
+    mask = torch.empty(w.B, w.H, w.n_q, w.n_kv, dtype=torch.float32, device=dev)
+    lam = torch.empty(w.B, w.H, w.n_q, dtype=torch.float32, device=dev)
+    kept = torch.empty(w.B, w.H, w.n_q, k, dtype=torch.int32, device=dev)
+    scores = torch.empty(w.B, w.H, w.n_q, w.n_kv, dtype=torch.float32, device=dev)
+    sla.sla_route(shape, q, kk, wq, wk, sla.SLA_MODE_SLA2_TOPK, k, 0, kept, None, scores, ws, stream)
+    for _ in range(args.warmup):
+        sla.sla_route_soft(shape, q, kk, wq, wk, k, tau, mask, lam, ws, stream)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        sla.sla_route_soft(shape, q, kk, wq, wk, k, tau, mask, lam, ws, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if sla.sla_read_device_status(ws, stream) != 0:
+        raise SystemExit("device-side error during the timed calls")
+    ms = t0.elapsed_time(t1) / args.steps
+    xs = (scores.cpu().numpy() / np.float32(tau)).astype(np.float32)
+    width = (-xs.min(-1) + 40.0) - (-xs.max(-1) - 40.0)
+    ulp = np.spacing(np.abs(lam.cpu().numpy()).astype(np.float32)).astype(np.float64)
+    iters = np.ceil(np.log2(width / ulp))
+    sig = float(((iters + 1.0) * w.n_kv).sum())
+    mhz = clk.get("sm_mhz") or 1965.0
+    peak = 148 * 8 * mhz * 1e6
+    achieved = sig / (ms * 1e-3)
+    print(json.dumps({
+        "metric": "SoftTop-k router forward ms @Wan-1.3B shape (sla_route_soft, tau = 0.1)", "value": ms,
+        "unit": "ms per call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": False, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
+                               f"budget={k}/{w.n_kv} key blocks"},
+        "roofline": {"bound": "alu", "achieved": achieved / 1e9, "peak": peak / 1e9, "unit": "G sigmoid/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": "special-function unit: 16 ops per SM per clock, 2 per sigmoid, 148 SMs",
+                     "algorithmic": "n_kv sigmoids per bisection probe and per row; mean probes per row "
+                                    f"{float(iters.mean()):.1f}"},
+        "gpu_launches": 2 * args.steps, "clocks": clk,
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -188,6 +250,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soft-topk", action="store_true",
+                    help="time the SoftTop-k router (sla_route_soft) instead of the forward step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -233,6 +297,10 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
+    if args.soft_topk:
+        if world == 1:
+            soft_topk_leg(args, w, dev, stream)
+        return
 
     x = inputs.make_inputs(w)
     k = keep_of(w)

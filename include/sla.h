@@ -126,6 +126,25 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k,
                      float* scores_dbg, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* SoftTop-k router mask, the differentiable stand-in for the hard Top-k while
+ * the router is trained [SLA2-deep §06, Stage 1]:
+ *   M[i,j] = sigmoid(s[i,j] / tau + lambda_i)
+ * with s the router scores exactly as sla_route computes them (same kernels,
+ * same bits) and lambda_i found by bisection so that sum_j M[i,j] = k_keep
+ * (the row's budget; the pages use tau = 0.1).  fp32: x = s / tau, the
+ * bracket [-max(x) - 40, -min(x) + 40], halved until its midpoint no longer
+ * moves; k_keep == 0 gives M = 0 (lambda = -inf), k_keep == n_kv gives M = 1
+ * (lambda = +inf).
+ * Outputs (device, caller-owned):
+ *   mask   fp32 [B,H,n_q,n_kv]
+ *   lambda fp32 [B,H,n_q] (nullable)
+ * tau must be positive and finite; 0 <= k_keep <= n_kv <= 2048.  Same
+ * workspace and argument rules as sla_route. */
+sla_status sla_route_soft(const sla_shape* shape, const void* q, const void* k,
+                          const float* Wq, const float* Wk, int k_keep, float tau,
+                          float* mask, float* lambda, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* Router without a workspace.  The pages have no counterpart to this entry
  * point: it exists for callers that cannot give the library device memory,
  * for example code that runs under another framework's memory manager and

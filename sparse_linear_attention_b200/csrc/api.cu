@@ -205,6 +205,26 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k, const
   return e == cudaSuccess ? SLA_OK : cuda_fail(e, "route");
 }
 
+sla_status sla_route_soft(const sla_shape* shape, const void* q, const void* k, const float* Wq, const float* Wk,
+                          int k_keep, float tau, float* mask, float* lambda, void* ws, size_t ws_bytes,
+                          void* stream) {
+  sla_status s = check_shape(shape);
+  if (s != SLA_OK) return s;
+  if (q == nullptr || k == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Q or K is null");
+  if (mask == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "mask is null");
+  if (!(tau > 0.0f) || !(tau < INFINITY)) return arg_fail(SLA_ERR_INVALID_ARG, "tau must be positive and finite");
+  if (!aligned16(q) || !aligned16(k)) return arg_fail(SLA_ERR_ALIGNMENT, "Q, K must be 16-byte aligned");
+  if (!aligned16(Wq) || !aligned16(Wk)) return arg_fail(SLA_ERR_ALIGNMENT, "Wq, Wk must be 16-byte aligned");
+  const int nkv = ceil_div(shape->N, shape->bkv);
+  if (nkv > kMaxNKV) return arg_fail(SLA_ERR_UNSUPPORTED, "router needs n_kv <= 2048");
+  if (k_keep < 0 || k_keep > nkv) return arg_fail(SLA_ERR_INVALID_ARG, "k_keep");
+  if ((s = check_ws(shape, SLA_MODE_SLA2_TOPK, ws, ws_bytes)) != SLA_OK) return s;
+  const WsLayout L = ws_layout(*shape, SLA_MODE_SLA2_TOPK);
+  cudaError_t e = launch_route(*shape, q, k, Wq, Wk, SLA_MODE_SLA2_TOPK, k_keep, 0, nullptr, nullptr, nullptr, L,
+                               static_cast<char*>(ws), static_cast<cudaStream_t>(stream), tau, mask, lambda);
+  return e == cudaSuccess ? SLA_OK : cuda_fail(e, "route_soft");
+}
+
 sla_status sla_prepare(const sla_shape* shape, const void* k, const void* v, int phi, void* ws, size_t ws_bytes,
                        void* stream) {
   sla_status s = check_shape(shape);

@@ -142,7 +142,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const float
                                                            int kstride, int d, int mode, int k_keep, int k_neg,
                                                            int32_t* __restrict__ kept_idx,
                                                            int8_t* __restrict__ labels,
-                                                           float* __restrict__ scores_dbg) {
+                                                           float* __restrict__ scores_dbg, float tau,
+                                                           float* __restrict__ soft_mask,
+                                                           float* __restrict__ soft_lambda) {
   extern __shared__ __align__(16) float sm[];
   float* qsT = sm;                                         // [128 channels][8 rows]
   float* kbuf = qsT + kDPad * kScoreRows;                  // kScoreStages x [kScoreC][kScoreKeys]
@@ -213,6 +215,67 @@ __global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const float
   __syncthreads();
 
   const int lane = tid % 32, warp = tid / 32;
+  if (soft_mask != nullptr) {
+    // SoftTop-k: M = sigmoid(s / tau + lambda), lambda by bisection so that the
+    // row's soft selections sum to k_keep (fp32).  The bracket
+    // [-max(x) - 40, -min(x) + 40] holds the root; the bisection stops when the
+    // midpoint no longer moves.  The row sum of each probe is broadcast from
+    // lane 0, so every lane takes the same branch.
+    auto sig = [](float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); };  // 0 when e^-z overflows
+    for (int r = warp; r < kScoreRows; r += kScoreThreads / 32) {
+      const int row = r0 + r;
+      if (row >= nq) break;
+      const float* srow = sc + r * kstride;
+      const long long grow = bh * nq + row;
+      const int nvl = nkv > lane ? (nkv - lane + 31) / 32 : 0;
+      float x[kKPL];
+      float xmax = -INFINITY, xmin = INFINITY;
+#pragma unroll
+      for (int t = 0; t < kKPL; ++t) {
+        x[t] = 0.0f;
+        if (t < nvl) {
+          const float sv = srow[lane + 32 * t];
+          if (scores_dbg) scores_dbg[grow * nkv + lane + 32 * t] = sv;
+          x[t] = __fdiv_rn(sv, tau);
+          xmax = fmaxf(xmax, x[t]);
+          xmin = fminf(xmin, x[t]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, o));
+        xmin = fminf(xmin, __shfl_xor_sync(0xffffffffu, xmin, o));
+      }
+      float lam = k_keep <= 0 ? -INFINITY : INFINITY;
+      if (k_keep > 0 && k_keep < nkv) {
+        const float kf = static_cast<float>(k_keep);
+        float lo = -xmax - 40.0f, hi = -xmin + 40.0f;
+        for (int it = 0; it < 256; ++it) {
+          const float mid = 0.5f * (lo + hi);
+          if (mid == lo || mid == hi) break;
+          float f = 0.0f;
+#pragma unroll
+          for (int t = 0; t < kKPL; ++t)
+            if (t < nvl) f += sig(x[t] + mid);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+          f = __shfl_sync(0xffffffffu, f, 0);
+          if (f < kf) lo = mid;
+          else hi = mid;
+        }
+        lam = 0.5f * (lo + hi);
+      }
+#pragma unroll
+      for (int t = 0; t < kKPL; ++t) {
+        if (t < nvl) {
+          const float m = k_keep <= 0 ? 0.0f : (k_keep >= nkv ? 1.0f : sig(x[t] + lam));
+          soft_mask[grow * nkv + lane + 32 * t] = m;
+        }
+      }
+      if (lane == 0 && soft_lambda != nullptr) soft_lambda[grow] = lam;
+    }
+    return;
+  }
   for (int r = warp; r < kScoreRows; r += kScoreThreads / 32) {
     const int row = r0 + r;
     if (row >= nq) break;
@@ -314,7 +377,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const float
 
 cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const float* Wq, const float* Wk,
                          int mode, int k_keep, int k_neg, int32_t* kept_idx, int8_t* labels,
-                         float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st) {
+                         float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st, float tau,
+                         float* soft_mask, float* soft_lambda) {
   const int BH = s.B * s.H;
   const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
   float* qtT = reinterpret_cast<float*>(ws + L.qt);
@@ -336,7 +400,7 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
       kernel<<<grid, kScoreThreads, smem, st>>>(qtT, ktT, nq, nkv, kt_stride(nkv), s.d, mode, k_keep, k_neg, kept_idx, labels,
-                                      scores_dbg);
+                                      scores_dbg, tau, soft_mask, soft_lambda);
       return cudaSuccess;
     };
     static_assert(kMaxNKV <= 32 * 64, "selection keys per lane");

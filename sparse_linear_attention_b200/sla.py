@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
                 4: "SLA_ERR_WORKSPACE", 5: "SLA_ERR_CUDA", 6: "SLA_ERR_TIMEOUT", 7: "SLA_ERR_DEVICE_INDEX"}
 
 EXPORTS = ("sla_status_string", "sla_last_error_detail", "sla_keep_count", "sla_workspace_size",
-           "sla_workspace_init", "sla_route", "sla_route_noalloc", "sla_prepare", "sla2_attn_fwd", "sla_attn_fwd",
+           "sla_workspace_init", "sla_route", "sla_route_noalloc", "sla_route_soft", "sla_prepare", "sla2_attn_fwd",
+           "sla_attn_fwd",
            "sla_read_device_status")
 
 
@@ -63,6 +64,7 @@ def lib() -> ctypes.CDLL:
         "sla_workspace_init": (i, [vp, sz, vp]),
         "sla_route": (i, [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp]),
         "sla_route_noalloc": (i, [sp, vp, vp, vp, vp, i, i, i, vp, vp, vp, vp]),
+        "sla_route_soft": (i, [sp, vp, vp, vp, vp, i, ctypes.c_float, vp, vp, vp, sz, vp]),
         "sla_prepare": (i, [sp, vp, vp, i, vp, sz, vp]),
         "sla2_attn_fwd": (i, [sp, vp, vp, vp, vp, i, vp, i, u, vp, i, vp, sz, vp]),
         "sla_attn_fwd": (i, [sp, vp, vp, vp, vp, vp, i, u, vp, i, vp, sz, vp]),
@@ -126,6 +128,11 @@ def sla_route_noalloc(shape: Shape, q, k, wq, wk, mode, k_keep, k_neg, kept_idx,
     _check("sla_route_noalloc", lib().sla_route_noalloc(ctypes.byref(shape), _p(q), _p(k), _p(wq), _p(wk), mode,
                                                         k_keep, k_neg, _p(kept_idx), _p(labels), _p(scores_dbg),
                                                         _s(stream)))
+
+
+def sla_route_soft(shape: Shape, q, k, wq, wk, k_keep, tau, mask, lam, ws, stream=None):
+    _check("sla_route_soft", lib().sla_route_soft(ctypes.byref(shape), _p(q), _p(k), _p(wq), _p(wk), k_keep,
+                                                  float(tau), _p(mask), _p(lam), _p(ws), ws.numel(), _s(stream)))
 
 
 def sla_prepare(shape: Shape, k, v, phi, ws, stream=None):

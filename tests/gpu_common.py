@@ -39,6 +39,22 @@ def run_route(q, k, wq, wk, bq, bkv, mode, k_keep, k_neg=0):
     return kept.cpu().numpy(), labels.cpu().numpy(), scores.cpu().numpy()
 
 
+def run_route_soft(q, k, wq, wk, bq, bkv, k_keep, tau):
+    """sla_route_soft through the C ABI: (mask [B,H,n_q,n_kv], lambda [B,H,n_q])."""
+    dev = "cuda"
+    qd, kd = q.to(dev), k.to(dev)
+    shape = sla.make_shape(qd, bq, bkv)
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, 0), dtype=torch.uint8, device=dev)
+    mask = torch.full((B, H, nq, nkv), float("nan"), dtype=torch.float32, device=dev)
+    lam = torch.full((B, H, nq), float("nan"), dtype=torch.float32, device=dev)
+    sla.sla_route_soft(shape, qd, kd, None if wq is None else wq.to(dev), None if wk is None else wk.to(dev),
+                       k_keep, tau, mask, lam, ws)
+    assert sla.sla_read_device_status(ws) == 0
+    return mask.cpu().numpy(), lam.cpu().numpy()
+
+
 def run_sla2(q, k, v, kept, alpha, bq, bkv, phi=sla.SLA_PHI_ELU1, out_dtype=torch.float32, flags=0, ws=None):
     dev = "cuda"
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
