@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_linear_attention_b200 import inputs, sla  # noqa: E402
+from sparse_linear_attention_b200 import dist_timing, inputs, sla  # noqa: E402
 
 METRIC = "SLA2 attn fwd ms & effective TOPS @Wan-1.3B shape, 97% sparse; % tensor peak"
 UNIT = "effective TOPS (4*N^2*d*H*B per forward / time)"
@@ -256,9 +256,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_timing.world_info()
     w = inputs.WORKLOADS[args.workload]
     if w.mode != "sla2" or w.fp8:
         raise SystemExit("bench.py times the SLA2 bf16 path; pick wan13, wan14 or tiny")
@@ -336,22 +334,16 @@ def main():
     clocks = ClockSampler(dev.index if world == 1 else local)
     clocks.start()
     time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
+    dist_timing.barrier()
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    dist_timing.barrier()
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = dist_timing.max_over_ranks(t_start.elapsed_time(t_end), dev)
     if sla.sla_read_device_status(ws, stream) != 0:
         raise SystemExit("device-side error during the timed steps")
     route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
@@ -360,7 +352,7 @@ def main():
 
     full_ops, sparse_flop = work_counts(w, kept.cpu())
     ms_step = elapsed_ms / args.steps
-    value = full_ops * world / (ms_step * 1e-3) / 1e12
+    value = dist_timing.job_throughput(full_ops, ms_step, world) / 1e12
 
     hbm, bf16_burst, bf16_sus, peak_src = peaks()
     achieved = sparse_flop / (sparse_ms * 1e-3) / 1e12
@@ -382,20 +374,15 @@ def main():
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    dist_timing.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_val = full_ops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = dist_timing.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+    e2e_val = dist_timing.job_throughput(full_ops, e2e_ms, world) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -408,7 +395,7 @@ def main():
 
     if world > 1:
         dist.destroy_process_group()
-    if rank != 0:
+    if not dist_timing.reports(rank):
         return
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
