@@ -250,6 +250,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--phi", default="elu1", choices=["elu1", "softmax"],
+                    help="linear-branch feature map (the pages' default for SLA2 is ELU+1)")
     ap.add_argument("--soft-topk", action="store_true",
                     help="time the SoftTop-k router (sla_route_soft) instead of the forward step")
     args = ap.parse_args()
@@ -258,8 +260,12 @@ def main():
 
     rank, world, local = dist_timing.world_info()
     w = inputs.WORKLOADS[args.workload]
-    if w.mode != "sla2" or w.fp8:
-        raise SystemExit("bench.py times the SLA2 bf16 path; pick wan13, wan14 or tiny")
+    if w.fp8:
+        raise SystemExit("bench.py times the bf16 path; pick a workload without fp8")
+    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk):
+        raise SystemExit("the reference arm and --soft-topk time the SLA2 router / forward")
+    phi = sla.SLA_PHI_ELU1 if args.phi == "elu1" else sla.SLA_PHI_SOFTMAX
+    sla_mode = w.mode == "sla"
 
     if args.impl == "reference":
         if rank != 0:
@@ -301,25 +307,34 @@ def main():
         return
 
     x = inputs.make_inputs(w)
-    k = keep_of(w)
+    # SLA: k = critical blocks (+1), k_neg negligible (-1) [SLA 关键设计 2]; SLA2: k kept blocks
+    k = sla.sla_keep_count(w.crit_ratio, w.n_kv) if sla_mode else keep_of(w)
+    k_neg = sla.sla_keep_count(w.negl_ratio, w.n_kv) if sla_mode else 0
+    mode = sla.SLA_MODE_SLA_3WAY if sla_mode else sla.SLA_MODE_SLA2_TOPK
     q, kk, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
     wq, wk, alpha = x["wq"].to(dev), x["wk"].to(dev), x["alpha"].to(dev)
+    wproj = x["wproj"].to(dev)
     shape = sla.make_shape(q, w.bq, w.bkv)
-    ws = torch.zeros(sla.sla_workspace_size(shape, sla.SLA_MODE_SLA2_TOPK), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(sla.sla_workspace_size(shape, mode), dtype=torch.uint8, device=dev)
     kept = torch.empty(w.B, w.H, w.n_q, k, dtype=torch.int32, device=dev)
+    labels = torch.empty(w.B, w.H, w.n_q, w.n_kv, dtype=torch.int8, device=dev) if sla_mode else None
     out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
-    launches_per_step = 3 + 2 + 1 + (1 if (w.d != 128 or w.dtype == "f32") else 0)
+    # route 2, prepare 3 (+ Q conversion off the d = 128 bf16 grid), attention 1 (+ SLA label lists 1)
+    launches_per_step = 2 + 3 + 1 + (1 if (w.d != 128 or w.dtype == "f32") else 0) + (1 if sla_mode else 0)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        sla.sla_route(shape, q, kk, wq, wk, sla.SLA_MODE_SLA2_TOPK, k, 0, kept, None, None, ws, stream)
+        sla.sla_route(shape, q, kk, wq, wk, mode, k, k_neg, kept, labels, None, ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        sla.sla_prepare(shape, kk, v, sla.SLA_PHI_ELU1, ws, stream)
+        sla.sla_prepare(shape, kk, v, phi, ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        sla.sla2_attn_fwd(shape, q, kk, v, kept, k, alpha, sla.SLA_PHI_ELU1, sla.SLA_FLAG_PREPARED, out, ws, stream)
+        if sla_mode:
+            sla.sla_attn_fwd(shape, q, kk, v, labels, wproj, phi, sla.SLA_FLAG_PREPARED, out, ws, stream)
+        else:
+            sla.sla2_attn_fwd(shape, q, kk, v, kept, k, alpha, phi, sla.SLA_FLAG_PREPARED, out, ws, stream)
         if ev is not None:
             ev[3].record(stream)
 
@@ -360,13 +375,13 @@ def main():
 
     # end to end through the public API: pinned host inputs in, output back out
     hq, hk, hv = (t.pin_memory() for t in (x["q"], x["k"], x["v"]))
-    hwq, hwk, hal = (t.pin_memory() for t in (x["wq"], x["wk"], x["alpha"]))
+    hwq, hwk, hal, hwp = (t.pin_memory() for t in (x["wq"], x["wk"], x["alpha"], x["wproj"]))
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hwq, hwk, hal))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hwq, hwk, hwp if sla_mode else hal))
     d2h = hout.numel() * hout.element_size()
 
     def e2e_step():
-        for dst, src in ((q, hq), (kk, hk), (v, hv), (wq, hwq), (wk, hwk), (alpha, hal)):
+        for dst, src in ((q, hq), (kk, hk), (v, hv), (wq, hwq), (wk, hwk), (wproj, hwp) if sla_mode else (alpha, hal)):
             dst.copy_(src, non_blocking=True)
         step()
         hout.copy_(out, non_blocking=True)
@@ -385,7 +400,7 @@ def main():
     e2e_val = dist_timing.job_throughput(full_ops, e2e_ms, world) / 1e12
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not sla_mode and phi == sla.SLA_PHI_ELU1:
         ot = OracleTimer(w, x)
         while ot.t_att < args.cpu_budget or ot.blocks < 4:
             ot.one_block()
@@ -404,7 +419,9 @@ def main():
         "config": {"workload": f"{w.name}: Wan2.1-1.3B-480P latent shape" if w.name == "wan13" else w.name,
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bkv": w.bkv,
                    "kept_blocks": f"{k}/{w.n_kv} per query block ({100.0 * (1 - k / w.n_kv):.2f}% sparse)",
-                   "phi": "elu+1", "global_batch": w.B * world,
+                   "phi": "elu+1" if phi == sla.SLA_PHI_ELU1 else "softmax over channels",
+                   "method": "SLA (critical / marginal / negligible, O_s + Proj(O_l))" if sla_mode
+                   else "SLA2 (top-k, alpha mix)", "global_batch": w.B * world,
                    "l2": "no flush: Q,K,V = %.0f MB per rank > 126 MB L2" % (3 * q.numel() * 2 / 1e6)},
         "breakdown_ms": {"route": route_ms, "prepare": prep_ms, "sparse_attention": sparse_ms},
         "sparse_tflops_executed": achieved,

@@ -227,6 +227,14 @@ def test_sla_wan13_sampled_blocks():
     _sla_check(w, x, lab, blocks=sample_blocks(w.B, w.H, w.n_q, 3, seed=2))
 
 
+def test_sla_64x64_sampled_blocks():
+    """SLA at the block sizes of its own page: b_q = b_kv = 64."""
+    w, x = workload("sla13_64")
+    kh, kl = orc.keep_count(w.crit_ratio, w.n_kv), orc.keep_count(w.negl_ratio, w.n_kv)
+    _, lab, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 1, kh, kl)
+    _sla_check(w, x, lab, blocks=sample_blocks(w.B, w.H, w.n_q, 3, seed=3))
+
+
 def test_sla_label_edge_cases():
     w, x = _rand_case(700, 128, scale=1.5)
     rng = np.random.default_rng(5)
