@@ -64,6 +64,12 @@ typedef enum { SLA_PHI_ELU1 = 0, SLA_PHI_SOFTMAX = 1 } sla_phi;
  * critical / marginal / negligible [SLA 关键设计 2]. */
 typedef enum { SLA_MODE_SLA2_TOPK = 0, SLA_MODE_SLA_3WAY = 1 } sla_route_mode;
 
+/* OR into sla_route's mode: take the key-block means from ws, where
+ * sla_prepare wrote them while it streamed K (bf16 inputs with d = 128 only),
+ * instead of reading K again.  Same arithmetic, so the same bits; sla_prepare
+ * must have run on these K and this ws, earlier on the same stream. */
+#define SLA_ROUTE_KBAR_FROM_WS 0x10
+
 /* flags for the attention entry points */
 #define SLA_FLAG_PREPARED 1u  /* ws already holds sla_prepare's results for these K, V */
 #define SLA_FLAG_FP8 2u       /* low-bit (e4m3) sparse branch [SLA2-deep §07], SLA2 only */
@@ -119,7 +125,8 @@ sla_status sla_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   kept_idx   int32 [B,H,n_q,k_keep], ascending per row (k_keep may be 0)
  *   labels     int8  [B,H,n_q,n_kv] (nullable): SLA2 1/0; SLA +1/0/-1
  *   scores_dbg fp32  [B,H,n_q,n_kv] (nullable): the raw scores s
- * Requires n_kv <= 2048 and k_keep + k_neg <= n_kv (k_neg = 0 for SLA2). */
+ * Requires n_kv <= 2048 and k_keep + k_neg <= n_kv (k_neg = 0 for SLA2).
+ * mode may carry SLA_ROUTE_KBAR_FROM_WS (bf16, d = 128; else UNSUPPORTED). */
 sla_status sla_route(const sla_shape* shape, const void* q, const void* k,
                      const float* Wq, const float* Wk, int mode, int k_keep,
                      int k_neg, int32_t* kept_idx, int8_t* labels,

@@ -189,7 +189,11 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k, const
                      void* ws, size_t ws_bytes, void* stream) {
   sla_status s = check_shape(shape);
   if (s != SLA_OK) return s;
+  const bool kbar_ws = (mode & SLA_ROUTE_KBAR_FROM_WS) != 0;
+  mode &= ~SLA_ROUTE_KBAR_FROM_WS;
   if (mode != SLA_MODE_SLA2_TOPK && mode != SLA_MODE_SLA_3WAY) return arg_fail(SLA_ERR_INVALID_ARG, "mode");
+  if (kbar_ws && (shape->in_dtype != SLA_BF16 || shape->d != kDPad))
+    return arg_fail(SLA_ERR_UNSUPPORTED, "SLA_ROUTE_KBAR_FROM_WS needs bf16 inputs with d = 128");
   if (q == nullptr || k == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Q or K is null");
   if (!aligned16(q) || !aligned16(k)) return arg_fail(SLA_ERR_ALIGNMENT, "Q, K must be 16-byte aligned");
   if (!aligned16(Wq) || !aligned16(Wk)) return arg_fail(SLA_ERR_ALIGNMENT, "Wq, Wk must be 16-byte aligned");
@@ -200,8 +204,10 @@ sla_status sla_route(const sla_shape* shape, const void* q, const void* k, const
   if (k_keep > 0 && kept_idx == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "kept_idx is null");
   if ((s = check_ws(shape, SLA_MODE_SLA2_TOPK, ws, ws_bytes)) != SLA_OK) return s;
   const WsLayout L = ws_layout(*shape, SLA_MODE_SLA2_TOPK);
-  cudaError_t e = launch_route(*shape, q, k, Wq, Wk, mode, k_keep, k_neg, kept_idx, labels, scores_dbg, L,
-                               static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+  char* w = static_cast<char*>(ws);
+  cudaError_t e = launch_route(*shape, q, k, Wq, Wk, mode, k_keep, k_neg, kept_idx, labels, scores_dbg, L, w,
+                               static_cast<cudaStream_t>(stream), 0.0f, nullptr, nullptr,
+                               kbar_ws ? reinterpret_cast<const float*>(w + L.kbar) : nullptr);
   return e == cudaSuccess ? SLA_OK : cuda_fail(e, "route");
 }
 

@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_tma_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __grid_constant__ CUtensorMap tmPhiOut, const __grid_constant__ CUtensorMap tmVOut,
     float* __restrict__ hpart, float* __restrict__ zpart, float* __restrict__ zblk, float* __restrict__ kstat,
-    float* __restrict__ vstat, int N, int nkv, int nsplit, int phi_kind, int* status) {
+    float* __restrict__ vstat, float* __restrict__ kbar, int N, int nkv, int nsplit, int phi_kind, int* status) {
   extern __shared__ __align__(1024) uint8_t sm[];
   if ((smem_u32(sm) & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned window
     if (threadIdx.x == 0) report_error(status, SLA_ERR_UNSUPPORTED);
@@ -427,6 +427,23 @@ __global__ void __launch_bounds__(kPreThreads, 2) lin_prepass_tma_kernel(
     ok = ok && mbar_wait(&full[stg], (it / kStagesP) & 1, abort_flag, status);
     ok = __syncthreads_and(ok) != 0;  // CTA-uniform verdict
     if (!ok) break;
+    {
+      // The router's mean of key block jb [SLA2-deep §05], from the raw K tile
+      // before it turns into phi(K) in place: channel tid, the block's tokens in
+      // ascending order from +0.0 in fp32, then one division by their count
+      // (the same arithmetic as the router's own pooling).
+      if (tid < 128) {
+        const int cnt = min(64, N - jb * 64);
+        const uint32_t cb = (tid >> 6) * 8192u + ((tid & 7) << 1);
+        const int u8 = (tid >> 3) & 7;
+        float acc = 0.0f;
+#pragma unroll 8
+        for (int t = 0; t < cnt; ++t)
+          acc = __fadd_rn(acc, __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sk + cb + sw128_off(t, u8))));
+        kbar[(static_cast<long long>(bh) * nkv + jb) * 128 + tid] = __fdiv_rn(acc, static_cast<float>(cnt));
+      }
+      __syncthreads();  // every column is summed before the tile is converted
+    }
     float csum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // this thread's rows, rounded phi(K)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -811,7 +828,8 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
     if (e != cudaSuccess) return e;
     lin_prepass_tma_kernel<<<grid, kPreThreads, kTPreSmem, st>>>(
         mk, mv, mpo, mvo, hpart, zpart, reinterpret_cast<float*>(ws + L.zblk), reinterpret_cast<float*>(ws + L.kstat),
-        reinterpret_cast<float*>(ws + L.vstat), s.N, nkv, L.nsplit, phi, status);
+        reinterpret_cast<float*>(ws + L.vstat), reinterpret_cast<float*>(ws + L.kbar), s.N, nkv, L.nsplit, phi,
+        status);
   } else if (s.in_dtype == SLA_BF16) {
     e = cudaFuncSetAttribute(lin_prepass_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kPreSmem);

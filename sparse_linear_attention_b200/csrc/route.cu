@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
                                                            const float* __restrict__ Wq,
                                                            const float* __restrict__ Wk,
                                                            float* __restrict__ qtT, float* __restrict__ ktT,
-                                                           int N, int d, int bq, int bkv, int kstride) {
+                                                           const float* __restrict__ kbar, int N, int d, int bq,
+                                                           int bkv, int kstride) {
   constexpr int VPU = 16 / sizeof(T);  // channels per 16-byte unit
   const bool isK = blockIdx.z == 1;
   const T* x = isK ? k : q;
@@ -52,6 +53,13 @@ __global__ void __launch_bounds__(256) pool_project_kernel(const T* __restrict__
   __shared__ __align__(16) float xs[kPPRows][kDPad];
   const int tid = threadIdx.x;
   const int upr = d / VPU;
+  if (isK && kbar != nullptr) {
+    // the key-block means from the prepass (same arithmetic, K read only once)
+    for (int i = tid; i < kPPRows * d; i += 256) {
+      const int r = i / d, c = i % d;
+      xs[r][c] = r0 + r < nrows ? kbar[(bh * nrows + r0 + r) * kDPad + c] : 0.0f;
+    }
+  } else
   for (int i = tid; i < kPPRows * upr; i += 256) {
     const int r = i / upr, u = i % upr;
     const int blk = r0 + r;
@@ -378,7 +386,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const float
 cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const float* Wq, const float* Wk,
                          int mode, int k_keep, int k_neg, int32_t* kept_idx, int8_t* labels,
                          float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st, float tau,
-                         float* soft_mask, float* soft_lambda) {
+                         float* soft_mask, float* soft_lambda, const float* kbar) {
   const int BH = s.B * s.H;
   const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
   float* qtT = reinterpret_cast<float*>(ws + L.qt);
@@ -388,10 +396,12 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
     if (s.in_dtype == SLA_BF16)
       pool_project_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                                 static_cast<const __nv_bfloat16*>(k), Wq, Wk,
-                                                                qtT, ktT, s.N, s.d, s.bq, s.bkv, kt_stride(nkv));
+                                                                qtT, ktT, kbar, s.N, s.d, s.bq, s.bkv,
+                                                                kt_stride(nkv));
     else
       pool_project_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                        Wq, Wk, qtT, ktT, s.N, s.d, s.bq, s.bkv, kt_stride(nkv));
+                                                        Wq, Wk, qtT, ktT, kbar, s.N, s.d, s.bq, s.bkv,
+                                                        kt_stride(nkv));
   }
   {
     const size_t smem = score_smem_bytes(kt_stride(nkv));

@@ -25,6 +25,7 @@ struct WsLayout {
   size_t hs16 = 0, ztot = 0;    // fp16 [BH, 128, 128] = H_tot / sigma, fp32 [BH, 128] = Z_tot
   size_t sigma = 0;             // fp32 [BH]: per-head power of two >= max_e Z_tot[e]
   size_t zblk = 0;              // fp32 [BH, n_kv, 128]: colsum of phi(K) per key block
+  size_t kbar = 0;              // fp32 [BH, n_kv, 128]: key-block means for the router (bf16, d = 128 prepass)
   size_t kstat = 0, vstat = 0;  // fp32 [BH, nsplit, 128]: per-split column sum of K, column absmax of V
   // low-bit sparse branch (only with SLA_WS_FP8)
   size_t q8 = 0, k8 = 0, v8 = 0;  // e4m3 [BH, N, 128]: Q, K - mean(K), V
@@ -81,6 +82,7 @@ inline WsLayout ws_layout(const sla_shape& s, int mode_flags) {
   L.ztot = take(BH * kDPad * 4);
   L.sigma = take(BH * 4);
   L.zblk = take(BH * static_cast<size_t>(nkv) * kDPad * 4);
+  L.kbar = take(BH * static_cast<size_t>(nkv) * kDPad * 4);
   L.kstat = take(BH * L.nsplit * kDPad * 4);
   L.vstat = take(BH * L.nsplit * kDPad * 4);
   if (L.fp8) {

@@ -9,11 +9,12 @@
 namespace sla {
 
 // Hard routing (kept_idx / labels) or, when soft_mask is non-null, the SoftTop-k
-// mask and lambda with temperature tau.
+// mask and lambda with temperature tau.  kbar (nullable): the key-block means
+// sla_prepare wrote, used instead of pooling K again.
 cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const float* Wq, const float* Wk,
                          int mode, int k_keep, int k_neg, int32_t* kept_idx, int8_t* labels,
                          float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st, float tau = 0.0f,
-                         float* soft_mask = nullptr, float* soft_lambda = nullptr);
+                         float* soft_mask = nullptr, float* soft_lambda = nullptr, const float* kbar = nullptr);
 
 cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
                            char* ws, cudaStream_t st);

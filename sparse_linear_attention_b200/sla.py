@@ -19,6 +19,7 @@ SLA_OK = 0
 SLA_F32, SLA_BF16 = 0, 1
 SLA_PHI_ELU1, SLA_PHI_SOFTMAX = 0, 1
 SLA_MODE_SLA2_TOPK, SLA_MODE_SLA_3WAY = 0, 1
+SLA_ROUTE_KBAR_FROM_WS = 0x10
 SLA_FLAG_PREPARED, SLA_FLAG_FP8 = 1, 2
 SLA_WS_FP8 = 0x100
 

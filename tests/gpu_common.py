@@ -39,6 +39,25 @@ def run_route(q, k, wq, wk, bq, bkv, mode, k_keep, k_neg=0):
     return kept.cpu().numpy(), labels.cpu().numpy(), scores.cpu().numpy()
 
 
+def run_route_after_prepare(q, k, v, wq, wk, bq, bkv, mode, k_keep, k_neg=0):
+    """sla_prepare, then sla_route with SLA_ROUTE_KBAR_FROM_WS (key-block means
+    from the prepass) on the same workspace."""
+    dev = "cuda"
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    shape = sla.make_shape(qd, bq, bkv)
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, mode), dtype=torch.uint8, device=dev)
+    kept = torch.full((B, H, nq, k_keep), -7, dtype=torch.int32, device=dev)
+    labels = torch.full((B, H, nq, nkv), 9, dtype=torch.int8, device=dev)
+    scores = torch.full((B, H, nq, nkv), float("nan"), dtype=torch.float32, device=dev)
+    sla.sla_prepare(shape, kd, vd, sla.SLA_PHI_ELU1, ws)
+    sla.sla_route(shape, qd, kd, None if wq is None else wq.to(dev), None if wk is None else wk.to(dev),
+                  mode | sla.SLA_ROUTE_KBAR_FROM_WS, k_keep, k_neg, kept, labels, scores, ws)
+    assert sla.sla_read_device_status(ws) == 0
+    return kept.cpu().numpy(), labels.cpu().numpy(), scores.cpu().numpy()
+
+
 def run_route_soft(q, k, wq, wk, bq, bkv, k_keep, tau):
     """sla_route_soft through the C ABI: (mask [B,H,n_q,n_kv], lambda [B,H,n_q])."""
     dev = "cuda"

@@ -8,7 +8,8 @@ import torch
 
 from oracle import sla_oracle as orc
 from sparse_linear_attention_b200 import inputs, sla
-from tests.gpu_common import (TOL_BF16, as32, as64, compare, run_route, run_sla, run_sla2, sample_blocks)
+from tests.gpu_common import (TOL_BF16, as32, as64, compare, run_route, run_route_after_prepare, run_sla, run_sla2,
+                              sample_blocks)
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +80,40 @@ def test_route_bitexact_odd_shapes(N, d, mode):
     assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32)), "scores differ"
     assert np.array_equal(kept, okept)
     assert np.array_equal(lab, olab)
+
+
+@pytest.mark.parametrize("name,mode", [("wan13", 0), ("sla13", 1)])
+def test_route_key_means_from_prepare_bitexact(name, mode):
+    """The router with the key-block means the prepass wrote (K read once):
+    the same bits as the oracle's own pooling."""
+    w, x = workload(name)
+    if mode == 0:
+        kh, kl = k_of(w), 0
+    else:
+        kh, kl = orc.keep_count(w.crit_ratio, w.n_kv), orc.keep_count(w.negl_ratio, w.n_kv)
+    kept, lab, sc = run_route_after_prepare(x["q"], x["k"], x["v"], x["wq"], x["wk"], w.bq, w.bkv, mode, kh, kl)
+    okept, olab, osc = orc.route(as32(x["q"]), as32(x["k"]), x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv,
+                                 "sla" if mode else "sla2", kh, kl)
+    assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32)), "scores differ"
+    assert np.array_equal(kept, okept)
+    assert np.array_equal(lab, olab)
+
+
+def test_route_key_means_from_prepare_ragged():
+    """A ragged last key block (N = 1000: 40 tokens) and no projections."""
+    g = torch.Generator().manual_seed(5)
+    q, k, v = ((torch.randn(1, 2, 1000, 128, generator=g) * 1.5).to(torch.bfloat16) for _ in range(3))
+    kept, lab, sc = run_route_after_prepare(q, k, v, None, None, 128, 64, 0, 4)
+    okept, olab, osc = orc.route(as32(q), as32(k), None, None, 128, 64, "sla2", 4)
+    assert np.array_equal(sc.view(np.uint32), osc.view(np.uint32))
+    assert np.array_equal(kept, okept)
+
+
+def test_route_key_means_from_prepare_needs_bf16_d128():
+    q = torch.zeros(1, 1, 256, 64, dtype=torch.bfloat16)
+    with pytest.raises(sla.SLAError) as e:
+        run_route_after_prepare(q, q, q, None, None, 64, 64, 0, 2)
+    assert e.value.status == 2  # SLA_ERR_UNSUPPORTED
 
 
 def test_route_ties_break_to_lower_index():
