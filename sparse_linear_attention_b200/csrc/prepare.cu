@@ -17,6 +17,9 @@
 // zsum_kernel / hsum_kernel: Z_tot, H_tot = sum of the partials in split
 //   order (fixed, so deterministic); H_tot is stored as fp16 H_tot / sigma
 //   with sigma an exact per-head power of two (see hsum_kernel).
+// lin_prepass_tma_kernel (bf16, d = 128) also writes the router's key-block
+//   means ("SLA2 深度解读 …" §05: pool(K)) while each key block sits in shared
+//   memory, so the router need not read K again (SLA_ROUTE_KBAR_FROM_WS).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
