@@ -92,6 +92,45 @@ def test_route_rejects_bad_arguments_before_launch():
     assert "kept_idx" in sla.lib().sla_last_error_detail().decode()
 
 
+def test_route_key_means_flag_checks():
+    """SLA_ROUTE_KBAR_FROM_WS (key-block means from the prepass) exists only
+    where the prepass writes them: bf16 inputs with d = 128."""
+    flag = sla.SLA_ROUTE_KBAR_FROM_WS
+    assert _route(_shape(d=64), mode=flag) == 2
+    assert _route(_shape(in_dtype=sla.SLA_F32), mode=flag) == 2
+    assert "d = 128" in sla.lib().sla_last_error_detail().decode()
+    assert _route(_shape(), mode=flag | 3) == 1       # the base mode is still checked
+    assert _route(_shape(), mode=flag, kept=None) == 1  # and the other arguments
+    # the route without a workspace takes no flag
+    L = sla.lib()
+    assert L.sla_route_noalloc(ctypes.byref(_shape()), FAKE, FAKE, None, None, flag, 15, 0, FAKE, None, None,
+                               None) == 1
+
+
+def test_route_soft_rejects_bad_arguments_before_launch():
+    s = _shape()
+    L = sla.lib()
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, wq=None, k_keep=15, tau=0.1, mask=FAKE, lam=None, ws=FAKE, wsb=1 << 40)
+        a.update(kw)
+        return L.sla_route_soft(ctypes.byref(a.pop("shape", s)), a["q"], a["k"], a["wq"], None, a["k_keep"],
+                                a["tau"], a["mask"], a["lam"], a["ws"], a["wsb"], None)
+
+    assert call(q=None) == 1
+    assert call(mask=None) == 1
+    assert "mask" in L.sla_last_error_detail().decode()
+    for tau in (0.0, -0.1, float("inf"), float("nan")):
+        assert call(tau=tau) == 1, tau
+    assert call(k_keep=-1) == 1
+    assert call(k_keep=513) == 1
+    assert call(q=FAKE + 8) == 3
+    assert call(wq=FAKE + 4) == 3
+    assert call(ws=None) == 1
+    assert call(wsb=1000) == 4
+    assert call(shape=_shape(N=131072 + 64)) == 2
+
+
 def test_attention_rejects_bad_arguments_before_launch():
     s = _shape()
     L = sla.lib()
