@@ -1,4 +1,5 @@
-"""CPU oracle for the SLA2 / SLA sparse-linear attention forward pass.
+"""CPU oracle for the SLA2 / SLA sparse-linear attention forward pass and its
+gradients.
 
 TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
 CPU-baseline / reference leg may import this module.  The library
@@ -473,3 +474,149 @@ def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None
             out["o_l"][b, h, rows] = o_l
             out["o"][b, h, rows] = a * o_s + (1.0 - a) * o_l
     return out
+
+
+# ----------------------------------------------------------------------------
+# Backward (fp64): gradients of sla2_forward / sla_forward with the block mask
+# held fixed.  [SLA 关键设计 4]: the sparse part returns dQ, dK, dV the way
+# FlashAttention does; the linear part follows the chain rule through dH_i and
+# dZ_i, formed per query block and then spread over the keys that built H_i
+# and Z_i.  [SLA2-deep §07], [SLA2-sum §2.C]: gradients are taken on the
+# original, unquantised inputs, so the low-bit forward has no backward of its
+# own.  The hard Top-k passes no gradient to the router; the stage that trains
+# the router uses SoftTop-k instead [SLA2-deep §06].
+# ----------------------------------------------------------------------------
+
+def phi_backward(x, dphi, kind="elu1"):
+    """dL/dx from dL/dphi(x) for the feature map phi above.  "elu1": phi'(x) is
+    1 for x > 0 and exp(x) otherwise.  "softmax" over the channels of a token:
+    dx = phi * (dphi - sum_c dphi_c phi_c)."""
+    x = np.asarray(x, dtype=F64)
+    if kind == "elu1":
+        return dphi * np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+    if kind == "softmax":
+        p = phi(x, "softmax")
+        return p * (dphi - (dphi * p).sum(axis=-1, keepdims=True))
+    raise ValueError(kind)
+
+
+def sparse_branch_backward(q, k, v, rows, keys, do_s):
+    """Gradients of sparse_branch's O_s for the given rows over the selected
+    keys.  With P the row softmax of S = Q K^T / sqrt(d) and O_s = P V:
+      dV = P^T dO_s,  dP = dO_s V^T,  D = rowsum(dO_s * O_s),
+      dS = P * (dP - D),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
+    No selected key -> O_s = 0 and nothing flows.
+    Returns (dq [rows, d], dk [keys, d], dv [keys, dv])."""
+    d = q.shape[-1]
+    if len(keys) == 0:
+        return np.zeros((len(rows), d)), np.zeros((0, d)), np.zeros((0, v.shape[-1]))
+    s = (q[rows] @ k[keys].T) / math.sqrt(d)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p = p / p.sum(axis=1, keepdims=True)
+    o = p @ v[keys]
+    dv = p.T @ do_s
+    dp = do_s @ v[keys].T
+    D = (do_s * o).sum(axis=1, keepdims=True)
+    ds = p * (dp - D)
+    dq = ds @ k[keys] / math.sqrt(d)
+    dk = ds.T @ q[rows] / math.sqrt(d)
+    return dq, dk, dv
+
+
+def linear_branch_backward(q, k, v, rows, keys, do_l, phi_kind="elu1"):
+    """Gradients of linear_branch's O_l = phi(Q) H / (phi(Q) Z) for the given
+    rows over the given (unselected) keys, through dH and dZ:
+      a = phi(q), num = a H, den = a . Z, O_l = num / den;
+      dnum = dO_l / den,  dden = -rowsum(dO_l * O_l) / den;
+      dphi(q) = dnum H^T + dden Z^T;
+      dH = a^T dnum,  dZ = a^T dden  (sums over the rows);
+      dphi(k_m) = dH v_m + dZ,  dv_m = dH^T phi(k_m)  for every key m;
+    then dq and dk through phi_backward.  No key -> O_l = 0 and nothing flows.
+    Returns (dq [rows, d], dk [keys, d], dv [keys, dv])."""
+    if len(keys) == 0:
+        return np.zeros((len(rows), q.shape[-1])), np.zeros((0, k.shape[-1])), np.zeros((0, v.shape[-1]))
+    pk = phi(k[keys], phi_kind)
+    Hm = pk.T @ v[keys]            # [d, dv]
+    Z = pk.sum(axis=0)             # [d]
+    pq = phi(q[rows], phi_kind)
+    num = pq @ Hm
+    den = pq @ Z
+    o = num / den[:, None]
+    dnum = do_l / den[:, None]
+    dden = -(do_l * o).sum(axis=1) / den
+    dpq = dnum @ Hm.T + dden[:, None] * Z[None, :]
+    dH = pq.T @ dnum               # [d, dv]
+    dZ = pq.T @ dden               # [d]
+    dpk = v[keys] @ dH.T + dZ[None, :]
+    dv = pk @ dH
+    return phi_backward(q[rows], dpq, phi_kind), phi_backward(k[keys], dpk, phi_kind), dv
+
+
+def sla2_backward(q, k, v, kept, alpha, do, bq, bkv, phi_kind="elu1"):
+    """Gradients of sla2_forward's O = alpha*O_s + (1-alpha)*O_l for the
+    upstream gradient do [B,H,N,d], the mask held fixed:
+      dO_s = alpha dO,  dO_l = (1 - alpha) dO,
+      dalpha_i = sum over the rows of query block i of dO * (O_s - O_l).
+    A key's gradient adds up over every query block that reads it: through the
+    sparse branch where its block is kept, through the linear branch elsewhere.
+    Returns dict dq, dk, dv (float64 [B,H,N,d]) and dalpha ([B,H,nq])."""
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    n_kv = -(-N // bkv)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dalpha = np.zeros((B, H, nq))
+    for b in range(B):
+        for h in range(H):
+            qs, ks, vs = q[b, h], k[b, h], v[b, h]
+            for i in range(nq):
+                rows = _rows(i, bq, N)
+                sel = sorted(int(j) for j in kept[b, h, i])
+                uns = [j for j in range(n_kv) if j not in set(sel)]
+                ts, tl = _tokens_of(sel, bkv, N), _tokens_of(uns, bkv, N)
+                a = float(alpha[b, h, i])
+                g = do[b, h, rows]
+                o_s = sparse_branch(qs, ks, vs, rows, ts)
+                o_l = linear_branch(qs, ks, vs, rows, tl, phi_kind)
+                dalpha[b, h, i] = (g * (o_s - o_l)).sum()
+                gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, ts, a * g)
+                dq[b, h, rows] += gq
+                dk[b, h, ts] += gk
+                dv[b, h, ts] += gv
+                gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tl, (1.0 - a) * g, phi_kind)
+                dq[b, h, rows] += gq
+                dk[b, h, tl] += gk
+                dv[b, h, tl] += gv
+    return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dalpha}
+
+
+def sla_backward(q, k, v, labels, wproj, do, bq, bkv, phi_kind="elu1"):
+    """Gradients of sla_forward's O = O_s + O_l Wp for the upstream gradient do,
+    the labels held fixed:  dO_s = dO,  dO_l = dO Wp^T,  dWp = sum over every
+    row of every head of O_l^T dO (Wp is shared).  Critical blocks (+1) take
+    the sparse branch, marginal ones (0) the linear branch, negligible ones
+    (-1) get no gradient.  Returns dict dq, dk, dv and dwproj ([d_in, d_out])."""
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    wp = np.asarray(wproj, dtype=F64)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dwp = np.zeros(wp.shape)
+    for b in range(B):
+        for h in range(H):
+            qs, ks, vs = q[b, h], k[b, h], v[b, h]
+            for i in range(nq):
+                rows = _rows(i, bq, N)
+                lab = labels[b, h, i]
+                tc = _tokens_of([int(j) for j in np.nonzero(lab == 1)[0]], bkv, N)
+                tm = _tokens_of([int(j) for j in np.nonzero(lab == 0)[0]], bkv, N)
+                g = do[b, h, rows]
+                o_l = linear_branch(qs, ks, vs, rows, tm, phi_kind)
+                dwp += o_l.T @ g
+                gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, tc, g)
+                dq[b, h, rows] += gq
+                dk[b, h, tc] += gk
+                dv[b, h, tc] += gv
+                gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tm, g @ wp.T, phi_kind)
+                dq[b, h, rows] += gq
+                dk[b, h, tm] += gk
+                dv[b, h, tm] += gv
+    return {"dq": dq, "dk": dk, "dv": dv, "dwproj": dwp}

@@ -602,6 +602,127 @@ def pin_soft_topk_edges_and_shift(orc):
     assert np.allclose(lam2, lam - 25.0, rtol=0, atol=1e-8)
 
 
+# ---------------------------------------------------------------- backward pins
+# The backward is pinned by central finite differences of the (pinned) forward,
+# by torch autograd on the two limits that are textbook attention, and by sum
+# rules that follow from the forward's structure.
+
+def _bwd_case(seed, N=45, d=8, H=2, bq=16, bkv=8, k_keep=2):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((1, H, N, d)) * 0.8
+    k = g.standard_normal((1, H, N, d)) * 0.8
+    v = g.standard_normal((1, H, N, d))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kept = np.array([[[np.sort(g.choice(nkv, k_keep, replace=False)) for _ in range(nq)] for _ in range(H)]])
+    alpha = g.uniform(0.15, 0.85, (1, H, nq))
+    do = g.standard_normal((1, H, N, d))
+    return q, k, v, kept, alpha, do
+
+
+def _fd_agree(loss, x, grad, n, seed, h=1e-5, tol=1e-6):
+    """Central differences of loss at n sampled entries of x against grad."""
+    idx = np.random.default_rng(seed).choice(x.size, size=min(n, x.size), replace=False)
+    for t in idx:
+        xp, xm = x.copy(), x.copy()
+        xp.flat[t] += h
+        xm.flat[t] -= h
+        fd = (loss(xp) - loss(xm)) / (2.0 * h)
+        assert abs(fd - grad.flat[t]) <= tol * (1.0 + abs(fd)), (int(t), fd, float(grad.flat[t]))
+
+
+def _sla2_fd(orc, kind, seed, n):
+    q, k, v, kept, alpha, do = _bwd_case(seed)
+    bq, bkv = 16, 8
+    gr = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
+
+    def L(q_=q, k_=k, v_=v, a_=alpha):
+        return float((orc.sla2_forward(q_, k_, v_, kept, a_, bq, bkv, kind)["o"] * do).sum())
+    _fd_agree(lambda x: L(q_=x), q, gr["dq"], n, seed + 1)
+    _fd_agree(lambda x: L(k_=x), k, gr["dk"], n, seed + 2)
+    _fd_agree(lambda x: L(v_=x), v, gr["dv"], n, seed + 3)
+    _fd_agree(lambda x: L(a_=x), alpha, gr["dalpha"], alpha.size, seed + 4)
+
+
+def pin_bwd_sla2_finite_differences(orc):
+    """SLA2 gradients (dQ, dK, dV, dalpha) against central differences of the
+    forward, ELU+1 feature map, ragged last blocks."""
+    _sla2_fd(orc, "elu1", 700, 24)
+
+
+def pin_bwd_sla2_softmax_phi_finite_differences(orc):
+    """The same with the softmax feature map."""
+    _sla2_fd(orc, "softmax", 710, 16)
+
+
+def pin_bwd_sla_finite_differences(orc):
+    """SLA gradients (dQ, dK, dV, dW_proj) against central differences, with
+    critical, marginal and negligible blocks in every row."""
+    q, k, v, _, _, do = _bwd_case(720)
+    bq, bkv, nq, nkv = 16, 8, 3, 6
+    g = np.random.default_rng(721)
+    labels = np.zeros((1, 2, nq, nkv), dtype=np.int8)
+    for h, i in np.ndindex(2, nq):
+        perm = g.permutation(nkv)
+        labels[0, h, i, perm[:2]] = 1
+        labels[0, h, i, perm[2:3]] = -1
+    wp = g.standard_normal((8, 8)) / math.sqrt(8)
+    gr = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv)
+
+    def L(q_=q, k_=k, v_=v, w_=wp):
+        return float((orc.sla_forward(q_, k_, v_, labels, w_, bq, bkv)["o"] * do).sum())
+    _fd_agree(lambda x: L(q_=x), q, gr["dq"], 20, 722)
+    _fd_agree(lambda x: L(k_=x), k, gr["dk"], 20, 723)
+    _fd_agree(lambda x: L(v_=x), v, gr["dv"], 20, 724)
+    _fd_agree(lambda x: L(w_=x), wp, gr["dwproj"], 20, 725)
+
+
+def pin_bwd_textbook_limits(orc):
+    """Every block kept with alpha = 1 is softmax attention, no block kept with
+    alpha = 0 is linear attention: their gradients equal torch autograd of
+    those textbook formulas (float64)."""
+    q, k, v, _, _, do = _bwd_case(730)
+    N, bq, bkv, nq, nkv = 45, 16, 8, 3, 6
+    tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)
+    o.backward(torch.from_numpy(do))
+    kept = np.broadcast_to(np.arange(nkv), (1, 2, nq, nkv))
+    gr = orc.sla2_backward(q, k, v, kept, np.ones((1, 2, nq)), do, bq, bkv)
+    for name, t in (("dq", tq), ("dk", tk), ("dv", tv)):
+        assert np.allclose(gr[name], t.grad.numpy(), atol=1e-12, rtol=1e-10), name
+    for kind in ("elu1", "softmax"):
+        tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k, v))
+        if kind == "elu1":
+            fq, fk = torch.nn.functional.elu(tq) + 1, torch.nn.functional.elu(tk) + 1
+        else:
+            fq, fk = torch.softmax(tq, -1), torch.softmax(tk, -1)
+        o = (fq @ (fk.transpose(-1, -2) @ tv)) / (fq @ fk.sum(-2, keepdim=True).transpose(-1, -2))
+        o.backward(torch.from_numpy(do))
+        gr = orc.sla2_backward(q, k, v, np.zeros((1, 2, nq, 0), dtype=np.int32), np.zeros((1, 2, nq)), do,
+                               bq, bkv, kind)
+        for name, t in (("dq", tq), ("dk", tk), ("dv", tv)):
+            assert np.allclose(gr[name], t.grad.numpy(), atol=1e-12, rtol=1e-10), (kind, name)
+
+
+def pin_bwd_sum_rules(orc):
+    """Rules that follow from the forward's structure:
+    - both branches weight the values convexly, so with 0 < k < n_kv the value
+      gradients of a head sum to the sum of its upstream gradients;
+    - with alpha = 1 only the softmax acts, and a common shift of the keys
+      leaves it unchanged, so the key gradients of a head sum to zero;
+    - the softmax feature map ignores a common shift of a token's channels, so
+      with alpha = 0 every row of dQ and of dK sums to zero."""
+    q, k, v, kept, alpha, do = _bwd_case(740)
+    gr = orc.sla2_backward(q, k, v, kept, alpha, do, 16, 8)
+    assert np.allclose(gr["dv"].sum(axis=2), do.sum(axis=2), atol=1e-10)
+    gr = orc.sla2_backward(q, k, v, kept, np.ones_like(alpha), do, 16, 8)
+    assert np.allclose(gr["dk"].sum(axis=2), 0.0, atol=1e-10)
+    assert np.abs(gr["dk"]).max() > 1e-3
+    gr = orc.sla2_backward(q, k, v, kept, np.zeros_like(alpha), do, 16, 8, "softmax")
+    assert np.allclose(gr["dq"].sum(axis=3), 0.0, atol=1e-10)
+    assert np.allclose(gr["dk"].sum(axis=3), 0.0, atol=1e-10)
+    assert np.abs(gr["dq"]).max() > 1e-3 and np.abs(gr["dk"]).max() > 1e-3
+
+
 ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
             pin_fp8_k_smoothing, pin_fp8_block_scales, pin_fp8_tile_width_exact_without_quantisation,
             pin_fp8_tile_width_moves_quantisation,
@@ -612,4 +733,6 @@ ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, p
     pin_sla_special_cases, pin_e4m3_codec,
     pin_soft_topk_two_blocks_closed_form, pin_soft_topk_equal_scores, pin_soft_topk_budget_and_order,
     pin_soft_topk_hard_limit, pin_soft_topk_edges_and_shift,
+    pin_bwd_sla2_finite_differences, pin_bwd_sla2_softmax_phi_finite_differences, pin_bwd_sla_finite_differences,
+    pin_bwd_textbook_limits, pin_bwd_sum_rules,
 ]

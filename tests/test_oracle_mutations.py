@@ -46,6 +46,22 @@ MUTATIONS = {
     "soft_topk_bisection_backwards": ("lo = np.where(below, mid, lo)\n        hi = np.where(below, hi, mid)",
                                       "lo = np.where(below, lo, mid)\n        hi = np.where(below, mid, hi)"),
     "sigmoid_sign_flipped": ("out[pos] = 1.0 / (1.0 + np.exp(-z[pos]))", "out[pos] = 1.0 / (1.0 + np.exp(z[pos]))"),
+    "bwd_softmax_drops_D": ("ds = p * (dp - D)", "ds = p * dp"),
+    "bwd_dq_no_sqrt_d": ("dq = ds @ k[keys] / math.sqrt(d)", "dq = ds @ k[keys]"),
+    "bwd_dk_uses_k": ("dk = ds.T @ q[rows] / math.sqrt(d)", "dk = ds.T @ k[keys] / math.sqrt(d)"),
+    "bwd_dv_from_unnormalised_p": ("dv = p.T @ do_s", "dv = np.exp(s - s.max(axis=1, keepdims=True)).T @ do_s"),
+    "bwd_denominator_sign": ("dden = -(do_l * o).sum(axis=1) / den", "dden = (do_l * o).sum(axis=1) / den"),
+    "bwd_phi_k_drops_dZ": ("dpk = v[keys] @ dH.T + dZ[None, :]", "dpk = v[keys] @ dH.T"),
+    "bwd_phi_q_drops_Z_term": ("dpq = dnum @ Hm.T + dden[:, None] * Z[None, :]", "dpq = dnum @ Hm.T"),
+    "bwd_dH_transposed": ("dv = pk @ dH\n", "dv = pk @ dH.T\n"),
+    "bwd_elu_derivative_one": ("return dphi * np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))", "return dphi"),
+    "bwd_softmax_phi_jacobian_sign": ("return p * (dphi - (dphi * p).sum(axis=-1, keepdims=True))",
+                                      "return p * (dphi + (dphi * p).sum(axis=-1, keepdims=True))"),
+    "bwd_alpha_not_applied": ("sparse_branch_backward(qs, ks, vs, rows, ts, a * g)",
+                              "sparse_branch_backward(qs, ks, vs, rows, ts, g)"),
+    "bwd_dalpha_sign": ("dalpha[b, h, i] = (g * (o_s - o_l)).sum()", "dalpha[b, h, i] = (g * (o_l - o_s)).sum()"),
+    "bwd_sla_proj_not_transposed": ("g @ wp.T, phi_kind)", "g @ wp, phi_kind)"),
+    "bwd_sla_dwproj_transposed": ("dwp += o_l.T @ g", "dwp += g.T @ o_l"),
 }
 
 
