@@ -212,6 +212,33 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k,
                         int phi, unsigned flags, void* out, int out_dtype,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace sla2_attn_bwd needs for this shape (0 for an
+ * invalid shape): the status word, H_tot, Z_tot and their gradients per
+ * (b,h), and a [B,H,N,128] fp32 buffer of key-side sums. */
+size_t sla2_attn_bwd_workspace_size(const sla_shape* shape);
+
+/* Gradients of the SLA2 forward [SLA 关键设计 4; SLA2-deep §07; SLA2-sum §2.C]
+ * for the upstream gradient dout, with the block mask held fixed (the hard
+ * Top-k passes no gradient):
+ *   dO_s = alpha dO, dO_l = (1 - alpha) dO, dalpha_i = sum over the rows of
+ *   query block i of dO . (O_s - O_l); the sparse branch back-propagated as
+ *   FlashAttention does, the linear branch through dH_i, dZ_i formed from the
+ *   totals minus the kept blocks' share.
+ * Inputs q, k, v, kept_idx, k_keep, alpha, phi as for sla2_attn_fwd (kept
+ * indices distinct per row); dout [B,H,N,d] of the input dtype.
+ * Outputs (fp32, caller-owned, fully overwritten): dq, dk, dv [B,H,N,d],
+ *   dalpha [B,H,n_q].  dk, dv and dalpha are accumulated with atomic adds
+ *   after a zero fill, so their last bits can differ between runs.
+ * ws: its own workspace of sla2_attn_bwd_workspace_size bytes, 256-byte
+ *   aligned, status word zeroed once (sla_workspace_init); the call zeroes
+ *   the rest itself.  Out-of-range block indices are skipped and reported in
+ *   the status word (sla_read_device_status). */
+sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k,
+                         const void* v, const int32_t* kept_idx, int k_keep,
+                         const float* alpha, int phi, const void* dout,
+                         float* dq, float* dk, float* dv, float* dalpha,
+                         void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, then return (and clear) the device status word that
  * kernels write when a bounded wait runs out or a block index is out of
  * range.  SLA_OK when no device error happened. */

@@ -39,6 +39,15 @@ struct WsLayout {
   bool need_hat = false;
 };
 
+// Workspace of the backward (sla2_attn_bwd): status word first, as in WsLayout.
+struct BwdLayout {
+  size_t status = 0;
+  size_t htot = 0, ztot = 0;    // fp32 [BH, 128, 128], [BH, 128]: H_tot, Z_tot
+  size_t dhtot = 0, dztot = 0;  // fp32 [BH, 128, 128], [BH, 128]: their gradients
+  size_t dphik = 0;             // fp32 [BH, N, 128]: kept blocks' share of dL/dphi(K)
+  size_t total = 0;
+};
+
 // Record the one-line detail that sla_last_error_detail() returns.
 void set_error_detail(const char* msg);
 

@@ -16,6 +16,14 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                          float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st, float tau = 0.0f,
                          float* soft_mask = nullptr, float* soft_lambda = nullptr, const float* kbar = nullptr);
 
+BwdLayout bwd_layout(const sla_shape& s);
+
+// Gradients of the SLA2 forward (backward.cu): zeroes dk, dv, dalpha and the
+// workspace sums, then runs the three backward kernels on st.
+cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                            const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
+                            float* dv, float* dalpha, char* ws, cudaStream_t st);
+
 cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
                            char* ws, cudaStream_t st);
 

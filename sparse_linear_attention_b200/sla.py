@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 
 EXPORTS = ("sla_status_string", "sla_last_error_detail", "sla_keep_count", "sla_workspace_size",
            "sla_workspace_init", "sla_route", "sla_route_noalloc", "sla_route_soft", "sla_prepare", "sla2_attn_fwd",
-           "sla_attn_fwd",
+           "sla_attn_fwd", "sla2_attn_bwd_workspace_size", "sla2_attn_bwd",
            "sla_read_device_status")
 
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         "sla_prepare": (i, [sp, vp, vp, i, vp, sz, vp]),
         "sla2_attn_fwd": (i, [sp, vp, vp, vp, vp, i, vp, i, u, vp, i, vp, sz, vp]),
         "sla_attn_fwd": (i, [sp, vp, vp, vp, vp, vp, i, u, vp, i, vp, sz, vp]),
+        "sla2_attn_bwd_workspace_size": (sz, [sp]),
+        "sla2_attn_bwd": (i, [sp, vp, vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sla_read_device_status": (i, [vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -151,6 +153,16 @@ def sla_attn_fwd(shape: Shape, q, k, v, labels, wproj, phi, flags, out, ws, stre
     out_dt = _dtype_code(out)
     _check("sla_attn_fwd", lib().sla_attn_fwd(ctypes.byref(shape), _p(q), _p(k), _p(v), _p(labels), _p(wproj), phi,
                                               flags, _p(out), out_dt, _p(ws), ws.numel(), _s(stream)))
+
+
+def sla2_attn_bwd_workspace_size(shape: Shape) -> int:
+    return lib().sla2_attn_bwd_workspace_size(ctypes.byref(shape))
+
+
+def sla2_attn_bwd(shape: Shape, q, k, v, kept_idx, k_keep, alpha, phi, dout, dq, dk, dv, dalpha, ws, stream=None):
+    _check("sla2_attn_bwd", lib().sla2_attn_bwd(ctypes.byref(shape), _p(q), _p(k), _p(v), _p(kept_idx), k_keep,
+                                                _p(alpha), phi, _p(dout), _p(dq), _p(dk), _p(dv), _p(dalpha),
+                                                _p(ws), ws.numel(), _s(stream)))
 
 
 def sla_read_device_status(ws, stream=None) -> int:

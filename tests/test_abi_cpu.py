@@ -180,3 +180,36 @@ def test_prepare_rejects_bad_arguments_before_launch():
     assert L.sla_prepare(ctypes.byref(s), None, FAKE, 0, FAKE, 1 << 40, None) == 1
     assert L.sla_prepare(ctypes.byref(s), FAKE, FAKE, 5, FAKE, 1 << 40, None) == 1
     assert L.sla_prepare(ctypes.byref(_shape(bkv=32)), FAKE, FAKE, 0, FAKE, 1 << 40, None) == 2
+
+
+def test_backward_rejects_bad_arguments_before_launch():
+    s = _shape()
+    L = sla.lib()
+    need = sla.sla2_attn_bwd_workspace_size(s)
+    # status + H_tot, Z_tot and their gradients + the [BH, N, 128] fp32 key-side sums
+    assert need >= 12 * 32760 * 128 * 4 and need % 256 == 0
+    assert sla.sla2_attn_bwd_workspace_size(_shape(d=100)) == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, kept=FAKE, k_keep=15, alpha=FAKE, phi=0, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+                 dal=FAKE, ws=FAKE, wsb=need)
+        a.update(kw)
+        return L.sla2_attn_bwd(ctypes.byref(s), a["q"], FAKE, FAKE, a["kept"], a["k_keep"], a["alpha"], a["phi"],
+                               a["dout"], a["dq"], a["dk"], a["dv"], a["dal"], a["ws"], a["wsb"], None)
+
+    assert call(q=None) == 1
+    assert call(q=FAKE + 2) == 3
+    assert call(k_keep=-1) == 1
+    assert call(k_keep=513) == 1
+    assert call(kept=None) == 1
+    assert call(alpha=None) == 1
+    assert call(phi=3) == 1
+    for name in ("dout", "dq", "dk", "dv", "dal"):
+        assert call(**{name: None}) == 1, name
+        assert call(**{name: FAKE + 4}) == 3, name
+    assert call(ws=None) == 1
+    assert call(ws=FAKE + 16) == 3
+    assert call(wsb=need - 1) == 4
+    assert "sla2_attn_bwd_workspace_size" in L.sla_last_error_detail().decode()
+    assert L.sla2_attn_bwd(ctypes.byref(_shape(bq=96)), FAKE, FAKE, FAKE, FAKE, 15, FAKE, 0, FAKE, FAKE, FAKE,
+                           FAKE, FAKE, FAKE, need, None) == 2

@@ -1,0 +1,110 @@
+"""GPU parity of sla2_attn_bwd (the gradients of the SLA2 forward with the
+block mask held fixed) against the oracle's sla2_backward on the same seeded
+inputs, element by element.
+
+Follows "SLA: Beyond Sparsity in Diffusion Transformers …" (papernotes.org)
+关键设计 4 and "SLA2 深度解读 …" (jefxiong.cn) §07.  The kernels compute in
+fp32 on the exact input values; the oracle in fp64.  The bound below is
+relative to each tensor's largest entry: fp32 rounding over a few thousand
+terms and the run-to-run order of the atomic adds stay orders of magnitude
+under it.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import sla_oracle as orc
+from sparse_linear_attention_b200 import inputs, sla
+
+pytestmark = pytest.mark.gpu
+
+TOL_BWD_REL = 1e-4
+
+
+def _kept(seed, B, H, nq, nkv, kk):
+    g = np.random.default_rng(seed)
+    out = np.zeros((B, H, nq, kk), dtype=np.int32)
+    for idx in np.ndindex(B, H, nq):
+        out[idx] = np.sort(g.choice(nkv, kk, replace=False))
+    return out
+
+
+def _case(seed, B, H, N, d, bq, kk, dtype):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(B, H, N, d, generator=g) * 0.8).to(dtype)
+    k = (torch.randn(B, H, N, d, generator=g) * 0.8).to(dtype)
+    v = torch.randn(B, H, N, d, generator=g).to(dtype)
+    do = torch.randn(B, H, N, d, generator=g).to(dtype)
+    nq, nkv = -(-N // bq), -(-N // 64)
+    alpha = torch.rand(B, H, nq, generator=g) * 0.8 + 0.1
+    return q, k, v, do, alpha, _kept(seed, B, H, nq, nkv, kk)
+
+
+def _run(q, k, v, kept, alpha, do, bq, phi):
+    dev = "cuda"
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
+    shape = sla.make_shape(qd, bq, 64)
+    B, H, N, d = q.shape
+    nq = -(-N // bq)
+    kk = kept.shape[-1]
+    keptd = torch.from_numpy(kept).to(dev).contiguous() if kk else None
+    ws = torch.zeros(sla.sla2_attn_bwd_workspace_size(shape), dtype=torch.uint8, device=dev)
+    dq = torch.full((B, H, N, d), float("nan"), device=dev)
+    dk = torch.full_like(dq, float("nan"))
+    dv = torch.full_like(dq, float("nan"))
+    dal = torch.full((B, H, nq), float("nan"), device=dev)
+    sla.sla2_attn_bwd(shape, qd, kd, vd, keptd, kk, alpha.to(dev).contiguous(), phi, dod, dq, dk, dv, dal, ws)
+    status = sla.sla_read_device_status(ws)
+    return status, {"dq": dq.cpu().numpy(), "dk": dk.cpu().numpy(), "dv": dv.cpu().numpy(),
+                    "dalpha": dal.cpu().numpy()}
+
+
+def _check(q, k, v, kept, alpha, do, bq, phi):
+    status, got = _run(q, k, v, kept, alpha, do, bq, phi)
+    assert status == 0
+    kind = "softmax" if phi == sla.SLA_PHI_SOFTMAX else "elu1"
+    f64 = lambda t: t.to(torch.float64).numpy()
+    ref = orc.sla2_backward(f64(q), f64(k), f64(v), kept, f64(alpha), f64(do), bq, 64, kind)
+    for name in ("dq", "dk", "dv", "dalpha"):
+        g, r = got[name], ref[name]
+        assert np.isfinite(g).all(), name
+        scale = max(np.abs(r).max(), 1e-30)
+        err = np.abs(g - r).max() / scale
+        assert err <= TOL_BWD_REL, (name, err)
+
+
+def test_backward_tiny_workload():
+    """The small SLA2 case (fp32, d = 64, b_q = 64, 4 of 16 blocks kept)."""
+    w = inputs.WORKLOADS["tiny"]
+    x = inputs.make_inputs(w)
+    g = torch.Generator().manual_seed(5)
+    do = torch.randn(x["q"].shape, generator=g).to(x["q"].dtype)
+    kept = _kept(5, w.B, w.H, w.n_q, w.n_kv, 4)
+    _check(x["q"], x["k"], x["v"], kept, x["alpha"], do, w.bq, sla.SLA_PHI_ELU1)
+
+
+@pytest.mark.parametrize("N,d,bq,kk", [(1000, 128, 128, 3), (777, 64, 64, 2), (130, 32, 128, 1)])
+def test_backward_bf16_ragged(N, d, bq, kk):
+    """bf16 inputs, ragged last query and key blocks."""
+    q, k, v, do, alpha, kept = _case(N + kk, 1, 2, N, d, bq, kk, torch.bfloat16)
+    _check(q, k, v, kept, alpha, do, bq, sla.SLA_PHI_ELU1)
+
+
+def test_backward_softmax_feature_map():
+    q, k, v, do, alpha, kept = _case(31, 1, 2, 700, 64, 64, 3, torch.bfloat16)
+    _check(q, k, v, kept, alpha, do, 64, sla.SLA_PHI_SOFTMAX)
+
+
+@pytest.mark.parametrize("kk", [0, 5])
+def test_backward_no_block_and_every_block(kk):
+    """k = 0 (linear branch only) and k = n_kv (sparse branch only, O_l = 0)."""
+    q, k, v, do, alpha, kept = _case(40 + kk, 2, 1, 300, 32, 64, kk, torch.bfloat16)
+    _check(q, k, v, kept, alpha, do, 64, sla.SLA_PHI_ELU1)
+
+
+def test_backward_reports_out_of_range_block():
+    q, k, v, do, alpha, kept = _case(50, 1, 1, 256, 64, 64, 2, torch.bfloat16)
+    kept[0, 0, 1, 1] = 4  # n_kv = 4
+    status, got = _run(q, k, v, kept, alpha, do, 64, sla.SLA_PHI_ELU1)
+    assert status == 7  # SLA_ERR_DEVICE_INDEX; the block is skipped
+    assert all(np.isfinite(t).all() for t in got.values())
