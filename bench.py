@@ -241,6 +241,64 @@ def soft_topk_leg(args, w, dev, stream):
     }), flush=True)
 
 
+def backward_leg(args, w, dev, stream):
+    """SLA2 backward (sla2_attn_bwd) at the same workload: ms per call with
+    every input resident, the kept blocks from the router, a seeded dO.  The
+    work is dense contractions, so the roofline is the measured bf16 tensor
+    peak; the algorithmic work is the FlashAttention-style backward of the
+    sparse branch, 10 d FLOP per (query row, kept valid key): S recomputed,
+    dP = dO V^T, dQ, dK and dV (the linear branch is not counted)."""
+    x = inputs.make_inputs(w)
+    q, kk, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    wq, wk, alpha = x["wq"].to(dev), x["wk"].to(dev), x["alpha"].to(dev)
+    k = keep_of(w)
+    shape = sla.make_shape(q, w.bq, w.bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, sla.SLA_MODE_SLA2_TOPK), dtype=torch.uint8, device=dev)
+    kept = torch.empty(w.B, w.H, w.n_q, k, dtype=torch.int32, device=dev)
+    sla.sla_route(shape, q, kk, wq, wk, sla.SLA_MODE_SLA2_TOPK, k, 0, kept, None, None, ws, stream)
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    do = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    wsb = torch.zeros(sla.sla2_attn_bwd_workspace_size(shape), dtype=torch.uint8, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk, dv = torch.empty_like(dq), torch.empty_like(dq)
+    dal = torch.empty(w.B, w.H, w.n_q, dtype=torch.float32, device=dev)
+    phi = sla.SLA_PHI_ELU1 if args.phi == "elu1" else sla.SLA_PHI_SOFTMAX
+    call = lambda: sla.sla2_attn_bwd(shape, q, kk, v, kept, k, alpha, phi, do, dq, dk, dv, dal, wsb, stream)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if sla.sla_read_device_status(wsb, stream) != 0:
+        raise SystemExit("device-side error during the timed calls")
+    ms = t0.elapsed_time(t1) / args.steps
+    _, executed = work_counts(w, kept.cpu())
+    flops = executed / 4.0 * 10.0  # work_counts' executed count is 4 d per (row, kept valid key)
+    _, peak, _, src = peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "SLA2 backward ms @Wan-1.3B shape (sla2_attn_bwd: dQ, dK, dV, dalpha)", "value": ms,
+        "unit": "ms per call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": False, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
+                               f"keep={k}/{w.n_kv} key blocks, phi={args.phi}"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense (burst)",
+                     "algorithmic": "10*d FLOP per (query row, kept valid key): the sparse branch's "
+                                    "FlashAttention-style backward; kernels are fp32 on the CUDA cores"},
+        "gpu_launches": 3 * args.steps, "clocks": clk,
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -255,6 +313,8 @@ def main():
                     help="linear-branch feature map (the pages' default for SLA2 is ELU+1)")
     ap.add_argument("--soft-topk", action="store_true",
                     help="time the SoftTop-k router (sla_route_soft) instead of the forward step")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the SLA2 backward (sla2_attn_bwd) instead of the forward step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -263,8 +323,8 @@ def main():
     w = inputs.WORKLOADS[args.workload]
     if w.fp8:
         raise SystemExit("bench.py times the bf16 path; pick a workload without fp8")
-    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk):
-        raise SystemExit("the reference arm and --soft-topk time the SLA2 router / forward")
+    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk or args.backward):
+        raise SystemExit("the reference arm, --soft-topk and --backward time the SLA2 router / forward / backward")
     phi = sla.SLA_PHI_ELU1 if args.phi == "elu1" else sla.SLA_PHI_SOFTMAX
     sla_mode = w.mode == "sla"
 
@@ -305,6 +365,10 @@ def main():
     if args.soft_topk:
         if world == 1:
             soft_topk_leg(args, w, dev, stream)
+        return
+    if args.backward:
+        if world == 1:
+            backward_leg(args, w, dev, stream)
         return
 
     x = inputs.make_inputs(w)
