@@ -1,0 +1,118 @@
+"""The decomposition the GPU backward is built on (sparse_linear_attention_b200/
+csrc/backward.cu, header comment) restated in numpy and checked against the
+oracle's sla2_backward, on the CPU.
+
+The kernel writes the linear branch as totals minus the kept blocks: H_i =
+H_tot - sum_kept phi(K_j)^T V_j, and the gradient that H_i, Z_i send to the
+unselected keys as (dH_tot, dZ_tot) minus the kept blocks' share.  It also
+recomputes the softmax in three passes over the kept blocks (row max; row sum,
+O_s, num, den; gradients) per 32-row tile.  This restatement follows those
+steps and shares no code with the kernel or the oracle; agreement to rounding
+shows the algebra is exact, including k = 0, k = n_kv, ragged blocks and both
+feature maps ("SLA: Beyond Sparsity …" (papernotes.org) 关键设计 4).
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import sla_oracle as orc
+
+
+def _phi(x, kind):
+    if kind == "elu1":
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    e = np.exp(x - x.max(-1, keepdims=True))
+    return e / e.sum(-1, keepdims=True)
+
+
+def _phi_grad(x, g, kind):
+    if kind == "elu1":
+        return g * np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+    f = _phi(x, kind)
+    return f * (g - (g * f).sum(-1, keepdims=True))
+
+
+def _decomposed(q, k, v, kept, alpha, do, bq, bkv, kind):
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dal = np.zeros((B, H, nq))
+    has_lin = kept.shape[-1] < nkv
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK = _phi(K, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            dHt, dZt, dPK = np.zeros((d, d)), np.zeros(d), np.zeros((N, d))
+            for i in range(nq):
+                a = alpha[b, h, i]
+                blocks = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in kept[b, h, i]]
+                for r0 in range(i * bq, min((i + 1) * bq, N), 32):
+                    rows = np.arange(r0, min(r0 + 32, N))
+                    Qt, Gt = Q[rows], G[rows]
+                    PQ = _phi(Qt, kind)
+                    num = PQ @ Ht
+                    m = np.full(len(rows), -np.inf)
+                    for ks in blocks:
+                        m = np.maximum(m, (sc * Qt @ K[ks].T).max(1))
+                    l, oacc, rsa = np.zeros(len(rows)), np.zeros((len(rows), d)), np.zeros(len(rows))
+                    for ks in blocks:
+                        P = np.exp(sc * Qt @ K[ks].T - m[:, None])
+                        A = PQ @ PK[ks].T
+                        l += P.sum(1)
+                        oacc += P @ V[ks]
+                        num -= A @ V[ks]
+                        rsa += A.sum(1)
+                    Os = oacc / l[:, None] if blocks else np.zeros_like(oacc)
+                    if has_lin:
+                        den = PQ @ Zt - rsa
+                        Ol = num / den[:, None]
+                        s = (1.0 - a) / den
+                        dd = -(1.0 - a) * (Gt * Ol).sum(1) / den
+                    else:
+                        Ol, s, dd = np.zeros_like(Os), np.zeros(len(rows)), np.zeros(len(rows))
+                    D = a * (Gt * Os).sum(1)
+                    dal[b, h, i] += (Gt * (Os - Ol)).sum()
+                    dqs, dpq = np.zeros((len(rows), d)), np.zeros((len(rows), d))
+                    for ks in blocks:
+                        P = np.exp(sc * Qt @ K[ks].T - m[:, None]) / l[:, None]
+                        A = PQ @ PK[ks].T
+                        Gk = Gt @ V[ks].T
+                        dS = P * (a * Gk - D[:, None])
+                        C = a * P - s[:, None] * A
+                        Bx = s[:, None] * Gk + dd[:, None]
+                        dqs += dS @ K[ks]
+                        dpq -= Bx @ PK[ks]
+                        dk[b, h, ks] += sc * dS.T @ Qt
+                        dv[b, h, ks] += C.T @ Gt
+                        if has_lin:
+                            dPK[ks] -= Bx.T @ PQ
+                    if has_lin:
+                        dpq += s[:, None] * (Gt @ Ht.T) + dd[:, None] * Zt[None, :]
+                        dHt += PQ.T @ (s[:, None] * Gt)
+                        dZt += PQ.T @ dd
+                    dq[b, h, rows] = sc * dqs + _phi_grad(Qt, dpq, kind)
+            dPK += V @ dHt.T + dZt[None, :]
+            dv[b, h] += PK @ dHt
+            dk[b, h] += _phi_grad(K, dPK, kind)
+    return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dal}
+
+
+@pytest.mark.parametrize("N,d,bq,kk,kind", [(200, 16, 64, 2, "elu1"), (333, 8, 128, 3, "softmax"),
+                                            (130, 16, 64, 0, "elu1"), (130, 16, 64, 3, "elu1"),
+                                            (97, 8, 64, 2, "softmax")])
+def test_decomposition_matches_oracle(N, d, bq, kk, kind):
+    rng = np.random.default_rng(N + kk)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kk = min(kk, nkv)
+    kept = np.array([[[np.sort(rng.choice(nkv, kk, replace=False)) for _ in range(nq)] for _ in range(H)]])
+    kept = kept.reshape(1, H, nq, kk)
+    alpha = rng.uniform(0.1, 0.9, (1, H, nq))
+    ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
+    got = _decomposed(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
