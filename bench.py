@@ -241,6 +241,30 @@ def soft_topk_leg(args, w, dev, stream):
     }), flush=True)
 
 
+def backward_oracle_ms(w, x, kept, do_cpu, budget_s):
+    """The oracle's sla2_backward timed on sampled query blocks (random heads
+    and positions, at least three, until budget_s seconds are spent), each
+    block's time extrapolated to every block of the workload.  Returns (ms per
+    backward, blocks timed, seconds spent)."""
+    import numpy as np
+
+    from oracle import sla_oracle as orc
+    rng = np.random.default_rng(1)
+    heads = {}
+    spent, n = 0.0, 0
+    while n < 3 or spent < budget_s:
+        h, i = int(rng.integers(0, w.H)), int(rng.integers(0, w.n_q))
+        if h not in heads:
+            heads[h] = tuple(t[:, h:h + 1].to(torch.float64).numpy() for t in (x["q"], x["k"], x["v"], do_cpu))
+        q64, k64, v64, do64 = heads[h]
+        t1 = time.perf_counter()
+        orc.sla2_backward(q64, k64, v64, kept[:, h:h + 1], x["alpha"][:, h:h + 1].to(torch.float64).numpy(), do64,
+                          w.bq, w.bkv, blocks=[(0, 0, i)])
+        spent += time.perf_counter() - t1
+        n += 1
+    return spent / n * (w.B * w.H * w.n_q) * 1e3, n, spent
+
+
 def backward_leg(args, w, dev, stream):
     """SLA2 backward (sla2_attn_bwd) at the same workload: ms per call with
     every input resident, the kept blocks from the router, a seeded dO.  The
@@ -281,8 +305,15 @@ def backward_leg(args, w, dev, stream):
     if sla.sla_read_device_status(wsb, stream) != 0:
         raise SystemExit("device-side error during the timed calls")
     ms = t0.elapsed_time(t1) / args.steps
-    _, executed = work_counts(w, kept.cpu())
+    kept_cpu = kept.cpu()
+    _, executed = work_counts(w, kept_cpu)
     flops = executed / 4.0 * 10.0  # work_counts' executed count is 4 d per (row, kept valid key)
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu_ms, nblk, t_cpu = backward_oracle_ms(w, x, kept_cpu.numpy(), do.cpu(), args.cpu_budget)
+        cpu = {"value": cpu_ms, "unit": "ms per call", "cores": OracleTimer.threads(), "kind": "oracle",
+               "sample": f"CPU oracle (numpy fp64) sla2_backward on {nblk} sampled query blocks of "
+                         f"{w.B * w.H * w.n_q} ({t_cpu:.2f} s), extrapolated per block"}
     _, peak, _, src = peaks()
     achieved = flops / (ms * 1e-3) / 1e12
     print(json.dumps({
@@ -295,7 +326,7 @@ def backward_leg(args, w, dev, stream):
                      "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense (burst)",
                      "algorithmic": "10*d FLOP per (query row, kept valid key): the sparse branch's "
                                     "FlashAttention-style backward; kernels are fp32 on the CUDA cores"},
-        "gpu_launches": 3 * args.steps, "clocks": clk,
+        "gpu_launches": 3 * args.steps, "clocks": clk, "cpu_baseline": cpu,
     }), flush=True)
 
 

@@ -552,40 +552,40 @@ def linear_branch_backward(q, k, v, rows, keys, do_l, phi_kind="elu1"):
     return phi_backward(q[rows], dpq, phi_kind), phi_backward(k[keys], dpk, phi_kind), dv
 
 
-def sla2_backward(q, k, v, kept, alpha, do, bq, bkv, phi_kind="elu1"):
+def sla2_backward(q, k, v, kept, alpha, do, bq, bkv, phi_kind="elu1", blocks=None):
     """Gradients of sla2_forward's O = alpha*O_s + (1-alpha)*O_l for the
     upstream gradient do [B,H,N,d], the mask held fixed:
       dO_s = alpha dO,  dO_l = (1 - alpha) dO,
       dalpha_i = sum over the rows of query block i of dO * (O_s - O_l).
     A key's gradient adds up over every query block that reads it: through the
     sparse branch where its block is kept, through the linear branch elsewhere.
+    blocks: optional list of (b,h,i) whose share to add (default: all, which
+    gives the full gradients).
     Returns dict dq, dk, dv (float64 [B,H,N,d]) and dalpha ([B,H,nq])."""
     B, H, N, d = q.shape
     nq = -(-N // bq)
     n_kv = -(-N // bkv)
     dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
     dalpha = np.zeros((B, H, nq))
-    for b in range(B):
-        for h in range(H):
-            qs, ks, vs = q[b, h], k[b, h], v[b, h]
-            for i in range(nq):
-                rows = _rows(i, bq, N)
-                sel = sorted(int(j) for j in kept[b, h, i])
-                uns = [j for j in range(n_kv) if j not in set(sel)]
-                ts, tl = _tokens_of(sel, bkv, N), _tokens_of(uns, bkv, N)
-                a = float(alpha[b, h, i])
-                g = do[b, h, rows]
-                o_s = sparse_branch(qs, ks, vs, rows, ts)
-                o_l = linear_branch(qs, ks, vs, rows, tl, phi_kind)
-                dalpha[b, h, i] = (g * (o_s - o_l)).sum()
-                gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, ts, a * g)
-                dq[b, h, rows] += gq
-                dk[b, h, ts] += gk
-                dv[b, h, ts] += gv
-                gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tl, (1.0 - a) * g, phi_kind)
-                dq[b, h, rows] += gq
-                dk[b, h, tl] += gk
-                dv[b, h, tl] += gv
+    for (b, h, i) in _blocks_to_do(B, H, nq, blocks):
+        qs, ks, vs = q[b, h], k[b, h], v[b, h]
+        rows = _rows(i, bq, N)
+        sel = sorted(int(j) for j in kept[b, h, i])
+        uns = [j for j in range(n_kv) if j not in set(sel)]
+        ts, tl = _tokens_of(sel, bkv, N), _tokens_of(uns, bkv, N)
+        a = float(alpha[b, h, i])
+        g = do[b, h, rows]
+        o_s = sparse_branch(qs, ks, vs, rows, ts)
+        o_l = linear_branch(qs, ks, vs, rows, tl, phi_kind)
+        dalpha[b, h, i] = (g * (o_s - o_l)).sum()
+        gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, ts, a * g)
+        dq[b, h, rows] += gq
+        dk[b, h, ts] += gk
+        dv[b, h, ts] += gv
+        gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tl, (1.0 - a) * g, phi_kind)
+        dq[b, h, rows] += gq
+        dk[b, h, tl] += gk
+        dv[b, h, tl] += gv
     return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dalpha}
 
 

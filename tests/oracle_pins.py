@@ -721,6 +721,11 @@ def pin_bwd_sum_rules(orc):
     assert np.allclose(gr["dq"].sum(axis=3), 0.0, atol=1e-10)
     assert np.allclose(gr["dk"].sum(axis=3), 0.0, atol=1e-10)
     assert np.abs(gr["dq"]).max() > 1e-3 and np.abs(gr["dk"]).max() > 1e-3
+    # the shares of single query blocks add up to the whole gradient
+    full = orc.sla2_backward(q, k, v, kept, alpha, do, 16, 8)
+    parts = [orc.sla2_backward(q, k, v, kept, alpha, do, 16, 8, blocks=[t]) for t in np.ndindex(1, 2, 3)]
+    for name in ("dq", "dk", "dv", "dalpha"):
+        assert np.allclose(sum(p[name] for p in parts), full[name], atol=1e-12), name
 
 
 ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, pin_fp8_identity_codec_is_fp64, pin_fp8_quantisation_error_bounded,
