@@ -379,6 +379,12 @@ def e4m3_round(x32: np.ndarray) -> np.ndarray:
     return e4m3_decode(e4m3_encode(x32))
 
 
+def int8_round(x32: np.ndarray) -> np.ndarray:
+    """Value of x after a symmetric INT8 round trip, float64: round to the
+    nearest integer (ties to even), saturate to [-127, 127]."""
+    return np.clip(np.rint(np.asarray(x32, dtype=F64)), -127.0, 127.0)
+
+
 # ----------------------------------------------------------------------------
 # Low-bit (FP8 e4m3) sparse branch  [SLA2-deep §07]
 #
@@ -401,34 +407,43 @@ def e4m3_round(x32: np.ndarray) -> np.ndarray:
 #     running row max including that tile, p8 = e4m3(fp32(p * 448)); the row
 #     sum uses the unquantised p.  Without quantisation the tile width does
 #     not change the result (online softmax is exact for any grouping).
+# The page names "INT8 or FP8" and points to SageAttention2++ for the scheme
+# without fixing it.  The INT8 variant read from that: Q and K' in INT8 with
+# the same per-block rule (qmax 127 in place of 448, codes rint(x * inv) ties
+# to even, saturated to +-127; their product is exact in integers), P and V
+# in e4m3 as above.
 # ----------------------------------------------------------------------------
 
 def _e4m3_q(x32, codec):
     return codec(np.asarray(x32, dtype=F32))
 
 
-def _quant_blocks(x32, blk, codec):
-    """Per block of `blk` tokens (rows of x32 [n, d]): (decoded values, scales)."""
+def _quant_blocks(x32, blk, codec, qmax=448.0):
+    """Per block of `blk` tokens (rows of x32 [n, d]): (decoded values, scales),
+    codes of x * qmax / amax and scale amax / qmax (both fp32)."""
     n = x32.shape[0]
     vals = np.empty(x32.shape, dtype=F64)
     scales = []
     for t0 in range(0, n, blk):
         xb = x32[t0:t0 + blk]
         amax = F32(np.abs(xb).max()) if xb.size else F32(0.0)
-        inv = F32(448.0) / amax if amax > 0 else F32(1.0)
+        inv = F32(qmax) / amax if amax > 0 else F32(1.0)
         vals[t0:t0 + blk] = _e4m3_q(xb * inv, codec)
-        scales.append(F64(F32(amax / F32(448.0))) if amax > 0 else F64(F32(1.0) / F32(448.0)))
+        scales.append(F64(F32(amax / F32(qmax))) if amax > 0 else F64(F32(1.0) / F32(qmax)))
     return vals, np.array(scales, dtype=F64)
 
 
 def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, codec=None, qblk=128,
-                     kv_tile=2):
+                     kv_tile=2, qk_codec=None, qk_max=448.0):
     """SLA2 output with the low-bit sparse branch described above; the linear
     branch and the combine are the fp64 ones of sla2_forward.  q, k, v: exact
     values of the inputs as float64 [B,H,N,d].  codec(x32) -> float64 values
     after the e4m3 round trip (e4m3_round by default; an identity codec turns
-    the quantisation off, which pins the bookkeeping to sla2_forward)."""
+    the quantisation off, which pins the bookkeeping to sla2_forward).
+    qk_codec, qk_max: the round trip and code range of Q and K' (default: codec
+    and 448; the INT8 variant passes int8_round and 127)."""
     codec = e4m3_round if codec is None else codec
+    qk_codec = codec if qk_codec is None else qk_codec
     B, H, N, d = q.shape
     nq = -(-N // bq)
     n_kv = -(-N // bkv)
@@ -439,8 +454,8 @@ def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None
         qs, ks, vs = q[b, h], k[b, h], v[b, h]
         mu = ks.mean(axis=0)
         kp32 = (ks - mu).astype(F32)
-        q8, sq = _quant_blocks(qs.astype(F32), qblk, codec)
-        k8, sk = _quant_blocks(kp32, qblk, codec)
+        q8, sq = _quant_blocks(qs.astype(F32), qblk, qk_codec, qk_max)
+        k8, sk = _quant_blocks(kp32, qblk, qk_codec, qk_max)
         v32 = vs.astype(F32)
         vamax = np.abs(v32).max(axis=0)
         vinv = np.where(vamax > 0, F32(448.0) / np.where(vamax > 0, vamax, F32(1.0)), F32(1.0)).astype(F32)
@@ -474,6 +489,14 @@ def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None
             out["o_l"][b, h, rows] = o_l
             out["o"][b, h, rows] = a * o_s + (1.0 - a) * o_l
     return out
+
+
+def sla2_forward_int8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, qblk=128, kv_tile=2):
+    """SLA2 output with the INT8 variant of the low-bit branch: Q and K' in
+    INT8 (int8_round, qmax 127, one scale per qblk-token block), P and V in
+    e4m3 as in sla2_forward_fp8."""
+    return sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind, blocks, None, qblk, kv_tile,
+                            qk_codec=int8_round, qk_max=127.0)
 
 
 # ----------------------------------------------------------------------------

@@ -602,6 +602,66 @@ def pin_soft_topk_edges_and_shift(orc):
     assert np.allclose(lam2, lam - 25.0, rtol=0, atol=1e-8)
 
 
+# ---------------------------------------------------------------- INT8 variant pins
+
+def pin_int8_codec(orc):
+    """INT8 round trip: round to nearest with ties to even (as torch.round),
+    saturated to [-127, 127]."""
+    x = np.array([2.5, 3.5, -2.5, -3.5, 0.49, 126.6, 127.4, 200.0, -300.0, -127.5, 0.0], dtype=np.float32)
+    want = np.array([2, 4, -2, -4, 0, 127, 127, 127, -127, -127, 0], dtype=np.float64)
+    assert np.array_equal(orc.int8_round(x), want)
+    g = _rand((4000,), 95, 80.0).astype(np.float32)
+    ref = torch.clamp(torch.round(torch.from_numpy(g).double()), -127, 127).numpy()
+    assert np.array_equal(orc.int8_round(g), ref)
+
+
+def pin_int8_integer_inputs_are_exact(orc):
+    """Q and K' integer-valued with |x| <= 127 and 127 reached in every 128-token
+    block: the INT8 codes are the values themselves, so with P and V left
+    unquantised the INT8 branch equals the fp64 sparse branch.  e4m3 cannot
+    hold these integers (3 mantissa bits), so the same case through e4m3 Q, K'
+    does move."""
+    g = np.random.default_rng(96)
+    N, d = 256, 16
+    q = g.integers(-127, 128, size=(1, 1, N, d)).astype(np.float64)
+    blocks = []
+    for blk in range(2):
+        q[0, 0, 128 * blk, 0] = 127.0
+        half = g.integers(-127, 128, size=(64, d)).astype(np.float64)
+        half[0, 1] = 127.0
+        blocks += [half, -half]  # every column of every block sums to zero
+    kp = np.concatenate(blocks)
+    k = (kp + 3.0)[None, None]  # column mean exactly 3, so K' = kp
+    v = _rand((1, 1, N, d), 97)
+    kept = np.array([[[[0, 2], [1, 3]]]])
+    alpha = np.array([[[0.5, 0.5]]])
+    ident = lambda x: np.asarray(x, np.float64)  # noqa: E731
+    sq, sk = q * 2.0 ** -6, k * 2.0 ** -6  # exact: amax 127/64, inv 64, scale 1/64
+    # P and V pass through fp32 on every path; only the Q, K' round trip differs
+    a = orc.sla2_forward_fp8(sq, sk, v, kept, alpha, 128, 64, codec=ident, qk_codec=ident, qk_max=127.0)["o_s"]
+    b = orc.sla2_forward_fp8(sq, sk, v, kept, alpha, 128, 64, codec=ident,
+                             qk_codec=orc.int8_round, qk_max=127.0)["o_s"]
+    assert np.abs(a - b).max() < 1e-12
+    assert np.abs(a - orc.sla2_forward(sq, sk, v, kept, alpha, 128, 64)["o_s"]).max() < 1e-6
+    c = orc.sla2_forward_fp8(sq, sk, v, kept, alpha, 128, 64, codec=ident,
+                             qk_codec=orc.e4m3_round, qk_max=448.0)["o_s"]
+    assert np.abs(a - c).max() > 1e-4
+
+
+def pin_int8_variant_error_bounded(orc):
+    """The INT8 variant (INT8 Q, K'; e4m3 P, V) moves the output by a bounded
+    amount, and its scale bookkeeping with qmax 127 is exact when every round
+    trip is the identity."""
+    q, k, v, kept, alpha = _fp8_case(98)
+    a = orc.sla2_forward(q, k, v, kept, alpha, 128, 64)["o"]
+    c = orc.sla2_forward_int8(q, k, v, kept, alpha, 128, 64)["o"]
+    err = np.abs(a - c).max()
+    assert 1e-4 < err < 0.2, err
+    ident = lambda x: np.asarray(x, np.float64)  # noqa: E731
+    b = orc.sla2_forward_fp8(q, k, v, kept, alpha, 128, 64, codec=ident, qk_codec=ident, qk_max=127.0)["o"]
+    assert np.abs(a - b).max() < 1e-6
+
+
 # ---------------------------------------------------------------- backward pins
 # The backward is pinned by central finite differences of the (pinned) forward,
 # by torch autograd on the two limits that are textbook attention, and by sum
@@ -740,4 +800,5 @@ ALL_PINS = [pin_hand_example, pin_fma32_exact, pin_fma32_double_rounding_case, p
     pin_soft_topk_hard_limit, pin_soft_topk_edges_and_shift,
     pin_bwd_sla2_finite_differences, pin_bwd_sla2_softmax_phi_finite_differences, pin_bwd_sla_finite_differences,
     pin_bwd_textbook_limits, pin_bwd_sum_rules,
+    pin_int8_codec, pin_int8_integer_inputs_are_exact, pin_int8_variant_error_bounded,
 ]

@@ -62,6 +62,12 @@ MUTATIONS = {
     "bwd_dalpha_sign": ("dalpha[b, h, i] = (g * (o_s - o_l)).sum()", "dalpha[b, h, i] = (g * (o_l - o_s)).sum()"),
     "bwd_sla_proj_not_transposed": ("g @ wp.T, phi_kind)", "g @ wp, phi_kind)"),
     "bwd_sla_dwproj_transposed": ("dwp += o_l.T @ g", "dwp += g.T @ o_l"),
+    "int8_rounds_half_up": ("np.clip(np.rint(np.asarray(x32, dtype=F64)), -127.0, 127.0)",
+                            "np.clip(np.floor(np.asarray(x32, dtype=F64) + 0.5), -127.0, 127.0)"),
+    "int8_saturates_at_128": ("np.clip(np.rint(np.asarray(x32, dtype=F64)), -127.0, 127.0)",
+                              "np.clip(np.rint(np.asarray(x32, dtype=F64)), -128.0, 128.0)"),
+    "int8_variant_keeps_448": ("qk_codec=int8_round, qk_max=127.0)", "qk_codec=int8_round, qk_max=448.0)"),
+    "quant_blocks_ignores_qmax": ("inv = F32(qmax) / amax", "inv = F32(448.0) / amax"),
 }
 
 
