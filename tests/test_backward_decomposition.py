@@ -10,6 +10,11 @@ O_s, num, den; gradients) per 32-row tile.  This restatement follows those
 steps and shares no code with the kernel or the oracle; agreement to rounding
 shows the algebra is exact, including k = 0, k = n_kv, ragged blocks and both
 feature maps ("SLA: Beyond Sparsity …" (papernotes.org) 关键设计 4).
+
+The same decomposition for SLA's three labels (critical blocks in the softmax,
+critical and negligible blocks both taken out of the linear totals, the
+W_proj gradient) is checked against the oracle's sla_backward; it is the
+algebra a GPU form of SLA's backward would follow.
 """
 import math
 
@@ -114,5 +119,101 @@ def test_decomposition_matches_oracle(N, d, bq, kk, kind):
     alpha = rng.uniform(0.1, 0.9, (1, H, nq))
     ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
     got = _decomposed(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
+
+
+def _decomposed_sla(q, k, v, labels, wp, do, bq, bkv, kind):
+    """SLA (O = O_s + O_l W_proj): the sparse passes run over the critical
+    blocks; the linear branch is the totals minus the critical AND the
+    negligible blocks (both leave it), so the kept share that goes back to the
+    keys is taken over both lists; dO_s = dO, dO_l = dO W_proj^T, and
+    dW_proj = sum O_l^T dO."""
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dwp = np.zeros(wp.shape)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK = _phi(K, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            dHt, dZt, dPK = np.zeros((d, d)), np.zeros(d), np.zeros((N, d))
+            for i in range(nq):
+                lab = labels[b, h, i]
+                crit = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in np.nonzero(lab == 1)[0]]
+                out = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in np.nonzero(lab != 0)[0]]
+                has_lin = (lab == 0).any()
+                for r0 in range(i * bq, min((i + 1) * bq, N), 32):
+                    rows = np.arange(r0, min(r0 + 32, N))
+                    Qt, Gs = Q[rows], G[rows]
+                    Gl = Gs @ wp.T
+                    PQ = _phi(Qt, kind)
+                    num, rsa = PQ @ Ht, np.zeros(len(rows))
+                    for ks in out:
+                        A = PQ @ PK[ks].T
+                        num -= A @ V[ks]
+                        rsa += A.sum(1)
+                    m = np.full(len(rows), -np.inf)
+                    for ks in crit:
+                        m = np.maximum(m, (sc * Qt @ K[ks].T).max(1))
+                    l, oacc = np.zeros(len(rows)), np.zeros((len(rows), d))
+                    for ks in crit:
+                        P = np.exp(sc * Qt @ K[ks].T - m[:, None])
+                        l += P.sum(1)
+                        oacc += P @ V[ks]
+                    Os = oacc / l[:, None] if crit else np.zeros_like(oacc)
+                    if has_lin:
+                        den = PQ @ Zt - rsa
+                        Ol = num / den[:, None]
+                        s = 1.0 / den
+                        dd = -(Gl * Ol).sum(1) / den
+                    else:
+                        Ol, s, dd = np.zeros_like(Os), np.zeros(len(rows)), np.zeros(len(rows))
+                    dwp += Ol.T @ Gs
+                    D = (Gs * Os).sum(1)
+                    dqs, dpq = np.zeros((len(rows), d)), np.zeros((len(rows), d))
+                    for ks in crit:
+                        P = np.exp(sc * Qt @ K[ks].T - m[:, None]) / l[:, None]
+                        dS = P * (Gs @ V[ks].T - D[:, None])
+                        dqs += dS @ K[ks]
+                        dk[b, h, ks] += sc * dS.T @ Qt
+                        dv[b, h, ks] += P.T @ Gs
+                    if has_lin:
+                        for ks in out:
+                            A = PQ @ PK[ks].T
+                            Bx = s[:, None] * (Gl @ V[ks].T) + dd[:, None]
+                            dpq -= Bx @ PK[ks]
+                            dv[b, h, ks] -= (s[:, None] * A).T @ Gl
+                            dPK[ks] -= Bx.T @ PQ
+                        dpq += s[:, None] * (Gl @ Ht.T) + dd[:, None] * Zt[None, :]
+                        dHt += PQ.T @ (s[:, None] * Gl)
+                        dZt += PQ.T @ dd
+                    dq[b, h, rows] = sc * dqs + _phi_grad(Qt, dpq, kind)
+            dPK += V @ dHt.T + dZt[None, :]
+            dv[b, h] += PK @ dHt
+            dk[b, h] += _phi_grad(K, dPK, kind)
+    return {"dq": dq, "dk": dk, "dv": dv, "dwproj": dwp}
+
+
+@pytest.mark.parametrize("N,d,bq,kind,n_crit,n_negl", [(200, 16, 64, "elu1", 1, 1), (333, 8, 128, "softmax", 2, 1),
+                                                        (130, 16, 64, "elu1", 0, 1), (130, 16, 64, "elu1", 2, 1),
+                                                        (130, 16, 64, "elu1", 3, 0)])
+def test_sla_decomposition_matches_oracle(N, d, bq, kind, n_crit, n_negl):
+    """Critical, marginal and negligible blocks; no critical block; no marginal
+    block (critical and negligible fill the row); every block critical."""
+    rng = np.random.default_rng(N + 10 * n_crit + n_negl)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    labels = np.zeros((1, H, nq, nkv), dtype=np.int8)
+    for h, i in np.ndindex(H, nq):
+        perm = rng.permutation(nkv)
+        labels[0, h, i, perm[:n_crit]] = 1
+        labels[0, h, i, perm[n_crit:n_crit + n_negl]] = -1
+    wp = rng.standard_normal((d, d)) / math.sqrt(d)
+    ref = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv, kind)
+    got = _decomposed_sla(q, k, v, labels, wp, do, bq, bkv, kind)
     for name in ref:
         assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
