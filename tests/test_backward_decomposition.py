@@ -217,3 +217,95 @@ def test_sla_decomposition_matches_oracle(N, d, bq, kind, n_crit, n_negl):
     got = _decomposed_sla(q, k, v, labels, wp, do, bq, bkv, kind)
     for name in ref:
         assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
+
+
+def _key_major(q, k, v, kept, alpha, do, bq, bkv, kind):
+    """The SLA2 backward restructured key-major: a query-major pass keeps per
+    row only the log-sum-exp of the kept scores, D, s and dden (and forms dH_tot,
+    dZ_tot and the linear dQ terms); then, per key block, the query blocks that
+    keep it (the inverse map of the kept lists, ascending) give
+      G^T = V dO^T,  dS^T = P^T * (alpha G^T - D),  C^T = alpha P^T - s A^T,
+      dK += dS^T Q / sqrt(d),  dV += C^T dO,  dphi(K) -= Bx^T phi(Q),
+    and dQ += dS K / sqrt(d) - Bx phi(K) is scattered back (Bx = s G + dden)."""
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dal = np.zeros((B, H, nq))
+    has_lin = kept.shape[-1] < nkv
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK, PQ = _phi(K, kind), _phi(Q, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            keys_of = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in range(nkv)]
+            lse, D, s, dd = np.zeros(N), np.zeros(N), np.zeros(N), np.zeros(N)
+            dHt, dZt, dPK = np.zeros((d, d)), np.zeros(d), np.zeros((N, d))
+            dpq_all = np.zeros((N, d))  # dphi(Q) from the totals; the kept share is added key-major
+            for i in range(nq):  # query-major statistics
+                rows = np.arange(i * bq, min((i + 1) * bq, N))
+                a = alpha[b, h, i]
+                ks = np.concatenate([keys_of[j] for j in kept[b, h, i]]) if kept.shape[-1] else np.zeros(0, int)
+                if len(ks):
+                    S = sc * Q[rows] @ K[ks].T
+                    mx = S.max(1)
+                    lse[rows] = mx + np.log(np.exp(S - mx[:, None]).sum(1))
+                    Os = np.exp(S - lse[rows][:, None]) @ V[ks]
+                else:
+                    Os = np.zeros((len(rows), d))
+                if has_lin:
+                    A = PQ[rows] @ PK[ks].T if len(ks) else np.zeros((len(rows), 0))
+                    den = PQ[rows] @ Zt - A.sum(1)
+                    Ol = (PQ[rows] @ Ht - A @ V[ks]) / den[:, None]
+                    s[rows] = (1 - a) / den
+                    dd[rows] = -(1 - a) * (G[rows] * Ol).sum(1) / den
+                else:
+                    Ol = np.zeros_like(Os)
+                D[rows] = a * (G[rows] * Os).sum(1)
+                dal[b, h, i] = (G[rows] * (Os - Ol)).sum()
+                dpq_all[rows] = s[rows][:, None] * (G[rows] @ Ht.T) + dd[rows][:, None] * Zt[None, :]
+                if has_lin:
+                    dHt += PQ[rows].T @ (s[rows][:, None] * G[rows])
+                    dZt += PQ[rows].T @ dd[rows]
+            users = [[i for i in range(nq) if j in set(int(x) for x in kept[b, h, i])] for j in range(nkv)]
+            dpq_kept = np.zeros((N, d))
+            dqs = np.zeros((N, d))
+            for j in range(nkv):  # key-major
+                ks = keys_of[j]
+                for i in users[j]:
+                    rows = np.arange(i * bq, min((i + 1) * bq, N))
+                    a = alpha[b, h, i]
+                    PT = np.exp(sc * K[ks] @ Q[rows].T - lse[rows][None, :])
+                    AT = PK[ks] @ PQ[rows].T
+                    GT = V[ks] @ G[rows].T
+                    dST = PT * (a * GT - D[rows][None, :])
+                    CT = a * PT - AT * s[rows][None, :]
+                    BxT = GT * s[rows][None, :] + dd[rows][None, :]
+                    dk[b, h, ks] += sc * dST @ Q[rows]
+                    dv[b, h, ks] += CT @ G[rows]
+                    if has_lin:
+                        dPK[ks] -= BxT @ PQ[rows]
+                        dpq_kept[rows] -= BxT.T @ PK[ks]
+                    dqs[rows] += sc * dST.T @ K[ks]
+            dq[b, h] = dqs + _phi_grad(Q, dpq_all + dpq_kept, kind)
+            dPK += V @ dHt.T + dZt[None, :]
+            dv[b, h] += PK @ dHt
+            dk[b, h] += _phi_grad(K, dPK, kind)
+    return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dal}
+
+
+@pytest.mark.parametrize("N,d,bq,kk,kind", [(200, 16, 64, 2, "elu1"), (333, 8, 128, 3, "softmax"),
+                                            (130, 16, 64, 0, "elu1"), (130, 16, 64, 3, "elu1")])
+def test_key_major_restatement_matches_oracle(N, d, bq, kk, kind):
+    rng = np.random.default_rng(7 * N + kk)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kk = min(kk, nkv)
+    kept = np.array([[[np.sort(rng.choice(nkv, kk, replace=False)) for _ in range(nq)] for _ in range(H)]])
+    kept = kept.reshape(1, H, nq, kk)
+    alpha = rng.uniform(0.1, 0.9, (1, H, nq))
+    ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
+    got = _key_major(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
