@@ -224,6 +224,9 @@ size_t sla2_attn_bwd_workspace_size(const sla_shape* shape);
  *   query block i of dO . (O_s - O_l); the sparse branch back-propagated as
  *   FlashAttention does, the linear branch through dH_i, dZ_i formed from the
  *   totals minus the kept blocks' share.
+ * The gradients are taken on the original (unquantised) inputs, so this is
+ *   also the backward of the e4m3 forward (SLA_FLAG_FP8): the low-bit
+ *   quantisation is forward-only [SLA2-deep §07].
  * Inputs q, k, v, kept_idx, k_keep, alpha, phi as for sla2_attn_fwd (kept
  * indices distinct per row); dout [B,H,N,d] of the input dtype.
  * Outputs (fp32, caller-owned, fully overwritten): dq, dk, dv [B,H,N,d],
