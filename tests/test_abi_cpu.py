@@ -213,3 +213,14 @@ def test_backward_rejects_bad_arguments_before_launch():
     assert "sla2_attn_bwd_workspace_size" in L.sla_last_error_detail().decode()
     assert L.sla2_attn_bwd(ctypes.byref(_shape(bq=96)), FAKE, FAKE, FAKE, FAKE, 15, FAKE, 0, FAKE, FAKE, FAKE,
                            FAKE, FAKE, FAKE, need, None) == 2
+
+
+def test_backward_workspace_layout():
+    """Status word, H_tot and Z_tot, their gradients, and the [BH, N, 128] fp32
+    key-side buffer, each rounded up to 256 bytes."""
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for B, H, N, d in [(1, 12, 32760, 128), (2, 3, 1000, 64), (1, 1, 1, 8), (1, 40, 75600, 128)]:
+        s = _shape(B=B, H=H, N=N, d=d)
+        BH = B * H
+        want = 256 + 2 * (a256(BH * 128 * 128 * 4) + a256(BH * 128 * 4)) + a256(BH * N * 128 * 4)
+        assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N, d)
