@@ -400,13 +400,14 @@ def int8_round(x32: np.ndarray) -> np.ndarray:
 #     inv = 448 / amax in fp32 (1 if amax = 0), x8 = e4m3(fp32(x * inv)),
 #     scale = amax / 448 in fp32;
 #   - V: one scale per (b,h) and channel over all valid tokens, same rule;
-#   - P: online softmax over the kept blocks in ascending order, taken a tile
-#     of kv_tile consecutive kept blocks at a time (the page leaves the tile
-#     width open; 2 blocks = 128 keys by default, the width of the attention
-#     kernel's softmax step); after each tile p = exp(S - m) with m the
-#     running row max including that tile, p8 = e4m3(fp32(p * 448)); the row
-#     sum uses the unquantised p.  Without quantisation the tile width does
-#     not change the result (online softmax is exact for any grouping).
+#   - P: online softmax over the kept blocks in ascending order, one kept
+#     block at a time: after each block p = exp(S - m) with m the running row
+#     max including that block, p8 = e4m3(fp32(p * 448)); the row sum uses
+#     the unquantised p.  The page fixes no tile, so the block, the unit the
+#     mask selects, is the tile here.  kv_tile > 1 groups that many
+#     consecutive kept blocks per step instead; it exists only so a pin can
+#     show that the grouping moves nothing but the rounding of P (without
+#     quantisation online softmax is exact for any grouping).
 # The page names "INT8 or FP8" and points to SageAttention2++ for the scheme
 # without fixing it.  The INT8 variant read from that: Q and K' in INT8 with
 # the same per-block rule (qmax 127 in place of 448, codes rint(x * inv) ties
@@ -434,7 +435,7 @@ def _quant_blocks(x32, blk, codec, qmax=448.0):
 
 
 def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, codec=None, qblk=128,
-                     kv_tile=2, qk_codec=None, qk_max=448.0):
+                     kv_tile=1, qk_codec=None, qk_max=448.0):
     """SLA2 output with the low-bit sparse branch described above; the linear
     branch and the combine are the fp64 ones of sla2_forward.  q, k, v: exact
     values of the inputs as float64 [B,H,N,d].  codec(x32) -> float64 values
@@ -491,7 +492,7 @@ def sla2_forward_fp8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None
     return out
 
 
-def sla2_forward_int8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, qblk=128, kv_tile=2):
+def sla2_forward_int8(q, k, v, kept, alpha, bq, bkv, phi_kind="elu1", blocks=None, qblk=128, kv_tile=1):
     """SLA2 output with the INT8 variant of the low-bit branch: Q and K' in
     INT8 (int8_round, qmax 127, one scale per qblk-token block), P and V in
     e4m3 as in sla2_forward_fp8."""
