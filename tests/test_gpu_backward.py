@@ -108,3 +108,35 @@ def test_backward_reports_out_of_range_block():
     status, got = _run(q, k, v, kept, alpha, do, 64, sla.SLA_PHI_ELU1)
     assert status == 7  # SLA_ERR_DEVICE_INDEX; the block is skipped
     assert all(np.isfinite(t).all() for t in got.values())
+
+
+def test_backward_wan13_sampled_query_blocks():
+    """The full 1.3B-shape backward (12 heads, N = 32760, d = 128, 15 of 512
+    key blocks kept by the router): dQ and dalpha of sampled query blocks
+    against the oracle.  A query block's dQ rows and its dalpha depend on that
+    block alone, so the oracle computes just those blocks (its blocks= path);
+    the bound is relative to the largest entry of the checked rows."""
+    w = inputs.WORKLOADS["wan13"]
+    x = inputs.make_inputs(w)
+    kk = w.keep_count if w.keep_count is not None else orc.keep_count(w.keep_ratio, w.n_kv)
+    kept, _, _ = orc.route(x["q"].float().numpy(), x["k"].float().numpy(), x["wq"].numpy(), x["wk"].numpy(),
+                           w.bq, w.bkv, "sla2", kk)
+    g = torch.Generator().manual_seed(13)
+    do = torch.randn(x["q"].shape, generator=g).to(torch.bfloat16)
+    status, got = _run(x["q"], x["k"], x["v"], kept, x["alpha"], do, w.bq, sla.SLA_PHI_ELU1)
+    assert status == 0
+    rng = np.random.default_rng(13)
+    blocks = [(0, h, int(i)) for h in (0, 6, 11) for i in sorted({0, w.n_q - 1, *rng.integers(0, w.n_q, 2)})]
+    f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    ref = orc.sla2_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), kept, f64(x["alpha"]), f64(do), w.bq, w.bkv,
+                            blocks=blocks)
+    sel = [(b, h, slice(i * w.bq, min((i + 1) * w.bq, w.N))) for (b, h, i) in blocks]
+    g_q = np.concatenate([got["dq"][b, h, r] for (b, h, r) in sel])
+    r_q = np.concatenate([ref["dq"][b, h, r] for (b, h, r) in sel])
+    assert np.isfinite(g_q).all()
+    err = np.abs(g_q - r_q).max() / max(np.abs(r_q).max(), 1e-30)
+    assert err <= TOL_BWD_REL, ("dq", err)
+    ga = np.array([got["dalpha"][b, h, i] for (b, h, i) in blocks])
+    ra = np.array([ref["dalpha"][b, h, i] for (b, h, i) in blocks])
+    err = np.abs(ga - ra).max() / max(np.abs(ra).max(), 1e-30)
+    assert err <= TOL_BWD_REL, ("dalpha", err)

@@ -201,6 +201,34 @@ def test_sla2_softmax_feature_map():
     _sla2_check(w, x, kept, phi=sla.SLA_PHI_SOFTMAX)
 
 
+def test_sla2_softmax_feature_map_production_path():
+    """Softmax-phi on the bf16 d = 128 path the benchmark times: the TMA
+    prepass (phi = softmax), the router on the prepass's key-block means, the
+    attention kernel on the prepared totals; sampled query blocks of the
+    full-size 1.3B-shape launch."""
+    w, x = workload("wan13")
+    kk = k_of(w)
+    dev = "cuda"
+    qd, kd, vd = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    shape = sla.make_shape(qd, w.bq, w.bkv)
+    ws = torch.zeros(sla.sla_workspace_size(shape, 0), dtype=torch.uint8, device=dev)
+    kept = torch.full((w.B, w.H, w.n_q, kk), -7, dtype=torch.int32, device=dev)
+    out = torch.full(x["q"].shape, float("nan"), dtype=torch.float32, device=dev)
+    sla.sla_prepare(shape, kd, vd, sla.SLA_PHI_SOFTMAX, ws)
+    sla.sla_route(shape, qd, kd, x["wq"].to(dev), x["wk"].to(dev),
+                  sla.SLA_MODE_SLA2_TOPK | sla.SLA_ROUTE_KBAR_FROM_WS, kk, 0, kept, None, None, ws)
+    sla.sla2_attn_fwd(shape, qd, kd, vd, kept, kk, x["alpha"].to(dev), sla.SLA_PHI_SOFTMAX, sla.SLA_FLAG_PREPARED,
+                      out, ws)
+    assert sla.sla_read_device_status(ws) == 0
+    kept_h = kept.cpu().numpy()
+    okept, _, _ = orc.route(as32(x["q"]), as32(x["k"]), x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv, "sla2", kk)
+    assert np.array_equal(kept_h, okept)
+    blocks = sample_blocks(w.B, w.H, w.n_q, 3, seed=6)
+    want = orc.sla2_forward(as64(x["q"]), as64(x["k"]), as64(x["v"]), kept_h, x["alpha"].numpy(), w.bq, w.bkv,
+                            phi_kind="softmax", blocks=blocks)["o"]
+    compare(out.cpu().numpy(), want, blocks, w.bq)
+
+
 def test_sla2_bf16_output():
     w, x = _rand_case(1500, 128, scale=1.5)
     kept = _rand_kept(w, 4)
@@ -310,15 +338,37 @@ def test_fp8_wan13_keep_sweep(ratio):
     _fp8_check(w, x, kept, blocks=sample_blocks(1, 3, w.n_q, 3, seed=4), heads=[0, 5, 11])
 
 
-def test_fp8_wan14_sampled_blocks():
+@pytest.mark.parametrize("ratio", [0.03, 0.05, 0.10])
+def test_fp8_wan14_keep_sweep(ratio):
+    """The e4m3 branch at the 14B shape for the keep sweep of that workload
+    (35 / 59 / 118 of 1182 key blocks): full launch, 3 heads x 3 query blocks
+    checked."""
     _, x = workload("wan14")  # same seeded inputs as the e4m3 14B workload
     w = inputs.WORKLOADS["fp8_14"]
-    kk = k_of(w)
+    kk = orc.keep_count(ratio, w.n_kv)
     kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, kk)
     _fp8_check(w, x, kept, blocks=sample_blocks(1, 3, w.n_q, 3, seed=5), heads=[0, 21, 39])
 
 
 @pytest.mark.parametrize("N,d,bq", [(777, 128, 64), (300, 64, 128)])
 def test_fp8_ragged_shapes(N, d, bq):
+    """Ragged shapes on plain N(0, 1.5^2) inputs (|V| up to 7, peaked rows).
+    The kernel quantises P once per softmax step of two kept blocks; the
+    oracle's default quantises it once per kept block.  The pages fix no tile,
+    so both are readings of the same step, and the grouping moves only the
+    rounding of P.  Here that rounding difference alone (the oracle against
+    itself, one block vs two per step) reaches 4e-2, above the 3e-2 gate that
+    the seeded workloads meet against the per-block oracle.  So the kernel is
+    held to the gate against the oracle with its own grouping, and to the gate
+    plus the oracle's own grouping spread against the per-block default."""
+    from tests.gpu_common import TOL_FP8
     w, x = _rand_case(N, d, bq=bq, scale=1.5)
-    _fp8_check(w, x, _rand_kept(w, min(3, w.n_kv)))
+    kept = _rand_kept(w, min(3, w.n_kv))
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, flags=sla.SLA_FLAG_FP8)
+    args = (as64(x["q"]), as64(x["k"]), as64(x["v"]), kept, x["alpha"].numpy(), w.bq, w.bkv)
+    per_block = orc.sla2_forward_fp8(*args)["o"]
+    per_step = orc.sla2_forward_fp8(*args, kv_tile=2)["o"]
+    spread = float(np.abs(per_block - per_step).max())
+    blocks = [(0, h, i) for h in range(w.H) for i in range(w.n_q)]
+    compare(got, per_step, blocks, w.bq, tol=TOL_FP8)
+    compare(got, per_block, blocks, w.bq, tol=TOL_FP8 + spread)
