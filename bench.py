@@ -2,22 +2,31 @@
 """Benchmark of the SLA2 attention forward (router + linear totals + sparse
 attention) on synthetic Wan2.1-shaped inputs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan13] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan13]
+                    [--fp8] [--keep-ratio R] [--impl reference]
 
-One process per GPU (torchrun for N > 1).  Each rank runs the whole hot path
-on its own batch (weak scaling; the heads of different ranks never interact,
-so there is no collective on the data path).  Rank 0 prints one JSON line.
+One process per GPU.  Under torchrun each process is one rank; `--gpus N`
+with N > 1 outside a launcher starts N ranks of itself under torchrun.  Each
+rank runs the whole hot path on its own batch (weak scaling; the heads of
+different ranks never interact, so there is no collective on the data path),
+the job's time is the maximum over ranks, and rank 0 prints one JSON line.
 
 A step = sla_prepare + sla_route(SLA_ROUTE_KBAR_FROM_WS) + sla2_attn_fwd(
 SLA_FLAG_PREPARED) on one batch already resident in HBM (bf16, d = 128: the
-router takes the key-block means the prepass wrote; other inputs route first).  Inputs (Q, K, V: 302 MB at the 1.3B shape)
-exceed the 126 MB L2, so the timed loop does not flush L2 between steps.
-`--impl reference` times the CPU oracle (the only reference that exists) on
-a bounded sample of the same workload on rank 0.
+router takes the key-block means the prepass wrote; other inputs route
+first).  Inputs (Q, K, V: 302 MB at the 1.3B shape) exceed the 126 MB L2, so
+the timed loop does not flush L2 between steps.  `--fp8` (or an fp8_*
+workload) runs the e4m3 sparse branch and reports its roofline against an
+e4m3 tensor peak measured in the same run.  The e2e figure times
+sla2_forward_host: pinned host inputs in, the output back to the host, one
+C-ABI call per step.  `--impl reference` times the CPU oracle (the only
+reference that exists) on a bounded sample of the same workload on rank 0,
+without loading the library.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -33,7 +42,19 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_linear_attention_b200 import dist_timing, inputs, sla  # noqa: E402
+from sparse_linear_attention_b200 import dist_timing, inputs  # noqa: E402
+
+# the library's binding, loaded only by the legs that run the GPU path (the
+# reference arm times the CPU oracle alone and never maps libsla.so)
+sla = None
+
+
+def _load_binding():
+    global sla
+    if sla is None:
+        from sparse_linear_attention_b200 import sla as binding
+        sla = binding
+    return sla
 
 METRIC = "SLA2 attn fwd ms & effective TOPS @Wan-1.3B shape, 97% sparse; % tensor peak"
 UNIT = "effective TOPS (4*N^2*d*H*B per forward / time)"
@@ -48,10 +69,18 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def keep_of(w):
+def keep_of(w, count=None):
+    """Kept blocks per query block: the workload's count, else its ratio through
+    `count` (the library's sla_keep_count on the GPU legs, the oracle's
+    keep_count on the CPU legs)."""
     if w.keep_count is not None:
         return w.keep_count
-    return sla.sla_keep_count(w.keep_ratio, w.n_kv)
+    return (count or sla.sla_keep_count)(w.keep_ratio, w.n_kv)
+
+
+def oracle_keep_of(w):
+    from oracle import sla_oracle as orc
+    return keep_of(w, orc.keep_count)
 
 
 def work_counts(w, kept_cpu):
@@ -141,7 +170,7 @@ class OracleTimer:
         self.orc, self.w, self.x = orc, w, x
         q32, k32 = x["q"].to(torch.float32).numpy(), x["k"].to(torch.float32).numpy()
         t0 = time.perf_counter()
-        self.kept, _, _ = orc.route(q32, k32, x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv, "sla2", keep_of(w))
+        self.kept, _, _ = orc.route(q32, k32, x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv, "sla2", oracle_keep_of(w))
         self.t_route = time.perf_counter() - t0
         self.heads = {}
         self.blocks = 0
@@ -330,6 +359,64 @@ def backward_leg(args, w, dev, stream):
     }), flush=True)
 
 
+def fp8_peak_tflops(dev, reps=10):
+    """Dense e4m3 tensor-core throughput measured here, the way the bf16 peak
+    is: torch._scaled_mm (cuBLASLt) on 8192^3 e4m3 operands with fp32 scales,
+    2*N^3 FLOP, best of `reps` CUDA-event timings after warm-up."""
+    n = 8192
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    one = torch.ones((), device=dev)
+    mm = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def hbm_roofline(name, bytes_, ms, hbm, src, what):
+    achieved = bytes_ / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "peak_source": f"{src} HBM copy", "algorithmic": what}
+
+
+def reference_arm(args, w):
+    """The CPU oracle (the only reference that exists) on a bounded sample of
+    the workload, rank 0 only; the library is never loaded here."""
+    rank, _, _ = dist_timing.world_info()
+    if rank != 0:
+        return
+    x = inputs.make_inputs(w)
+    ot = OracleTimer(w, x)
+    for _ in range(args.warmup):
+        ot.one_block()
+    ot.t_att, ot.blocks = 0.0, 0
+    vals = [ot.one_block() for _ in range(args.steps)]
+    full = 4.0 * w.N * w.N * w.d * w.H * w.B
+    t = statistics.median(vals)
+    val = full / t / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
+                               f"keep={oracle_keep_of(w)}/{w.n_kv} key blocks"},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": OracleTimer.threads(), "kind": "oracle",
+                         "sample": ot.describe() + "; each step = one sampled query block"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -342,6 +429,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--phi", default="elu1", choices=["elu1", "softmax"],
                     help="linear-branch feature map (the pages' default for SLA2 is ELU+1)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the e4m3 (low-bit) sparse branch; implied by the fp8_* workloads")
+    ap.add_argument("--int8", action="store_true",
+                    help="the INT8 variant of the low-bit sparse branch (INT8 Q, K'; e4m3 P, V)")
+    ap.add_argument("--keep-ratio", type=float, default=None,
+                    help="SLA2 keep fraction instead of the workload's (the e4m3 sweep: 0.03, 0.05, 0.10)")
     ap.add_argument("--soft-topk", action="store_true",
                     help="time the SoftTop-k router (sla_route_soft) instead of the forward step")
     ap.add_argument("--backward", action="store_true",
@@ -349,39 +442,31 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
 
+    # --gpus N outside a launcher: start N ranks of this script under torchrun
+    if args.gpus > 1 and not dist_timing.launched():
+        raise SystemExit(dist_timing.run_ranks(os.path.abspath(__file__), sys.argv[1:], args.gpus))
     rank, world, local = dist_timing.world_info()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
+
     w = inputs.WORKLOADS[args.workload]
-    if w.fp8:
-        raise SystemExit("bench.py times the bf16 path; pick a workload without fp8")
-    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk or args.backward):
-        raise SystemExit("the reference arm, --soft-topk and --backward time the SLA2 router / forward / backward")
+    if args.keep_ratio is not None:
+        w = dataclasses.replace(w, keep_ratio=args.keep_ratio, keep_count=None)
+    int8 = args.int8
+    fp8 = (args.fp8 or w.fp8) and not int8
+    low = fp8 or int8
+    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk or args.backward or low):
+        raise SystemExit("the reference arm, --fp8, --int8, --soft-topk and --backward are SLA2 legs")
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+
+    _load_binding()
     phi = sla.SLA_PHI_ELU1 if args.phi == "elu1" else sla.SLA_PHI_SOFTMAX
     sla_mode = w.mode == "sla"
-
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        x = inputs.make_inputs(w)
-        ot = OracleTimer(w, x)
-        for _ in range(args.warmup):
-            ot.one_block()
-        ot.t_att, ot.blocks = 0.0, 0
-        vals = [ot.one_block() for _ in range(args.steps)]
-        full, _ = work_counts(w, torch.zeros(w.B, w.H, w.n_q, 0, dtype=torch.int32))
-        t = statistics.median(vals)
-        val = full / t / 1e12
-        print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
-                                   f"keep={keep_of(w)}/{w.n_kv} key blocks"},
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": OracleTimer.threads(), "kind": "oracle",
-                             "sample": ot.describe() + "; each step = one sampled query block"},
-            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }), flush=True)
-        return
 
     if world > 1:
         import datetime
@@ -411,12 +496,17 @@ def main():
     wq, wk, alpha = x["wq"].to(dev), x["wk"].to(dev), x["alpha"].to(dev)
     wproj = x["wproj"].to(dev)
     shape = sla.make_shape(q, w.bq, w.bkv)
-    ws = torch.zeros(sla.sla_workspace_size(shape, mode), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(sla.sla_workspace_size(shape, mode | (sla.SLA_WS_FP8 if low else 0)), dtype=torch.uint8,
+                     device=dev)
     kept = torch.empty(w.B, w.H, w.n_q, k, dtype=torch.int32, device=dev)
     labels = torch.empty(w.B, w.H, w.n_q, w.n_kv, dtype=torch.int8, device=dev) if sla_mode else None
     out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
-    # route 2, prepare 3 (+ Q conversion off the d = 128 bf16 grid), attention 1 (+ SLA label lists 1)
-    launches_per_step = 2 + 3 + 1 + (1 if (w.d != 128 or w.dtype == "f32") else 0) + (1 if sla_mode else 0)
+    low_flag = sla.SLA_FLAG_INT8 if int8 else (sla.SLA_FLAG_FP8 if fp8 else 0)
+    attn_flags = sla.SLA_FLAG_PREPARED | low_flag
+    # route 2, prepare 3 (+ Q conversion off the d = 128 bf16 grid), attention 1 (+ SLA label lists 1,
+    # + e4m3 statistics and quantisation 2)
+    launches_per_step = (2 + 3 + 1 + (1 if (w.d != 128 or w.dtype == "f32") else 0) + (1 if sla_mode else 0)
+                         + (2 if low else 0))
 
     # bf16, d = 128: the prepass also writes the key-block means, so the router
     # runs after it and reads K only through the prepass (SLA_ROUTE_KBAR_FROM_WS)
@@ -441,7 +531,7 @@ def main():
         if sla_mode:
             sla.sla_attn_fwd(shape, q, kk, v, labels, wproj, phi, sla.SLA_FLAG_PREPARED, out, ws, stream)
         else:
-            sla.sla2_attn_fwd(shape, q, kk, v, kept, k, alpha, phi, sla.SLA_FLAG_PREPARED, out, ws, stream)
+            sla.sla2_attn_fwd(shape, q, kk, v, kept, k, alpha, phi, attn_flags, out, ws, stream)
         if ev is not None:
             ev[3].record(stream)
 
@@ -479,20 +569,50 @@ def main():
 
     hbm, bf16_burst, bf16_sus, peak_src = peaks()
     achieved = sparse_flop / (sparse_ms * 1e-3) / 1e12
-    traffic = profile_traffic(os.path.join(ROOT, "sparse_linear_attention_b200", "csrc", "sparse_fwd.cu"))
+    if low:
+        tc_peak, tc_src = fp8_peak_tflops(dev), "measured here: torch._scaled_mm e4m3 8192^3, best of 10 (burst)"
+        if int8:
+            tc_src += "; the INT8 variant's S runs kind::i8, whose nominal dense rate equals e4m3's"
+    else:
+        tc_peak, tc_src = bf16_burst, f"{peak_src} bf16 dense (burst)"
+    traffic = None if low else profile_traffic(os.path.join(ROOT, "sparse_linear_attention_b200", "csrc",
+                                                            "sparse_fwd.cu"))
+    # HBM-bound stages by their algorithmic bytes: the prepass reads K and V, the
+    # router reads Q (and K too unless the prepass handed it the key-block means)
+    elt = 2 if w.dtype == "bf16" else 4
+    tensor_bytes = w.B * w.H * w.N * w.d * elt
+    hbm_lines = {
+        "prepare": hbm_roofline("lin_prepass_tma_kernel + zsum/hsum", 2 * tensor_bytes, prep_ms, hbm, peak_src,
+                                "read K, V once (2*B*H*N*d*elt bytes)"),
+        "route": hbm_roofline("pool_project_kernel + score_select_kernel",
+                              tensor_bytes * (1 if kbar_first else 2), route_ms, hbm, peak_src,
+                              "read Q" + ("" if kbar_first else " and K") + " once"),
+    }
 
-    # end to end through the public API: pinned host inputs in, output back out
+    # end to end through the public API: pinned host buffers in, the output back
+    # out, inside one C-ABI call per step (sla2_forward_host); SLA copies with torch
     hq, hk, hv = (t.pin_memory() for t in (x["q"], x["k"], x["v"]))
     hwq, hwk, hal, hwp = (t.pin_memory() for t in (x["wq"], x["wk"], x["alpha"], x["wproj"]))
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hwq, hwk, hwp if sla_mode else hal))
     d2h = hout.numel() * hout.element_size()
+    if sla_mode:
+        e2e_api = "torch copies around sla_route + sla_prepare + sla_attn_fwd"
 
-    def e2e_step():
-        for dst, src in ((q, hq), (kk, hk), (v, hv), (wq, hwq), (wk, hwk), (wproj, hwp) if sla_mode else (alpha, hal)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
+        def e2e_step():
+            for dst, src in ((q, hq), (kk, hk), (v, hv), (wq, hwq), (wk, hwk), (wproj, hwp)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+    else:
+        e2e_api = "sla2_forward_host (host buffers in and out, one C-ABI call per step)"
+        hflags = low_flag
+        dbuf = torch.zeros(sla.sla2_forward_host_device_bytes(shape, k, sla.SLA_BF16, hflags), dtype=torch.uint8,
+                           device=dev)
+        del ws  # the host call carries its own workspace inside dbuf
+
+        def e2e_step():
+            sla.sla2_forward_host(shape, hq, hk, hv, hwq, hwk, hal, k, phi, hflags, hout, None, dbuf, stream)
 
     for _ in range(3):
         e2e_step()
@@ -504,11 +624,14 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
+    if not sla_mode and sla.sla_read_device_status(dbuf, stream) != 0:
+        raise SystemExit("device-side error during the end-to-end steps")
     e2e_ms = dist_timing.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
     e2e_val = dist_timing.job_throughput(full_ops, e2e_ms, world) / 1e12
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not sla_mode and phi == sla.SLA_PHI_ELU1:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not sla_mode and not low
+            and phi == sla.SLA_PHI_ELU1):
         ot = OracleTimer(w, x)
         while ot.t_att < args.cpu_budget or ot.blocks < 4:
             ot.one_block()
@@ -520,26 +643,33 @@ def main():
         dist.destroy_process_group()
     if not dist_timing.reports(rank):
         return
+    shape_names = {"wan13": "Wan2.1-1.3B-480P latent shape", "wan14": "Wan2.1-14B-720P latent shape",
+                   "fp8_13": "Wan2.1-1.3B-480P latent shape, e4m3 sparse branch",
+                   "fp8_14": "Wan2.1-14B-720P latent shape, e4m3 sparse branch"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: Wan2.1-1.3B-480P latent shape" if w.name == "wan13" else w.name,
+        "vs_baseline": None, "dtype": "int8+e4m3" if int8 else ("e4m3" if fp8 else "bf16"), "data": "synthetic",
+        "config": {"workload": f"{w.name}: {shape_names[w.name]}" if w.name in shape_names else w.name,
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bkv": w.bkv,
                    "kept_blocks": f"{k}/{w.n_kv} per query block ({100.0 * (1 - k / w.n_kv):.2f}% sparse)",
                    "phi": "elu+1" if phi == sla.SLA_PHI_ELU1 else "softmax over channels",
                    "method": "SLA (critical / marginal / negligible, O_s + Proj(O_l))" if sla_mode
-                   else "SLA2 (top-k, alpha mix)", "global_batch": w.B * world,
+                   else "SLA2 (top-k, alpha mix)" + (", e4m3 sparse branch" if fp8 else "")
+                   + (", INT8 Q/K' with e4m3 P/V sparse branch" if int8 else ""),
+                   "global_batch": w.B * world,
                    "l2": "no flush: Q,K,V = %.0f MB per rank > 126 MB L2" % (3 * q.numel() * 2 / 1e6)},
         "breakdown_ms": {"route": route_ms, "prepare": prep_ms, "sparse_attention": sparse_ms},
         "sparse_tflops_executed": achieved,
         "roofline": {"bound": "tensor", "kernel": "sparse_fwd_kernel", "achieved": achieved,
-                     "peak": bf16_burst, "unit": "TFLOP/s", "frac": achieved / bf16_burst,
-                     "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": traffic,
-                     "algorithmic": "4*d FLOP per (query row, kept valid key): QK^T + PV on kept tiles"},
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
+                     "peak_source": tc_src, "traffic": traffic,
+                     "algorithmic": "4*d FLOP per (query row, kept valid key): QK^T + PV on kept tiles"
+                                    + ("; the attention call includes the 8-bit quantisation" if low else "")},
+        "hbm_rooflines": hbm_lines,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": UNIT, "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "api": e2e_api},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }

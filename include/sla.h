@@ -73,6 +73,20 @@ typedef enum { SLA_MODE_SLA2_TOPK = 0, SLA_MODE_SLA_3WAY = 1 } sla_route_mode;
 /* flags for the attention entry points */
 #define SLA_FLAG_PREPARED 1u  /* ws already holds sla_prepare's results for these K, V */
 #define SLA_FLAG_FP8 2u       /* low-bit (e4m3) sparse branch [SLA2-deep §07], SLA2 only */
+/* The page's other low-bit format ("INT8 or FP8" [SLA2-deep §07]): Q and
+ * K - mean(K) as INT8 codes rint(x * 127 / amax) (ties to even, saturated to
+ * +-127, one scale amax / 127 per 128-token block), S as an exact integer
+ * product; P and V in e4m3 as with SLA_FLAG_FP8.  SLA2 only; excludes
+ * SLA_FLAG_FP8; the workspace is sized with SLA_WS_FP8. */
+#define SLA_FLAG_INT8 4u
+/* Test hook for the device-side failure detection, not for production use:
+ * every bounded wait of the attention kernel gives up as soon as it is not
+ * already satisfied (limit 0 instead of 1 s), as a wait that ran out would.
+ * The kernel then stops issuing work, drains the copies and tensor-core
+ * products it started, frees its tensor memory and returns; the call's output
+ * is undefined and sla_read_device_status reports SLA_ERR_TIMEOUT.  No wait
+ * is left unsatisfied on purpose: the limit, not a missing arrival, ends it. */
+#define SLA_FLAG_WAIT_TEST 8u
 
 /* OR into the mode of sla_workspace_size to include the buffers of the
  * low-bit sparse branch (e4m3 copies of Q, K - mean(K), V and their scales). */
@@ -157,8 +171,10 @@ sla_status sla_route_soft(const sla_shape* shape, const void* q, const void* k,
  * for example code that runs under another framework's memory manager and
  * may not allocate outside it, or that must not call cudaMalloc where it
  * routes.  It computes exactly what sla_route computes (same kernels, same
- * bit-exact results) with the same arguments minus ws / ws_bytes; its scratch
- * is a 16 MiB array compiled into the library, held by every GPU that loads
+ * bit-exact results) with the same arguments minus ws / ws_bytes, except that
+ * mode may not carry SLA_ROUTE_KBAR_FROM_WS (there is no workspace holding
+ * the prepass's key-block means: SLA_ERR_INVALID_ARG).  Its scratch is a
+ * 16 MiB array compiled into the library, held by every GPU that loads
  * libsla until the process exits.
  *   - Shapes whose scratch, B*H*(n_q + n_kv)*d floats (the projected block
  *     means of Q and K, each piece rounded up to 256 bytes), exceeds 16 MiB
@@ -167,9 +183,14 @@ sla_status sla_route_soft(const sla_shape* shape, const void* q, const void* k,
  *     workload needs 4.7 MB.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept with the id of the
+ *     CUDA context it belongs to; a call that finds another context current
+ *     (after cudaDeviceReset, say) looks it up again, so that call too should
+ *     come before any capture.
  *   - All calls share the array: calls that overlap on the GPU race.  Nothing
- *     in it needs to start at zero; each call overwrites what it reads.
+ *     in it needs to start at zero: each call writes every value that reaches
+ *     its results before reading it.
+ *   - Every rejected argument also sets sla_last_error_detail.
  *   - Nothing is allocated or freed. */
 sla_status sla_route_noalloc(const sla_shape* shape, const void* q, const void* k,
                              const float* Wq, const float* Wk, int mode, int k_keep,
@@ -241,6 +262,36 @@ sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k,
                          const float* alpha, int phi, const void* dout,
                          float* dq, float* dk, float* dv, float* dalpha,
                          void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device memory sla2_forward_host needs (0 for invalid arguments):
+ * the workspace of sla_workspace_size (with SLA_WS_FP8 when flags carry
+ * SLA_FLAG_FP8 or SLA_FLAG_INT8) followed by device copies of Q, K, V, Wq, Wk, alpha, the kept
+ * lists and the output, each 256-byte aligned. */
+size_t sla2_forward_host_device_bytes(const sla_shape* shape, int k_keep, int out_dtype, unsigned flags);
+
+/* One whole SLA2 forward from host memory [SLA2-deep §04, §05, §08]: the
+ * router (top-k_keep per query block), the linear-branch totals and the
+ * attention call, exactly as sla_route + sla_prepare + sla2_attn_fwd compute
+ * them, with the inputs copied in and the output copied out on `stream`.
+ *   q, k, v  host [B,H,N,d] of shape->in_dtype;  Wq, Wk host d x d fp32
+ *            (nullable = identity);  alpha host fp32 [B,H,n_q];
+ *   out      host [B,H,N,d] of out_dtype (SLA_F32 / SLA_BF16);
+ *   kept_out host int32 [B,H,n_q,k_keep] (nullable): the router's kept lists.
+ *   flags    0, SLA_FLAG_FP8 or SLA_FLAG_INT8 (the low-bit sparse branches).
+ *   dev      device memory of sla2_forward_host_device_bytes bytes, 256-byte
+ *            aligned, caller-owned; its first 256 bytes are the workspace
+ *            status word (zero it once with sla_workspace_init, read it with
+ *            sla_read_device_status(dev, stream)).
+ * Everything is enqueued on `stream`; the call returns without waiting, so
+ * the host buffers must stay valid (and out unread) until the stream is
+ * synchronised.  Page-locked host memory lets the copies run asynchronously;
+ * one cudaMemcpyAsync is issued per buffer.  Same argument rules as the calls
+ * it combines. */
+sla_status sla2_forward_host(const sla_shape* shape, const void* q, const void* k,
+                             const void* v, const float* Wq, const float* Wk,
+                             const float* alpha, int k_keep, int phi, unsigned flags,
+                             void* out, int out_dtype, int32_t* kept_out, void* dev,
+                             size_t dev_bytes, void* stream);
 
 /* Synchronise `stream`, then return (and clear) the device status word that
  * kernels write when a bounded wait runs out or a block index is out of

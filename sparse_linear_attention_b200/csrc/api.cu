@@ -114,10 +114,12 @@ sla_status run_attention(const sla_shape* s, const void* q, const void* k, const
   if (L.need_hat) {
     if ((e = launch_qhat(*s, q, L, ws, st)) != cudaSuccess) return cuda_fail(e, "qhat");
   }
-  a.fp8 = (flags & SLA_FLAG_FP8) ? 1 : 0;
+  a.fp8 = (flags & SLA_FLAG_INT8) ? 2 : ((flags & SLA_FLAG_FP8) ? 1 : 0);
+  a.wait_ns = (flags & SLA_FLAG_WAIT_TEST) ? 0ull : kWaitLimitNs;
   a.nb128 = ceil_div(s->N, 128);
   if (a.fp8) {
-    if ((e = launch_fp8_quant(*s, q, k, v, L, ws, st)) != cudaSuccess) return cuda_fail(e, "fp8 quantisation");
+    if ((e = launch_fp8_quant(*s, q, k, v, L, ws, st, a.fp8 == 2)) != cudaSuccess)
+      return cuda_fail(e, "low-bit quantisation");
     a.sq = reinterpret_cast<const float*>(ws + L.sq);
     a.sk = reinterpret_cast<const float*>(ws + L.sk);
     a.vamax = reinterpret_cast<const float*>(ws + L.sv);
@@ -255,11 +257,14 @@ sla_status sla2_attn_fwd(const sla_shape* shape, const void* q, const void* k, c
   if (k_keep > 0 && kept_idx == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "kept_idx is null");
   if (alpha == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "alpha is null");
   if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
-  if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8)) return arg_fail(SLA_ERR_INVALID_ARG, "flags");
+  if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8 | SLA_FLAG_INT8 | SLA_FLAG_WAIT_TEST))
+    return arg_fail(SLA_ERR_INVALID_ARG, "flags");
+  if ((flags & SLA_FLAG_FP8) && (flags & SLA_FLAG_INT8))
+    return arg_fail(SLA_ERR_INVALID_ARG, "flags: SLA_FLAG_FP8 and SLA_FLAG_INT8 exclude each other");
   if (out == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "out is null");
   if (!aligned16(out)) return arg_fail(SLA_ERR_ALIGNMENT, "out must be 16-byte aligned");
   if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return arg_fail(SLA_ERR_INVALID_ARG, "out_dtype");
-  const int wsmode = SLA_MODE_SLA2_TOPK | ((flags & SLA_FLAG_FP8) ? SLA_WS_FP8 : 0);
+  const int wsmode = SLA_MODE_SLA2_TOPK | ((flags & (SLA_FLAG_FP8 | SLA_FLAG_INT8)) ? SLA_WS_FP8 : 0);
   if ((s = check_ws(shape, wsmode, ws, ws_bytes)) != SLA_OK) return s;
   const WsLayout L = ws_layout(*shape, wsmode);
   SparseArgs a{};
@@ -316,8 +321,10 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k, co
   if (Wproj == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Wproj is null");
   if (!aligned16(Wproj)) return arg_fail(SLA_ERR_ALIGNMENT, "Wproj must be 16-byte aligned");
   if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
-  if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8)) return arg_fail(SLA_ERR_INVALID_ARG, "flags");
-  if (flags & SLA_FLAG_FP8) return arg_fail(SLA_ERR_UNSUPPORTED, "the e4m3 sparse branch is built for SLA2 only");
+  if (flags & ~(SLA_FLAG_PREPARED | SLA_FLAG_FP8 | SLA_FLAG_INT8 | SLA_FLAG_WAIT_TEST))
+    return arg_fail(SLA_ERR_INVALID_ARG, "flags");
+  if (flags & (SLA_FLAG_FP8 | SLA_FLAG_INT8))
+    return arg_fail(SLA_ERR_UNSUPPORTED, "the low-bit sparse branch is built for SLA2 only");
   if (out == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "out is null");
   if (!aligned16(out)) return arg_fail(SLA_ERR_ALIGNMENT, "out must be 16-byte aligned");
   if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return arg_fail(SLA_ERR_INVALID_ARG, "out_dtype");
@@ -340,6 +347,104 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k, co
   a.out = out;
   a.out_bf16 = out_dtype == SLA_BF16;
   return run_attention(shape, q, k, v, phi, flags, L, w, st, a);
+}
+
+// Device layout of sla2_forward_host: the workspace first (its status word at
+// offset 0), then the device copies of the inputs, the kept lists and the output.
+struct HostLayout {
+  WsLayout ws;
+  size_t q = 0, k = 0, v = 0, wq = 0, wk = 0, alpha = 0, kept = 0, out = 0, total = 0;
+  size_t in_bytes = 0, out_bytes = 0;
+};
+
+static HostLayout host_layout(const sla_shape& s, int k_keep, int out_dtype, unsigned flags) {
+  HostLayout H;
+  H.ws = ws_layout(s, SLA_MODE_SLA2_TOPK | ((flags & (SLA_FLAG_FP8 | SLA_FLAG_INT8)) ? SLA_WS_FP8 : 0));
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t nq = static_cast<size_t>(ceil_div(s.N, s.bq));
+  const size_t elt = s.in_dtype == SLA_BF16 ? 2 : 4;
+  H.in_bytes = BH * s.N * s.d * elt;
+  H.out_bytes = BH * s.N * s.d * (out_dtype == SLA_BF16 ? 2 : 4);
+  size_t off = H.ws.total;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  H.q = take(H.in_bytes);
+  H.k = take(H.in_bytes);
+  H.v = take(H.in_bytes);
+  H.wq = take(static_cast<size_t>(s.d) * s.d * 4);
+  H.wk = take(static_cast<size_t>(s.d) * s.d * 4);
+  H.alpha = take(BH * nq * 4);
+  H.kept = take(BH * nq * static_cast<size_t>(k_keep > 0 ? k_keep : 0) * 4);
+  H.out = take(H.out_bytes);
+  H.total = off;
+  return H;
+}
+
+size_t sla2_forward_host_device_bytes(const sla_shape* shape, int k_keep, int out_dtype, unsigned flags) {
+  if (check_shape(shape) != SLA_OK || k_keep < 0 || k_keep > ceil_div(shape->N, shape->bkv)) return 0;
+  if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return 0;
+  return host_layout(*shape, k_keep, out_dtype, flags).total;
+}
+
+sla_status sla2_forward_host(const sla_shape* shape, const void* q, const void* k, const void* v, const float* Wq,
+                             const float* Wk, const float* alpha, int k_keep, int phi, unsigned flags, void* out,
+                             int out_dtype, int32_t* kept_out, void* dev, size_t dev_bytes, void* stream) {
+  sla_status s = check_shape(shape);
+  if (s != SLA_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Q, K or V is null");
+  if (alpha == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "alpha is null");
+  if (out == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "out is null");
+  if (out_dtype != SLA_F32 && out_dtype != SLA_BF16) return arg_fail(SLA_ERR_INVALID_ARG, "out_dtype");
+  if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
+  if (flags & ~(SLA_FLAG_FP8 | SLA_FLAG_INT8))
+    return arg_fail(SLA_ERR_INVALID_ARG, "flags (only SLA_FLAG_FP8 or SLA_FLAG_INT8 is accepted)");
+  const int nkv = ceil_div(shape->N, shape->bkv);
+  if (nkv > kMaxNKV) return arg_fail(SLA_ERR_UNSUPPORTED, "router needs n_kv <= 2048");
+  if (k_keep < 0 || k_keep > nkv) return arg_fail(SLA_ERR_INVALID_ARG, "k_keep outside [0, n_kv]");
+  if (dev == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "dev is null");
+  if ((reinterpret_cast<uintptr_t>(dev) & 255u) != 0) return arg_fail(SLA_ERR_ALIGNMENT, "dev must be 256-byte aligned");
+  const HostLayout H = host_layout(*shape, k_keep, out_dtype, flags);
+  if (dev_bytes < H.total) return arg_fail(SLA_ERR_WORKSPACE, "dev smaller than sla2_forward_host_device_bytes");
+  char* d = static_cast<char*>(dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t nq = static_cast<size_t>(ceil_div(shape->N, shape->bq));
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const size_t wbytes = static_cast<size_t>(shape->d) * shape->d * 4;
+  // one plain asynchronous copy per buffer (pinned host memory lets them overlap the host)
+  struct { void* dst; const void* src; size_t n; } in[] = {
+      {d + H.q, q, H.in_bytes}, {d + H.k, k, H.in_bytes}, {d + H.v, v, H.in_bytes},
+      {d + H.wq, Wq, Wq ? wbytes : 0}, {d + H.wk, Wk, Wk ? wbytes : 0}, {d + H.alpha, alpha, BH * nq * 4}};
+  for (const auto& c : in) {
+    if (c.n == 0) continue;
+    cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  }
+  const float* wq_d = Wq ? reinterpret_cast<const float*>(d + H.wq) : nullptr;
+  const float* wk_d = Wk ? reinterpret_cast<const float*>(d + H.wk) : nullptr;
+  int32_t* kept_d = reinterpret_cast<int32_t*>(d + H.kept);
+  // bf16, d = 128: the prepass writes the key-block means and the router reuses them
+  const bool kbar_first = shape->in_dtype == SLA_BF16 && shape->d == kDPad;
+  const size_t wsb = H.ws.total;
+  if (kbar_first && (s = sla_prepare(shape, d + H.k, d + H.v, phi, d, wsb, stream)) != SLA_OK) return s;
+  if ((s = sla_route(shape, d + H.q, d + H.k, wq_d, wk_d, SLA_MODE_SLA2_TOPK | (kbar_first ? SLA_ROUTE_KBAR_FROM_WS : 0),
+                     k_keep, 0, kept_d, nullptr, nullptr, d, wsb, stream)) != SLA_OK)
+    return s;
+  if (!kbar_first && (s = sla_prepare(shape, d + H.k, d + H.v, phi, d, wsb, stream)) != SLA_OK) return s;
+  if ((s = sla2_attn_fwd(shape, d + H.q, d + H.k, d + H.v, kept_d, k_keep, reinterpret_cast<const float*>(d + H.alpha),
+                         phi, SLA_FLAG_PREPARED | (flags & (SLA_FLAG_FP8 | SLA_FLAG_INT8)), d + H.out, out_dtype, d,
+                         wsb, stream)) !=
+      SLA_OK)
+    return s;
+  cudaError_t e = cudaMemcpyAsync(out, d + H.out, H.out_bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  if (kept_out != nullptr && k_keep > 0) {
+    e = cudaMemcpyAsync(kept_out, kept_d, BH * nq * k_keep * 4, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  return SLA_OK;
 }
 
 sla_status sla_read_device_status(void* ws, void* stream) {

@@ -702,6 +702,18 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
+// Four signed INT8 codes: rint(x) with ties to even, saturated to [-127, 127].
+__device__ __forceinline__ uint32_t i8x4(float a, float b, float c, float d) {
+  const float x[4] = {a, b, c, d};
+  uint32_t w = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int q = max(-127, min(127, __float2int_rn(x[e])));
+    w |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * e);
+  }
+  return w;
+}
+
 __device__ __forceinline__ float block_absmax(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -715,9 +727,11 @@ __device__ __forceinline__ float block_absmax(float v, float* red) {
 }
 
 // One 128-token block of one head per CTA (256 threads, 8 channel units each):
-// e4m3 copies of Q and K - mean(K) with the block's scale, and of V with the
-// per-channel scale.  Channels past d and rows past N stay zero.
-template <typename T>
+// 8-bit copies of Q and K - mean(K) with the block's scale (e4m3 codes of
+// x * 448 / amax, or with kInt8 the INT8 codes of x * 127 / amax), and the e4m3
+// copy of V with the per-channel scale.  Channels past d and rows past N stay
+// zero.
+template <typename T, bool kInt8>
 __global__ void __launch_bounds__(256) fp8_quant_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ mu,
                                                         const float* __restrict__ vamax, uint8_t* __restrict__ q8,
@@ -755,9 +769,10 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const T* __restrict__ q,
     }
     float inv[8];
     if (which < 2) {
+      const float qmax = kInt8 ? 127.0f : 448.0f;
       const float amax = block_absmax(am, red);
-      const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : __fdiv_rn(1.0f, 448.0f);
-      const float iv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+      const float sc = amax > 0.0f ? __fdiv_rn(amax, qmax) : __fdiv_rn(1.0f, qmax);
+      const float iv = amax > 0.0f ? __fdiv_rn(qmax, amax) : 1.0f;
       if (tid == 0) (which == 0 ? sq : sk)[bh * nb128 + blk] = sc;
 #pragma unroll
       for (int e = 0; e < 8; ++e) inv[e] = iv;
@@ -770,6 +785,14 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const T* __restrict__ q,
       const int tok = blk * 128 + tid / 16 + 16 * i;
       if (tok < N) {
         const float* y = x[i];
+        if (kInt8 && which < 2) {
+          const uint2 w = make_uint2(i8x4(__fmul_rn(y[0], inv[0]), __fmul_rn(y[1], inv[1]), __fmul_rn(y[2], inv[2]),
+                                          __fmul_rn(y[3], inv[3])),
+                                     i8x4(__fmul_rn(y[4], inv[4]), __fmul_rn(y[5], inv[5]), __fmul_rn(y[6], inv[6]),
+                                          __fmul_rn(y[7], inv[7])));
+          *reinterpret_cast<uint2*>(dst + (base + tok) * kDPad + 8 * u) = w;
+          continue;
+        }
         const uint2 w = make_uint2(e4m3x4(__fmul_rn(y[0], inv[0]), __fmul_rn(y[1], inv[1]), __fmul_rn(y[2], inv[2]),
                                           __fmul_rn(y[3], inv[3])),
                                    e4m3x4(__fmul_rn(y[4], inv[4]), __fmul_rn(y[5], inv[5]), __fmul_rn(y[6], inv[6]),
@@ -783,7 +806,7 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const T* __restrict__ q,
 }  // namespace
 
 cudaError_t launch_fp8_quant(const sla_shape& s, const void* q, const void* k, const void* v, const WsLayout& L,
-                             char* ws, cudaStream_t st) {
+                             char* ws, cudaStream_t st, bool int8_qk) {
   const int BH = s.B * s.H;
   const int nb128 = ceil_div(s.N, 128);
   float* mu = reinterpret_cast<float*>(ws + L.mu);
@@ -796,14 +819,23 @@ cudaError_t launch_fp8_quant(const sla_shape& s, const void* q, const void* k, c
   auto* v8 = reinterpret_cast<uint8_t*>(ws + L.v8);
   auto* sq = reinterpret_cast<float*>(ws + L.sq);
   auto* sk = reinterpret_cast<float*>(ws + L.sk);
-  if (s.in_dtype == SLA_BF16)
-    fp8_quant_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), mu, vam, q8, k8, v8, sq, sk, s.N, s.d, nb128);
-  else
-    fp8_quant_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                   static_cast<const float*>(v), mu, vam, q8, k8, v8, sq, sk, s.N,
-                                                   s.d, nb128);
+  auto run = [&](auto kernel, const auto* tq, const auto* tk, const auto* tv) {
+    kernel<<<grid, 256, 0, st>>>(tq, tk, tv, mu, vam, q8, k8, v8, sq, sk, s.N, s.d, nb128);
+  };
+  using BF = __nv_bfloat16;
+  if (s.in_dtype == SLA_BF16) {
+    const auto* tq = static_cast<const BF*>(q);
+    const auto* tk = static_cast<const BF*>(k);
+    const auto* tv = static_cast<const BF*>(v);
+    if (int8_qk) run(fp8_quant_kernel<BF, true>, tq, tk, tv);
+    else run(fp8_quant_kernel<BF, false>, tq, tk, tv);
+  } else {
+    const auto* tq = static_cast<const float*>(q);
+    const auto* tk = static_cast<const float*>(k);
+    const auto* tv = static_cast<const float*>(v);
+    if (int8_qk) run(fp8_quant_kernel<float, true>, tq, tk, tv);
+    else run(fp8_quant_kernel<float, false>, tq, tk, tv);
+  }
   return cudaGetLastError();
 }
 

@@ -29,9 +29,6 @@ __device__ __forceinline__ void report_error(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
-// Every wait in these kernels gives up after this long and reports
-// SLA_ERR_TIMEOUT instead of hanging the GPU.
-constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -70,17 +67,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Gives up when
-// *abort becomes nonzero (another role of the CTA failed) or after
-// kWaitLimitNs; in that case sets *abort, reports SLA_ERR_TIMEOUT and returns
-// false.  The caller must then stop issuing work.
+// *abort becomes nonzero (another role of the CTA failed) or after limit_ns
+// (kWaitLimitNs unless a test shortens it); in that case sets *abort, reports
+// SLA_ERR_TIMEOUT and returns false.  The caller must then stop issuing work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;  // the common case touches nothing else
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       report_error(status, SLA_ERR_TIMEOUT);
       return false;
@@ -122,6 +119,21 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier that also ANDs a predicate over its nthreads participants:
+// every participant gets the same verdict (so a group leaves a loop together).
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------- cp.async
 
 // 16-byte asynchronous copy global -> shared (L2 only), completed by
@@ -147,6 +159,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), completing on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -221,6 +243,18 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Same with kind::i8 (signed 8-bit integer operands, s32 accumulate, K = 32
+// per MMA): exact integer dot products.
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -372,6 +406,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab, uint32_t a_mn, uin
 // Instruction descriptor, kind::f8f6f4 with e4m3 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_f8(uint32_t a_mn, uint32_t b_mn, uint32_t M, uint32_t N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::i8 with signed 8-bit A and B, s32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_i8(uint32_t a_mn, uint32_t b_mn, uint32_t M, uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // Byte offset of 16-byte unit u (0..7) of row r inside a swizzled 128-byte-row tile.

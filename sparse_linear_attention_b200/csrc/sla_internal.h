@@ -14,6 +14,10 @@ constexpr int kMaxNKV = 2048;     // router limit on key blocks per head
 constexpr int kMaxN = 131072;     // token limit (n_kv <= 2048 at bkv = 64)
 constexpr int kNumSMs = 148;
 
+// Every wait in the kernels gives up after this long and reports
+// SLA_ERR_TIMEOUT instead of hanging the GPU.
+constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
 // Device workspace layout.  All offsets are 256-byte aligned.
 struct WsLayout {
   size_t status = 0;  // int32 status word (+ padding)

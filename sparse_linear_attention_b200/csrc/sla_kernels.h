@@ -28,8 +28,10 @@ cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int
                            char* ws, cudaStream_t st);
 
 // e4m3 copies of Q, K - mean(K), V and their scales (needs sla_prepare's statistics).
+// 8-bit copies for the low-bit sparse branch: e4m3 Q, K - mean(K), V; with
+// int8_qk the Q and K - mean(K) codes are INT8 instead (V stays e4m3).
 cudaError_t launch_fp8_quant(const sla_shape& s, const void* q, const void* k, const void* v, const WsLayout& L,
-                             char* ws, cudaStream_t st);
+                             char* ws, cudaStream_t st, bool int8_qk);
 
 cudaError_t launch_qhat(const sla_shape& s, const void* q, const WsLayout& L, char* ws, cudaStream_t st);
 
@@ -54,13 +56,14 @@ struct SparseArgs {
   int tma_out;               // bf16 output, d = 128, bq = 128: 128-row tiles leave through a TMA store
   int phi;
   int* status;
-  // e4m3 sparse branch
+  // low-bit sparse branch: 0 none (bf16), 1 e4m3 Q, K', P, V; 2 INT8 Q, K' with e4m3 P, V
   int fp8;
   int nb128;                 // ceil(N / 128)
   const float* sq;           // [BH, nb128] per-block scale of Q
   const float* sk;           // [BH, nb128] per-block scale of K - mean(K)
   const float* vamax;        // [BH, 128] column absmax of V
   const void* qsrc;          // bf16 [BH, N, 128] Q (for phi(Q) when the smem tile holds e4m3)
+  unsigned long long wait_ns;  // limit of every bounded wait (the exit drains keep their own)
 };
 
 // 3-D tensor map over a [BH][N][128] 16-bit array: boxes of 64 channels x

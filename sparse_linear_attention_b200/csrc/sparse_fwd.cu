@@ -172,17 +172,21 @@ __device__ __forceinline__ int block_at(const Tile& T, int it, int nkv, int* sta
 
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the verdict.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                          int* status, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xffffffffu, ok) != 0;
 }
 
-template <bool kFP8>
+// kLow: 0 = bf16 sparse branch; 1 = e4m3 Q, K', P, V; 2 = INT8 Q, K' (S as an
+// exact integer product, kind::i8) with e4m3 P, V.
+template <int kLow>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmV8,
                       const __grid_constant__ CUtensorMap tmO, const SparseArgs a) {
+  constexpr bool kFP8 = kLow != 0;  // the low-bit layout (8-bit Q, K', V)
+  constexpr bool kI8 = kLow == 2;
   using L = Lay<kFP8>;
   constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V;
   constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_RED = L::OFF_RED, OFF_Z = L::OFF_Z;
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the key tiles of step s (list positions 2s, 2s+1) into the next pair slot
       auto load_k = [&](const Tile& T, int s) -> bool {
         const int sl = gk % kKSlots;
-        if (gk >= kKSlots && !mbar_wait(&bars[B_SFULL + sl], ((gk / kKSlots) - 1) & 1, abort_flag, a.status))
+        if (gk >= kKSlots && !mbar_wait(&bars[B_SFULL + sl], ((gk / kKSlots) - 1) & 1, abort_flag, a.status, a.wait_ns))
           return false;  // S of the step two back has read this slot
         const bool two = 2 * s + 1 < T.n_crit;
         const int ra = block_at(T, 2 * s, a.nkv, a.status) * kBlockKV;
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto v_slot = [&](uint64_t*& fb) -> uint8_t* {
         const int sl = gv % kVSlots;
-        if (gv >= kVSlots && !mbar_wait(&bars[B_VEMPTY + sl], ((gv / kVSlots) - 1) & 1, abort_flag, a.status))
+        if (gv >= kVSlots && !mbar_wait(&bars[B_VEMPTY + sl], ((gv / kVSlots) - 1) & 1, abort_flag, a.status, a.wait_ns))
           return nullptr;
         fb = &bars[B_VFULL + sl];
         ++gv;
@@ -313,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ti = 0;
       for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++ti) {
         const Tile T = tile_at(a, t, true);
-        if (ti > 0 && !mbar_wait(&bars[B_QFREE], (ti - 1) & 1, abort_flag, a.status)) break;
+        if (ti > 0 && !mbar_wait(&bars[B_QFREE], (ti - 1) & 1, abort_flag, a.status, a.wait_ns)) break;
         mbar_arrive_expect_tx(&bars[B_QFULL], L::QBYTES);
         tma_load_3d(sm + OFF_Q, &tmQ, &bars[B_QFULL], 0, T.qb * a.bq, T.bh);
         if constexpr (!kFP8) tma_load_3d(sm + OFF_Q + 16384, &tmQ, &bars[B_QFULL], 64, T.qb * a.bq, T.bh);
@@ -350,6 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_bf = idesc_f16(1, 0, 1, 128, 128);  // TMEM A (bf16) x MN-major B
       const uint32_t id_qk8 = idesc_f8(0, 0, 128, 128);     // Q8 x [K8_a|K8_b], e4m3
       const uint32_t id_qk81 = idesc_f8(0, 0, 128, 64);
+      const uint32_t id_qki8 = idesc_i8(0, 0, 128, 128);    // Q8 x [K8_a|K8_b], INT8, s32 accumulate
+      const uint32_t id_qki81 = idesc_i8(0, 0, 128, 64);
       const uint32_t id_pv8 = idesc_f8(0, 1, 128, 128);     // P8 (TMEM) x V8 (MN-major), e4m3
       // Descriptors built once; a byte offset d inside the window adds d >> 4 to
       // the start-address field (addresses stay below 2^18, so it cannot carry).
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // data right after the previous PV.
       auto wait_k = [&]() -> bool {  // the next key pair has landed (TMA data: no tcgen05 fence needed)
         const int sl = gk % kKSlots;
-        return mbar_wait(&bars[B_KFULL + sl], (gk / kKSlots) & 1, abort_flag, a.status);
+        return mbar_wait(&bars[B_KFULL + sl], (gk / kKSlots) & 1, abort_flag, a.status, a.wait_ns);
       };
       // S for step s of T into buffer g & 1 (key pair already waited for); frees the slot when done
       auto issue_s = [&](const Tile& T, int s, int g, bool last_s) {
@@ -377,7 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + T_S0 + (g & 1) * 128;
         if constexpr (kFP8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + kk * 2u, kb + kk * 2u, two ? id_qk8 : id_qk81, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            if constexpr (kI8)
+              mma_i8_ss(d, dQ + kk * 2u, kb + kk * 2u, two ? id_qki8 : id_qki81, kk > 0 ? 1u : 0u);
+            else
+              mma_f8_ss(d, dQ + kk * 2u, kb + kk * 2u, two ? id_qk8 : id_qk81, kk > 0 ? 1u : 0u);
+          }
         } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -391,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto take_v = [&]() -> int {  // next V-ring entry, once it has landed
         const int sl = gv % kVSlots;
-        if (!mbar_wait(&bars[B_VFULL + sl], (gv / kVSlots) & 1, abort_flag, a.status)) return -1;
+        if (!mbar_wait(&bars[B_VFULL + sl], (gv / kVSlots) & 1, abort_flag, a.status, a.wait_ns)) return -1;
         ++gv;
         return sl;
       };
@@ -428,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pend_ti = 0;
       auto wait_epidone = [&]() -> bool {
         pend = false;
-        if (!mbar_wait(&bars[B_EPIDONE], pend_ti & 1, abort_flag, a.status)) return false;
+        if (!mbar_wait(&bars[B_EPIDONE], pend_ti & 1, abort_flag, a.status, a.wait_ns)) return false;
         tc_fence_after();
         return true;
       };
@@ -437,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile T = tile_at(a, t, false);
         if (sp) {
           // ---------------------------------------------- warp 9: S, PV
-          if (!mbar_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status)) break;
+          if (!mbar_wait(&bars[B_QFULL], ti & 1, abort_flag, a.status, a.wait_ns)) break;
           tc_fence_after();
           const int ns = T.nsteps;
           if (ns > 0) {
@@ -456,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               issue_s(T, i + 1, g + 1, i + 1 == ns - 1);
             }
-            if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status)) {
+            if (!mbar_wait(&bars[B_PFULL + b], (g >> 1) & 1, abort_flag, a.status, a.wait_ns)) {
               ok = false;
               break;
             }
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           mma_commit(&bars[B_HFIN]);
           // epilogue: phi(Q) (TMEM, the tile's last S buffer) x H_i / sigma (smem, the H tile's slot)
-          if (!mbar_wait(&bars[B_EPI], ti & 1, abort_flag, a.status)) break;
+          if (!mbar_wait(&bars[B_EPI], ti & 1, abort_flag, a.status, a.wait_ns)) break;
           tc_fence_after();
           const uint32_t ecol = T_S0 + ((gs + T.nsteps - 1) & 1) * 128;
           gs += T.nsteps;
@@ -514,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&bars[B_NUM]);
           if (a.wproj != nullptr) {
-            if (!mbar_wait(&bars[B_PROJR], ti & 1, abort_flag, a.status)) break;
+            if (!mbar_wait(&bars[B_PROJR], ti & 1, abort_flag, a.status, a.wait_ns)) break;
             tc_fence_after();
             if (T.has_lin) {
               const uint64_t hb = dH + ((hs * VSLOT) >> 4);
@@ -564,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Q tile can be replaced early.
     uint32_t phq[32];
     auto form_phi_q = [&](const Tile& Tq, int tiq) {
-      ok = ok && warp_wait(&bars[B_QFULL], tiq & 1, abort_flag, a.status);
+      ok = ok && warp_wait(&bars[B_QFULL], tiq & 1, abort_flag, a.status, a.wait_ns);
       const int tokq = Tq.qb * a.bq + r;
       {
         uint4 qw[8];
@@ -663,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i > 0 && (i & 31) == 0) jl = list_chunk(T, i >> 5);
         const int j_cur = __shfl_sync(0xffffffffu, jl, i & 31);
         const float zv = (T.has_lin && j_cur >= 0) ? zb[static_cast<long long>(j_cur) * kDPad] : 0.0f;
-        ok = ok && warp_wait(&bars[B_SFULL + b], (g >> 1) & 1, abort_flag, a.status);
+        ok = ok && warp_wait(&bars[B_SFULL + b], (g >> 1) & 1, abort_flag, a.status, a.wait_ns);
         const bool live = ok && j_cur >= 0;  // this half has a key block in this step
         const uint32_t scol = tmem + lrow + T_S0 + b * 128 + 64 * half;  // this half's 64 S columns
         const int nvalid = (tail && j_cur == a.nkv - 1) ? a.N - j_cur * kBlockKV : kBlockKV;
@@ -679,6 +690,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(scol, s);
           tmem_ld32(scol + 32, s + 32);
           tmem_wait_ld();
+          if constexpr (kI8) {  // s32 accumulators: exact below 2^24, so the conversion is exact
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = static_cast<float>(__float_as_int(s[c]));
+          }
           if (nvalid < kBlockKV) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -701,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float f = need ? ex2_approx(m_run - m_new) : 1.0f;
           if (i > 0) {
             // O holds P V of the previous steps: wait for the last PV, rescale
-            ok = ok && warp_wait(&bars[B_PEMPTY + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag, a.status);
+            ok = ok && warp_wait(&bars[B_PEMPTY + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag, a.status, a.wait_ns);
             if (ok) {
               tc_fence_after();
 #pragma unroll 1
@@ -729,6 +744,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float sk[32];
             tmem_ld32(scol + 32 * cc, sk);
             tmem_wait_ld();
+            if constexpr (kI8) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) sk[c] = static_cast<float>(__float_as_int(sk[c]));
+            }
             if (nvalid < kBlockKV) {
 #pragma unroll
               for (int c = 0; c < 32; ++c)
@@ -813,11 +832,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           dp = fmaf(f.y, zsh[c0 + 2 * c + 1], dp);
         }
         den = dp + xchg(dp);
-        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status);
+        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status, a.wait_ns);
         if (ok) tc_fence_after();
         // H_i / sigma = H_tot / sigma (fp16 tile from TMA) - H_ex / sigma, row e = r,
         // channels 64*half.., in place in the MN-major H tile
-        ok = ok && warp_wait(&bars[B_VFULL + hsl], (hidx / kVSlots) & 1, abort_flag, a.status);
+        ok = ok && warp_wait(&bars[B_VFULL + hsl], (hidx / kVSlots) & 1, abort_flag, a.status, a.wait_ns);
         const float inv_sigma = 1.0f / sigma;  // exact: sigma is a power of two
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -842,9 +861,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status);  // (every tile: phases stay aligned)
+        ok = ok && warp_wait(&bars[B_HFIN], ti & 1, abort_flag, a.status, a.wait_ns);  // (every tile: phases stay aligned)
       }
-      ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status);
+      ok = ok && warp_wait(&bars[B_OFINAL], ti & 1, abort_flag, a.status, a.wait_ns);
       if (ok) tc_fence_after();
       if (T.has_lin) {
         if (ok) {
@@ -860,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the next tile's phi(Q) while phi(Q) H_i runs
       if (t + static_cast<int>(gridDim.x) < ntiles) form_phi_q(tile_at(a, t + gridDim.x, false), ti + 1);
-      ok = ok && warp_wait(&bars[B_NUM], ti & 1, abort_flag, a.status);
+      ok = ok && warp_wait(&bars[B_NUM], ti & 1, abort_flag, a.status, a.wait_ns);
       if (ok) tc_fence_after();
 
       const float inv_l = (T.n_crit > 0 && l_run > 0.0f) ? 1.0f / l_run : 0.0f;
@@ -908,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&bars[B_PROJR]);
         }
-        ok = ok && warp_wait(&bars[B_PROJF], ti & 1, abort_flag, a.status);
+        ok = ok && warp_wait(&bars[B_PROJF], ti & 1, abort_flag, a.status, a.wait_ns);
         if (ok) tc_fence_after();
       } else {
         w_s = alpha_t * inv_l;
@@ -994,18 +1013,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <bool kFP8>
+template <int kLow>
 static cudaError_t launch_sparse_t(const SparseArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
                                    const CUtensorMap& mp, const CUtensorMap& mv, const CUtensorMap& mh,
                                    const CUtensorMap& mv8, const CUtensorMap& mo, cudaStream_t st) {
-  constexpr uint32_t smem = Lay<kFP8>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(sparse_fwd_kernel<kFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr uint32_t smem = Lay<kLow != 0>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(sparse_fwd_kernel<kLow>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long ntiles = static_cast<long long>(a.BH) * a.nq;
   const unsigned grid = static_cast<unsigned>(ntiles < sms ? ntiles : sms);
-  sparse_fwd_kernel<kFP8><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, mo, a);
+  sparse_fwd_kernel<kLow><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, mo, a);
   return cudaGetLastError();
 }
 
@@ -1029,11 +1048,12 @@ cudaError_t launch_sparse(const SparseArgs& a_in, const void* q_bf16_128, const 
     if ((e = encode_map8(&mq, q8, a.N, a.BH, 128)) != cudaSuccess) return e;
     if ((e = encode_map8(&mk, k8, a.N, a.BH, 64)) != cudaSuccess) return e;
     if ((e = encode_map8(&mv8, v8, a.N, a.BH, 64)) != cudaSuccess) return e;
-    return launch_sparse_t<true>(a, mq, mk, mp, mv, mh, mv8, mo, st);
+    if (a.fp8 == 2) return launch_sparse_t<2>(a, mq, mk, mp, mv, mh, mv8, mo, st);
+    return launch_sparse_t<1>(a, mq, mk, mp, mv, mh, mv8, mo, st);
   }
   if ((e = encode_map(&mq, q_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
   if ((e = encode_map(&mk, k_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
-  return launch_sparse_t<false>(a, mq, mk, mp, mv, mh, mv, mo, st);
+  return launch_sparse_t<0>(a, mq, mk, mp, mv, mh, mv, mo, st);
 }
 
 }  // namespace sla

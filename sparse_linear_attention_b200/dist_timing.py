@@ -7,6 +7,9 @@ on the GPUs, gloo in the CPU tests)."""
 from __future__ import annotations
 
 import os
+import socket
+import subprocess
+import sys
 
 import torch
 import torch.distributed as dist
@@ -47,3 +50,31 @@ def job_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
 def reports(rank: int) -> bool:
     """Only rank 0 prints the result line."""
     return rank == 0
+
+
+def launched() -> bool:
+    """True inside a process that a launcher (torchrun) started as one rank."""
+    return "WORLD_SIZE" in os.environ
+
+
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launcher_argv(script: str, argv: list[str], nproc: int, port: int) -> list[str]:
+    """The torchrun command that starts `nproc` ranks of `script argv` on this
+    node, rendezvous on 127.0.0.1."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nproc}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", script, *argv]
+
+
+def run_ranks(script: str, argv: list[str], nproc: int, timeout_s: float | None = None) -> int:
+    """Start `nproc` ranks of `script argv` under torchrun and return its exit
+    code (output goes to this process's stdout / stderr)."""
+    cmd = launcher_argv(script, argv, nproc, free_port())
+    try:
+        return subprocess.run(cmd, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        return 124

@@ -80,6 +80,7 @@ WORKLOADS = {
     "sla13_64": Workload("sla13_64", 1, 12, (21, 30, 52), 128, 64, 64, "bf16", mode="sla",
                          crit_ratio=0.05, negl_ratio=0.10, seed=1),
     "wan14": Workload("wan14", 1, 40, (21, 45, 80), 128, 128, 64, "bf16", keep_ratio=0.03, seed=2),
+    "fp8_13": Workload("fp8_13", 1, 12, (21, 30, 52), 128, 128, 64, "bf16", keep_ratio=0.03, fp8=True, seed=1),
     "fp8_14": Workload("fp8_14", 1, 40, (21, 45, 80), 128, 128, 64, "bf16", keep_ratio=0.03,
                        fp8=True, seed=2),
 }

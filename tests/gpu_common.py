@@ -79,7 +79,7 @@ def run_sla2(q, k, v, kept, alpha, bq, bkv, phi=sla.SLA_PHI_ELU1, out_dtype=torc
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     shape = sla.make_shape(qd, bq, bkv)
     if ws is None:
-        mode = sla.SLA_WS_FP8 if flags & sla.SLA_FLAG_FP8 else 0
+        mode = sla.SLA_WS_FP8 if flags & (sla.SLA_FLAG_FP8 | sla.SLA_FLAG_INT8) else 0
         ws = torch.zeros(sla.sla_workspace_size(shape, mode), dtype=torch.uint8, device=dev)
     kt = torch.as_tensor(np.ascontiguousarray(kept), dtype=torch.int32).to(dev)
     out = torch.full(q.shape, float("nan"), dtype=out_dtype, device=dev)

@@ -148,10 +148,13 @@ def test_attention_rejects_bad_arguments_before_launch():
     assert call(kept=None) == 1
     assert call(alpha=None) == 1
     assert call(phi=2) == 1
-    assert call(flags=8) == 1
-    # the e4m3 branch needs the larger workspace (sla_workspace_size with SLA_WS_FP8)
+    assert call(flags=16) == 1
+    assert call(flags=sla.SLA_FLAG_FP8 | sla.SLA_FLAG_INT8) == 1  # the two low-bit formats exclude each other
+    assert "exclude" in L.sla_last_error_detail().decode()
+    # the low-bit branches need the larger workspace (sla_workspace_size with SLA_WS_FP8)
     need = sla.sla_workspace_size(s, 0)
     assert call(flags=sla.SLA_FLAG_FP8, wsb=need) == 4
+    assert call(flags=sla.SLA_FLAG_INT8, wsb=need) == 4
     assert call(out=None) == 1
     assert call(out=FAKE + 4) == 3
     assert call(odt=9) == 1
@@ -167,8 +170,9 @@ def test_attention_rejects_bad_arguments_before_launch():
     assert call3(labels=None) == 1
     assert call3(wp=None) == 1
     assert call3(wp=FAKE + 2) == 3
-    assert L.sla_attn_fwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, 0, sla.SLA_FLAG_FP8, FAKE, 1, FAKE,
-                          1 << 40, None) == 2  # e4m3 branch: SLA2 only
+    for low in (sla.SLA_FLAG_FP8, sla.SLA_FLAG_INT8):  # the low-bit branches: SLA2 only
+        assert L.sla_attn_fwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, 0, low, FAKE, 1, FAKE,
+                              1 << 40, None) == 2
     # the SLA workspace also holds the per-row block lists
     need2 = sla.sla_workspace_size(s, 0)
     assert call3(wsb=need2) == 4
@@ -224,3 +228,57 @@ def test_backward_workspace_layout():
         BH = B * H
         want = 256 + 2 * (a256(BH * 128 * 128 * 4) + a256(BH * 128 * 4)) + a256(BH * N * 128 * 4)
         assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N, d)
+
+
+def _noalloc(shape, q=FAKE, k=FAKE, mode=0, k_keep=15, k_neg=0, kept=FAKE, wq=None):
+    L = sla.lib()
+    sp = ctypes.byref(shape) if shape is not None else None
+    st = L.sla_route_noalloc(sp, q, k, wq, None, mode, k_keep, k_neg, kept, None, None, None)
+    return st, L.sla_last_error_detail().decode()
+
+
+def test_route_noalloc_rejects_with_a_detail_naming_the_argument():
+    """Every early reject of the workspace-free router replaces the thread's
+    last error detail with one naming the rejected argument (and none of these
+    calls reaches the GPU)."""
+    s = _shape()
+    cases = [
+        (dict(shape=None), 1, "shape is null"),
+        (dict(shape=_shape(d=100)), 2, "d must be"),
+        (dict(shape=_shape(bq=96)), 2, "bq"),
+        (dict(shape=_shape(B=0)), 1, "positive"),
+        (dict(shape=s, mode=sla.SLA_MODE_SLA2_TOPK | sla.SLA_ROUTE_KBAR_FROM_WS), 1, "SLA_ROUTE_KBAR_FROM_WS"),
+        (dict(shape=s, mode=9), 1, "mode"),
+        (dict(shape=s, q=None), 1, "Q or K is null"),
+        (dict(shape=s, k=FAKE + 8), 3, "16-byte"),
+        (dict(shape=s, wq=FAKE + 4), 3, "Wq, Wk"),
+        (dict(shape=s, k_keep=600), 1, "k_keep"),
+        (dict(shape=s, k_neg=2), 1, "k_neg"),
+        (dict(shape=s, kept=None), 1, "kept_idx"),
+    ]
+    for kw, code, words in cases:
+        # a different failure first, so a stale detail would show
+        _route(_shape(), q=None)
+        st, detail = _noalloc(**kw)
+        assert st == code, (kw, st, detail)
+        assert words in detail and detail.startswith("sla_route_noalloc"), (kw, detail)
+
+
+def test_binding_refuses_host_tensors():
+    """The binding checks where each tensor lives before passing its pointer:
+    a CPU tensor never reaches the C side as a device pointer."""
+    import torch
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    shape = sla.make_shape(q, 64)
+    ws = torch.zeros(256, dtype=torch.uint8)
+    kept = torch.zeros(1, 2, 1, 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla_route(shape, q, q, None, None, 0, 1, 0, kept, None, None, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla_prepare(shape, q, q, 0, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla2_attn_fwd(shape, q, q, q, kept, 1, torch.zeros(1, 2, 1), 0, 0, torch.zeros_like(q), ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla_read_device_status(ws)
+    with pytest.raises(TypeError):
+        sla.sla_route(shape, "q", q, None, None, 0, 1, 0, kept, None, None, ws)

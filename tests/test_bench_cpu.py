@@ -40,3 +40,35 @@ def test_work_counts_at_the_headline_shape():
     assert full == 4.0 * 32760 ** 2 * 128 * 12
     assert executed == 4.0 * 128 * 12 * 32760 * 15 * 64
     assert abs(full / 6.594e12 - 1) < 1e-3
+
+
+def test_reference_arm_uses_the_oracle_alone(tmp_path):
+    """bench.py --impl reference: the CPU oracle on a bounded sample, its keep
+    count from the oracle, and libsla.so never mapped into the process."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'tiny', "
+            "'--steps', '2', '--warmup', '3']; runpy.run_path('bench.py', run_name='__main__'); "
+            "maps = open('/proc/self/maps').read(); print('LIBSLA_MAPPED' if 'libsla.so' in maps else 'NO_LIBSLA')")
+    out = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = out.stdout.strip().splitlines()
+    assert lines[-1] == "NO_LIBSLA"
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["cpu_baseline"]["kind"] == "oracle"
+    assert "keep=4/16" in rec["config"]["workload"]
+
+
+def test_gpus_flag_must_match_the_launcher():
+    """Under a launcher, --gpus N must equal the number of ranks it started."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference"], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=120)
+    assert out.returncode != 0 and "launcher started 1 ranks" in out.stderr

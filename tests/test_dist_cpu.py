@@ -90,3 +90,47 @@ def test_single_process_needs_no_group():
     assert dist_timing.job_throughput(10.0, 2.0, 1) == pytest.approx(5000.0)
     with pytest.raises(ValueError):
         dist_timing.job_throughput(1.0, 0.0, 1)
+
+
+_RANK_SCRIPT = '''
+import datetime, json, os, sys
+sys.path.insert(0, {root!r})
+from sparse_linear_attention_b200 import dist_timing
+n = int(sys.argv[sys.argv.index("--gpus") + 1])
+if n > 1 and not dist_timing.launched():
+    raise SystemExit(dist_timing.run_ranks(os.path.abspath(__file__), sys.argv[1:], n, timeout_s=120))
+import torch.distributed as dist
+rank, world, _ = dist_timing.world_info()
+assert world == n
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=30))
+got = dist_timing.max_over_ranks(float(rank + 1))
+dist.destroy_process_group()
+if dist_timing.reports(rank):
+    print(json.dumps({{"n_gpus": world, "max": got}}), flush=True)
+'''
+
+
+def test_gpus_flag_starts_its_own_ranks(tmp_path):
+    """bench.py's launcher path: `--gpus 2` outside torchrun starts two ranks of
+    the same script under torchrun (gloo here), every rank sees world size 2,
+    and rank 0 alone reports the max over ranks."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = tmp_path / "ranks.py"
+    script.write_text(_RANK_SCRIPT.format(root=root))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, str(script), "--gpus", "2"], capture_output=True, text=True,
+                         timeout=180, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    recs = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert recs == [{"n_gpus": 2, "max": 2.0}]
+
+
+def test_launcher_command_uses_loopback_rendezvous():
+    from sparse_linear_attention_b200 import dist_timing
+    cmd = dist_timing.launcher_argv("bench.py", ["--gpus", "4"], 4, 29511)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd and "--master-port=29511" in cmd
+    assert cmd[-3:] == ["bench.py", "--gpus", "4"]

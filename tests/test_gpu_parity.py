@@ -372,3 +372,104 @@ def test_fp8_ragged_shapes(N, d, bq):
     blocks = [(0, h, i) for h in range(w.H) for i in range(w.n_q)]
     compare(got, per_step, blocks, w.bq, tol=TOL_FP8)
     compare(got, per_block, blocks, w.bq, tol=TOL_FP8 + spread)
+
+
+# ------------------------------------------------------------------ host-buffer entry point
+
+@pytest.mark.parametrize("name,fp8", [("tiny", False), ("smoke128", False), ("smoke128", True)])
+def test_forward_host_matches_the_device_calls(name, fp8):
+    """sla2_forward_host (host inputs in, host output out, one C-ABI call) runs
+    the same kernels as sla_prepare + sla_route + sla2_attn_fwd on device
+    buffers: outputs and kept lists identical bit for bit, and the oracle's
+    router agrees."""
+    if name == "tiny":
+        w, x = workload("tiny")
+    else:
+        w = inputs.Workload("smoke128", 1, 2, (4, 16, 16), 128, 128, 64, "bf16", keep_count=4, seed=3)
+        x = inputs.make_inputs(w)
+    kk = k_of(w)
+    flags = sla.SLA_FLAG_FP8 if fp8 else 0
+    dev = "cuda"
+    shape = sla.make_shape(x["q"], w.bq, w.bkv)
+    hout = torch.full(x["q"].shape, float("nan"), dtype=torch.float32).pin_memory()
+    hkept = torch.full((w.B, w.H, w.n_q, kk), -1, dtype=torch.int32).pin_memory()
+    pin = {n: x[n].contiguous().pin_memory() for n in ("q", "k", "v", "wq", "wk", "alpha")}
+    dbuf = torch.zeros(sla.sla2_forward_host_device_bytes(shape, kk, sla.SLA_F32, flags), dtype=torch.uint8,
+                       device=dev)
+    sla.sla2_forward_host(shape, pin["q"], pin["k"], pin["v"], pin["wq"], pin["wk"], pin["alpha"], kk,
+                          sla.SLA_PHI_ELU1, flags, hout, hkept, dbuf)
+    assert sla.sla_read_device_status(dbuf) == 0
+    # the same forward through the device-pointer calls
+    qd, kd, vd = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    ws = torch.zeros(sla.sla_workspace_size(shape, sla.SLA_WS_FP8 if fp8 else 0), dtype=torch.uint8, device=dev)
+    kept = torch.empty(w.B, w.H, w.n_q, kk, dtype=torch.int32, device=dev)
+    out = torch.empty(x["q"].shape, dtype=torch.float32, device=dev)
+    kbar = w.dtype == "bf16" and w.d == 128
+    if kbar:
+        sla.sla_prepare(shape, kd, vd, sla.SLA_PHI_ELU1, ws)
+    sla.sla_route(shape, qd, kd, x["wq"].to(dev), x["wk"].to(dev), sla.SLA_ROUTE_KBAR_FROM_WS if kbar else 0, kk,
+                  0, kept, None, None, ws)
+    if not kbar:
+        sla.sla_prepare(shape, kd, vd, sla.SLA_PHI_ELU1, ws)
+    sla.sla2_attn_fwd(shape, qd, kd, vd, kept, kk, x["alpha"].to(dev), sla.SLA_PHI_ELU1,
+                      sla.SLA_FLAG_PREPARED | flags, out, ws)
+    assert sla.sla_read_device_status(ws) == 0
+    assert np.array_equal(hkept.numpy(), kept.cpu().numpy())
+    assert np.array_equal(hout.numpy().view(np.uint32), out.cpu().numpy().view(np.uint32))
+    okept, _, _ = orc.route(as32(x["q"]), as32(x["k"]), x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv, "sla2", kk)
+    assert np.array_equal(hkept.numpy(), okept)
+
+
+# ------------------------------------------------------------------ INT8 variant of the low-bit branch
+
+def _int8_check(w, x, kept, blocks=None, heads=None, extra_tol=0.0):
+    from tests.gpu_common import TOL_FP8
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, flags=sla.SLA_FLAG_INT8)
+    hs = list(range(w.H)) if heads is None else heads
+    sub = lambda t: t[:, hs]  # noqa: E731
+    args = (as64(sub(x["q"])), as64(sub(x["k"])), as64(sub(x["v"])), kept[:, hs], x["alpha"][:, hs].numpy(),
+            w.bq, w.bkv)
+    want = orc.sla2_forward_int8(*args, blocks=blocks)["o"]
+    if blocks is None:
+        blocks = [(0, h, i) for h in range(len(hs)) for i in range(w.n_q)]
+    return compare(got[:, hs], want, blocks, w.bq, tol=TOL_FP8 + extra_tol)
+
+
+def test_int8_tiny_all_rows():
+    """INT8 Q, K' (kind::i8 S), e4m3 P, V on the tiny workload, every row."""
+    w, x = workload("tiny")
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, k_of(w))
+    _int8_check(w, x, kept)
+
+
+@pytest.mark.parametrize("ratio", [0.03, 0.10])
+def test_int8_wan13_sampled_blocks(ratio):
+    w, x = workload("wan13")
+    kk = orc.keep_count(ratio, w.n_kv)
+    kept, _, _ = run_route(x["q"], x["k"], x["wq"], x["wk"], w.bq, w.bkv, 0, kk)
+    _int8_check(w, x, kept, blocks=sample_blocks(1, 3, w.n_q, 3, seed=7), heads=[0, 4, 9])
+
+
+@pytest.mark.parametrize("N,d,bq", [(777, 128, 64), (300, 64, 128)])
+def test_int8_ragged_shapes(N, d, bq):
+    """As test_fp8_ragged_shapes: held to the gate against the oracle with the
+    kernel's two-block softmax step, and to the gate plus the oracle's own
+    grouping spread against the per-block default."""
+    from tests.gpu_common import TOL_FP8
+    w, x = _rand_case(N, d, bq=bq, scale=1.5)
+    kept = _rand_kept(w, min(3, w.n_kv))
+    got = run_sla2(x["q"], x["k"], x["v"], kept, x["alpha"], w.bq, w.bkv, flags=sla.SLA_FLAG_INT8)
+    args = (as64(x["q"]), as64(x["k"]), as64(x["v"]), kept, x["alpha"].numpy(), w.bq, w.bkv)
+    per_block = orc.sla2_forward_int8(*args)["o"]
+    per_step = orc.sla2_forward_int8(*args, kv_tile=2)["o"]
+    spread = float(np.abs(per_block - per_step).max())
+    blocks = [(0, h, i) for h in range(w.H) for i in range(w.n_q)]
+    compare(got, per_step, blocks, w.bq, tol=TOL_FP8)
+    compare(got, per_block, blocks, w.bq, tol=TOL_FP8 + spread)
+
+
+def test_low_bit_flags_exclude_each_other():
+    w, x = _rand_case(300, 64, bq=128)
+    with pytest.raises(sla.SLAError, match="exclude"):
+        run_sla2(x["q"], x["k"], x["v"], _rand_kept(w, 2), x["alpha"], w.bq, w.bkv,
+                 flags=sla.SLA_FLAG_INT8 | sla.SLA_FLAG_FP8)
