@@ -270,11 +270,12 @@ def soft_topk_leg(args, w, dev, stream):
     }), flush=True)
 
 
-def backward_oracle_ms(w, x, kept, do_cpu, budget_s):
-    """The oracle's sla2_backward timed on sampled query blocks (random heads
-    and positions, at least three, until budget_s seconds are spent), each
-    block's time extrapolated to every block of the workload.  Returns (ms per
-    backward, blocks timed, seconds spent)."""
+def backward_oracle_ms(w, x, kept, do_cpu, budget_s, labels=None):
+    """The oracle's backward (sla2_backward, or sla_backward when SLA labels
+    are given) timed on sampled query blocks (random heads and positions, at
+    least three, until budget_s seconds are spent), each block's time
+    extrapolated to every block of the workload.  Returns (ms per backward,
+    blocks timed, seconds spent)."""
     import numpy as np
 
     from oracle import sla_oracle as orc
@@ -287,36 +288,51 @@ def backward_oracle_ms(w, x, kept, do_cpu, budget_s):
             heads[h] = tuple(t[:, h:h + 1].to(torch.float64).numpy() for t in (x["q"], x["k"], x["v"], do_cpu))
         q64, k64, v64, do64 = heads[h]
         t1 = time.perf_counter()
-        orc.sla2_backward(q64, k64, v64, kept[:, h:h + 1], x["alpha"][:, h:h + 1].to(torch.float64).numpy(), do64,
-                          w.bq, w.bkv, blocks=[(0, 0, i)])
+        if labels is not None:
+            orc.sla_backward(q64, k64, v64, labels[:, h:h + 1], x["wproj"].to(torch.float64).numpy(), do64, w.bq,
+                             w.bkv, blocks=[(0, 0, i)])
+        else:
+            orc.sla2_backward(q64, k64, v64, kept[:, h:h + 1], x["alpha"][:, h:h + 1].to(torch.float64).numpy(),
+                              do64, w.bq, w.bkv, blocks=[(0, 0, i)])
         spent += time.perf_counter() - t1
         n += 1
     return spent / n * (w.B * w.H * w.n_q) * 1e3, n, spent
 
 
 def backward_leg(args, w, dev, stream):
-    """SLA2 backward (sla2_attn_bwd) at the same workload: ms per call with
-    every input resident, the kept blocks from the router, a seeded dO.  The
-    work is dense contractions, so the roofline is the measured bf16 tensor
-    peak; the algorithmic work is the FlashAttention-style backward of the
-    sparse branch, 10 d FLOP per (query row, kept valid key): S recomputed,
+    """SLA2 backward (sla2_attn_bwd), or for an SLA workload sla_attn_bwd, at
+    the same workload: ms per call with every input resident, the kept
+    (critical) blocks from the router, a seeded dO.  The work is dense
+    contractions, so the roofline is the measured bf16 tensor peak; the
+    algorithmic work is the FlashAttention-style backward of the sparse
+    branch, 10 d FLOP per (query row, kept valid key): S recomputed,
     dP = dO V^T, dQ, dK and dV (the linear branch is not counted)."""
     x = inputs.make_inputs(w)
+    sla_mode = w.mode == "sla"
     q, kk, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
     wq, wk, alpha = x["wq"].to(dev), x["wk"].to(dev), x["alpha"].to(dev)
-    k = keep_of(w)
+    k = sla.sla_keep_count(w.crit_ratio, w.n_kv) if sla_mode else keep_of(w)
+    k_neg = sla.sla_keep_count(w.negl_ratio, w.n_kv) if sla_mode else 0
+    mode = sla.SLA_MODE_SLA_3WAY if sla_mode else sla.SLA_MODE_SLA2_TOPK
     shape = sla.make_shape(q, w.bq, w.bkv)
-    ws = torch.zeros(sla.sla_workspace_size(shape, sla.SLA_MODE_SLA2_TOPK), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(sla.sla_workspace_size(shape, mode), dtype=torch.uint8, device=dev)
     kept = torch.empty(w.B, w.H, w.n_q, k, dtype=torch.int32, device=dev)
-    sla.sla_route(shape, q, kk, wq, wk, sla.SLA_MODE_SLA2_TOPK, k, 0, kept, None, None, ws, stream)
+    labels = torch.empty(w.B, w.H, w.n_q, w.n_kv, dtype=torch.int8, device=dev) if sla_mode else None
+    sla.sla_route(shape, q, kk, wq, wk, mode, k, k_neg, kept, labels, None, ws, stream)
     g = torch.Generator().manual_seed(w.seed + 1000)
     do = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
-    wsb = torch.zeros(sla.sla2_attn_bwd_workspace_size(shape), dtype=torch.uint8, device=dev)
+    wsize = sla.sla_attn_bwd_workspace_size(shape) if sla_mode else sla.sla2_attn_bwd_workspace_size(shape)
+    wsb = torch.zeros(wsize, dtype=torch.uint8, device=dev)
     dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
     dk, dv = torch.empty_like(dq), torch.empty_like(dq)
     dal = torch.empty(w.B, w.H, w.n_q, dtype=torch.float32, device=dev)
     phi = sla.SLA_PHI_ELU1 if args.phi == "elu1" else sla.SLA_PHI_SOFTMAX
-    call = lambda: sla.sla2_attn_bwd(shape, q, kk, v, kept, k, alpha, phi, do, dq, dk, dv, dal, wsb, stream)
+    if sla_mode:
+        wproj = x["wproj"].to(dev)
+        dwp = torch.empty(w.d, w.d, dtype=torch.float32, device=dev)
+        call = lambda: sla.sla_attn_bwd(shape, q, kk, v, labels, wproj, phi, do, dq, dk, dv, dwp, wsb, stream)
+    else:
+        call = lambda: sla.sla2_attn_bwd(shape, q, kk, v, kept, k, alpha, phi, do, dq, dk, dv, dal, wsb, stream)
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
@@ -339,23 +355,28 @@ def backward_leg(args, w, dev, stream):
     flops = executed / 4.0 * 10.0  # work_counts' executed count is 4 d per (row, kept valid key)
     cpu = None
     if not args.no_cpu_baseline:
-        cpu_ms, nblk, t_cpu = backward_oracle_ms(w, x, kept_cpu.numpy(), do.cpu(), args.cpu_budget)
+        lab_cpu = labels.cpu().numpy() if sla_mode else None
+        cpu_ms, nblk, t_cpu = backward_oracle_ms(w, x, kept_cpu.numpy(), do.cpu(), args.cpu_budget, lab_cpu)
+        fn = "sla_backward" if sla_mode else "sla2_backward"
         cpu = {"value": cpu_ms, "unit": "ms per call", "cores": OracleTimer.threads(), "kind": "oracle",
-               "sample": f"CPU oracle (numpy fp64) sla2_backward on {nblk} sampled query blocks of "
+               "sample": f"CPU oracle (numpy fp64) {fn} on {nblk} sampled query blocks of "
                          f"{w.B * w.H * w.n_q} ({t_cpu:.2f} s), extrapolated per block"}
     _, peak, _, src = peaks()
     achieved = flops / (ms * 1e-3) / 1e12
+    metric = ("SLA backward ms @Wan-1.3B shape (sla_attn_bwd: dQ, dK, dV, dW_proj)" if sla_mode else
+              "SLA2 backward ms @Wan-1.3B shape (sla2_attn_bwd: dQ, dK, dV, dalpha)")
+    keep_txt = f"critical={k} negligible={k_neg}/{w.n_kv}" if sla_mode else f"keep={k}/{w.n_kv}"
     print(json.dumps({
-        "metric": "SLA2 backward ms @Wan-1.3B shape (sla2_attn_bwd: dQ, dK, dV, dalpha)", "value": ms,
+        "metric": metric, "value": ms,
         "unit": "ms per call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": False, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
-                               f"keep={k}/{w.n_kv} key blocks, phi={args.phi}"},
+                               f"{keep_txt} key blocks, phi={args.phi}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense (burst)",
                      "algorithmic": "10*d FLOP per (query row, kept valid key): the sparse branch's "
                                     "FlashAttention-style backward; kernels are fp32 on the CUDA cores"},
-        "gpu_launches": 3 * args.steps, "clocks": clk, "cpu_baseline": cpu,
+        "gpu_launches": (6 if sla_mode else 3) * args.steps, "clocks": clk, "cpu_baseline": cpu,
     }), flush=True)
 
 
@@ -458,8 +479,8 @@ def main():
     int8 = args.int8
     fp8 = (args.fp8 or w.fp8) and not int8
     low = fp8 or int8
-    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk or args.backward or low):
-        raise SystemExit("the reference arm, --fp8, --int8, --soft-topk and --backward are SLA2 legs")
+    if w.mode != "sla2" and (args.impl == "reference" or args.soft_topk or low):
+        raise SystemExit("the reference arm, --fp8, --int8 and --soft-topk are SLA2 legs")
     if args.impl == "reference":
         reference_arm(args, w)
         return

@@ -263,6 +263,34 @@ sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k,
                          float* dq, float* dk, float* dv, float* dalpha,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace sla_attn_bwd needs for this shape (0 for an
+ * invalid shape): sla2_attn_bwd's, plus the critical / negligible block lists,
+ * a [B,H,N,128] fp32 buffer of the O_l rows and the dW_proj partial sums. */
+size_t sla_attn_bwd_workspace_size(const sla_shape* shape);
+
+/* Gradients of the SLA forward [SLA 关键设计 4] for the upstream gradient
+ * dout, with the labels held fixed:
+ *   dO_s = dO, dO_l = dO W_proj^T, dW_proj = sum over the rows of every head
+ *   of O_l^T dO (W_proj is shared by the heads); the critical blocks take the
+ *   sparse branch back-propagated as FlashAttention does, the marginal blocks
+ *   the linear branch through dH_i, dZ_i (the totals minus the critical and
+ *   negligible blocks' share), the negligible blocks get nothing.
+ * Inputs q, k, v, labels, Wproj, phi as for sla_attn_fwd; dout [B,H,N,d] of
+ *   the input dtype.
+ * Outputs (fp32, caller-owned, fully overwritten): dq, dk, dv [B,H,N,d],
+ *   dWproj [d][d] (d_in x d_out, as Wproj).  dk and dv are accumulated with
+ *   atomic adds after a zero fill, so their last bits can differ between runs;
+ *   dWproj is summed in a fixed order.
+ * ws: its own workspace of sla_attn_bwd_workspace_size bytes, 256-byte
+ *   aligned, status word zeroed once (sla_workspace_init).  A label outside
+ *   {-1, 0, 1} is reported in the status word (sla_read_device_status) and
+ *   the block is treated as marginal. */
+sla_status sla_attn_bwd(const sla_shape* shape, const void* q, const void* k,
+                        const void* v, const int8_t* labels, const void* Wproj,
+                        int phi, const void* dout, float* dq, float* dk,
+                        float* dv, float* dWproj, void* ws, size_t ws_bytes,
+                        void* stream);
+
 /* Bytes of device memory sla2_forward_host needs (0 for invalid arguments):
  * the workspace of sla_workspace_size (with SLA_WS_FP8 when flags carry
  * SLA_FLAG_FP8 or SLA_FLAG_INT8) followed by device copies of Q, K, V, Wq, Wk, alpha, the kept

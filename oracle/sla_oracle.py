@@ -613,34 +613,34 @@ def sla2_backward(q, k, v, kept, alpha, do, bq, bkv, phi_kind="elu1", blocks=Non
     return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dalpha}
 
 
-def sla_backward(q, k, v, labels, wproj, do, bq, bkv, phi_kind="elu1"):
+def sla_backward(q, k, v, labels, wproj, do, bq, bkv, phi_kind="elu1", blocks=None):
     """Gradients of sla_forward's O = O_s + O_l Wp for the upstream gradient do,
     the labels held fixed:  dO_s = dO,  dO_l = dO Wp^T,  dWp = sum over every
     row of every head of O_l^T dO (Wp is shared).  Critical blocks (+1) take
     the sparse branch, marginal ones (0) the linear branch, negligible ones
-    (-1) get no gradient.  Returns dict dq, dk, dv and dwproj ([d_in, d_out])."""
+    (-1) get no gradient.  blocks: optional list of (b,h,i) whose share to add
+    (default: all, which gives the full gradients).
+    Returns dict dq, dk, dv and dwproj ([d_in, d_out])."""
     B, H, N, d = q.shape
     nq = -(-N // bq)
     wp = np.asarray(wproj, dtype=F64)
     dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
     dwp = np.zeros(wp.shape)
-    for b in range(B):
-        for h in range(H):
-            qs, ks, vs = q[b, h], k[b, h], v[b, h]
-            for i in range(nq):
-                rows = _rows(i, bq, N)
-                lab = labels[b, h, i]
-                tc = _tokens_of([int(j) for j in np.nonzero(lab == 1)[0]], bkv, N)
-                tm = _tokens_of([int(j) for j in np.nonzero(lab == 0)[0]], bkv, N)
-                g = do[b, h, rows]
-                o_l = linear_branch(qs, ks, vs, rows, tm, phi_kind)
-                dwp += o_l.T @ g
-                gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, tc, g)
-                dq[b, h, rows] += gq
-                dk[b, h, tc] += gk
-                dv[b, h, tc] += gv
-                gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tm, g @ wp.T, phi_kind)
-                dq[b, h, rows] += gq
-                dk[b, h, tm] += gk
-                dv[b, h, tm] += gv
+    for (b, h, i) in _blocks_to_do(B, H, nq, blocks):
+        qs, ks, vs = q[b, h], k[b, h], v[b, h]
+        rows = _rows(i, bq, N)
+        lab = labels[b, h, i]
+        tc = _tokens_of([int(j) for j in np.nonzero(lab == 1)[0]], bkv, N)
+        tm = _tokens_of([int(j) for j in np.nonzero(lab == 0)[0]], bkv, N)
+        g = do[b, h, rows]
+        o_l = linear_branch(qs, ks, vs, rows, tm, phi_kind)
+        dwp += o_l.T @ g
+        gq, gk, gv = sparse_branch_backward(qs, ks, vs, rows, tc, g)
+        dq[b, h, rows] += gq
+        dk[b, h, tc] += gk
+        dv[b, h, tc] += gv
+        gq, gk, gv = linear_branch_backward(qs, ks, vs, rows, tm, g @ wp.T, phi_kind)
+        dq[b, h, rows] += gq
+        dk[b, h, tm] += gk
+        dv[b, h, tm] += gv
     return {"dq": dq, "dk": dk, "dv": dv, "dwproj": dwp}

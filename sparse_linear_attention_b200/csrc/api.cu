@@ -284,7 +284,7 @@ sla_status sla2_attn_fwd(const sla_shape* shape, const void* q, const void* k, c
 
 size_t sla2_attn_bwd_workspace_size(const sla_shape* shape) {
   if (shape == nullptr || check_shape(shape) != SLA_OK) return 0;
-  return bwd_layout(*shape).total;
+  return bwd_layout(*shape, false).total;
 }
 
 sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k, const void* v,
@@ -304,10 +304,37 @@ sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k, c
     return arg_fail(SLA_ERR_ALIGNMENT, "dout, dq, dk, dv, dalpha must be 16-byte aligned");
   if (ws == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "ws is null");
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return arg_fail(SLA_ERR_ALIGNMENT, "ws must be 256-byte aligned");
-  if (ws_bytes < bwd_layout(*shape).total)
+  if (ws_bytes < bwd_layout(*shape, false).total)
     return arg_fail(SLA_ERR_WORKSPACE, "ws smaller than sla2_attn_bwd_workspace_size");
   cudaError_t e = launch_backward(*shape, q, k, v, dout, kept_idx, k_keep, alpha, phi, dq, dk, dv, dalpha,
                                   static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SLA_OK : cuda_fail(e, "backward");
+}
+
+size_t sla_attn_bwd_workspace_size(const sla_shape* shape) {
+  if (shape == nullptr || check_shape(shape) != SLA_OK) return 0;
+  return bwd_layout(*shape, true).total;
+}
+
+sla_status sla_attn_bwd(const sla_shape* shape, const void* q, const void* k, const void* v, const int8_t* labels,
+                        const void* Wproj, int phi, const void* dout, float* dq, float* dk, float* dv,
+                        float* dWproj, void* ws, size_t ws_bytes, void* stream) {
+  sla_status s = check_shape(shape);
+  if (s != SLA_OK) return s;
+  if ((s = check_qkv(q, k, v)) != SLA_OK) return s;
+  if (labels == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "labels is null");
+  if (Wproj == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "Wproj is null");
+  if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_SOFTMAX) return arg_fail(SLA_ERR_INVALID_ARG, "phi");
+  if (dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || dWproj == nullptr)
+    return arg_fail(SLA_ERR_INVALID_ARG, "dout, dq, dk, dv or dWproj is null");
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return arg_fail(SLA_ERR_ALIGNMENT, "dout, dq, dk, dv must be 16-byte aligned");
+  if (ws == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "ws is null");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return arg_fail(SLA_ERR_ALIGNMENT, "ws must be 256-byte aligned");
+  if (ws_bytes < bwd_layout(*shape, true).total)
+    return arg_fail(SLA_ERR_WORKSPACE, "ws smaller than sla_attn_bwd_workspace_size");
+  cudaError_t e = launch_sla_backward(*shape, q, k, v, dout, labels, Wproj, phi, dq, dk, dv, dWproj,
+                                      static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SLA_OK : cuda_fail(e, "backward");
 }
 

@@ -209,6 +209,13 @@ struct BwdArgs {
   float *dHtot, *dZtot, *dphik;
   float *dq, *dk, *dv, *dalpha;
   int* status;
+  // SLA (sla != 0): per query block the critical and negligible lists
+  // [rows][2][nkv] with their counts [rows][2], W_proj [d][d], and the O_l
+  // rows [BH][N][128] kept for dW_proj.  kept, kk, alpha and dalpha unused.
+  int sla;
+  const int32_t *lists, *counts;
+  const __nv_bfloat16* wproj;
+  float* ol;
 };
 
 // Shared-memory layout of bwd_query_kernel (floats)
@@ -224,7 +231,9 @@ constexpr int kOffT3 = kOffT2 + kRowsB * kLdT;    // G -> Bx
 constexpr int kOffRV = kOffT3 + kRowsB * kLdT;    // row scalars: m, l, rsA, D, s, dden  [6][32]
 constexpr int kOffZ = kOffRV + 6 * kRowsB;        // Z_tot [128]
 constexpr int kOffRed = kOffZ + kDPad;            // [8] block reduction
-constexpr int kQuerySmemFloats = kOffRed + 8;
+constexpr int kOffE = kOffRed + 8;                // SLA: dO_l = dO W_proj^T  [32][kLd]
+constexpr int kOffT4 = kOffE + kRowsB * kLd;      // SLA: -s A  [32][kLdT]
+constexpr int kQuerySmemFloats = kOffT4 + kRowsB * kLdT;
 static_assert(3 * kBlockKV * kLd >= kDPad * kLd, "H_tot staging fits the key tiles");
 static_assert(kQuerySmemFloats * 4 <= 232448, "shared memory budget");
 
@@ -331,6 +340,8 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
   float* rv_dd = rv_s + kRowsB;
   float* Zs = smq + kOffZ;
   float* red = smq + kOffRed;
+  float* Es = smq + kOffE;
+  float* T4 = smq + kOffT4;
 
   const int tid = threadIdx.x, lane = tid & 31, wr = tid >> 5;
   const int rg = tid >> 4, kl = tid & 15;  // 32 x 64 tile map
@@ -346,14 +357,56 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
   const T* vb = static_cast<const T*>(a.v) + bh * N * d;
   const T* gb = static_cast<const T*>(a.dout) + bh * N * d;
   const long long rowq = bh * a.nq + i;
-  const int32_t* list = a.kept + rowq * a.kk;
-  const float alpha = a.alpha[rowq];
-  const bool has_lin = a.kk < a.nkv;
+  // The blocks whose linear share is taken out of the totals: SLA2 the kept
+  // list; SLA the critical list, then the negligible one.  The first n_crit
+  // of them also take the sparse branch.
+  const int32_t* clist;
+  const int32_t* nlist = nullptr;
+  int n_crit, n_all;
+  if (a.sla) {
+    clist = a.lists + rowq * 2 * a.nkv;
+    nlist = clist + a.nkv;
+    n_crit = a.counts[2 * rowq];
+    n_all = n_crit + a.counts[2 * rowq + 1];
+  } else {
+    clist = a.kept + rowq * a.kk;
+    n_crit = n_all = a.kk;
+  }
+  auto entry = [&](int jj) { return jj < n_crit ? clist[jj] : nlist[jj - n_crit]; };
+  // dO_s = c_s dO; dO_l = c_l dO (SLA2) or dO W_proj^T (SLA, held in Es)
+  const float alpha = a.sla ? 1.0f : a.alpha[rowq];
+  const float lin_w = a.sla ? 1.0f : 1.0f - alpha;
+  const bool has_lin = n_all < a.nkv;
+  const float* LD = a.sla ? Es : DO;
   auto block_ok = [&](int j) { return j >= 0 && j < a.nkv; };
 
   // rows, phi(rows) (phi of the zero vector past N keeps den > 0), dO, Z_tot, H_tot
   load_rows(qb, N, d, row0, kRowsB, Qs, PQ, a.phi, false);
   load_rows(gb, N, d, row0, kRowsB, DO, nullptr, a.phi, false);
+  if (a.sla) {
+    // W_proj^T staged [c][e], then E = dO W_proj^T (32 x 128 map)
+    for (int x = tid; x < kDPad * kDPad; x += kBT) {
+      const int e = x / kDPad, c = x % kDPad;
+      Ks[c * kLd + e] = (e < d && c < d) ? __bfloat162float(a.wproj[e * d + c]) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int r = 4 * wr + u;
+      for (int c = 0; c < d; ++c) {
+        const float g = DO[r * kLd + c];
+        const float4 wv = *reinterpret_cast<const float4*>(Ks + c * kLd + cc);
+        acc[0] = fmaf(g, wv.x, acc[0]);
+        acc[1] = fmaf(g, wv.y, acc[1]);
+        acc[2] = fmaf(g, wv.z, acc[2]);
+        acc[3] = fmaf(g, wv.w, acc[3]);
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) Es[r * kLd + cc + w] = acc[w];
+    }
+    __syncthreads();
+  }
   const float* Hg = a.Htot + bh * kDPad * kDPad;
   for (int x = tid; x < kDPad * kDPad; x += kBT) Ks[(x / kDPad) * kLd + x % kDPad] = Hg[x];
   for (int x = tid; x < kDPad; x += kBT) Zs[x] = a.Ztot[bh * kDPad + x];
@@ -388,7 +441,7 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
     const float4 h = *reinterpret_cast<const float4*>(Ks + c * kLd + cc);  // H_tot[cc + w][c]
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float g = DO[(4 * wr + u) * kLd + c];
+      const float g = LD[(4 * wr + u) * kLd + c];
       hdo[u][0] = fmaf(g, h.x, hdo[u][0]);
       hdo[u][1] = fmaf(g, h.y, hdo[u][1]);
       hdo[u][2] = fmaf(g, h.z, hdo[u][2]);
@@ -398,8 +451,8 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
 
   // ------------------------------------------------ pass 0: row max of the scaled scores
   float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};
-  for (int jj = 0; jj < a.kk; ++jj) {
-    const int j = list[jj];
+  for (int jj = 0; jj < n_crit; ++jj) {
+    const int j = entry(jj);
     if (!block_ok(j)) {
       if (tid == 0) report_error(a.status, SLA_ERR_DEVICE_INDEX);
       continue;
@@ -427,16 +480,20 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int w = 0; w < 4; ++w) oacc[u][w] = 0.0f;
-  for (int jj = 0; jj < a.kk; ++jj) {
-    const int j = list[jj];
-    if (!block_ok(j)) continue;
+  for (int jj = 0; jj < n_all; ++jj) {
+    const int j = entry(jj);
+    if (!block_ok(j)) {
+      if (jj >= n_crit && tid == 0) report_error(a.status, SLA_ERR_DEVICE_INDEX);
+      continue;
+    }
+    const bool crit = jj < n_crit;
     __syncthreads();
     load_rows(kb, N, d, j * kBlockKV, kBlockKV, Ks, PK, a.phi, true);
     load_rows(vb, N, d, j * kBlockKV, kBlockKV, Vs, nullptr, a.phi, true);
     __syncthreads();
     const int nvalid = min(kBlockKV, N - j * kBlockKV);
     float s[2][4], al[2][4];
-    rows_x_keys_over_channels(Qs, Ks, d, s);
+    if (crit) rows_x_keys_over_channels(Qs, Ks, d, s);
     rows_x_keys_over_channels(PQ, PK, d, al);
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -444,7 +501,7 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const int c = kl + 16 * w;
-        const float p = c < nvalid ? expf(s[u][w] * a.scale - m2[u]) : 0.0f;
+        const float p = (crit && c < nvalid) ? expf(s[u][w] * a.scale - m2[u]) : 0.0f;
         T1[(2 * rg + u) * kLdT + c] = p;
         T2[(2 * rg + u) * kLdT + c] = al[u][w];  // phi(K) rows past N are zero
         ls += p;
@@ -454,7 +511,7 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
       rsa2[u] += half_sum(as);
     }
     __syncthreads();
-    rows_x_channels_over_keys(T1, Vs, 1.0f, oacc);
+    if (crit) rows_x_channels_over_keys(T1, Vs, 1.0f, oacc);
     rows_x_channels_over_keys(T2, Vs, -1.0f, num);
   }
   if (kl == 0) {
@@ -484,18 +541,25 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
     }
 #pragma unroll
     for (int w = 0; w < 4; ++w) ol[w] = has_lin ? num[u][w] / den : 0.0f;
-    float dos = 0.0f, dol = 0.0f;
+    float dos = 0.0f, dol = 0.0f, dlo = 0.0f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const float g = DO[r * kLd + cc + w];
       dos = fmaf(g, os[w], dos);
       dol = fmaf(g, ol[w], dol);
+      dlo = fmaf(LD[r * kLd + cc + w], ol[w], dlo);
     }
     dos = warp_sum(dos);
     dol = warp_sum(dol);
+    dlo = warp_sum(dlo);
     dal += dos - dol;
-    sr4[u] = has_lin ? (1.0f - alpha) / den : 0.0f;
-    dd4[u] = has_lin ? -(1.0f - alpha) * dol / den : 0.0f;
+    // SLA2: s = (1 - alpha) / den with dO; SLA: s = 1 / den with dO W_proj^T
+    sr4[u] = has_lin ? lin_w / den : 0.0f;
+    dd4[u] = has_lin ? -lin_w * dlo / den : 0.0f;
+    if (a.sla && row0 + r < N) {
+      float* olr = a.ol + (bh * N + row0 + r) * kDPad + cc;
+      *reinterpret_cast<float4*>(olr) = make_float4(ol[0], ol[1], ol[2], ol[3]);
+    }
     if (lane == 0) {
       rv_D[r] = alpha * dos;
       rv_s[r] = sr4[u];
@@ -504,7 +568,7 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
   }
   if (lane == 0) red[wr] = dal;
   __syncthreads();
-  if (tid == 0) {
+  if (tid == 0 && !a.sla) {
     float t = 0.0f;
     for (int w = 0; w < kBT / 32; ++w) t += red[w];
     atomicAdd(a.dalpha + rowq, t);
@@ -522,19 +586,23 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
   float* dkh = a.dk + bh * N * d;
   float* dvh = a.dv + bh * N * d;
   float* dpkh = a.dphik + bh * N * kDPad;
-  for (int jj = 0; jj < a.kk; ++jj) {
-    const int j = list[jj];
+  for (int jj = 0; jj < n_all; ++jj) {
+    const int j = entry(jj);
     if (!block_ok(j)) continue;
+    const bool crit = jj < n_crit;
     __syncthreads();
     load_rows(kb, N, d, j * kBlockKV, kBlockKV, Ks, PK, a.phi, true);
     load_rows(vb, N, d, j * kBlockKV, kBlockKV, Vs, nullptr, a.phi, true);
     __syncthreads();
     const int nvalid = min(kBlockKV, N - j * kBlockKV);
     {
-      float s[2][4], al[2][4], g[2][4];
-      rows_x_keys_over_channels(Qs, Ks, d, s);
+      float s[2][4], al[2][4], g[2][4], gl[2][4];
+      if (crit) {
+        rows_x_keys_over_channels(Qs, Ks, d, s);
+        rows_x_keys_over_channels(DO, Vs, d, g);
+      }
       rows_x_keys_over_channels(PQ, PK, d, al);
-      rows_x_keys_over_channels(DO, Vs, d, g);
+      if (a.sla) rows_x_keys_over_channels(Es, Vs, d, gl);  // SLA2: dO_l V^T = (1 - alpha) G
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int r = 2 * rg + u;
@@ -543,21 +611,39 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
         for (int w = 0; w < 4; ++w) {
           const int c = kl + 16 * w;
           const bool kv = c < nvalid;
-          const float p = kv ? expf(s[u][w] * a.scale - m) / l : 0.0f;
-          T1[r * kLdT + c] = p * (alpha * g[u][w] - D);   // dS
-          T2[r * kLdT + c] = alpha * p - sr * al[u][w];    // C
-          T3[r * kLdT + c] = kv ? sr * g[u][w] + dd : 0.0f;  // Bx
+          const float p = (crit && kv) ? expf(s[u][w] * a.scale - m) / l : 0.0f;
+          const float gs = crit ? g[u][w] : 0.0f;
+          const float glv = a.sla ? gl[u][w] : gs;
+          T1[r * kLdT + c] = p * (alpha * gs - D);                  // dS
+          T2[r * kLdT + c] = a.sla ? p : alpha * p - sr * al[u][w];  // C (SLA: P)
+          T3[r * kLdT + c] = kv ? sr * glv + dd : 0.0f;             // Bx
+          if (a.sla) T4[r * kLdT + c] = -sr * al[u][w];
         }
       }
     }
     __syncthreads();
-    rows_x_channels_over_keys(T1, Ks, 1.0f, dqa);
+    if (crit) rows_x_channels_over_keys(T1, Ks, 1.0f, dqa);
     rows_x_channels_over_keys(T3, PK, -1.0f, dpq);
     {
       float kt[8][4];
-      keys_x_channels_over_rows(T1, Qs, kt);
-      add_key_tile(dkh, d, N, d, j * kBlockKV, a.scale, kt);
-      keys_x_channels_over_rows(T2, DO, kt);
+      if (crit) {
+        keys_x_channels_over_rows(T1, Qs, kt);
+        add_key_tile(dkh, d, N, d, j * kBlockKV, a.scale, kt);
+      }
+      if (a.sla) {
+        // dV = P^T dO (critical) - (s A)^T dO_l
+        keys_x_channels_over_rows(T4, Es, kt);
+        if (crit) {
+          float kp[8][4];
+          keys_x_channels_over_rows(T2, DO, kp);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) kt[u][w] += kp[u][w];
+        }
+      } else {
+        keys_x_channels_over_rows(T2, DO, kt);
+      }
       add_key_tile(dvh, d, N, d, j * kBlockKV, 1.0f, kt);
       if (has_lin) {
         keys_x_channels_over_rows(T3, PQ, kt);
@@ -597,7 +683,7 @@ __global__ void __launch_bounds__(kBT, 1) bwd_query_kernel(const BwdArgs a) {
       for (int r = 0; r < kRowsB; ++r) {
         const float pe = PQ[r * kLd + e];
         const float ps = pe * rv_s[r];
-        const float4* gr = reinterpret_cast<const float4*>(DO + r * kLd + c0);
+        const float4* gr = reinterpret_cast<const float4*>(LD + r * kLd + c0);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const float4 g = gr[u];
@@ -692,6 +778,71 @@ __global__ void __launch_bounds__(kBT, 1) bwd_keys_kernel(const T* __restrict__ 
   }
 }
 
+// ---------------------------------------------------------------- dW_proj (SLA)
+// grid (nsplit): this split's share of dW_proj[e][c] = sum over the rows of
+// every head of O_l[e] dO[c], rows [split * per, ...) of the flat [BH * N]
+// row range; thread: e = tid / 2, columns 64 (tid % 2) .. +63.  The partials
+// are summed in split order by bwd_wproj_sum_kernel, so dW_proj is the same
+// on every run.
+template <typename T>
+__global__ void __launch_bounds__(kBT) bwd_wproj_kernel(const float* __restrict__ ol, const T* __restrict__ dout,
+                                                        long long rows, int d, long long per,
+                                                        float* __restrict__ wpart) {
+  extern __shared__ __align__(16) float smw[];
+  float* Ot = smw;                   // [32][kLd]
+  float* Gt = smw + kTokTile * kLd;  // [32][kLd]
+  const long long r_begin = blockIdx.x * per;
+  const long long r_end = min(rows, r_begin + per);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, e = tid >> 1, c0 = (tid & 1) * 64;
+  float h[64];
+#pragma unroll
+  for (int u = 0; u < 64; ++u) h[u] = 0.0f;
+  for (long long t0 = r_begin; t0 < r_end; t0 += kTokTile) {
+    __syncthreads();
+    for (int r = warp; r < kTokTile; r += kBT / 32) {
+      const long long row = t0 + r;
+      const bool valid = row < r_end;
+      float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (valid) o = *reinterpret_cast<const float4*>(ol + row * kDPad + 4 * lane);
+      *reinterpret_cast<float4*>(Ot + r * kLd + 4 * lane) = o;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = 4 * lane + u;
+        Gt[r * kLd + c] = (valid && c < d) ? ld_in(dout + row * d + c) : 0.0f;
+      }
+    }
+    __syncthreads();
+    const int nt = static_cast<int>(min(static_cast<long long>(kTokTile), r_end - t0));
+    for (int t = 0; t < nt; ++t) {
+      const float oe = Ot[t * kLd + e];
+      const float4* gr = reinterpret_cast<const float4*>(Gt + t * kLd + c0);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float4 g = gr[u];
+        h[4 * u] = fmaf(oe, g.x, h[4 * u]);
+        h[4 * u + 1] = fmaf(oe, g.y, h[4 * u + 1]);
+        h[4 * u + 2] = fmaf(oe, g.z, h[4 * u + 2]);
+        h[4 * u + 3] = fmaf(oe, g.w, h[4 * u + 3]);
+      }
+    }
+  }
+  float* dst = wpart + (static_cast<long long>(blockIdx.x) * kDPad + e) * kDPad + c0;
+#pragma unroll
+  for (int u = 0; u < 64; u += 4)
+    *reinterpret_cast<float4*>(dst + u) = make_float4(h[u], h[u + 1], h[u + 2], h[u + 3]);
+}
+
+// dW_proj [d][d] = the partials summed in split order.
+__global__ void __launch_bounds__(kBT) bwd_wproj_sum_kernel(const float* __restrict__ wpart, int nsplit, int d,
+                                                            float* __restrict__ dwproj) {
+  const int x = blockIdx.x * kBT + threadIdx.x;
+  if (x >= d * d) return;
+  const int e = x / d, c = x % d;
+  float t = 0.0f;
+  for (int sp = 0; sp < nsplit; ++sp) t += wpart[(static_cast<long long>(sp) * kDPad + e) * kDPad + c];
+  dwproj[x] = t;
+}
+
 template <typename T>
 cudaError_t run_backward(const sla_shape& s, const BwdArgs& a, cudaStream_t st) {
   const int BH = s.B * s.H;
@@ -728,9 +879,30 @@ cudaError_t run_backward(const sla_shape& s, const BwdArgs& a, cudaStream_t st) 
   return cudaGetLastError();
 }
 
+// Rows per split of the dW_proj reduction: about two CTAs per SM, whole
+// 32-row tiles.
+long long wproj_rows_per_split(long long rows) {
+  long long per = (rows + 2 * kNumSMs - 1) / (2 * kNumSMs);
+  per = (per + kTokTile - 1) / kTokTile * kTokTile;
+  return per < kTokTile ? kTokTile : per;
+}
+
+template <typename T>
+cudaError_t run_wproj(const sla_shape& s, const BwdLayout& L, const float* ol, const void* dout, char* ws,
+                      float* dwproj, cudaStream_t st) {
+  const long long rows = static_cast<long long>(s.B) * s.H * s.N;
+  const long long per = wproj_rows_per_split(rows);
+  const int nsplit = static_cast<int>((rows + per - 1) / per);
+  float* wpart = reinterpret_cast<float*>(ws + L.wpart);
+  bwd_wproj_kernel<T><<<nsplit, kBT, 2 * kTokTile * kLd * sizeof(float), st>>>(ol, static_cast<const T*>(dout), rows,
+                                                                               s.d, per, wpart);
+  bwd_wproj_sum_kernel<<<(s.d * s.d + kBT - 1) / kBT, kBT, 0, st>>>(wpart, nsplit, s.d, dwproj);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-BwdLayout bwd_layout(const sla_shape& s) {
+BwdLayout bwd_layout(const sla_shape& s, bool sla_mode) {
   BwdLayout L;
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   size_t off = 0;
@@ -745,14 +917,29 @@ BwdLayout bwd_layout(const sla_shape& s) {
   L.dhtot = take(BH * kDPad * kDPad * 4);
   L.dztot = take(BH * kDPad * 4);
   L.dphik = take(BH * static_cast<size_t>(s.N) * kDPad * 4);
+  if (sla_mode) {
+    const size_t rows = BH * static_cast<size_t>(ceil_div(s.N, s.bq));
+    const size_t nkv = static_cast<size_t>(ceil_div(s.N, s.bkv));
+    const long long flat = static_cast<long long>(BH) * s.N;
+    const long long per = wproj_rows_per_split(flat);
+    const size_t nsplit = static_cast<size_t>((flat + per - 1) / per);
+    L.lists = take(rows * 2 * nkv * 4);
+    L.counts = take(rows * 2 * 4);
+    L.ol = take(BH * static_cast<size_t>(s.N) * kDPad * 4);
+    L.wpart = take(nsplit * kDPad * kDPad * 4);
+  }
   L.total = off;
   return L;
 }
 
-cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
-                            const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
-                            float* dv, float* dalpha, char* ws, cudaStream_t st) {
-  const BwdLayout L = bwd_layout(s);
+namespace {
+
+cudaError_t launch_backward_common(const sla_shape& s, const void* q, const void* k, const void* v,
+                                   const void* dout, const int32_t* kept, int k_keep, const float* alpha,
+                                   const int8_t* labels, const void* wproj, int phi, float* dq, float* dk, float* dv,
+                                   float* dalpha, float* dwproj, char* ws, cudaStream_t st) {
+  const bool sla_mode = labels != nullptr;
+  const BwdLayout L = bwd_layout(s, sla_mode);
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const size_t nqkv = BH * static_cast<size_t>(s.N) * s.d * sizeof(float);
   const int nq = ceil_div(s.N, s.bq);
@@ -760,8 +947,15 @@ cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, co
   // accumulators: the key gradients, d alpha and the workspace sums start at zero
   if ((e = cudaMemsetAsync(dk, 0, nqkv, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dv, 0, nqkv, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(dalpha, 0, BH * nq * sizeof(float), st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(ws + L.htot, 0, L.total - L.htot, st)) != cudaSuccess) return e;
+  if (!sla_mode && (e = cudaMemsetAsync(dalpha, 0, BH * nq * sizeof(float), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ws + L.htot, 0, L.dphik + BH * static_cast<size_t>(s.N) * kDPad * 4 - L.htot, st)) !=
+      cudaSuccess)
+    return e;
+  if (sla_mode) {
+    e = launch_labels_to_lists(s, labels, reinterpret_cast<int32_t*>(ws + L.lists),
+                               reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int*>(ws + L.status), st);
+    if (e != cudaSuccess) return e;
+  }
   BwdArgs a;
   a.q = q;
   a.k = k;
@@ -787,7 +981,32 @@ cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, co
   a.dv = dv;
   a.dalpha = dalpha;
   a.status = reinterpret_cast<int*>(ws + L.status);
-  return s.in_dtype == SLA_BF16 ? run_backward<__nv_bfloat16>(s, a, st) : run_backward<float>(s, a, st);
+  a.sla = sla_mode ? 1 : 0;
+  a.lists = sla_mode ? reinterpret_cast<const int32_t*>(ws + L.lists) : nullptr;
+  a.counts = sla_mode ? reinterpret_cast<const int32_t*>(ws + L.counts) : nullptr;
+  a.wproj = static_cast<const __nv_bfloat16*>(wproj);
+  a.ol = sla_mode ? reinterpret_cast<float*>(ws + L.ol) : nullptr;
+  const bool bf = s.in_dtype == SLA_BF16;
+  e = bf ? run_backward<__nv_bfloat16>(s, a, st) : run_backward<float>(s, a, st);
+  if (e != cudaSuccess || !sla_mode) return e;
+  return bf ? run_wproj<__nv_bfloat16>(s, L, a.ol, dout, ws, dwproj, st)
+            : run_wproj<float>(s, L, a.ol, dout, ws, dwproj, st);
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                            const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
+                            float* dv, float* dalpha, char* ws, cudaStream_t st) {
+  return launch_backward_common(s, q, k, v, dout, kept, k_keep, alpha, nullptr, nullptr, phi, dq, dk, dv, dalpha,
+                                nullptr, ws, st);
+}
+
+cudaError_t launch_sla_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                                const int8_t* labels, const void* wproj, int phi, float* dq, float* dk, float* dv,
+                                float* dwproj, char* ws, cudaStream_t st) {
+  return launch_backward_common(s, q, k, v, dout, nullptr, 0, nullptr, labels, wproj, phi, dq, dk, dv, nullptr,
+                                dwproj, ws, st);
 }
 
 }  // namespace sla

@@ -47,14 +47,19 @@ __global__ void __launch_bounds__(256) labels_to_lists_kernel(const int8_t* __re
 
 }  // namespace
 
-cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, const WsLayout& L, char* ws,
-                                   cudaStream_t st) {
+cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, int32_t* lists, int32_t* counts,
+                                   int* status, cudaStream_t st) {
   const long long rows = static_cast<long long>(s.B) * s.H * ceil_div(s.N, s.bq);
   const int nkv = ceil_div(s.N, s.bkv);
-  labels_to_lists_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(
-      labels, reinterpret_cast<int32_t*>(ws + L.lists), reinterpret_cast<int32_t*>(ws + L.counts), rows, nkv,
-      reinterpret_cast<int*>(ws + L.status));
+  labels_to_lists_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(labels, lists, counts, rows,
+                                                                                        nkv, status);
   return cudaGetLastError();
+}
+
+cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, const WsLayout& L, char* ws,
+                                   cudaStream_t st) {
+  return launch_labels_to_lists(s, labels, reinterpret_cast<int32_t*>(ws + L.lists),
+                                reinterpret_cast<int32_t*>(ws + L.counts), reinterpret_cast<int*>(ws + L.status), st);
 }
 
 }  // namespace sla

@@ -49,6 +49,9 @@ struct BwdLayout {
   size_t htot = 0, ztot = 0;    // fp32 [BH, 128, 128], [BH, 128]: H_tot, Z_tot
   size_t dhtot = 0, dztot = 0;  // fp32 [BH, 128, 128], [BH, 128]: their gradients
   size_t dphik = 0;             // fp32 [BH, N, 128]: kept blocks' share of dL/dphi(K)
+  size_t lists = 0, counts = 0;  // SLA: int32 [BH, n_q, 2, n_kv] critical / negligible lists, [BH, n_q, 2] counts
+  size_t ol = 0;                // SLA: fp32 [BH, N, 128]: O_l rows for dW_proj
+  size_t wpart = 0;             // SLA: fp32 [splits, 128, 128]: dW_proj partial sums
   size_t total = 0;
 };
 

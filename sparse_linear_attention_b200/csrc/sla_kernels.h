@@ -16,13 +16,19 @@ cudaError_t launch_route(const sla_shape& s, const void* q, const void* k, const
                          float* scores_dbg, const WsLayout& L, char* ws, cudaStream_t st, float tau = 0.0f,
                          float* soft_mask = nullptr, float* soft_lambda = nullptr, const float* kbar = nullptr);
 
-BwdLayout bwd_layout(const sla_shape& s);
+BwdLayout bwd_layout(const sla_shape& s, bool sla_mode);
 
 // Gradients of the SLA2 forward (backward.cu): zeroes dk, dv, dalpha and the
 // workspace sums, then runs the three backward kernels on st.
 cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
                             const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
                             float* dv, float* dalpha, char* ws, cudaStream_t st);
+
+// Gradients of the SLA forward (backward.cu): the labels turned into lists,
+// the same three kernels with the SLA weights, then the dW_proj reduction.
+cudaError_t launch_sla_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                                const int8_t* labels, const void* wproj, int phi, float* dq, float* dk, float* dv,
+                                float* dwproj, char* ws, cudaStream_t st);
 
 cudaError_t launch_prepare(const sla_shape& s, const void* k, const void* v, int phi, const WsLayout& L,
                            char* ws, cudaStream_t st);
@@ -37,6 +43,8 @@ cudaError_t launch_qhat(const sla_shape& s, const void* q, const WsLayout& L, ch
 
 cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, const WsLayout& L, char* ws,
                                    cudaStream_t st);
+cudaError_t launch_labels_to_lists(const sla_shape& s, const int8_t* labels, int32_t* lists, int32_t* counts,
+                                   int* status, cudaStream_t st);
 
 struct SparseArgs {
   int BH, N, d, bq, nq, nkv;

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 
 EXPORTS = ("sla_status_string", "sla_last_error_detail", "sla_keep_count", "sla_workspace_size",
            "sla_workspace_init", "sla_route", "sla_route_noalloc", "sla_route_soft", "sla_prepare", "sla2_attn_fwd",
-           "sla_attn_fwd", "sla2_attn_bwd_workspace_size", "sla2_attn_bwd",
+           "sla_attn_fwd", "sla2_attn_bwd_workspace_size", "sla2_attn_bwd", "sla_attn_bwd_workspace_size", "sla_attn_bwd",
            "sla2_forward_host_device_bytes", "sla2_forward_host", "sla_read_device_status")
 
 
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         "sla_attn_fwd": (i, [sp, vp, vp, vp, vp, vp, i, u, vp, i, vp, sz, vp]),
         "sla2_attn_bwd_workspace_size": (sz, [sp]),
         "sla2_attn_bwd": (i, [sp, vp, vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sla_attn_bwd_workspace_size": (sz, [sp]),
+        "sla_attn_bwd": (i, [sp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sla2_forward_host_device_bytes": (sz, [sp, i, i, u]),
         "sla2_forward_host": (i, [sp, vp, vp, vp, vp, vp, vp, i, i, u, vp, i, vp, vp, sz, vp]),
         "sla_read_device_status": (i, [vp, vp]),
@@ -263,6 +265,23 @@ def sla2_attn_bwd(shape: Shape, q, k, v, kept_idx, k_keep, alpha, phi, dout, dq,
     _check("sla2_attn_bwd", lib().sla2_attn_bwd(ctypes.byref(shape), _p(q), _p(k), _p(v), _p(kept_idx), k_keep,
                                                 _p(alpha), phi, _p(dout), _p(dq), _p(dk), _p(dv), _p(dalpha),
                                                 _p(ws), nb, _s(stream)))
+
+
+def sla_attn_bwd_workspace_size(shape: Shape) -> int:
+    return lib().sla_attn_bwd_workspace_size(ctypes.byref(shape))
+
+
+def sla_attn_bwd(shape: Shape, q, k, v, labels, wproj, phi, dout, dq, dk, dv, dwproj, ws, stream=None):
+    a = _Args("sla_attn_bwd", shape)
+    a.qkv(q=q, k=k, v=v, dout=dout)
+    a("labels", labels, (a.B, a.H, a.nq, a.nkv), (torch.int8,))
+    a("wproj", wproj, (a.d, a.d), (torch.bfloat16,))
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        a(name, t, (a.B, a.H, a.N, a.d), (torch.float32,))
+    a("dwproj", dwproj, (a.d, a.d), (torch.float32,))
+    nb = a.ws(ws)
+    _check("sla_attn_bwd", lib().sla_attn_bwd(ctypes.byref(shape), _p(q), _p(k), _p(v), _p(labels), _p(wproj), phi,
+                                              _p(dout), _p(dq), _p(dk), _p(dv), _p(dwproj), _p(ws), nb, _s(stream)))
 
 
 def sla2_forward_host_device_bytes(shape: Shape, k_keep: int, out_dtype: int = SLA_BF16, flags: int = 0) -> int:

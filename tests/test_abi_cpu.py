@@ -230,6 +230,50 @@ def test_backward_workspace_layout():
         assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N, d)
 
 
+def test_sla_backward_rejects_bad_arguments_before_launch():
+    s = _shape()
+    L = sla.lib()
+    need = sla.sla_attn_bwd_workspace_size(s)
+    assert need > sla.sla2_attn_bwd_workspace_size(s) and need % 256 == 0
+    assert sla.sla_attn_bwd_workspace_size(_shape(d=100)) == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, labels=FAKE, wp=FAKE, phi=0, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, dwp=FAKE, ws=FAKE,
+                 wsb=need)
+        a.update(kw)
+        return L.sla_attn_bwd(ctypes.byref(s), a["q"], FAKE, FAKE, a["labels"], a["wp"], a["phi"], a["dout"],
+                              a["dq"], a["dk"], a["dv"], a["dwp"], a["ws"], a["wsb"], None)
+
+    assert call(q=None) == 1
+    assert call(labels=None) == 1
+    assert call(wp=None) == 1
+    assert call(phi=2) == 1
+    for name in ("dout", "dq", "dk", "dv"):
+        assert call(**{name: None}) == 1, name
+        assert call(**{name: FAKE + 4}) == 3, name
+    assert call(dwp=None) == 1
+    assert call(ws=None) == 1
+    assert call(ws=FAKE + 16) == 3
+    assert call(wsb=need - 1) == 4
+    assert "sla_attn_bwd_workspace_size" in L.sla_last_error_detail().decode()
+
+
+def test_sla_backward_workspace_layout():
+    """sla2_attn_bwd's workspace, then the critical / negligible lists and
+    their counts, the [BH, N, 128] fp32 O_l rows and the dW_proj partials of
+    about two row splits per SM, each rounded up to 256 bytes."""
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for B, H, N, d, bq in [(1, 12, 32760, 128, 128), (2, 3, 1000, 64, 64), (1, 1, 1, 8, 64)]:
+        s = _shape(B=B, H=H, N=N, d=d, bq=bq)
+        BH, nq, nkv = B * H, -(-N // bq), -(-N // 64)
+        rows = BH * N
+        per = max(32, -(-(-(-rows // 296)) // 32) * 32)
+        nsplit = -(-rows // per)
+        want = (sla.sla2_attn_bwd_workspace_size(s) + a256(BH * nq * 2 * nkv * 4) + a256(BH * nq * 2 * 4)
+                + a256(rows * 128 * 4) + a256(nsplit * 128 * 128 * 4))
+        assert sla.sla_attn_bwd_workspace_size(s) == want, (B, H, N, d)
+
+
 def _noalloc(shape, q=FAKE, k=FAKE, mode=0, k_keep=15, k_neg=0, kept=FAKE, wq=None):
     L = sla.lib()
     sp = ctypes.byref(shape) if shape is not None else None

@@ -140,3 +140,152 @@ def test_backward_wan13_sampled_query_blocks():
     ra = np.array([ref["dalpha"][b, h, i] for (b, h, i) in blocks])
     err = np.abs(ga - ra).max() / max(np.abs(ra).max(), 1e-30)
     assert err <= TOL_BWD_REL, ("dalpha", err)
+
+
+# ---------------------------------------------------------------- SLA (three labels, W_proj)
+
+def _labels(seed, B, H, nq, nkv, kh, kl):
+    """Per query block: kh critical and kl negligible blocks drawn at random."""
+    g = np.random.default_rng(seed)
+    lab = np.zeros((B, H, nq, nkv), dtype=np.int8)
+    for idx in np.ndindex(B, H, nq):
+        perm = g.permutation(nkv)
+        lab[idx][perm[:kh]] = 1
+        lab[idx][perm[kh:kh + kl]] = -1
+    return lab
+
+
+def _run_sla(q, k, v, labels, wp, do, bq, phi):
+    dev = "cuda"
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
+    shape = sla.make_shape(qd, bq, 64)
+    B, H, N, d = q.shape
+    ws = torch.zeros(sla.sla_attn_bwd_workspace_size(shape), dtype=torch.uint8, device=dev)
+    dq = torch.full((B, H, N, d), float("nan"), device=dev)
+    dk = torch.full_like(dq, float("nan"))
+    dv = torch.full_like(dq, float("nan"))
+    dwp = torch.full((d, d), float("nan"), device=dev)
+    sla.sla_attn_bwd(shape, qd, kd, vd, torch.from_numpy(labels).to(dev).contiguous(), wp.to(dev).contiguous(), phi,
+                     dod, dq, dk, dv, dwp, ws)
+    status = sla.sla_read_device_status(ws)
+    return status, {"dq": dq.cpu().numpy(), "dk": dk.cpu().numpy(), "dv": dv.cpu().numpy(),
+                    "dwproj": dwp.cpu().numpy()}
+
+
+def _check_sla(q, k, v, labels, wp, do, bq, phi, blocks=None):
+    status, got = _run_sla(q, k, v, labels, wp, do, bq, phi)
+    assert status == 0
+    kind = "softmax" if phi == sla.SLA_PHI_SOFTMAX else "elu1"
+    f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    ref = orc.sla_backward(f64(q), f64(k), f64(v), labels, f64(wp), f64(do), bq, 64, kind, blocks=blocks)
+    for name in ("dq", "dk", "dv", "dwproj"):
+        g, r = got[name], ref[name]
+        assert np.isfinite(g).all(), name
+        scale = max(np.abs(r).max(), 1e-30)
+        err = np.abs(g - r).max() / scale
+        assert err <= TOL_BWD_REL, (name, err)
+    return got
+
+
+def _wproj(seed, d):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(d, d, generator=g) / d ** 0.5).to(torch.bfloat16)
+
+
+def test_sla_backward_tiny_workload():
+    """The small case (fp32, d = 64, b_q = 64) with the oracle router's SLA
+    labels: 2 critical and 3 negligible of 16 blocks per query block."""
+    w = inputs.WORKLOADS["tiny"]
+    x = inputs.make_inputs(w)
+    _, labels, _ = orc.route(x["q"].numpy(), x["k"].numpy(), x["wq"].numpy(), x["wk"].numpy(), w.bq, w.bkv, "sla",
+                             2, 3)
+    g = torch.Generator().manual_seed(6)
+    do = torch.randn(x["q"].shape, generator=g).to(x["q"].dtype)
+    _check_sla(x["q"], x["k"], x["v"], labels, x["wproj"], do, w.bq, sla.SLA_PHI_ELU1)
+
+
+@pytest.mark.parametrize("N,d,bq,kh,kl,phi", [(1000, 128, 128, 3, 4, 0), (777, 64, 64, 2, 3, 0),
+                                              (130, 32, 128, 1, 1, 0), (700, 64, 64, 3, 2, 1)])
+def test_sla_backward_bf16_ragged(N, d, bq, kh, kl, phi):
+    """bf16 inputs, ragged last query and key blocks, both feature maps."""
+    q, k, v, do, _, _ = _case(N + kh + 7 * kl, 1, 2, N, d, bq, 0, torch.bfloat16)
+    labels = _labels(N + kh, 1, 2, -(-N // bq), -(-N // 64), kh, kl)
+    _check_sla(q, k, v, labels, _wproj(N, d), do, bq, phi)
+
+
+@pytest.mark.parametrize("kh,kl", [(5, 0), (0, 0), (0, 5), (0, 2), (4, 1)])
+def test_sla_backward_degenerate_labels(kh, kl):
+    """Every block critical (O_l = 0, dW_proj = 0), every block marginal
+    (linear only), every block negligible (O = 0, all gradients 0), no critical
+    block, no marginal block."""
+    q, k, v, do, _, _ = _case(60 + kh + kl, 2, 1, 300, 32, 64, 0, torch.bfloat16)
+    labels = _labels(kh * 7 + kl, 2, 1, 5, 5, kh, kl)
+    got = _check_sla(q, k, v, labels, _wproj(3, 32), do, 64, sla.SLA_PHI_ELU1)
+    if kh + kl == 5:
+        assert not got["dwproj"].any()
+    if kh == 0 and kl == 5:
+        assert not any(t.any() for t in got.values())
+
+
+def test_sla_backward_reports_bad_label():
+    q, k, v, do, _, _ = _case(70, 1, 1, 256, 64, 64, 0, torch.bfloat16)
+    labels = _labels(70, 1, 1, 4, 4, 1, 1)
+    labels[0, 0, 2, 3] = 2
+    status, got = _run_sla(q, k, v, labels, _wproj(4, 64), do, 64, sla.SLA_PHI_ELU1)
+    assert status == 7  # SLA_ERR_DEVICE_INDEX; the block counts as marginal
+    assert all(np.isfinite(t).all() for t in got.values())
+
+
+def _sampled_blocks(w, heads, seed):
+    rng = np.random.default_rng(seed)
+    return [(0, h, int(i)) for h in heads for i in sorted({0, w.n_q - 1, *rng.integers(0, w.n_q, 2)})]
+
+
+def _do_on_blocks(w, blocks, seed):
+    """An upstream gradient that is zero outside the given query blocks, so
+    that every key-side gradient and dW_proj are those blocks' shares alone."""
+    g = torch.Generator().manual_seed(seed)
+    do = torch.zeros(w.B, w.H, w.N, w.d, dtype=torch.bfloat16)
+    for (b, h, i) in blocks:
+        r = slice(i * w.bq, min((i + 1) * w.bq, w.N))
+        do[b, h, r] = torch.randn(do[b, h, r].shape, generator=g).to(torch.bfloat16)
+    return do
+
+
+def test_sla_backward_sla13_full_gradients_of_sampled_blocks():
+    """The 1.3B-shape SLA backward (12 heads, N = 32760, d = 128, 26 critical and
+    51 negligible of 512 key blocks from the oracle router) with dO non-zero
+    on sampled query blocks only, the first and the ragged last among them:
+    then dQ, dK, dV and dW_proj over the whole tensors are those blocks'
+    shares, which the oracle's blocks= path computes in full."""
+    w = inputs.WORKLOADS["sla13"]
+    x = inputs.make_inputs(w)
+    kh, kl = orc.keep_count(w.crit_ratio, w.n_kv), orc.keep_count(w.negl_ratio, w.n_kv)
+    _, labels, _ = orc.route(x["q"].float().numpy(), x["k"].float().numpy(), x["wq"].numpy(), x["wk"].numpy(),
+                             w.bq, w.bkv, "sla", kh, kl)
+    blocks = _sampled_blocks(w, (0, 11), 21)
+    do = _do_on_blocks(w, blocks, 21)
+    _check_sla(x["q"], x["k"], x["v"], labels, x["wproj"], do, w.bq, sla.SLA_PHI_ELU1, blocks=blocks)
+
+
+def test_backward_wan13_full_key_gradients_of_sampled_blocks():
+    """The SLA2 counterpart at the 1.3B shape: dO non-zero on sampled query
+    blocks only, so dK, dV (whole tensors), dQ and dalpha are the oracle's
+    blocks= result in full."""
+    w = inputs.WORKLOADS["wan13"]
+    x = inputs.make_inputs(w)
+    kk = orc.keep_count(w.keep_ratio, w.n_kv)
+    kept, _, _ = orc.route(x["q"].float().numpy(), x["k"].float().numpy(), x["wq"].numpy(), x["wk"].numpy(),
+                           w.bq, w.bkv, "sla2", kk)
+    blocks = _sampled_blocks(w, (3, 9), 22)
+    do = _do_on_blocks(w, blocks, 22)
+    status, got = _run(x["q"], x["k"], x["v"], kept, x["alpha"], do, w.bq, sla.SLA_PHI_ELU1)
+    assert status == 0
+    f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    ref = orc.sla2_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), kept, f64(x["alpha"]), f64(do), w.bq, w.bkv,
+                            blocks=blocks)
+    for name in ("dq", "dk", "dv", "dalpha"):
+        g, r = got[name], ref[name]
+        assert np.isfinite(g).all(), name
+        err = np.abs(g - r).max() / max(np.abs(r).max(), 1e-30)
+        assert err <= TOL_BWD_REL, (name, err)
