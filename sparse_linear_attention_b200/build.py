@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsla.so")
-SOURCES = ["api.cu", "route.cu", "route_noalloc.cu", "prepare.cu", "sparse_fwd.cu", "labels.cu", "backward.cu"]
+SOURCES = ["api.cu", "route.cu", "route_noalloc.cu", "prepare.cu", "sparse_fwd.cu", "labels.cu", "backward.cu", "backward_tc.cu"]
 HEADERS = ["sla_device.cuh", "sla_internal.h", "sla_kernels.h"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

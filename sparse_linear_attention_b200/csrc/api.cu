@@ -284,7 +284,7 @@ sla_status sla2_attn_fwd(const sla_shape* shape, const void* q, const void* k, c
 
 size_t sla2_attn_bwd_workspace_size(const sla_shape* shape) {
   if (shape == nullptr || check_shape(shape) != SLA_OK) return 0;
-  return bwd_layout(*shape, false).total;
+  return bwd_tc_eligible(*shape) ? bwd_tc_layout(*shape).total : bwd_layout(*shape, false).total;
 }
 
 sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k, const void* v,
@@ -304,10 +304,13 @@ sla_status sla2_attn_bwd(const sla_shape* shape, const void* q, const void* k, c
     return arg_fail(SLA_ERR_ALIGNMENT, "dout, dq, dk, dv, dalpha must be 16-byte aligned");
   if (ws == nullptr) return arg_fail(SLA_ERR_INVALID_ARG, "ws is null");
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return arg_fail(SLA_ERR_ALIGNMENT, "ws must be 256-byte aligned");
-  if (ws_bytes < bwd_layout(*shape, false).total)
+  const bool tc = bwd_tc_eligible(*shape);
+  if (ws_bytes < (tc ? bwd_tc_layout(*shape).total : bwd_layout(*shape, false).total))
     return arg_fail(SLA_ERR_WORKSPACE, "ws smaller than sla2_attn_bwd_workspace_size");
-  cudaError_t e = launch_backward(*shape, q, k, v, dout, kept_idx, k_keep, alpha, phi, dq, dk, dv, dalpha,
-                                  static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+  cudaError_t e = tc ? launch_backward_tc(*shape, q, k, v, dout, kept_idx, k_keep, alpha, phi, dq, dk, dv, dalpha,
+                                          static_cast<char*>(ws), static_cast<cudaStream_t>(stream))
+                     : launch_backward(*shape, q, k, v, dout, kept_idx, k_keep, alpha, phi, dq, dk, dv, dalpha,
+                                       static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SLA_OK : cuda_fail(e, "backward");
 }
 

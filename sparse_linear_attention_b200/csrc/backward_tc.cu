@@ -1,0 +1,964 @@
+// backward_tc.cu -- the SLA2 backward on the tensor cores (bf16 inputs,
+// d = 128, b_q = 128, b_kv = 64).
+//
+// Same gradients as backward.cu ("SLA: Beyond Sparsity in Diffusion
+// Transformers …" (papernotes.org) 关键设计 4: the sparse part back-propagated
+// the FlashAttention way, the linear part through dH_i, dZ_i written as totals
+// minus the kept blocks; "SLA2 深度解读 …" (jefxiong.cn) §07: gradients on
+// the unquantised inputs), with A_j = phi(Q) phi(K_j)^T, G_j = dO V_j^T,
+// s = (1 - alpha) / den, dden = -(1 - alpha) dO . O_l / den:
+//   dS_j = P_j * (alpha G_j - D),  Bx_j = s G_j + dden,  C_j = alpha P_j - s A_j
+//   dQ   = dS K / sqrt(d) + phi'(Q) [ s dO H_tot^T + dden Z_tot^T - sum_j Bx_j phi(K_j) ]
+//   dK_j = dS_j^T Q / sqrt(d),  dV_j = C_j^T dO,  dphi(K_j) = -Bx_j^T phi(Q)  (kept shares)
+//   dH_tot = sum phi(Q)^T (s dO),  dZ_tot = sum phi(Q)^T dden
+// and the per-key step of backward.cu for the totals' share.
+//
+// The per-row quantities (the log2-sum-exp of the kept scores, D, s, dden and
+// the row's share of dalpha) come from the attention kernel itself, run once
+// more with the upstream gradient (SparseArgs::bwd_rows): it already forms
+// O_s, O_l, the row sums and the denominators.  Then:
+//   qphi_kernel      phi(Q) as fp16 [BH, N, 128] (the forward's rounding)
+//   inv_lists_kernel per key block the query blocks that keep it, ascending
+//   bwd_dq_kernel    per query tile: S, G (tcgen05, bf16) per kept block;
+//                    dS (bf16), -Bx sigma (fp16) to smem; dQ_s += dS K,
+//                    dQ_l += (-Bx sigma) phi(K); then s sigma dO H_tot^T / sigma
+//                    and dH_i = phi(Q)^T (s sigma dO) / sigma; epilogue dQ.
+//   bwd_dkv_kernel   per key block: for each query tile keeping it, S, G, A
+//                    (tcgen05); dS, C (bf16), -Bx sigma (fp16) to smem;
+//                    dV^T += dO^T C, dK^T += Q^T dS, dphi(K)^T += phi(Q)^T (-Bx sigma)
+//                    accumulated in TMEM over the tiles; no atomics.
+//   dh_reduce_kernel dH_tot, dZ_tot: the tiles' partials summed in tile order
+//   dalpha_kernel    dalpha per query block: its rows' shares in row order
+// sigma is the forward's per-head power of two (>= max_e Z_tot[e]); it scales
+// Bx and s dO into the fp16 range and is divided out exactly.
+// Every result is written once in a fixed order: the gradients are the same
+// on every run.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "sla_device.cuh"
+#include "sla_internal.h"
+#include "sla_kernels.h"
+
+namespace sla {
+
+namespace {
+
+constexpr int kTcThreads = 192;  // warps 0..3: one row (or channel) per thread; warp 4 TMA; warp 5 MMA
+constexpr int kRowsT = 128;      // query rows per tile
+
+struct TcArgs {
+  int BH, N, nq, nkv, kk, phi;
+  float sl2, scale;
+  const int32_t* kept;   // [BH, nq, kk]
+  const float* alpha;    // [BH, nq]
+  const float* rows;     // [BH * N, 8] from the attention kernel's statistics epilogue
+  const float* sigma;    // [BH]
+  const float* ztot;     // [BH, 128]
+  const int32_t* inv;    // [BH, nkv, nq] query blocks keeping each key block
+  const int32_t* inv_n;  // [BH, nkv]
+  const __nv_bfloat16* q;
+  float *dq, *dk, *dv, *dphik;  // dq, dk, dv [BH, N, 128]; dphik fp32 [BH, N, 128]
+  float *dhpart, *dzpart;       // [BH * nq, 128, 128], [BH * nq, 128]
+  int* status;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ int clamp_block(int j, int nkv, int* status, bool report) {
+  if (j < 0 || j >= nkv) {
+    if (report) report_error(status, SLA_ERR_DEVICE_INDEX);
+    return 0;
+  }
+  return j;
+}
+
+__device__ __forceinline__ bool warp_wait_tc(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                             uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+// Eight 16-bit values of row r into unit u of a 128-byte-swizzled tile.
+__device__ __forceinline__ void put_unit(uint8_t* tile, int r, int u, uint32_t a, uint32_t b, uint32_t c,
+                                         uint32_t d) {
+  *reinterpret_cast<uint4*>(tile + sw128_off(r, u)) = make_uint4(a, b, c, d);
+}
+
+// ---------------------------------------------------------------- phi(Q)
+// fp16 phi(Q) [rows][128] with the attention kernel's rounding (ELU+1 or the
+// channel softmax through ex2.approx).  16 threads per row, 8 channels each.
+__global__ void __launch_bounds__(256) qphi_kernel(const __nv_bfloat16* __restrict__ q, __half* __restrict__ out,
+                                                   long long rows, int phi) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = idx >> 4;
+  const int u = static_cast<int>(idx & 15);
+  const bool live = row < rows;
+  float x[8];
+  {
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (live) w = *reinterpret_cast<const uint4*>(q + row * kDPad + 8 * u);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf162(ww[e]);
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+  }
+  float y[8];
+  if (phi == SLA_PHI_SOFTMAX) {
+    float mx = x[0];
+#pragma unroll
+    for (int e = 1; e < 8; ++e) mx = fmaxf(mx, x[e]);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      y[e] = ex2_approx((x[e] - mx) * 1.4426950408889634f);
+      sum += y[e];
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] *= inv;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = elu1(x[e]);
+  }
+  if (live)
+    *reinterpret_cast<uint4*>(out + row * kDPad + 8 * u) =
+        make_uint4(pack_half2(y[0], y[1]), pack_half2(y[2], y[3]), pack_half2(y[4], y[5]), pack_half2(y[6], y[7]));
+}
+
+// ---------------------------------------------------------------- inverse lists
+// One warp per (bh, key block j): the query blocks whose kept list holds j,
+// ascending (the kept lists are scanned 32 query blocks at a time).
+__global__ void __launch_bounds__(256) inv_lists_kernel(const int32_t* __restrict__ kept, int nq, int nkv, int kk,
+                                                        int32_t* __restrict__ inv, int32_t* __restrict__ inv_n) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  const long long bh = blockIdx.y;
+  if (j >= nkv) return;
+  int32_t* dst = inv + (bh * nkv + j) * nq;
+  int n = 0;
+  for (int i0 = 0; i0 < nq; i0 += 32) {
+    const int i = i0 + lane;
+    bool hit = false;
+    if (i < nq) {
+      const int32_t* lst = kept + (bh * nq + i) * kk;
+      for (int t = 0; t < kk; ++t) hit = hit || (lst[t] == j);
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, hit);
+    if (hit) dst[n + __popc(m & ((1u << lane) - 1u))] = i;
+    n += __popc(m);
+  }
+  if (lane == 0) inv_n[bh * nkv + j] = n;
+}
+
+// ---------------------------------------------------------------- dQ (query-major)
+namespace dq {
+constexpr uint32_t OFF_Q = 0;          // bf16 [128 rows] x 2 chunks
+constexpr uint32_t OFF_DO = 32768;     // bf16 [128 rows] x 2 chunks
+constexpr uint32_t OFF_ST = 65536;     // 2 stages: K | V | phi(K), each 2 chunks of [64 rows][128 B]
+constexpr uint32_t STAGE = 49152;
+constexpr uint32_t OFF_OPS = OFF_ST + 2 * STAGE;  // dS bf16 [128][64] | -Bx sigma fp16 [128][64]; end: s sigma dO fp16 [128][128]
+constexpr uint32_t OFF_BAR = OFF_OPS + 32768;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t OFF_DD = OFF_MISC + 64;  // dden per row [128] floats
+constexpr uint32_t SMEM = OFF_DD + 512;
+static_assert(SMEM <= 232448, "shared memory budget");
+// TMEM columns: S_b at 128 b, G_b at 128 b + 64 (b = 0, 1); dQ_s 256; dQ_l 384.
+// End phase: s dO H_tot^T at 0, sigma dH_i at 128.
+constexpr uint32_t T_DQS = 256, T_DQL = 384, T_HT = 0, T_DH = 128;
+enum { B_QD = 0, B_STF = 1, B_STE = 3, B_SGF = 5, B_SGE = 7, B_OPF = 9, B_OPE = 10, B_LOOP = 11, B_ENDL = 12,
+       B_SDO = 13, B_END = 14, B_DRAIN = 15, NBAR = 16 };
+}  // namespace dq
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmH,
+                  const __grid_constant__ CUtensorMap tmPQ, const TcArgs a) {
+  using namespace dq;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(a.status, SLA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  float* ddsh = reinterpret_cast<float*>(sm + OFF_DD);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qb = blockIdx.x % a.nq;
+  const int bh = blockIdx.x / a.nq;
+  const long long tile = blockIdx.x;
+  const int kk = a.kk;
+  const int32_t* lst = a.kept + tile * kk;
+
+  if (tid == 0) {
+    mbar_init(&bars[B_QD], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[B_STF + s], 1);
+      mbar_init(&bars[B_STE + s], 1);
+      mbar_init(&bars[B_SGF + s], 1);
+      mbar_init(&bars[B_SGE + s], kRowsT);
+    }
+    mbar_init(&bars[B_OPF], kRowsT);
+    mbar_init(&bars[B_OPE], 1);
+    mbar_init(&bars[B_LOOP], 1);
+    mbar_init(&bars[B_ENDL], 1);
+    mbar_init(&bars[B_SDO], kRowsT);
+    mbar_init(&bars[B_END], 1);
+    mbar_init(&bars[B_DRAIN], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float sigma = a.sigma[bh];
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;  // stage loads issued
+      mbar_arrive_expect_tx(&bars[B_QD], 65536);
+      tma_load_3d(sm + OFF_Q, &tmQ, &bars[B_QD], 0, qb * kRowsT, bh);
+      tma_load_3d(sm + OFF_Q + 16384, &tmQ, &bars[B_QD], 64, qb * kRowsT, bh);
+      tma_load_3d(sm + OFF_DO, &tmDO, &bars[B_QD], 0, qb * kRowsT, bh);
+      tma_load_3d(sm + OFF_DO + 16384, &tmDO, &bars[B_QD], 64, qb * kRowsT, bh);
+      for (int n = 0; n < kk; ++n) {
+        const int s = n & 1;
+        if (n >= 2 && !mbar_wait(&bars[B_STE + s], ((n >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        const int krow = clamp_block(lst[n], a.nkv, a.status, true) * kBlockKV;
+        uint8_t* st = sm + OFF_ST + s * STAGE;
+        uint64_t* fb = &bars[B_STF + s];
+        mbar_arrive_expect_tx(fb, STAGE);
+        tma_load_3d(st, &tmK, fb, 0, krow, bh);
+        tma_load_3d(st + 8192, &tmK, fb, 64, krow, bh);
+        tma_load_3d(st + 16384, &tmV, fb, 0, krow, bh);
+        tma_load_3d(st + 16384 + 8192, &tmV, fb, 64, krow, bh);
+        tma_load_3d(st + 32768, &tmPK, fb, 0, krow, bh);
+        tma_load_3d(st + 32768 + 8192, &tmPK, fb, 64, krow, bh);
+        ++issued;
+      }
+      bool end_issued = false;
+      if (ok && mbar_wait(&bars[B_LOOP], 0, abort_flag, a.status, a.wait_ns)) {
+        // every product of the loop is done: the stage area takes H_tot / sigma and phi(Q)
+        mbar_arrive_expect_tx(&bars[B_ENDL], 65536);
+        tma_load_3d(sm + OFF_ST, &tmH, &bars[B_ENDL], 0, 0, bh);
+        tma_load_3d(sm + OFF_ST + 16384, &tmH, &bars[B_ENDL], 64, 0, bh);
+        tma_load_3d(sm + OFF_ST + 32768, &tmPQ, &bars[B_ENDL], 0, qb * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 49152, &tmPQ, &bars[B_ENDL], 64, qb * kRowsT, bh);
+        end_issued = true;
+      }
+      // every issued copy lands before the CTA exits
+      mbar_wait_drain(&bars[B_QD], 0);
+      for (int g = issued > 2 ? issued - 2 : 0; g < issued; ++g) mbar_wait_drain(&bars[B_STF + (g & 1)], (g >> 1) & 1);
+      if (end_issued) mbar_wait_drain(&bars[B_ENDL], 0);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);    // Q x K_j^T, dO x V_j^T (bf16, K-major)
+      const uint32_t id_qk = idesc_f16(1, 0, 1, 128, 128);  // dS (K-major) x K_j (MN-major), bf16
+      const uint32_t id_ql = idesc_f16(0, 0, 1, 128, 128);  // -Bx sigma x phi(K_j) (MN-major), f16
+      const uint32_t id_ht = idesc_f16(0, 0, 0, 128, 128);  // s sigma dO (K-major) x H_tot / sigma (K-major), f16
+      const uint32_t id_dh = idesc_f16(0, 1, 1, 128, 128);  // phi(Q)^T (MN-major) x s sigma dO (MN-major), f16
+      const uint64_t dQd = sdesc_sw128(smem_u32(sm + OFF_Q), 16, 1024);
+      const uint64_t dOd = sdesc_sw128(smem_u32(sm + OFF_DO), 16, 1024);
+      const uint64_t dStK = sdesc_sw128(smem_u32(sm + OFF_ST), 16, 1024);         // K-major key tiles
+      const uint64_t dStMN = sdesc_sw128(smem_u32(sm + OFF_ST), 8192, 1024);      // the same as MN-major
+      const uint64_t dOps = sdesc_sw128(smem_u32(sm + OFF_OPS), 16, 1024);        // dS, Bx (K-major, one chunk)
+      const uint64_t dSdoK = sdesc_sw128(smem_u32(sm + OFF_OPS), 16, 1024);       // s sigma dO as K-major A
+      const uint64_t dSdoMN = sdesc_sw128(smem_u32(sm + OFF_OPS), 16384, 1024);   // ... as MN-major B
+      const uint64_t dH = sdesc_sw128(smem_u32(sm + OFF_ST), 16, 1024);           // H_tot / sigma (K-major B)
+      const uint64_t dPQ = sdesc_sw128(smem_u32(sm + OFF_ST + 32768), 16384, 1024);  // phi(Q)^T (MN-major A)
+      bool ok = mbar_wait(&bars[B_QD], 0, abort_flag, a.status, a.wait_ns);
+      auto ops = [&](int m) -> bool {
+        if (!mbar_wait(&bars[B_OPF], m & 1, abort_flag, a.status, a.wait_ns)) return false;
+        tc_fence_after();
+        const uint32_t so = ((m & 1) * STAGE) >> 4;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)  // K = 64 keys: A +32 B, B +2048 B per 16
+          mma_f16_ss(tmem + T_DQS, dOps + k4 * 2u, dStMN + so + k4 * 128u, id_qk, (m > 0 || k4 > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)
+          mma_f16_ss(tmem + T_DQL, dOps + (16384u >> 4) + k4 * 2u, dStMN + so + (32768u >> 4) + k4 * 128u, id_ql,
+                     (m > 0 || k4 > 0) ? 1u : 0u);
+        mma_commit(&bars[B_OPE]);
+        mma_commit(&bars[B_STE + (m & 1)]);
+        return true;
+      };
+      for (int n = 0; ok && n < kk; ++n) {
+        const int b = n & 1;
+        if (!mbar_wait(&bars[B_STF + b], (n >> 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (n >= 2 && !mbar_wait(&bars[B_SGE + b], ((n >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t so = (b * STAGE) >> 4;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          const uint32_t ob = ((k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + 128 * b, dQd + oa, dStK + so + ob, id_s, k8 > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          const uint32_t ob = (16384u + (k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + 128 * b + 64, dOd + oa, dStK + so + ob, id_s, k8 > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[B_SGF + b]);
+        if (n >= 1 && !ops(n - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && kk > 0) ok = ops(kk - 1);
+      if (ok) mma_commit(&bars[B_LOOP]);
+      if (ok && mbar_wait(&bars[B_ENDL], 0, abort_flag, a.status, a.wait_ns) &&
+          mbar_wait(&bars[B_SDO], 0, abort_flag, a.status, a.wait_ns)) {
+        tc_fence_after();
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {  // s dO H_tot^T: K = 128 channels
+          const uint32_t o = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + T_HT, dSdoK + o, dH + o, id_ht, k8 > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8)  // sigma dH_i: K = 128 rows, +2048 B per 16
+          mma_f16_ss(tmem + T_DH, dPQ + k8 * 128u, dSdoMN + k8 * 128u, id_dh, k8 > 0 ? 1u : 0u);
+        mma_commit(&bars[B_END]);
+      }
+      mma_commit(&bars[B_DRAIN]);
+      mbar_wait_drain(&bars[B_DRAIN], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ rows (warps 0..3)
+    const int r = tid;  // tile row = TMEM lane
+    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
+    const int tok = qb * kRowsT + r;
+    const bool valid = tok < a.N;
+    float lse2 = 0.0f, D = 0.0f, sr = 0.0f, dd = 0.0f;
+    if (valid) {
+      const float4 st = *reinterpret_cast<const float4*>(a.rows + (static_cast<long long>(bh) * a.N + tok) * 8);
+      lse2 = st.x;
+      D = st.y;
+      sr = st.z;
+      dd = st.w;
+    }
+    const float alpha = a.alpha[tile];
+    const bool tail = (a.N & (kBlockKV - 1)) != 0;
+    bool ok = true;
+    uint8_t* opS = sm + OFF_OPS;
+    uint8_t* opB = sm + OFF_OPS + 16384;
+    for (int n = 0; n < kk; ++n) {
+      const int b = n & 1;
+      ok = ok && warp_wait_tc(&bars[B_SGF + b], (n >> 1) & 1, abort_flag, a.status, a.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      const int j = clamp_block(lst[n], a.nkv, a.status, false);
+      const int nvalid = (tail && j == a.nkv - 1) ? a.N - j * kBlockKV : kBlockKV;
+      uint32_t pS[32], pB[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float sv[32], gv[32];
+        tmem_ld32(tmem + lrow + 128 * b + 32 * h, sv);
+        tmem_ld32(tmem + lrow + 128 * b + 64 + 32 * h, gv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float ds[2], bx[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool kv = valid && (32 * h + c + e < nvalid);
+            const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
+            ds[e] = p * fmaf(alpha, gv[c + e], -D);
+            bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
+          }
+          pS[16 * h + c / 2] = pack_bf162(ds[0], ds[1]);
+          pB[16 * h + c / 2] = pack_half2(bx[0], bx[1]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_SGE + b]);
+      ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
+      if (!ok) break;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        put_unit(opS, r, u, pS[4 * u], pS[4 * u + 1], pS[4 * u + 2], pS[4 * u + 3]);
+        put_unit(opB, r, u, pB[4 * u], pB[4 * u + 1], pB[4 * u + 2], pB[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_OPF]);
+    }
+    // s sigma dO (fp16) over the operand tiles once the loop's products are done
+    ok = ok && warp_wait_tc(&bars[B_LOOP], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) {
+      const float f = sr * sigma;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_DO + ch * 16384u + sw128_off(r, u));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 g = unpack_bf162(ww[e]);
+            o4[e] = pack_half2(g.x * f, g.y * f);
+          }
+          put_unit(sm + OFF_OPS + ch * 16384u, r, u, o4[0], o4[1], o4[2], o4[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_SDO]);
+    }
+    ddsh[r] = dd;
+    named_bar_sync(1, kRowsT);
+    // dZ_i[e] = sum over the rows of phi(Q)[row][e] dden[row], e = r (phi(Q) tile in smem)
+    ok = ok && warp_wait_tc(&bars[B_ENDL], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) {
+      const int e = r, ch = e >> 6, u = (e & 63) >> 3, w = e & 7;
+      float z = 0.0f;
+      for (int rr = 0; rr < kRowsT; ++rr) {
+        const __half* hp =
+            reinterpret_cast<const __half*>(sm + OFF_ST + 32768 + ch * 16384u + sw128_off(rr, u)) + w;
+        z = fmaf(__half2float(*hp), ddsh[rr], z);
+      }
+      a.dzpart[tile * kDPad + e] = z;
+    }
+    ok = ok && warp_wait_tc(&bars[B_END], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      const float inv_sigma = 1.0f / sigma;  // exact: a power of two
+      // sigma dH_i: lane e, 128 columns c
+      float* dh = a.dhpart + (tile * kDPad + r) * kDPad;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float hv[32];
+        tmem_ld32(tmem + lrow + T_DH + 32 * cc, hv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          *reinterpret_cast<float4*>(dh + 32 * cc + c) =
+              make_float4(hv[c] * inv_sigma, hv[c + 1] * inv_sigma, hv[c + 2] * inv_sigma, hv[c + 3] * inv_sigma);
+      }
+      // dQ of row r: scale dQ_s + phi'(Q) (dQ_l / sigma + s dO H_tot^T + dden Z_tot)
+      const float* zt = a.ztot + static_cast<long long>(bh) * kDPad;
+      const bool have = kk > 0;
+      // 32 channels of Q row r from the smem tile
+      auto q32 = [&](int cc, float* x) {
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_Q + (cc >> 1) * 16384u +
+                                                          sw128_off(r, (cc & 1) * 4 + u4));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf162(ww[e]);
+            x[8 * u4 + 2 * e] = f.x;
+            x[8 * u4 + 2 * e + 1] = f.y;
+          }
+        }
+      };
+      // the gradient reaching phi(Q) for 32 channels
+      auto gphi = [&](int cc, float* g) {
+        float l[32], h[32];
+        tmem_ld32(tmem + lrow + T_DQL + 32 * cc, l);
+        tmem_ld32(tmem + lrow + T_HT + 32 * cc, h);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) g[c] = (have ? l[c] * inv_sigma : 0.0f) + h[c] + dd * zt[32 * cc + c];
+      };
+      // the softmax feature map: phi'(q) g = phi (g - sum_c phi_c g_c), phi from the row max and sum
+      const bool smx = a.phi == SLA_PHI_SOFTMAX;
+      float mx = -INFINITY, inv_sum = 0.0f, dot = 0.0f;
+      if (smx) {
+        float x[32];
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          q32(cc, x);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, x[c]);
+        }
+        float sum = 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          q32(cc, x);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sum += expf(x[c] - mx);
+        }
+        inv_sum = 1.0f / sum;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float g[32];
+          q32(cc, x);
+          gphi(cc, g);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) dot = fmaf(expf(x[c] - mx) * inv_sum, g[c], dot);
+        }
+      }
+      float* dqr = a.dq + (static_cast<long long>(bh) * a.N + tok) * kDPad;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float g[32], sq[32], x[32];
+        q32(cc, x);
+        gphi(cc, g);
+        tmem_ld32(tmem + lrow + T_DQS + 32 * cc, sq);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float dphi = smx ? expf(x[c] - mx) * inv_sum * (g[c] - dot) : g[c] * (x[c] > 0.0f ? 1.0f : expf(x[c]));
+          o[c] = (have ? sq[c] * a.scale : 0.0f) + dphi;
+        }
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dqr + 32 * cc + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV (key-major)
+namespace dkv {
+constexpr uint32_t OFF_K = 0;          // K_j | V_j | phi(K_j): each 2 chunks of [64 rows][128 B]
+constexpr uint32_t OFF_V = 16384;
+constexpr uint32_t OFF_PK = 32768;
+constexpr uint32_t OFF_ST = 49152;     // Q_i | dO_i | phi(Q_i): each 2 chunks of [128 rows][128 B]
+constexpr uint32_t OFF_OPS = OFF_ST + 98304;  // dS bf16 | C bf16 | -Bx sigma fp16, each [128 rows][64 keys]
+constexpr uint32_t OFF_BAR = OFF_OPS + 49152;
+constexpr uint32_t OFF_MISC = OFF_BAR + 128;
+constexpr uint32_t SMEM = OFF_MISC + 64;
+static_assert(SMEM <= 232448, "shared memory budget");
+// TMEM: S 0, G 64, A 128; dV^T 256, dK^T 320, dphi(K)^T 384
+constexpr uint32_t T_S = 0, T_G = 64, T_A = 128, T_DV = 256, T_DK = 320, T_DP = 384;
+enum { B_KV = 0, B_STF = 1, B_STE = 2, B_SGF = 3, B_OPF = 4, B_OPE = 5, B_DONE = 6, B_DRAIN = 7, NBAR = 8 };
+}  // namespace dkv
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
+                   const TcArgs a) {
+  using namespace dkv;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(a.status, SLA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x % a.nkv;
+  const int bh = blockIdx.x / a.nkv;
+  const long long kb = static_cast<long long>(bh) * a.nkv + j;
+  int cnt = a.inv_n[kb];
+  if (cnt < 0 || cnt > a.nq) cnt = 0;
+  const int32_t* il = a.inv + kb * a.nq;
+
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == B_OPF) ? kRowsT : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float sigma = a.sigma[bh];
+
+  if (warp == 4) {
+    if (lane == 0 && cnt > 0) {
+      int issued = 0;
+      mbar_arrive_expect_tx(&bars[B_KV], 49152);
+      tma_load_3d(sm + OFF_K, &tmK, &bars[B_KV], 0, j * kBlockKV, bh);
+      tma_load_3d(sm + OFF_K + 8192, &tmK, &bars[B_KV], 64, j * kBlockKV, bh);
+      tma_load_3d(sm + OFF_V, &tmV, &bars[B_KV], 0, j * kBlockKV, bh);
+      tma_load_3d(sm + OFF_V + 8192, &tmV, &bars[B_KV], 64, j * kBlockKV, bh);
+      tma_load_3d(sm + OFF_PK, &tmPK, &bars[B_KV], 0, j * kBlockKV, bh);
+      tma_load_3d(sm + OFF_PK + 8192, &tmPK, &bars[B_KV], 64, j * kBlockKV, bh);
+      for (int n = 0; n < cnt; ++n) {
+        if (n >= 1 && !mbar_wait(&bars[B_STE], (n - 1) & 1, abort_flag, a.status, a.wait_ns)) break;
+        int i = il[n];
+        if (i < 0 || i >= a.nq) i = 0;
+        uint64_t* fb = &bars[B_STF];
+        mbar_arrive_expect_tx(fb, 98304);
+        tma_load_3d(sm + OFF_ST, &tmQ, fb, 0, i * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 16384, &tmQ, fb, 64, i * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 32768, &tmDO, fb, 0, i * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 49152, &tmDO, fb, 64, i * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 65536, &tmPQ, fb, 0, i * kRowsT, bh);
+        tma_load_3d(sm + OFF_ST + 81920, &tmPQ, fb, 64, i * kRowsT, bh);
+        ++issued;
+      }
+      mbar_wait_drain(&bars[B_KV], 0);
+      if (issued > 0) mbar_wait_drain(&bars[B_STF], (issued - 1) & 1);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);   // Q_i K_j^T, dO_i V_j^T (bf16)
+      const uint32_t id_a = idesc_f16(0, 0, 0, 128, 64);   // phi(Q_i) phi(K_j)^T (f16)
+      const uint32_t id_t = idesc_f16(1, 1, 1, 128, 64);   // dO^T C, Q^T dS (bf16, both MN-major)
+      const uint32_t id_tp = idesc_f16(0, 1, 1, 128, 64);  // phi(Q)^T (-Bx sigma) (f16)
+      const uint64_t dKd = sdesc_sw128(smem_u32(sm + OFF_K), 16, 1024);
+      const uint64_t dStK = sdesc_sw128(smem_u32(sm + OFF_ST), 16, 1024);
+      const uint64_t dStMN = sdesc_sw128(smem_u32(sm + OFF_ST), 16384, 1024);
+      const uint64_t dOpsMN = sdesc_sw128(smem_u32(sm + OFF_OPS), 16, 1024);  // N = 64 fits one atom
+      bool ok = cnt > 0 && mbar_wait(&bars[B_KV], 0, abort_flag, a.status, a.wait_ns);
+      for (int n = 0; ok && n < cnt; ++n) {
+        if (!mbar_wait(&bars[B_STF], n & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // S, G, A: M = 128 rows, N = 64 keys, K = 128 channels
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          const uint32_t ob = ((k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + T_S, dStK + oa, dKd + ob, id_s, k8 > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + T_G, dStK + (32768u >> 4) + oa, dKd + (16384u >> 4) + ob, id_s, k8 > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + T_A, dStK + (65536u >> 4) + oa, dKd + (32768u >> 4) + ob, id_a, k8 > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[B_SGF]);
+        if (!mbar_wait(&bars[B_OPF], n & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dV^T, dK^T, dphi(K)^T: M = 128 channels, N = 64 keys, K = 128 rows (+2048 B per 16)
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t acc = (n > 0 || k8 > 0) ? 1u : 0u;
+          mma_f16_ss(tmem + T_DV, dStMN + (32768u >> 4) + k8 * 128u, dOpsMN + (16384u >> 4) + k8 * 128u, id_t, acc);
+          mma_f16_ss(tmem + T_DK, dStMN + k8 * 128u, dOpsMN + k8 * 128u, id_t, acc);
+          mma_f16_ss(tmem + T_DP, dStMN + (65536u >> 4) + k8 * 128u, dOpsMN + (32768u >> 4) + k8 * 128u, id_tp, acc);
+        }
+        mma_commit(&bars[B_OPE]);
+        mma_commit(&bars[B_STE]);
+      }
+      mma_commit(&bars[B_DONE]);
+      mma_commit(&bars[B_DRAIN]);
+      mbar_wait_drain(&bars[B_DRAIN], 0);
+    }
+  } else {
+    const int r = tid;
+    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
+    const bool tail = (a.N & (kBlockKV - 1)) != 0;
+    const int nvalid = (tail && j == a.nkv - 1) ? a.N - j * kBlockKV : kBlockKV;
+    bool ok = true;
+    uint8_t* opS = sm + OFF_OPS;
+    uint8_t* opC = sm + OFF_OPS + 16384;
+    uint8_t* opB = sm + OFF_OPS + 32768;
+    for (int n = 0; n < cnt; ++n) {
+      int i = il[n];
+      if (i < 0 || i >= a.nq) i = 0;
+      const int tok = i * kRowsT + r;
+      const bool valid = tok < a.N;
+      float lse2 = 0.0f, D = 0.0f, sr = 0.0f, dd = 0.0f;
+      if (valid) {
+        const float4 st = *reinterpret_cast<const float4*>(a.rows + (static_cast<long long>(bh) * a.N + tok) * 8);
+        lse2 = st.x;
+        D = st.y;
+        sr = st.z;
+        dd = st.w;
+      }
+      const float alpha = a.alpha[static_cast<long long>(bh) * a.nq + i];
+      ok = ok && warp_wait_tc(&bars[B_SGF], n & 1, abort_flag, a.status, a.wait_ns);
+      // The products of the previous tile read the operand tiles; they were
+      // issued before this tile's S, G, A, so they are done (the wait is immediate).
+      ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float sv[32], gv[32], av[32];
+        tmem_ld32(tmem + lrow + T_S + 32 * h, sv);
+        tmem_ld32(tmem + lrow + T_G + 32 * h, gv);
+        tmem_ld32(tmem + lrow + T_A + 32 * h, av);
+        tmem_wait_ld();
+        uint32_t pS[16], pC[16], pB[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float ds[2], cv[2], bx[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool kv = valid && (32 * h + c + e < nvalid);
+            const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
+            ds[e] = p * fmaf(alpha, gv[c + e], -D);
+            cv[e] = kv ? fmaf(alpha, p, -sr * av[c + e]) : 0.0f;
+            bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
+          }
+          pS[c / 2] = pack_bf162(ds[0], ds[1]);
+          pC[c / 2] = pack_bf162(cv[0], cv[1]);
+          pB[c / 2] = pack_half2(bx[0], bx[1]);
+        }
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int u = 4 * h + u4;
+          put_unit(opS, r, u, pS[4 * u4], pS[4 * u4 + 1], pS[4 * u4 + 2], pS[4 * u4 + 3]);
+          put_unit(opC, r, u, pC[4 * u4], pC[4 * u4 + 1], pC[4 * u4 + 2], pC[4 * u4 + 3]);
+          put_unit(opB, r, u, pB[4 * u4], pB[4 * u4 + 1], pB[4 * u4 + 2], pB[4 * u4 + 3]);
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_OPF]);
+    }
+    // epilogue: lane = channel c; columns = the block's 64 keys
+    if (cnt > 0) ok = ok && warp_wait_tc(&bars[B_DONE], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      const int c = r;
+      const float inv_sigma = 1.0f / sigma;
+      const long long base = (static_cast<long long>(bh) * a.N + static_cast<long long>(j) * kBlockKV) * kDPad + c;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float vv[32], kv[32], pv[32];
+        if (cnt > 0) {
+          tmem_ld32(tmem + lrow + T_DV + 32 * h, vv);
+          tmem_ld32(tmem + lrow + T_DK + 32 * h, kv);
+          tmem_ld32(tmem + lrow + T_DP + 32 * h, pv);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) vv[x] = kv[x] = pv[x] = 0.0f;
+        }
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int key = 32 * h + x;
+          if (key < nvalid) {
+            const long long o = base + static_cast<long long>(key) * kDPad;
+            a.dv[o] = vv[x];
+            a.dk[o] = kv[x] * a.scale;
+            a.dphik[o] = pv[x] * inv_sigma;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- reductions
+// grid (64, BH): dH_tot[bh][e][c] and dZ_tot[bh][e] as the tiles' partials summed in tile order.
+__global__ void __launch_bounds__(256) dh_reduce_kernel(const float* __restrict__ dhpart,
+                                                        const float* __restrict__ dzpart, int nq,
+                                                        float* __restrict__ dhtot, float* __restrict__ dztot) {
+  const long long bh = blockIdx.y;
+  const int x = blockIdx.x * 256 + threadIdx.x;  // element of the 128 x 128 block
+  const float* src = dhpart + bh * nq * kDPad * kDPad + x;
+  float t = 0.0f;
+  for (int i = 0; i < nq; ++i) t += src[static_cast<long long>(i) * kDPad * kDPad];
+  dhtot[bh * kDPad * kDPad + x] = t;
+  if (blockIdx.x == 0 && threadIdx.x < kDPad) {
+    const float* zs = dzpart + bh * nq * kDPad + threadIdx.x;
+    float z = 0.0f;
+    for (int i = 0; i < nq; ++i) z += zs[static_cast<long long>(i) * kDPad];
+    dztot[bh * kDPad + threadIdx.x] = z;
+  }
+}
+
+// One warp per (bh, query block): dalpha = its rows' dO . (O_s - O_l), lane-strided then a fixed tree.
+__global__ void __launch_bounds__(256) dalpha_kernel(const float* __restrict__ rows, int N, int nq, long long ntile,
+                                                     float* __restrict__ dalpha) {
+  const long long t = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= ntile) return;
+  const long long bh = t / nq;
+  const int i = static_cast<int>(t % nq);
+  float s = 0.0f;
+  for (int r = lane; r < kRowsT; r += 32) {
+    const int tok = i * kRowsT + r;
+    if (tok < N) s += rows[(bh * N + tok) * 8 + 4];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) dalpha[t] = s;
+}
+
+}  // namespace
+
+BwdTcLayout bwd_tc_layout(const sla_shape& s) {
+  BwdTcLayout L;
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t N = static_cast<size_t>(s.N);
+  const size_t nq = static_cast<size_t>(ceil_div(s.N, s.bq)), nkv = static_cast<size_t>(ceil_div(s.N, s.bkv));
+  L.fwd = ws_layout(s, SLA_MODE_SLA2_TOPK);
+  size_t off = L.fwd.total;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.rows = take(BH * N * 8 * 4);
+  L.phiq = take(BH * N * kDPad * 2);
+  L.inv = take(BH * nkv * nq * 4);
+  L.inv_n = take(BH * nkv * 4);
+  L.dhpart = take(BH * nq * kDPad * kDPad * 4);
+  L.dzpart = take(BH * nq * kDPad * 4);
+  L.dhtot = take(BH * kDPad * kDPad * 4);
+  L.dztot = take(BH * kDPad * 4);
+  L.dphik = take(BH * N * kDPad * 4);
+  L.total = off;
+  return L;
+}
+
+bool bwd_tc_eligible(const sla_shape& s) { return s.in_dtype == SLA_BF16 && s.d == kDPad && s.bq == 128; }
+
+cudaError_t launch_backward_tc(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                               const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
+                               float* dv, float* dalpha, char* ws, cudaStream_t st) {
+  const BwdTcLayout L = bwd_tc_layout(s);
+  const int BH = s.B * s.H;
+  const int nq = ceil_div(s.N, s.bq), nkv = ceil_div(s.N, s.bkv);
+  cudaError_t e;
+  // 1. sla_prepare, then the attention kernel with the statistics epilogue
+  if ((e = launch_prepare(s, k, v, phi, L.fwd, ws, st)) != cudaSuccess) return e;
+  {
+    SparseArgs fa{};
+    static const int32_t kNoBlocks = 0;
+    fa.crit_idx = kept ? kept : &kNoBlocks;
+    fa.negl_idx = nullptr;
+    fa.list_stride = k_keep;
+    fa.crit_max = k_keep;
+    fa.negl_max = 0;
+    fa.counts = nullptr;
+    fa.alpha = alpha;
+    fa.wproj = nullptr;
+    fa.out = nullptr;
+    fa.out_bf16 = 0;
+    fa.bwd_do = dout;
+    fa.bwd_rows = reinterpret_cast<float*>(ws + L.rows);
+    fa.fp8 = 0;
+    fa.wait_ns = kWaitLimitNs;
+    fa.nb128 = ceil_div(s.N, 128);
+    fa.BH = BH;
+    fa.N = s.N;
+    fa.d = s.d;
+    fa.bq = s.bq;
+    fa.nq = nq;
+    fa.nkv = nkv;
+    fa.sl2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s.d)));
+    fa.sigma = reinterpret_cast<const float*>(ws + L.fwd.sigma);
+    fa.zblk = reinterpret_cast<const float*>(ws + L.fwd.zblk);
+    fa.ztot = reinterpret_cast<const float*>(ws + L.fwd.ztot);
+    fa.phi = phi;
+    fa.status = reinterpret_cast<int*>(ws + L.fwd.status);
+    fa.qsrc = q;
+    if ((e = launch_sparse(fa, q, k, ws + L.fwd.phik, ws + L.fwd.v16, ws + L.fwd.hs16, nullptr, nullptr, nullptr,
+                           st)) != cudaSuccess)
+      return e;
+  }
+  const long long rows = static_cast<long long>(BH) * s.N;
+  __half* phiq = reinterpret_cast<__half*>(ws + L.phiq);
+  qphi_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), phiq, rows, phi);
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  int32_t* inv_n = reinterpret_cast<int32_t*>(ws + L.inv_n);
+  if (k_keep > 0) {
+    inv_lists_kernel<<<dim3((nkv + 7) / 8, BH), 256, 0, st>>>(kept, nq, nkv, k_keep, inv, inv_n);
+  } else if ((e = cudaMemsetAsync(inv_n, 0, static_cast<size_t>(BH) * nkv * 4, st)) != cudaSuccess) {
+    return e;
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  CUtensorMap mq, mdo, mk, mv, mpk, mh, mpq;
+  using CU = CUtensorMapDataType;
+  const CU BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if ((e = encode_map(&mq, q, BF, s.N, BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mdo, dout, BF, s.N, BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mk, k, BF, s.N, BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mv, v, BF, s.N, BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mpk, ws + L.fwd.phik, F16, s.N, BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mh, ws + L.fwd.hs16, F16, kDPad, BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mpq, phiq, F16, s.N, BH, 128)) != cudaSuccess) return e;
+
+  TcArgs a{};
+  a.BH = BH;
+  a.N = s.N;
+  a.nq = nq;
+  a.nkv = nkv;
+  a.kk = k_keep;
+  a.phi = phi;
+  a.sl2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s.d)));
+  a.scale = 1.0f / sqrtf(static_cast<float>(s.d));
+  a.kept = kept;
+  a.alpha = alpha;
+  a.rows = reinterpret_cast<const float*>(ws + L.rows);
+  a.sigma = reinterpret_cast<const float*>(ws + L.fwd.sigma);
+  a.ztot = reinterpret_cast<const float*>(ws + L.fwd.ztot);
+  a.inv = inv;
+  a.inv_n = inv_n;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dphik = reinterpret_cast<float*>(ws + L.dphik);
+  a.dhpart = reinterpret_cast<float*>(ws + L.dhpart);
+  a.dzpart = reinterpret_cast<float*>(ws + L.dzpart);
+  a.status = reinterpret_cast<int*>(ws + L.fwd.status);
+  a.wait_ns = kWaitLimitNs;
+
+  // 2. dQ per query tile; dH_i, dZ_i partials
+  if ((e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM)) != cudaSuccess)
+    return e;
+  bwd_dq_kernel<<<static_cast<unsigned>(BH * nq), kTcThreads, dq::SMEM, st>>>(mq, mdo, mk, mv, mpk, mh, mpq, a);
+  // 3. kept shares of dK, dV, dphi(K) per key block
+  if ((e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM)) !=
+      cudaSuccess)
+    return e;
+  bwd_dkv_kernel<<<static_cast<unsigned>(BH * nkv), kTcThreads, dkv::SMEM, st>>>(mq, mdo, mk, mv, mpk, mpq, a);
+  // 4. dH_tot, dZ_tot; dalpha
+  float* dhtot = reinterpret_cast<float*>(ws + L.dhtot);
+  float* dztot = reinterpret_cast<float*>(ws + L.dztot);
+  dh_reduce_kernel<<<dim3(kDPad * kDPad / 256, BH), 256, 0, st>>>(a.dhpart, a.dzpart, nq, dhtot, dztot);
+  const long long ntile = static_cast<long long>(BH) * nq;
+  dalpha_kernel<<<static_cast<unsigned>((ntile * 32 + 255) / 256), 256, 0, st>>>(a.rows, s.N, nq, ntile, dalpha);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 5. the totals' share of every key
+  return launch_bwd_keys(s, k, v, phi, dhtot, dztot, a.dphik, dk, dv, st);
+}
+
+}  // namespace sla

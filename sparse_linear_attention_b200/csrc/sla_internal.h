@@ -58,6 +58,20 @@ struct BwdLayout {
 // Record the one-line detail that sla_last_error_detail() returns.
 void set_error_detail(const char* msg);
 
+// Workspace of the tensor-core backward (bf16, d = 128, b_q = 128): the
+// forward's workspace first (its status word at offset 0), then the per-row
+// statistics, phi(Q), the inverse block lists and the reduction buffers.
+struct BwdTcLayout {
+  WsLayout fwd;
+  size_t rows = 0;            // fp32 [BH * N, 8]: lse2, D, s, dden, dalpha share
+  size_t phiq = 0;            // fp16 [BH, N, 128]
+  size_t inv = 0, inv_n = 0;  // int32 [BH, n_kv, n_q], [BH, n_kv]
+  size_t dhpart = 0, dzpart = 0;  // fp32 [BH * n_q, 128, 128], [BH * n_q, 128]
+  size_t dhtot = 0, dztot = 0;    // fp32 [BH, 128, 128], [BH, 128]
+  size_t dphik = 0;           // fp32 [BH, N, 128]: kept blocks' share of dL/dphi(K)
+  size_t total = 0;
+};
+
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }

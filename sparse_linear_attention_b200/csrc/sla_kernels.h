@@ -24,6 +24,20 @@ cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, co
                             const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
                             float* dv, float* dalpha, char* ws, cudaStream_t st);
 
+// The per-key step of the backward (backward.cu): with dk, dv holding the
+// kept blocks' shares, adds the totals' share: dphi(k) = dphik + dH_tot v +
+// dZ_tot, dv += dH_tot^T phi(k), dk += phi'(k) dphi(k).
+cudaError_t launch_bwd_keys(const sla_shape& s, const void* k, const void* v, int phi, const float* dhtot,
+                            const float* dztot, const float* dphik, float* dk, float* dv, cudaStream_t st);
+
+// The tensor-core SLA2 backward (backward_tc.cu) for bf16 inputs, d = 128,
+// b_q = 128: same arguments as launch_backward, its own workspace layout.
+BwdTcLayout bwd_tc_layout(const sla_shape& s);
+bool bwd_tc_eligible(const sla_shape& s);
+cudaError_t launch_backward_tc(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
+                               const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
+                               float* dv, float* dalpha, char* ws, cudaStream_t st);
+
 // Gradients of the SLA forward (backward.cu): the labels turned into lists,
 // the same three kernels with the SLA weights, then the dW_proj reduction.
 cudaError_t launch_sla_backward(const sla_shape& s, const void* q, const void* k, const void* v, const void* dout,
@@ -72,6 +86,13 @@ struct SparseArgs {
   const float* vamax;        // [BH, 128] column absmax of V
   const void* qsrc;          // bf16 [BH, N, 128] Q (for phi(Q) when the smem tile holds e4m3)
   unsigned long long wait_ns;  // limit of every bounded wait (the exit drains keep their own)
+  // Backward statistics (SLA2, bf16 branch, d = 128; null otherwise): with the
+  // upstream gradient bwd_do (bf16 [BH, N, 128]) the epilogue writes per row
+  // bwd_rows[row * 8 + 0..4] = log2-sum-exp of the scaled kept scores,
+  // D = alpha dO . O_s, s = (1 - alpha) / den, dden = -(1 - alpha) dO . O_l / den
+  // and dO . (O_s - O_l).  out may then be null (no output written).
+  const void* bwd_do;
+  float* bwd_rows;
 };
 
 // 3-D tensor map over a [BH][N][128] 16-bit array: boxes of 64 channels x

@@ -938,6 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // are done) and leave as two 64-channel boxes.
       const bool tma_o = a.tma_out && T.has_lin;
       const long long obase = (static_cast<long long>(T.bh) * a.N + tok) * a.d;
+      float bs = 0.0f, bl = 0.0f;  // backward statistics: dO . O_s, dO . O_l over this half's channels
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int ch0 = 64 * half + 32 * cc;
@@ -957,6 +958,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
         }
         const bool use_s = ok && T.n_crit > 0, use_l = ok && T.has_lin;
+        if constexpr (!kFP8) {
+          if (a.bwd_rows != nullptr && row_valid) {
+            const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(a.bwd_do) + obase + ch0;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              const uint4 w = *reinterpret_cast<const uint4*>(gp + 8 * q8);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 g2 = unpack_bf162(ww[e]);
+                const int c = 8 * q8 + 2 * e;
+                bs = fmaf(g2.x, use_s ? o[c] * inv_l : 0.0f, bs);
+                bs = fmaf(g2.y, use_s ? o[c + 1] * inv_l : 0.0f, bs);
+                bl = fmaf(g2.x, use_l ? nmv[c] * lin_scale : 0.0f, bl);
+                bl = fmaf(g2.y, use_l ? nmv[c + 1] * lin_scale : 0.0f, bl);
+              }
+            }
+          }
+        }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float os = use_s ? o[c] * w_s : 0.0f;
@@ -969,7 +989,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(hbuf + half * 16384u + sw128_off(r, 4 * cc + q8)) =
                 make_uint4(pack_bf162(o[8 * q8], o[8 * q8 + 1]), pack_bf162(o[8 * q8 + 2], o[8 * q8 + 3]),
                            pack_bf162(o[8 * q8 + 4], o[8 * q8 + 5]), pack_bf162(o[8 * q8 + 6], o[8 * q8 + 7]));
-        } else if (ok && row_valid) {
+        } else if (ok && row_valid && a.out != nullptr) {
           if (a.out_bf16) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + obase;
 #pragma unroll
@@ -986,6 +1006,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float4*>(dst + ch0 + 4 * q4) =
                     make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
           }
+        }
+      }
+      if (a.bwd_rows != nullptr) {
+        bs += xchg(bs);
+        bl += xchg(bl);
+        if (half == 0 && row_valid) {
+          const bool lin = T.has_lin && den > 0.0f;
+          float4* rp = reinterpret_cast<float4*>(a.bwd_rows + (static_cast<long long>(T.bh) * a.N + tok) * 8);
+          rp[0] = make_float4((T.n_crit > 0 && l_run > 0.0f) ? m_run + log2f(l_run) : 0.0f, alpha_t * bs,
+                              lin ? (1.0f - alpha_t) / den : 0.0f, lin ? -(1.0f - alpha_t) * bl / den : 0.0f);
+          rp[1] = make_float4(bs - bl, 0.0f, 0.0f, 0.0f);
         }
       }
       if (tma_o) {

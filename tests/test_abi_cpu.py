@@ -220,21 +220,33 @@ def test_backward_rejects_bad_arguments_before_launch():
 
 
 def test_backward_workspace_layout():
-    """Status word, H_tot and Z_tot, their gradients, and the [BH, N, 128] fp32
-    key-side buffer, each rounded up to 256 bytes."""
+    """CUDA-core path: status word, H_tot and Z_tot, their gradients, and the
+    [BH, N, 128] fp32 key-side buffer, each rounded up to 256 bytes.
+    Tensor-core path (bf16, d = 128, b_q = 128): the forward's SLA2 workspace,
+    then the per-row statistics, phi(Q) in fp16, the inverse block lists, the
+    dH / dZ partials per query tile, dH_tot, dZ_tot and the key-side buffer."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    for B, H, N, d in [(1, 12, 32760, 128), (2, 3, 1000, 64), (1, 1, 1, 8), (1, 40, 75600, 128)]:
-        s = _shape(B=B, H=H, N=N, d=d)
+    for B, H, N, d, dt in [(1, 12, 32760, 64, sla.SLA_BF16), (2, 3, 1000, 64, sla.SLA_BF16), (1, 1, 1, 8, sla.SLA_F32),
+                           (1, 40, 75600, 128, sla.SLA_F32)]:
+        s = _shape(B=B, H=H, N=N, d=d, in_dtype=dt)
         BH = B * H
         want = 256 + 2 * (a256(BH * 128 * 128 * 4) + a256(BH * 128 * 4)) + a256(BH * N * 128 * 4)
         assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N, d)
+    for B, H, N in [(1, 12, 32760), (2, 3, 1000), (1, 1, 1), (1, 40, 75600)]:
+        s = _shape(B=B, H=H, N=N, d=128, bq=128, in_dtype=sla.SLA_BF16)
+        BH, nq, nkv = B * H, -(-N // 128), -(-N // 64)
+        want = (sla.sla_workspace_size(s, sla.SLA_MODE_SLA2_TOPK) + a256(BH * N * 32) + a256(BH * N * 256)
+                + a256(BH * nkv * nq * 4) + a256(BH * nkv * 4) + a256(BH * nq * 65536) + a256(BH * nq * 512)
+                + a256(BH * 65536) + a256(BH * 512) + a256(BH * N * 512))
+        assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N)
 
 
 def test_sla_backward_rejects_bad_arguments_before_launch():
     s = _shape()
     L = sla.lib()
     need = sla.sla_attn_bwd_workspace_size(s)
-    assert need > sla.sla2_attn_bwd_workspace_size(s) and need % 256 == 0
+    # the key-side buffer and the O_l rows, both fp32 [BH, N, 128], among the rest
+    assert need >= 2 * 12 * 32760 * 128 * 4 and need % 256 == 0
     assert sla.sla_attn_bwd_workspace_size(_shape(d=100)) == 0
 
     def call(**kw):
@@ -259,7 +271,7 @@ def test_sla_backward_rejects_bad_arguments_before_launch():
 
 
 def test_sla_backward_workspace_layout():
-    """sla2_attn_bwd's workspace, then the critical / negligible lists and
+    """The CUDA-core backward's workspace, then the critical / negligible lists and
     their counts, the [BH, N, 128] fp32 O_l rows and the dW_proj partials of
     about two row splits per SM, each rounded up to 256 bytes."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
@@ -269,8 +281,9 @@ def test_sla_backward_workspace_layout():
         rows = BH * N
         per = max(32, -(-(-(-rows // 296)) // 32) * 32)
         nsplit = -(-rows // per)
-        want = (sla.sla2_attn_bwd_workspace_size(s) + a256(BH * nq * 2 * nkv * 4) + a256(BH * nq * 2 * 4)
-                + a256(rows * 128 * 4) + a256(nsplit * 128 * 128 * 4))
+        fp32_ws = 256 + 2 * (a256(BH * 128 * 128 * 4) + a256(BH * 128 * 4)) + a256(BH * N * 128 * 4)
+        want = (fp32_ws + a256(BH * nq * 2 * nkv * 4) + a256(BH * nq * 2 * 4) + a256(rows * 128 * 4)
+                + a256(nsplit * 128 * 128 * 4))
         assert sla.sla_attn_bwd_workspace_size(s) == want, (B, H, N, d)
 
 
