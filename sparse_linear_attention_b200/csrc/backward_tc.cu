@@ -800,6 +800,206 @@ __global__ void __launch_bounds__(256) dh_reduce_kernel(const float* __restrict_
   }
 }
 
+// One block per head: tau = a power of two with tau max|dH_tot| < 2^14 (1 if dH_tot = 0)
+// and the fp16 copy tau dH_tot for the per-key products.
+__global__ void __launch_bounds__(256) dh_pack_kernel(const float* __restrict__ dhtot, __half* __restrict__ dh16,
+                                                      float* __restrict__ tau) {
+  __shared__ float red[8];
+  const long long bh = blockIdx.x;
+  const float* src = dhtot + bh * kDPad * kDPad;
+  float m = 0.0f;
+  for (int x = threadIdx.x; x < kDPad * kDPad; x += 256) m = fmaxf(m, fabsf(src[x]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0.0f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+  int ex = 0;
+  if (m > 0.0f) frexpf(m, &ex);  // m < 2^ex
+  const float t = m > 0.0f ? ldexpf(1.0f, 14 - ex) : 1.0f;
+  if (threadIdx.x == 0) tau[bh] = t;
+  for (int x = threadIdx.x; x < kDPad * kDPad; x += 256) dh16[bh * kDPad * kDPad + x] = __float2half_rn(src[x] * t);
+}
+
+// ---------------------------------------------------------------- the totals' share per key (tensor cores)
+// One CTA per 128-key tile of a head.  With dH = dH_tot (fp16, times tau):
+//   acc1 = V dH^T   (fp16 V copy x dH K-major)    -> dphi(k) = acc1 / tau + dZ_tot + kept share
+//   acc2 = phi(K) dH (fp16 phi(K) x dH MN-major)  -> dv += acc2 / tau
+// then dk += phi'(k) dphi(k).  Warps 0..3 one key row per thread, warp 4 loads and issues.
+namespace kt {
+constexpr uint32_t OFF_V = 0, OFF_PK = 32768, OFF_H = 65536, OFF_BAR = 98304, OFF_MISC = OFF_BAR + 64;
+constexpr uint32_t SMEM = OFF_MISC + 64;
+constexpr int kThreads = 160;
+enum { B_LD = 0, B_MMA = 1, NBAR = 2 };
+}  // namespace kt
+
+__global__ void __launch_bounds__(kt::kThreads)
+    bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmPK,
+                       const __grid_constant__ CUtensorMap tmH, const __nv_bfloat16* __restrict__ k, int N, int ntile,
+                       int phi, const float* __restrict__ tau, const float* __restrict__ dztot,
+                       const float* __restrict__ dphik, float* __restrict__ dk, float* __restrict__ dv, int* status,
+                       unsigned long long wait_ns) {
+  using namespace kt;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(status, SLA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = blockIdx.x % ntile;
+  const int bh = blockIdx.x / ntile;
+  if (tid == 0) {
+    mbar_init(&bars[B_LD], 1);
+    mbar_init(&bars[B_MMA], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[B_LD], 98304);
+      tma_load_3d(sm + OFF_V, &tmV16, &bars[B_LD], 0, t * 128, bh);
+      tma_load_3d(sm + OFF_V + 16384, &tmV16, &bars[B_LD], 64, t * 128, bh);
+      tma_load_3d(sm + OFF_PK, &tmPK, &bars[B_LD], 0, t * 128, bh);
+      tma_load_3d(sm + OFF_PK + 16384, &tmPK, &bars[B_LD], 64, t * 128, bh);
+      tma_load_3d(sm + OFF_H, &tmH, &bars[B_LD], 0, 0, bh);
+      tma_load_3d(sm + OFF_H + 16384, &tmH, &bars[B_LD], 64, 0, bh);
+      if (mbar_wait(&bars[B_LD], 0, abort_flag, status, wait_ns)) {
+        tc_fence_after();
+        const uint32_t id1 = idesc_f16(0, 0, 0, 128, 128);
+        const uint32_t id2 = idesc_f16(0, 0, 1, 128, 128);
+        const uint64_t dVd = sdesc_sw128(smem_u32(sm + OFF_V), 16, 1024);
+        const uint64_t dPd = sdesc_sw128(smem_u32(sm + OFF_PK), 16, 1024);
+        const uint64_t dHk = sdesc_sw128(smem_u32(sm + OFF_H), 16, 1024);
+        const uint64_t dHm = sdesc_sw128(smem_u32(sm + OFF_H), 16384, 1024);
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t o = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem, dVd + o, dHk + o, id1, k8 > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + 128, dPd + o, dHm + k8 * 128u, id2, k8 > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[B_MMA]);
+      } else {
+        mbar_wait_drain(&bars[B_LD], 0);
+      }
+    }
+  } else {
+    const int r = tid, tok = t * 128 + r;
+    const bool valid = tok < N;
+    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
+    const bool ok = warp_wait_tc(&bars[B_MMA], 0, abort_flag, status, wait_ns);
+    if (ok) {
+      tc_fence_after();
+      const float it = 1.0f / tau[bh];  // exact: a power of two
+      const float* zt = dztot + static_cast<long long>(bh) * kDPad;
+      const long long row = static_cast<long long>(bh) * N + (valid ? tok : 0);
+      const __nv_bfloat16* kr = k + row * kDPad;
+      const float* pk = dphik + row * kDPad;
+      auto k32 = [&](int cc, float* x) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(kr + 32 * cc + 8 * u);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf162(ww[e]);
+            x[8 * u + 2 * e] = f.x;
+            x[8 * u + 2 * e + 1] = f.y;
+          }
+        }
+      };
+      auto dphi32 = [&](int cc, float* g) {
+        float a1[32];
+        tmem_ld32(tmem + lrow + 32 * cc, a1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) g[c] = a1[c] * it + zt[32 * cc + c] + pk[32 * cc + c];
+      };
+      const bool smx = phi == SLA_PHI_SOFTMAX;
+      float mx = -INFINITY, inv_sum = 0.0f, dot = 0.0f;
+      // warp-uniform: dphi32 reads TMEM with a warp-collective load (rows past N
+      // read row 0 of the head and store nothing)
+      if (smx) {
+        float x[32];
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          k32(cc, x);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, x[c]);
+        }
+        float sum = 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          k32(cc, x);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sum += expf(x[c] - mx);
+        }
+        inv_sum = 1.0f / sum;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float g[32];
+          k32(cc, x);
+          dphi32(cc, g);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) dot = fmaf(expf(x[c] - mx) * inv_sum, g[c], dot);
+        }
+      }
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float g[32], x[32], a2[32];
+        dphi32(cc, g);
+        tmem_ld32(tmem + lrow + 128 + 32 * cc, a2);
+        tmem_wait_ld();
+        if (valid) {
+          k32(cc, x);
+          float* dkr = dk + row * kDPad + 32 * cc;
+          float* dvr = dv + row * kDPad + 32 * cc;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            float4 kk4 = *reinterpret_cast<float4*>(dkr + c);
+            float4 vv4 = *reinterpret_cast<float4*>(dvr + c);
+            float o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float xe = x[c + e], ge = g[c + e];
+              o[e] = smx ? expf(xe - mx) * inv_sum * (ge - dot) : ge * (xe > 0.0f ? 1.0f : expf(xe));
+            }
+            kk4.x += o[0];
+            kk4.y += o[1];
+            kk4.z += o[2];
+            kk4.w += o[3];
+            vv4.x += a2[c] * it;
+            vv4.y += a2[c + 1] * it;
+            vv4.z += a2[c + 2] * it;
+            vv4.w += a2[c + 3] * it;
+            *reinterpret_cast<float4*>(dkr + c) = kk4;
+            *reinterpret_cast<float4*>(dvr + c) = vv4;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // One warp per (bh, query block): dalpha = its rows' dO . (O_s - O_l), lane-strided then a fixed tree.
 __global__ void __launch_bounds__(256) dalpha_kernel(const float* __restrict__ rows, int N, int nq, long long ntile,
                                                      float* __restrict__ dalpha) {
@@ -841,6 +1041,8 @@ BwdTcLayout bwd_tc_layout(const sla_shape& s) {
   L.dhtot = take(BH * kDPad * kDPad * 4);
   L.dztot = take(BH * kDPad * 4);
   L.dphik = take(BH * N * kDPad * 4);
+  L.dh16 = take(BH * kDPad * kDPad * 2);
+  L.tau = take(BH * 4);
   L.total = off;
   return L;
 }
@@ -956,9 +1158,23 @@ cudaError_t launch_backward_tc(const sla_shape& s, const void* q, const void* k,
   dh_reduce_kernel<<<dim3(kDPad * kDPad / 256, BH), 256, 0, st>>>(a.dhpart, a.dzpart, nq, dhtot, dztot);
   const long long ntile = static_cast<long long>(BH) * nq;
   dalpha_kernel<<<static_cast<unsigned>((ntile * 32 + 255) / 256), 256, 0, st>>>(a.rows, s.N, nq, ntile, dalpha);
+  // 5. the totals' share of every key, on the tensor cores
+  __half* dh16 = reinterpret_cast<__half*>(ws + L.dh16);
+  float* tau = reinterpret_cast<float*>(ws + L.tau);
+  dh_pack_kernel<<<BH, 256, 0, st>>>(dhtot, dh16, tau);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // 5. the totals' share of every key
-  return launch_bwd_keys(s, k, v, phi, dhtot, dztot, a.dphik, dk, dv, st);
+  CUtensorMap mv16, mpk128, mdh;
+  if ((e = encode_map(&mv16, ws + L.fwd.v16, F16, s.N, BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mpk128, ws + L.fwd.phik, F16, s.N, BH, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mdh, dh16, F16, kDPad, BH, 128)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bwd_keys_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kt::SMEM)) !=
+      cudaSuccess)
+    return e;
+  const int ntk = ceil_div(s.N, 128);
+  bwd_keys_tc_kernel<<<static_cast<unsigned>(BH * ntk), kt::kThreads, kt::SMEM, st>>>(
+      mv16, mpk128, mdh, static_cast<const __nv_bfloat16*>(k), s.N, ntk, phi, tau, dztot, a.dphik, dk, dv, a.status,
+      kWaitLimitNs);
+  return cudaGetLastError();
 }
 
 }  // namespace sla

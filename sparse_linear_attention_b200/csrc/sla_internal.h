@@ -69,6 +69,7 @@ struct BwdTcLayout {
   size_t dhpart = 0, dzpart = 0;  // fp32 [BH * n_q, 128, 128], [BH * n_q, 128]
   size_t dhtot = 0, dztot = 0;    // fp32 [BH, 128, 128], [BH, 128]
   size_t dphik = 0;           // fp32 [BH, N, 128]: kept blocks' share of dL/dphi(K)
+  size_t dh16 = 0, tau = 0;   // fp16 [BH, 128, 128] = tau dH_tot; fp32 [BH] power-of-two scale tau
   size_t total = 0;
 };
 
