@@ -363,20 +363,26 @@ def backward_leg(args, w, dev, stream):
                          f"{w.B * w.H * w.n_q} ({t_cpu:.2f} s), extrapolated per block"}
     _, peak, _, src = peaks()
     achieved = flops / (ms * 1e-3) / 1e12
+    # the SLA2 backward of bf16 inputs at d = 128, b_q = 128 runs on the tensor cores:
+    # prepare (3), the attention kernel with its statistics epilogue, phi(Q), the
+    # inverse lists, dQ, dK/dV, the dH reduction, dalpha, the dH packing, the per-key step
+    tc_path = (not sla_mode) and w.dtype == "bf16" and w.d == 128 and w.bq == 128
+    launches = 6 if sla_mode else (12 if tc_path else 3)
     metric = ("SLA backward ms @Wan-1.3B shape (sla_attn_bwd: dQ, dK, dV, dW_proj)" if sla_mode else
               "SLA2 backward ms @Wan-1.3B shape (sla2_attn_bwd: dQ, dK, dV, dalpha)")
     keep_txt = f"critical={k} negligible={k_neg}/{w.n_kv}" if sla_mode else f"keep={k}/{w.n_kv}"
     print(json.dumps({
         "metric": metric, "value": ms,
         "unit": "ms per call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "higher_is_better": False, "dtype": "f32", "data": "synthetic",
+        "higher_is_better": False, "dtype": "bf16" if tc_path else "f32", "data": "synthetic",
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} bq={w.bq} bkv={w.bkv} "
                                f"{keep_txt} key blocks, phi={args.phi}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense (burst)",
                      "algorithmic": "10*d FLOP per (query row, kept valid key): the sparse branch's "
-                                    "FlashAttention-style backward; kernels are fp32 on the CUDA cores"},
-        "gpu_launches": (6 if sla_mode else 3) * args.steps, "clocks": clk, "cpu_baseline": cpu,
+                                    "FlashAttention-style backward",
+                     "path": "tensor cores (tcgen05)" if tc_path else "fp32 CUDA cores"},
+        "gpu_launches": launches * args.steps, "clocks": clk, "cpu_baseline": cpu,
     }), flush=True)
 
 
