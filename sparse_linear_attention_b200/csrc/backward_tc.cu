@@ -46,7 +46,14 @@ namespace sla {
 
 namespace {
 
-constexpr int kTcThreads = 192;  // warps 0..3: one row (or channel) per thread; warp 4 TMA; warp 5 MMA
+// Warps 0..15 work on the 128 rows (or channels) of a tile: warp w takes the
+// 32 rows of its TMEM lane quarter w % 4 and column group w / 4 (16 keys of a
+// key block, 32 channels in the epilogues), so four warps share each SM
+// sub-partition and hide each other's latencies.  Warp 16 issues the TMA
+// copies, warp 17 the tensor-core products.
+constexpr int kCompute = 512;
+constexpr int kTcThreads = kCompute + 64;
+constexpr int kProdWarp = 16, kMmaWarp = 17;
 constexpr int kRowsT = 128;      // query rows per tile
 
 struct TcArgs {
@@ -169,7 +176,8 @@ constexpr uint32_t OFF_OPS = OFF_ST + 2 * STAGE;  // dS bf16 [128][64] | -Bx sig
 constexpr uint32_t OFF_BAR = OFF_OPS + 32768;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t OFF_DD = OFF_MISC + 64;  // dden per row [128] floats
-constexpr uint32_t SMEM = OFF_DD + 512;
+constexpr uint32_t OFF_RED = OFF_DD + 512;  // softmax feature map: [3][4 groups][128 rows] floats
+constexpr uint32_t SMEM = OFF_RED + 6144;
 static_assert(SMEM <= 232448, "shared memory budget");
 // TMEM columns: S_b at 128 b, G_b at 128 b + 64 (b = 0, 1); dQ_s 256; dQ_l 384.
 // End phase: s dO H_tot^T at 0, sigma dH_i at 128.
@@ -206,19 +214,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&bars[B_STF + s], 1);
       mbar_init(&bars[B_STE + s], 1);
       mbar_init(&bars[B_SGF + s], 1);
-      mbar_init(&bars[B_SGE + s], kRowsT);
+      mbar_init(&bars[B_SGE + s], kCompute);
     }
-    mbar_init(&bars[B_OPF], kRowsT);
+    mbar_init(&bars[B_OPF], kCompute);
     mbar_init(&bars[B_OPE], 1);
     mbar_init(&bars[B_LOOP], 1);
     mbar_init(&bars[B_ENDL], 1);
-    mbar_init(&bars[B_SDO], kRowsT);
+    mbar_init(&bars[B_SDO], kCompute);
     mbar_init(&bars[B_END], 1);
     mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -229,7 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const float sigma = a.sigma[bh];
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int g = issued > 2 ? issued - 2 : 0; g < issued; ++g) mbar_wait_drain(&bars[B_STF + (g & 1)], (g >> 1) & 1);
       if (end_issued) mbar_wait_drain(&bars[B_ENDL], 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);    // Q x K_j^T, dO x V_j^T (bf16, K-major)
@@ -354,9 +362,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait_drain(&bars[B_DRAIN], 0);
     }
   } else {
-    // ------------------------------------------------------------ rows (warps 0..3)
-    const int r = tid;  // tile row = TMEM lane
-    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------------------------ rows (warps 0..15)
+    const int q4 = warp & 3, g = warp >> 2;
+    const int r = q4 * 32 + lane;  // tile row = TMEM lane
+    const uint32_t lrow = static_cast<uint32_t>(q4 * 32) << 16;
     const int tok = qb * kRowsT + r;
     const bool valid = tok < a.N;
     float lse2 = 0.0f, D = 0.0f, sr = 0.0f, dd = 0.0f;
@@ -379,66 +388,61 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       const int j = clamp_block(lst[n], a.nkv, a.status, false);
       const int nvalid = (tail && j == a.nkv - 1) ? a.N - j * kBlockKV : kBlockKV;
-      uint32_t pS[32], pB[32];
+      float sv[16], gv[16];
+      tmem_ld16(tmem + lrow + 128 * b + 16 * g, sv);
+      tmem_ld16(tmem + lrow + 128 * b + 64 + 16 * g, gv);
+      tmem_wait_ld();
+      uint32_t pS[8], pB[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float sv[32], gv[32];
-        tmem_ld32(tmem + lrow + 128 * b + 32 * h, sv);
-        tmem_ld32(tmem + lrow + 128 * b + 64 + 32 * h, gv);
-        tmem_wait_ld();
+      for (int c = 0; c < 16; c += 2) {
+        float ds[2], bx[2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float ds[2], bx[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool kv = valid && (32 * h + c + e < nvalid);
-            const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
-            ds[e] = p * fmaf(alpha, gv[c + e], -D);
-            bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
-          }
-          pS[16 * h + c / 2] = pack_bf162(ds[0], ds[1]);
-          pB[16 * h + c / 2] = pack_half2(bx[0], bx[1]);
+        for (int e = 0; e < 2; ++e) {
+          const bool kv = valid && (16 * g + c + e < nvalid);
+          const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
+          ds[e] = p * fmaf(alpha, gv[c + e], -D);
+          bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
         }
+        pS[c / 2] = pack_bf162(ds[0], ds[1]);
+        pB[c / 2] = pack_half2(bx[0], bx[1]);
       }
       tc_fence_before();
       mbar_arrive(&bars[B_SGE + b]);
       ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
       if (!ok) break;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        put_unit(opS, r, u, pS[4 * u], pS[4 * u + 1], pS[4 * u + 2], pS[4 * u + 3]);
-        put_unit(opB, r, u, pB[4 * u], pB[4 * u + 1], pB[4 * u + 2], pB[4 * u + 3]);
-      }
+      put_unit(opS, r, 2 * g, pS[0], pS[1], pS[2], pS[3]);
+      put_unit(opS, r, 2 * g + 1, pS[4], pS[5], pS[6], pS[7]);
+      put_unit(opB, r, 2 * g, pB[0], pB[1], pB[2], pB[3]);
+      put_unit(opB, r, 2 * g + 1, pB[4], pB[5], pB[6], pB[7]);
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_OPF]);
     }
-    // s sigma dO (fp16) over the operand tiles once the loop's products are done
+    // s sigma dO (fp16, channels 32 g ..) over the operand tiles once the loop's products are done
     ok = ok && warp_wait_tc(&bars[B_LOOP], 0, abort_flag, a.status, a.wait_ns);
     if (ok) {
       const float f = sr * sigma;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int u = (g & 1) * 4 + u4;
+        const uint32_t ch = static_cast<uint32_t>(g >> 1) * 16384u;
+        const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_DO + ch + sw128_off(r, u));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o4[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_DO + ch * 16384u + sw128_off(r, u));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-          uint32_t o4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 g = unpack_bf162(ww[e]);
-            o4[e] = pack_half2(g.x * f, g.y * f);
-          }
-          put_unit(sm + OFF_OPS + ch * 16384u, r, u, o4[0], o4[1], o4[2], o4[3]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 gg = unpack_bf162(ww[e]);
+          o4[e] = pack_half2(gg.x * f, gg.y * f);
         }
+        put_unit(sm + OFF_OPS + ch, r, u, o4[0], o4[1], o4[2], o4[3]);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_SDO]);
     }
-    ddsh[r] = dd;
-    named_bar_sync(1, kRowsT);
+    if (g == 0) ddsh[r] = dd;
+    named_bar_sync(1, kCompute);
     // dZ_i[e] = sum over the rows of phi(Q)[row][e] dden[row], e = r (phi(Q) tile in smem)
     ok = ok && warp_wait_tc(&bars[B_ENDL], 0, abort_flag, a.status, a.wait_ns);
-    if (ok) {
+    if (ok && g == 0) {
       const int e = r, ch = e >> 6, u = (e & 63) >> 3, w = e & 7;
       float z = 0.0f;
       for (int rr = 0; rr < kRowsT; ++rr) {
@@ -449,101 +453,112 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       a.dzpart[tile * kDPad + e] = z;
     }
     ok = ok && warp_wait_tc(&bars[B_END], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) tc_fence_after();
+    const float inv_sigma = 1.0f / sigma;  // exact: a power of two
     if (ok) {
-      tc_fence_after();
-      const float inv_sigma = 1.0f / sigma;  // exact: a power of two
-      // sigma dH_i: lane e, 128 columns c
-      float* dh = a.dhpart + (tile * kDPad + r) * kDPad;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        float hv[32];
-        tmem_ld32(tmem + lrow + T_DH + 32 * cc, hv);
-        tmem_wait_ld();
+      // sigma dH_i: lane e = r, columns c = 32 g ..
+      float* dh = a.dhpart + (tile * kDPad + r) * kDPad + 32 * g;
+      float hv[32];
+      tmem_ld32(tmem + lrow + T_DH + 32 * g, hv);
+      tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          *reinterpret_cast<float4*>(dh + 32 * cc + c) =
-              make_float4(hv[c] * inv_sigma, hv[c + 1] * inv_sigma, hv[c + 2] * inv_sigma, hv[c + 3] * inv_sigma);
-      }
-      // dQ of row r: scale dQ_s + phi'(Q) (dQ_l / sigma + s dO H_tot^T + dden Z_tot)
-      const float* zt = a.ztot + static_cast<long long>(bh) * kDPad;
-      const bool have = kk > 0;
-      // 32 channels of Q row r from the smem tile
-      auto q32 = [&](int cc, float* x) {
+      for (int c = 0; c < 32; c += 4)
+        *reinterpret_cast<float4*>(dh + c) =
+            make_float4(hv[c] * inv_sigma, hv[c + 1] * inv_sigma, hv[c + 2] * inv_sigma, hv[c + 3] * inv_sigma);
+    }
+    // dQ of row r, channels 32 g + 16 h ..: scale dQ_s + phi'(Q) (dQ_l / sigma + s dO H_tot^T + dden Z_tot)
+    const float* zt = a.ztot + static_cast<long long>(bh) * kDPad;
+    const bool have = kk > 0;
+    auto q16 = [&](int h, float* x) {  // 16 channels of Q row r from the smem tile
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_Q + (cc >> 1) * 16384u +
-                                                          sw128_off(r, (cc & 1) * 4 + u4));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      for (int u2 = 0; u2 < 2; ++u2) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sm + OFF_Q + (g >> 1) * 16384u +
+                                                        sw128_off(r, (g & 1) * 4 + 2 * h + u2));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf162(ww[e]);
-            x[8 * u4 + 2 * e] = f.x;
-            x[8 * u4 + 2 * e + 1] = f.y;
-          }
-        }
-      };
-      // the gradient reaching phi(Q) for 32 channels
-      auto gphi = [&](int cc, float* g) {
-        float l[32], h[32];
-        tmem_ld32(tmem + lrow + T_DQL + 32 * cc, l);
-        tmem_ld32(tmem + lrow + T_HT + 32 * cc, h);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) g[c] = (have ? l[c] * inv_sigma : 0.0f) + h[c] + dd * zt[32 * cc + c];
-      };
-      // the softmax feature map: phi'(q) g = phi (g - sum_c phi_c g_c), phi from the row max and sum
-      const bool smx = a.phi == SLA_PHI_SOFTMAX;
-      float mx = -INFINITY, inv_sum = 0.0f, dot = 0.0f;
-      if (smx) {
-        float x[32];
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          q32(cc, x);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, x[c]);
-        }
-        float sum = 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          q32(cc, x);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sum += expf(x[c] - mx);
-        }
-        inv_sum = 1.0f / sum;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float g[32];
-          q32(cc, x);
-          gphi(cc, g);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) dot = fmaf(expf(x[c] - mx) * inv_sum, g[c], dot);
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf162(ww[e]);
+          x[8 * u2 + 2 * e] = f.x;
+          x[8 * u2 + 2 * e + 1] = f.y;
         }
       }
-      float* dqr = a.dq + (static_cast<long long>(bh) * a.N + tok) * kDPad;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        float g[32], sq[32], x[32];
-        q32(cc, x);
-        gphi(cc, g);
-        tmem_ld32(tmem + lrow + T_DQS + 32 * cc, sq);
-        tmem_wait_ld();
-        float o[32];
+    };
+    auto gphi16 = [&](int h, float* gp) {  // the gradient reaching phi(Q), 16 channels
+      float l[16], hh[16];
+      tmem_ld16(tmem + lrow + T_DQL + 32 * g + 16 * h, l);
+      tmem_ld16(tmem + lrow + T_HT + 32 * g + 16 * h, hh);
+      tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float dphi = smx ? expf(x[c] - mx) * inv_sum * (g[c] - dot) : g[c] * (x[c] > 0.0f ? 1.0f : expf(x[c]));
+      for (int c = 0; c < 16; ++c) gp[c] = (have ? l[c] * inv_sigma : 0.0f) + hh[c] + dd * zt[32 * g + 16 * h + c];
+    };
+    // the softmax feature map: phi'(q) gp = phi (gp - sum_c phi_c gp_c); the row's
+    // max, sum and dot are combined over the four column groups in smem
+    const bool smx = a.phi == SLA_PHI_SOFTMAX;
+    float mx = -INFINITY, inv_sum = 0.0f, dot = 0.0f;
+    if (smx) {
+      float* red = reinterpret_cast<float*>(sm + OFF_RED);
+      float x[16];
+      float pm = -INFINITY;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        q16(h, x);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pm = fmaxf(pm, x[c]);
+      }
+      red[g * 128 + r] = pm;
+      named_bar_sync(1, kCompute);
+      mx = fmaxf(fmaxf(red[r], red[128 + r]), fmaxf(red[256 + r], red[384 + r]));
+      float ps = 0.0f;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        q16(h, x);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) ps += expf(x[c] - mx);
+      }
+      red[512 + g * 128 + r] = ps;
+      named_bar_sync(1, kCompute);
+      inv_sum = 1.0f / ((red[512 + r] + red[640 + r]) + (red[768 + r] + red[896 + r]));
+      float pd = 0.0f;
+      if (ok) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float gp[16];
+          q16(h, x);
+          gphi16(h, gp);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pd = fmaf(expf(x[c] - mx) * inv_sum, gp[c], pd);
+        }
+      }
+      red[1024 + g * 128 + r] = pd;
+      named_bar_sync(1, kCompute);
+      dot = (red[1024 + r] + red[1152 + r]) + (red[1280 + r] + red[1408 + r]);
+    }
+    if (ok) {
+      float* dqr = a.dq + (static_cast<long long>(bh) * a.N + tok) * kDPad + 32 * g;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float gp[16], sq[16], x[16];
+        q16(h, x);
+        gphi16(h, gp);
+        tmem_ld16(tmem + lrow + T_DQS + 32 * g + 16 * h, sq);
+        tmem_wait_ld();
+        float o[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float dphi = smx ? expf(x[c] - mx) * inv_sum * (gp[c] - dot) : gp[c] * (x[c] > 0.0f ? 1.0f : expf(x[c]));
           o[c] = (have ? sq[c] * a.scale : 0.0f) + dphi;
         }
         if (valid) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(dqr + 32 * cc + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          for (int c = 0; c < 16; c += 4)
+            *reinterpret_cast<float4*>(dqr + 16 * h + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -588,11 +603,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int32_t* il = a.inv + kb * a.nq;
 
   if (tid == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == B_OPF) ? kRowsT : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == B_OPF) ? kCompute : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -603,7 +618,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const float sigma = a.sigma[bh];
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     if (lane == 0 && cnt > 0) {
       int issued = 0;
       mbar_arrive_expect_tx(&bars[B_KV], 49152);
@@ -630,7 +645,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait_drain(&bars[B_KV], 0);
       if (issued > 0) mbar_wait_drain(&bars[B_STF], (issued - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);   // Q_i K_j^T, dO_i V_j^T (bf16)
       const uint32_t id_a = idesc_f16(0, 0, 0, 128, 64);   // phi(Q_i) phi(K_j)^T (f16)
@@ -678,8 +693,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait_drain(&bars[B_DRAIN], 0);
     }
   } else {
-    const int r = tid;
-    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
+    // warp w: rows (epilogue: channels) 32 (w % 4) .., keys 16 (w / 4) .. of the block
+    const int q4 = warp & 3, g = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const uint32_t lrow = static_cast<uint32_t>(q4 * 32) << 16;
     const bool tail = (a.N & (kBlockKV - 1)) != 0;
     const int nvalid = (tail && j == a.nkv - 1) ? a.N - j * kBlockKV : kBlockKV;
     bool ok = true;
@@ -706,76 +723,69 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float sv[32], gv[32], av[32];
-        tmem_ld32(tmem + lrow + T_S + 32 * h, sv);
-        tmem_ld32(tmem + lrow + T_G + 32 * h, gv);
-        tmem_ld32(tmem + lrow + T_A + 32 * h, av);
-        tmem_wait_ld();
-        uint32_t pS[16], pC[16], pB[16];
+      float sv[16], gv[16], av[16];
+      tmem_ld16(tmem + lrow + T_S + 16 * g, sv);
+      tmem_ld16(tmem + lrow + T_G + 16 * g, gv);
+      tmem_ld16(tmem + lrow + T_A + 16 * g, av);
+      tmem_wait_ld();
+      uint32_t pS[8], pC[8], pB[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float ds[2], cv[2], bx[2];
+      for (int c = 0; c < 16; c += 2) {
+        float ds[2], cv[2], bx[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool kv = valid && (32 * h + c + e < nvalid);
-            const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
-            ds[e] = p * fmaf(alpha, gv[c + e], -D);
-            cv[e] = kv ? fmaf(alpha, p, -sr * av[c + e]) : 0.0f;
-            bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
-          }
-          pS[c / 2] = pack_bf162(ds[0], ds[1]);
-          pC[c / 2] = pack_bf162(cv[0], cv[1]);
-          pB[c / 2] = pack_half2(bx[0], bx[1]);
+        for (int e = 0; e < 2; ++e) {
+          const bool kv = valid && (16 * g + c + e < nvalid);
+          const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
+          ds[e] = p * fmaf(alpha, gv[c + e], -D);
+          cv[e] = kv ? fmaf(alpha, p, -sr * av[c + e]) : 0.0f;
+          bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
         }
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const int u = 4 * h + u4;
-          put_unit(opS, r, u, pS[4 * u4], pS[4 * u4 + 1], pS[4 * u4 + 2], pS[4 * u4 + 3]);
-          put_unit(opC, r, u, pC[4 * u4], pC[4 * u4 + 1], pC[4 * u4 + 2], pC[4 * u4 + 3]);
-          put_unit(opB, r, u, pB[4 * u4], pB[4 * u4 + 1], pB[4 * u4 + 2], pB[4 * u4 + 3]);
-        }
+        pS[c / 2] = pack_bf162(ds[0], ds[1]);
+        pC[c / 2] = pack_bf162(cv[0], cv[1]);
+        pB[c / 2] = pack_half2(bx[0], bx[1]);
       }
+      put_unit(opS, r, 2 * g, pS[0], pS[1], pS[2], pS[3]);
+      put_unit(opS, r, 2 * g + 1, pS[4], pS[5], pS[6], pS[7]);
+      put_unit(opC, r, 2 * g, pC[0], pC[1], pC[2], pC[3]);
+      put_unit(opC, r, 2 * g + 1, pC[4], pC[5], pC[6], pC[7]);
+      put_unit(opB, r, 2 * g, pB[0], pB[1], pB[2], pB[3]);
+      put_unit(opB, r, 2 * g + 1, pB[4], pB[5], pB[6], pB[7]);
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_OPF]);
     }
-    // epilogue: lane = channel c; columns = the block's 64 keys
+    // epilogue: lane = channel c; keys 16 g .. of the block
     if (cnt > 0) ok = ok && warp_wait_tc(&bars[B_DONE], 0, abort_flag, a.status, a.wait_ns);
     if (ok) {
       tc_fence_after();
       const int c = r;
       const float inv_sigma = 1.0f / sigma;
       const long long base = (static_cast<long long>(bh) * a.N + static_cast<long long>(j) * kBlockKV) * kDPad + c;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float vv[32], kv[32], pv[32];
-        if (cnt > 0) {
-          tmem_ld32(tmem + lrow + T_DV + 32 * h, vv);
-          tmem_ld32(tmem + lrow + T_DK + 32 * h, kv);
-          tmem_ld32(tmem + lrow + T_DP + 32 * h, pv);
-          tmem_wait_ld();
-        } else {
+      float vv[16], kv[16], pv[16];
+      if (cnt > 0) {
+        tmem_ld16(tmem + lrow + T_DV + 16 * g, vv);
+        tmem_ld16(tmem + lrow + T_DK + 16 * g, kv);
+        tmem_ld16(tmem + lrow + T_DP + 16 * g, pv);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) vv[x] = kv[x] = pv[x] = 0.0f;
-        }
+        for (int x = 0; x < 16; ++x) vv[x] = kv[x] = pv[x] = 0.0f;
+      }
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int key = 32 * h + x;
-          if (key < nvalid) {
-            const long long o = base + static_cast<long long>(key) * kDPad;
-            a.dv[o] = vv[x];
-            a.dk[o] = kv[x] * a.scale;
-            a.dphik[o] = pv[x] * inv_sigma;
-          }
+      for (int x = 0; x < 16; ++x) {
+        const int key = 16 * g + x;
+        if (key < nvalid) {
+          const long long o = base + static_cast<long long>(key) * kDPad;
+          a.dv[o] = vv[x];
+          a.dk[o] = kv[x] * a.scale;
+          a.dphik[o] = pv[x] * inv_sigma;
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
