@@ -178,8 +178,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // kLow: 0 = bf16 sparse branch; 1 = e4m3 Q, K', P, V; 2 = INT8 Q, K' (S as an
-// exact integer product, kind::i8) with e4m3 P, V.
-template <int kLow>
+// exact integer product, kind::i8) with e4m3 P, V.  kStats: the backward's
+// per-row statistics epilogue (SparseArgs::bwd_rows; bf16 branch only).
+template <int kLow, bool kStats>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmV,
@@ -958,8 +959,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             o[c] *= __fdiv_rn(va[c] > 0.0f ? __fdiv_rn(va[c], 448.0f) : __fdiv_rn(1.0f, 448.0f), 448.0f);
         }
         const bool use_s = ok && T.n_crit > 0, use_l = ok && T.has_lin;
-        if constexpr (!kFP8) {
-          if (a.bwd_rows != nullptr && row_valid) {
+        if constexpr (kStats && !kFP8) {
+          if (row_valid) {
             const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(a.bwd_do) + obase + ch0;
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
@@ -989,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(hbuf + half * 16384u + sw128_off(r, 4 * cc + q8)) =
                 make_uint4(pack_bf162(o[8 * q8], o[8 * q8 + 1]), pack_bf162(o[8 * q8 + 2], o[8 * q8 + 3]),
                            pack_bf162(o[8 * q8 + 4], o[8 * q8 + 5]), pack_bf162(o[8 * q8 + 6], o[8 * q8 + 7]));
-        } else if (ok && row_valid && a.out != nullptr) {
+        } else if (ok && row_valid && (!kStats || a.out != nullptr)) {
           if (a.out_bf16) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + obase;
 #pragma unroll
@@ -1008,7 +1009,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (a.bwd_rows != nullptr) {
+      if constexpr (kStats) {
         bs += xchg(bs);
         bl += xchg(bl);
         if (half == 0 && row_valid) {
@@ -1044,18 +1045,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int kLow>
+template <int kLow, bool kStats = false>
 static cudaError_t launch_sparse_t(const SparseArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
                                    const CUtensorMap& mp, const CUtensorMap& mv, const CUtensorMap& mh,
                                    const CUtensorMap& mv8, const CUtensorMap& mo, cudaStream_t st) {
   constexpr uint32_t smem = Lay<kLow != 0>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(sparse_fwd_kernel<kLow>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(sparse_fwd_kernel<kLow, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long ntiles = static_cast<long long>(a.BH) * a.nq;
   const unsigned grid = static_cast<unsigned>(ntiles < sms ? ntiles : sms);
-  sparse_fwd_kernel<kLow><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, mo, a);
+  sparse_fwd_kernel<kLow, kStats><<<grid, kThreads, smem, st>>>(mq, mk, mp, mv, mh, mv8, mo, a);
   return cudaGetLastError();
 }
 
@@ -1084,6 +1086,7 @@ cudaError_t launch_sparse(const SparseArgs& a_in, const void* q_bf16_128, const 
   }
   if ((e = encode_map(&mq, q_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 128)) != cudaSuccess) return e;
   if ((e = encode_map(&mk, k_bf16_128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.BH, 64)) != cudaSuccess) return e;
+  if (a.bwd_rows != nullptr) return launch_sparse_t<0, true>(a, mq, mk, mp, mv, mh, mv, mo, st);
   return launch_sparse_t<0>(a, mq, mk, mp, mv, mh, mv, mo, st);
 }
 
