@@ -234,8 +234,12 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k,
                         void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace sla2_attn_bwd needs for this shape (0 for an
- * invalid shape): the status word, H_tot, Z_tot and their gradients per
- * (b,h), and a [B,H,N,128] fp32 buffer of key-side sums. */
+ * invalid shape).  CUDA-core path: the status word, H_tot, Z_tot and their
+ * gradients per (b,h), and a [B,H,N,128] fp32 buffer of key-side sums.
+ * Tensor-core path (bf16, d = 128, bq = 128): the forward's SLA2 workspace
+ * (sla_workspace_size with SLA_MODE_SLA2_TOPK) followed by the per-row
+ * statistics, fp16 phi(Q), the inverse block lists, the per-tile dH / dZ
+ * partials and the key-side sums. */
 size_t sla2_attn_bwd_workspace_size(const sla_shape* shape);
 
 /* Gradients of the SLA2 forward [SLA 关键设计 4; SLA2-deep §07; SLA2-sum §2.C]
@@ -251,8 +255,13 @@ size_t sla2_attn_bwd_workspace_size(const sla_shape* shape);
  * Inputs q, k, v, kept_idx, k_keep, alpha, phi as for sla2_attn_fwd (kept
  * indices distinct per row); dout [B,H,N,d] of the input dtype.
  * Outputs (fp32, caller-owned, fully overwritten): dq, dk, dv [B,H,N,d],
- *   dalpha [B,H,n_q].  dk, dv and dalpha are accumulated with atomic adds
- *   after a zero fill, so their last bits can differ between runs.
+ *   dalpha [B,H,n_q].
+ * Two paths: bf16 inputs with d = 128 and bq = 128 run on the tensor cores
+ *   (bf16 / fp16 operands, fp32 accumulation; every output written once in a
+ *   fixed order, so runs agree bit for bit; errors about 2e-3 of each tensor's
+ *   largest entry); every other shape runs in fp32 on the CUDA cores, where dk,
+ *   dv and dalpha are accumulated with atomic adds after a zero fill, so their
+ *   last bits can differ between runs.
  * ws: its own workspace of sla2_attn_bwd_workspace_size bytes, 256-byte
  *   aligned, status word zeroed once (sla_workspace_init); the call zeroes
  *   the rest itself.  Out-of-range block indices are skipped and reported in
