@@ -13,8 +13,13 @@ feature maps ("SLA: Beyond Sparsity …" (papernotes.org) 关键设计 4).
 
 The same decomposition for SLA's three labels (critical blocks in the softmax,
 critical and negligible blocks both taken out of the linear totals, the
-W_proj gradient) is checked against the oracle's sla_backward; it is the
-algebra a GPU form of SLA's backward would follow.
+W_proj gradient) is checked against the oracle's sla_backward; backward.cu
+follows it for SLA.
+
+Two rearrangements of the SLA2 decomposition follow: a key-major one, and the
+arrangement of the tensor-core kernels (csrc/backward_tc.cu: statistics from
+the attention kernel, query-major dQ, key-major kept shares, per-tile dH_i
+partials, power-of-two scalings), each in fp64 against the oracle.
 """
 import math
 
@@ -307,5 +312,130 @@ def test_key_major_restatement_matches_oracle(N, d, bq, kk, kind):
     alpha = rng.uniform(0.1, 0.9, (1, H, nq))
     ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
     got = _key_major(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
+
+
+def _tensor_core_arrangement(q, k, v, kept, alpha, do, bq, bkv, kind):
+    """The arrangement of sparse_linear_attention_b200/csrc/backward_tc.cu, in
+    fp64: per-row statistics as the attention kernel's epilogue writes them
+    (log2-sum-exp from a stale running max, D, s, dden, the row's dalpha share);
+    a query-major dQ pass with Bx and s dO scaled by the power of two sigma >=
+    max Z_tot and H_tot entering as H_tot / sigma, which also forms the per-tile
+    dH_i, dZ_i; a key-major pass over the inverse lists accumulating the
+    transposed key-side products; dH_tot, dZ_tot as sums of the tile partials;
+    the per-key step with dH_tot scaled by the power of two tau."""
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    l2e = 1.0 / math.log(2.0)
+    kk = kept.shape[-1]
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dal = np.zeros((B, H, nq))
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK, PQ = _phi(K, kind), _phi(Q, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            sigma = 2.0 ** math.ceil(math.log2(max(Zt.max(), 1e-300)))
+            keys_of = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in range(nkv)]
+            stats = np.zeros((N, 5))
+            # 1. the attention kernel's statistics epilogue
+            for i in range(nq):
+                rows = np.arange(i * bq, min((i + 1) * bq, N))
+                a = alpha[b, h, i]
+                ks = np.concatenate([keys_of[j] for j in kept[b, h, i]]) if kk else np.zeros(0, int)
+                Os, Ol = np.zeros((len(rows), d)), np.zeros((len(rows), d))
+                lse2 = np.zeros(len(rows))
+                if len(ks):
+                    S2 = sc * l2e * (Q[rows] @ K[ks].T)
+                    m = S2.max(1) - 3.0  # a stale running max: lse2 does not depend on it
+                    p = np.exp2(S2 - m[:, None])
+                    lse2 = m + np.log2(p.sum(1))
+                    Os = (p @ V[ks]) / p.sum(1)[:, None]
+                lin = kk < nkv
+                s_r, dd_r = np.zeros(len(rows)), np.zeros(len(rows))
+                if lin:
+                    A = PQ[rows] @ PK[ks].T if len(ks) else np.zeros((len(rows), 0))
+                    den = PQ[rows] @ Zt - A.sum(1)
+                    Ol = (PQ[rows] @ Ht - A @ V[ks]) / den[:, None]
+                    s_r = (1 - a) / den
+                    dd_r = -(1 - a) * (G[rows] * Ol).sum(1) / den
+                stats[rows] = np.stack([lse2, a * (G[rows] * Os).sum(1), s_r, dd_r,
+                                        (G[rows] * (Os - Ol)).sum(1)], axis=1)
+                dal[b, h, i] = stats[rows, 4].sum()
+            users = [[i for i in range(nq) if j in set(int(x) for x in kept[b, h, i])] for j in range(nkv)]
+            dh_parts, dz_parts = [], []
+            # 2. query-major dQ, per-tile dH_i, dZ_i
+            for i in range(nq):
+                rows = np.arange(i * bq, min((i + 1) * bq, N))
+                a = alpha[b, h, i]
+                lse2, D, s_r, dd_r = (stats[rows, c] for c in range(4))
+                dqs, dql = np.zeros((len(rows), d)), np.zeros((len(rows), d))
+                for j in kept[b, h, i]:
+                    ks = keys_of[j]
+                    P = np.exp2(sc * l2e * (Q[rows] @ K[ks].T) - lse2[:, None])
+                    Gm = G[rows] @ V[ks].T
+                    dS = P * (a * Gm - D[:, None])
+                    nbx = -(s_r[:, None] * Gm + dd_r[:, None]) * sigma
+                    dqs += dS @ K[ks]
+                    dql += nbx @ PK[ks]
+                ssd = (s_r * sigma)[:, None] * G[rows]
+                hterm = ssd @ (Ht / sigma).T
+                dh_parts.append(PQ[rows].T @ ssd / sigma)
+                dz_parts.append(PQ[rows].T @ dd_r)
+                gphi = dql / sigma + hterm + dd_r[:, None] * Zt[None, :]
+                dq[b, h, rows] = sc * dqs + _phi_grad(Q[rows], gphi, kind)
+            # 3. key-major kept shares (transposed accumulators)
+            dphik = np.zeros((N, d))
+            for j in range(nkv):
+                ks = keys_of[j]
+                dVT, dKT, dPT = np.zeros((d, len(ks))), np.zeros((d, len(ks))), np.zeros((d, len(ks)))
+                for i in users[j]:
+                    rows = np.arange(i * bq, min((i + 1) * bq, N))
+                    a = alpha[b, h, i]
+                    lse2, D, s_r, dd_r = (stats[rows, c] for c in range(4))
+                    P = np.exp2(sc * l2e * (Q[rows] @ K[ks].T) - lse2[:, None])
+                    Gm = G[rows] @ V[ks].T
+                    A = PQ[rows] @ PK[ks].T
+                    dS = P * (a * Gm - D[:, None])
+                    C = a * P - s_r[:, None] * A
+                    nbx = -(s_r[:, None] * Gm + dd_r[:, None]) * sigma
+                    dVT += G[rows].T @ C
+                    dKT += Q[rows].T @ dS
+                    dPT += PQ[rows].T @ nbx
+                dv[b, h, ks] = dVT.T
+                dk[b, h, ks] = sc * dKT.T
+                dphik[ks] = dPT.T / sigma
+            # 4. totals: the tile partials summed, tau, the per-key step
+            dHt = np.sum(dh_parts, axis=0)
+            dZt = np.sum(dz_parts, axis=0)
+            mh = np.abs(dHt).max()
+            tau = 2.0 ** (14 - math.frexp(mh)[1]) if mh > 0 else 1.0
+            acc1 = V @ (tau * dHt).T
+            acc2 = PK @ (tau * dHt)
+            dphi = acc1 / tau + dZt[None, :] + dphik
+            dk[b, h] += _phi_grad(K, dphi, kind)
+            dv[b, h] += acc2 / tau
+    return {"dq": dq, "dk": dk, "dv": dv, "dalpha": dal}
+
+
+@pytest.mark.parametrize("N,d,bq,kk,kind", [(300, 16, 128, 2, "elu1"), (333, 8, 128, 3, "softmax"),
+                                            (130, 16, 128, 0, "elu1"), (256, 16, 128, 4, "elu1"),
+                                            (100, 8, 128, 1, "softmax")])
+def test_tensor_core_arrangement_matches_oracle(N, d, bq, kk, kind):
+    """The tensor-core backward's order of work and its exact power-of-two
+    scalings reproduce the oracle's gradients in fp64 (k = 0, k = n_kv, ragged
+    tiles, both feature maps)."""
+    rng = np.random.default_rng(11 * N + kk)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kk = min(kk, nkv)
+    kept = np.array([[[np.sort(rng.choice(nkv, kk, replace=False)) for _ in range(nq)] for _ in range(H)]])
+    kept = kept.reshape(1, H, nq, kk)
+    alpha = rng.uniform(0.1, 0.9, (1, H, nq))
+    ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
+    got = _tensor_core_arrangement(q, k, v, kept, alpha, do, bq, bkv, kind)
     for name in ref:
         assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name

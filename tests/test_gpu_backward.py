@@ -134,11 +134,20 @@ def test_backward_tensor_core_is_deterministic_and_matches_the_fp32_kernels():
         _close(name, a1[name], f[name], True)
 
 
-@pytest.mark.parametrize("kk", [0, 5])
-def test_backward_no_block_and_every_block(kk):
-    """k = 0 (linear branch only) and k = n_kv (sparse branch only, O_l = 0)."""
-    q, k, v, do, alpha, kept = _case(40 + kk, 2, 1, 300, 32, 64, kk, torch.bfloat16)
-    _check(q, k, v, kept, alpha, do, 64, sla.SLA_PHI_ELU1)
+@pytest.mark.parametrize("kk,d,bq", [(0, 32, 64), (5, 32, 64), (0, 128, 128), (5, 128, 128)])
+def test_backward_no_block_and_every_block(kk, d, bq):
+    """k = 0 (linear branch only) and k = n_kv (sparse branch only, O_l = 0), on
+    both paths (d = 128 with b_q = 128 is the tensor-core one)."""
+    q, k, v, do, alpha, kept = _case(40 + kk, 2, 1, 300, d, bq, kk, torch.bfloat16)
+    _check(q, k, v, kept, alpha, do, bq, sla.SLA_PHI_ELU1)
+
+
+def test_backward_tensor_core_short_sequence():
+    """N below one query tile and one key block short of a second: a single
+    ragged tile on both sides."""
+    q, k, v, do, alpha, kept = _case(88, 1, 3, 100, 128, 128, 1, torch.bfloat16)
+    _check(q, k, v, kept, alpha, do, 128, sla.SLA_PHI_ELU1)
+    _check(q, k, v, kept, alpha, do, 128, sla.SLA_PHI_SOFTMAX)
 
 
 def test_backward_reports_out_of_range_block():
