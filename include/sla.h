@@ -238,8 +238,8 @@ sla_status sla_attn_fwd(const sla_shape* shape, const void* q, const void* k,
  * gradients per (b,h), and a [B,H,N,128] fp32 buffer of key-side sums.
  * Tensor-core path (bf16, d = 128, bq = 128): the forward's SLA2 workspace
  * (sla_workspace_size with SLA_MODE_SLA2_TOPK) followed by the per-row
- * statistics, fp16 phi(Q), the inverse block lists, the per-tile dH / dZ
- * partials and the key-side sums. */
+ * statistics, fp16 phi(Q), the inverse block lists, the per-tile dH (fp16)
+ * and dZ partials, dH_tot, dZ_tot and a scaled fp16 copy of dH_tot. */
 size_t sla2_attn_bwd_workspace_size(const sla_shape* shape);
 
 /* Gradients of the SLA2 forward [SLA 关键设计 4; SLA2-deep §07; SLA2-sum §2.C]

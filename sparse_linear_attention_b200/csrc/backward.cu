@@ -932,29 +932,6 @@ BwdLayout bwd_layout(const sla_shape& s, bool sla_mode) {
   return L;
 }
 
-cudaError_t launch_bwd_keys(const sla_shape& s, const void* k, const void* v, int phi, const float* dhtot,
-                            const float* dztot, const float* dphik, float* dk, float* dv, cudaStream_t st) {
-  const size_t smem = kKeysSmemFloats * sizeof(float);
-  const int BH = s.B * s.H;
-  const dim3 grid((s.N + kTokTile - 1) / kTokTile, BH);
-  cudaError_t e;
-  if (s.in_dtype == SLA_BF16) {
-    if ((e = cudaFuncSetAttribute(bwd_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(smem))) != cudaSuccess)
-      return e;
-    bwd_keys_kernel<__nv_bfloat16><<<grid, kBT, smem, st>>>(static_cast<const __nv_bfloat16*>(k),
-                                                            static_cast<const __nv_bfloat16*>(v), s.N, s.d, phi,
-                                                            dhtot, dztot, dphik, dk, dv);
-  } else {
-    if ((e = cudaFuncSetAttribute(bwd_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(smem))) != cudaSuccess)
-      return e;
-    bwd_keys_kernel<float><<<grid, kBT, smem, st>>>(static_cast<const float*>(k), static_cast<const float*>(v), s.N,
-                                                    s.d, phi, dhtot, dztot, dphik, dk, dv);
-  }
-  return cudaGetLastError();
-}
-
 namespace {
 
 cudaError_t launch_backward_common(const sla_shape& s, const void* q, const void* k, const void* v,

@@ -22,15 +22,21 @@
 //   bwd_dq_kernel    per query tile: S, G (tcgen05, bf16) per kept block;
 //                    dS (bf16), -Bx sigma (fp16) to smem; dQ_s += dS K,
 //                    dQ_l += (-Bx sigma) phi(K); then s sigma dO H_tot^T / sigma
-//                    and dH_i = phi(Q)^T (s sigma dO) / sigma; epilogue dQ.
-//   bwd_dkv_kernel   per key block: for each query tile keeping it, S, G, A
-//                    (tcgen05); dS, C (bf16), -Bx sigma (fp16) to smem;
-//                    dV^T += dO^T C, dK^T += Q^T dS, dphi(K)^T += phi(Q)^T (-Bx sigma)
-//                    accumulated in TMEM over the tiles; no atomics.
+//                    and sigma dH_i = phi(Q)^T (s sigma dO), written as -sigma dH_i
+//                    in fp16 with dZ_i; epilogue dQ.
 //   dh_reduce_kernel dH_tot, dZ_tot: the tiles' partials summed in tile order
+//   dh_pack_kernel   tau dH_tot in fp16 (tau a power of two)
 //   dalpha_kernel    dalpha per query block: its rows' shares in row order
+//   bwd_dkv_kernel   per key block j, with M_j = dH_tot - sum of the dH_i of the
+//                    query tiles keeping j (exact regrouping of the kept linear
+//                    shares):  dV_j = sum_i (alpha P_ij)^T dO_i + phi(K_j) M_j,
+//                    dphi(K_j) = V_j M_j^T + dZ_tot - sum_i dZ_i,
+//                    dK_j = sum_i dS_ij^T Q_i / sqrt(d) + phi'(K_j) dphi(K_j):
+//                    phase 1 over the tiles keeping j (S, G, then dV^T, dK^T in
+//                    TMEM), phase 2 the partials and the totals through
+//                    (.) V_j^T and (.)^T phi(K_j)^T, one combined epilogue.
 // sigma is the forward's per-head power of two (>= max_e Z_tot[e]); it scales
-// Bx and s dO into the fp16 range and is divided out exactly.
+// Bx, s dO and dH_i into the fp16 range and is divided out exactly.
 // Every result is written once in a fixed order: the gradients are the same
 // on every run.
 #include <cuda.h>
@@ -67,8 +73,11 @@ struct TcArgs {
   const int32_t* inv;    // [BH, nkv, nq] query blocks keeping each key block
   const int32_t* inv_n;  // [BH, nkv]
   const __nv_bfloat16* q;
-  float *dq, *dk, *dv, *dphik;  // dq, dk, dv [BH, N, 128]; dphik fp32 [BH, N, 128]
-  float *dhpart, *dzpart;       // [BH * nq, 128, 128], [BH * nq, 128]
+  float *dq, *dk, *dv;          // [BH, N, 128]
+  __half* dhpart;               // [BH * nq, 128, 128]: -sigma dH_i per query tile
+  float* dzpart;                // [BH * nq, 128]: dZ_i per query tile
+  const float* dztot;           // [BH, 128]
+  const float* tau;             // [BH]: the power of two scaling dH_tot into fp16
   int* status;
   unsigned long long wait_ns;
 };
@@ -417,8 +426,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_OPF]);
     }
-    // s sigma dO (fp16, channels 32 g ..) over the operand tiles once the loop's products are done
+    // s sigma dO (fp16, channels 32 g ..) over the operand tiles once the loop's products
+    // are done (the Q and dO tiles read from here on landed on B_QD, long complete)
     ok = ok && warp_wait_tc(&bars[B_LOOP], 0, abort_flag, a.status, a.wait_ns);
+    ok = ok && warp_wait_tc(&bars[B_QD], 0, abort_flag, a.status, a.wait_ns);
     if (ok) {
       const float f = sr * sigma;
 #pragma unroll
@@ -456,15 +467,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok) tc_fence_after();
     const float inv_sigma = 1.0f / sigma;  // exact: a power of two
     if (ok) {
-      // sigma dH_i: lane e = r, columns c = 32 g ..
-      float* dh = a.dhpart + (tile * kDPad + r) * kDPad + 32 * g;
+      // -sigma dH_i as fp16 (the key kernel subtracts the tiles keeping each key
+      // block from the totals): lane e = r, columns c = 32 g ..
+      __half* dh = a.dhpart + (tile * kDPad + r) * kDPad + 32 * g;
       float hv[32];
       tmem_ld32(tmem + lrow + T_DH + 32 * g, hv);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 32; c += 4)
-        *reinterpret_cast<float4*>(dh + c) =
-            make_float4(hv[c] * inv_sigma, hv[c + 1] * inv_sigma, hv[c + 2] * inv_sigma, hv[c + 3] * inv_sigma);
+      for (int c = 0; c < 32; c += 8)
+        *reinterpret_cast<uint4*>(dh + c) = make_uint4(pack_half2(-hv[c], -hv[c + 1]), pack_half2(-hv[c + 2], -hv[c + 3]),
+                                                       pack_half2(-hv[c + 4], -hv[c + 5]),
+                                                       pack_half2(-hv[c + 6], -hv[c + 7]));
     }
     // dQ of row r, channels 32 g + 16 h ..: scale dQ_s + phi'(Q) (dQ_l / sigma + s dO H_tot^T + dden Z_tot)
     const float* zt = a.ztot + static_cast<long long>(bh) * kDPad;
@@ -565,25 +578,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------- dK, dV (key-major)
+// One CTA per key block j of a head (64 keys).  With M_j = dH_tot minus the
+// dH_i of the query tiles i keeping j:
+//   dV_j = sum_i (alpha_i P_ij)^T dO_i + phi(K_j) M_j
+//   dphi(K_j) = V_j M_j^T + dZ_tot - sum_i dZ_i,  dK_j = sum_i dS_ij^T Q_i / sqrt(d) + phi'(K_j) dphi(K_j)
+// (the linear shares through the query tiles' partials, so the loop over the
+// tiles keeping j needs S, G, P and dS only).  Phase 1, per such tile i (two
+// operand stages, two S/G buffers): S = Q_i K_j^T, G = dO_i V_j^T; the row warps
+// write dS and alpha P (bf16); dV^T += dO_i^T (alpha P), dK^T += Q_i^T dS.  Phase 2:
+// the tiles' -sigma dH_i (fp16, from bwd_dq_kernel) and tau dH_tot through
+// (.) V16_j^T and (.)^T phi(K_j)^T, four 32 KB slots in the stage area.  The
+// epilogue combines everything; each gradient is written once.
 namespace dkv {
-constexpr uint32_t OFF_K = 0;          // K_j | V_j | phi(K_j): each 2 chunks of [64 rows][128 B]
+constexpr uint32_t OFF_K = 0;          // K_j bf16 | V_j bf16 | V_j fp16 | phi(K_j) fp16: each 2 chunks of [64 rows][128 B]
 constexpr uint32_t OFF_V = 16384;
-constexpr uint32_t OFF_PK = 32768;
-constexpr uint32_t OFF_ST = 49152;     // Q_i | dO_i | phi(Q_i): each 2 chunks of [128 rows][128 B]
-constexpr uint32_t OFF_OPS = OFF_ST + 98304;  // dS bf16 | C bf16 | -Bx sigma fp16, each [128 rows][64 keys]
-constexpr uint32_t OFF_BAR = OFF_OPS + 49152;
-constexpr uint32_t OFF_MISC = OFF_BAR + 128;
+constexpr uint32_t OFF_V16 = 32768;
+constexpr uint32_t OFF_PK = 49152;
+constexpr uint32_t OFF_ST = 65536;     // phase 1: 2 stages of Q_i | dO_i (2 chunks of [128 rows][128 B] each)
+constexpr uint32_t STAGE = 65536;      // phase 2: 4 slots of one [128][128] fp16 tile
+constexpr uint32_t SLOT = 32768;
+constexpr uint32_t OFF_OPS = OFF_ST + 2 * STAGE;  // dS bf16 | alpha P bf16, each [128 rows][64 keys]; epilogue reductions
+constexpr uint32_t OFF_BAR = OFF_OPS + 32768;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t SMEM = OFF_MISC + 64;
 static_assert(SMEM <= 232448, "shared memory budget");
-// TMEM: S 0, G 64, A 128; dV^T 256, dK^T 320, dphi(K)^T 384
-constexpr uint32_t T_S = 0, T_G = 64, T_A = 128, T_DV = 256, T_DK = 320, T_DP = 384;
-enum { B_KV = 0, B_STF = 1, B_STE = 2, B_SGF = 3, B_OPF = 4, B_OPE = 5, B_DONE = 6, B_DRAIN = 7, NBAR = 8 };
+// TMEM: phase 1 S_b at 128 b, G_b at 128 b + 64; then tau dH_tot V^T at 0, (tau dH_tot)^T phi(K)^T at 64;
+// dV^T 256, dK^T 320, the tiles' -sigma dH_i V^T 384, (-sigma dH_i)^T phi(K)^T 448
+constexpr uint32_t T_TP = 0, T_TV = 64, T_DV = 256, T_DK = 320, T_KP = 384, T_KV = 448;
+enum { B_KV = 0, B_STF = 1, B_STE = 3, B_SGF = 5, B_SGE = 7, B_OPF = 9, B_OPE = 10, B_SLOOP = 11, B_LF = 12,
+       B_LE = 16, B_DONE = 20, B_DRAIN = 21, NBAR = 22 };
+static_assert(NBAR * 8 <= 256, "barrier area");
 }  // namespace dkv
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                   const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
+                   const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmPK,
+                   const __grid_constant__ CUtensorMap tmDHi, const __grid_constant__ CUtensorMap tmDH,
                    const TcArgs a) {
   using namespace dkv;
   extern __shared__ __align__(1024) uint8_t sm[];
@@ -601,9 +632,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int cnt = a.inv_n[kb];
   if (cnt < 0 || cnt > a.nq) cnt = 0;
   const int32_t* il = a.inv + kb * a.nq;
+  auto tile_of = [&](int n) -> int {
+    const int i = il[n];
+    return (i < 0 || i >= a.nq) ? 0 : i;
+  };
 
   if (tid == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], (i == B_OPF) ? kCompute : 1);
+    for (int b = 0; b < NBAR; ++b)
+      mbar_init(&bars[b], (b == B_OPF || b == B_SGE || b == B_SGE + 1) ? kCompute : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -619,76 +655,136 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const float sigma = a.sigma[bh];
 
   if (warp == kProdWarp) {
-    if (lane == 0 && cnt > 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(&bars[B_KV], 49152);
-      tma_load_3d(sm + OFF_K, &tmK, &bars[B_KV], 0, j * kBlockKV, bh);
-      tma_load_3d(sm + OFF_K + 8192, &tmK, &bars[B_KV], 64, j * kBlockKV, bh);
-      tma_load_3d(sm + OFF_V, &tmV, &bars[B_KV], 0, j * kBlockKV, bh);
-      tma_load_3d(sm + OFF_V + 8192, &tmV, &bars[B_KV], 64, j * kBlockKV, bh);
-      tma_load_3d(sm + OFF_PK, &tmPK, &bars[B_KV], 0, j * kBlockKV, bh);
-      tma_load_3d(sm + OFF_PK + 8192, &tmPK, &bars[B_KV], 64, j * kBlockKV, bh);
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0, lissued = 0;
+      mbar_arrive_expect_tx(&bars[B_KV], 65536);
+      const int krow = j * kBlockKV;
+      tma_load_3d(sm + OFF_K, &tmK, &bars[B_KV], 0, krow, bh);
+      tma_load_3d(sm + OFF_K + 8192, &tmK, &bars[B_KV], 64, krow, bh);
+      tma_load_3d(sm + OFF_V, &tmV, &bars[B_KV], 0, krow, bh);
+      tma_load_3d(sm + OFF_V + 8192, &tmV, &bars[B_KV], 64, krow, bh);
+      tma_load_3d(sm + OFF_V16, &tmV16, &bars[B_KV], 0, krow, bh);
+      tma_load_3d(sm + OFF_V16 + 8192, &tmV16, &bars[B_KV], 64, krow, bh);
+      tma_load_3d(sm + OFF_PK, &tmPK, &bars[B_KV], 0, krow, bh);
+      tma_load_3d(sm + OFF_PK + 8192, &tmPK, &bars[B_KV], 64, krow, bh);
       for (int n = 0; n < cnt; ++n) {
-        if (n >= 1 && !mbar_wait(&bars[B_STE], (n - 1) & 1, abort_flag, a.status, a.wait_ns)) break;
-        int i = il[n];
-        if (i < 0 || i >= a.nq) i = 0;
-        uint64_t* fb = &bars[B_STF];
-        mbar_arrive_expect_tx(fb, 98304);
-        tma_load_3d(sm + OFF_ST, &tmQ, fb, 0, i * kRowsT, bh);
-        tma_load_3d(sm + OFF_ST + 16384, &tmQ, fb, 64, i * kRowsT, bh);
-        tma_load_3d(sm + OFF_ST + 32768, &tmDO, fb, 0, i * kRowsT, bh);
-        tma_load_3d(sm + OFF_ST + 49152, &tmDO, fb, 64, i * kRowsT, bh);
-        tma_load_3d(sm + OFF_ST + 65536, &tmPQ, fb, 0, i * kRowsT, bh);
-        tma_load_3d(sm + OFF_ST + 81920, &tmPQ, fb, 64, i * kRowsT, bh);
+        const int s = n & 1;
+        if (n >= 2 && !mbar_wait(&bars[B_STE + s], ((n >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        const int i = tile_of(n);
+        uint8_t* st = sm + OFF_ST + s * STAGE;
+        uint64_t* fb = &bars[B_STF + s];
+        mbar_arrive_expect_tx(fb, STAGE);
+        tma_load_3d(st, &tmQ, fb, 0, i * kRowsT, bh);
+        tma_load_3d(st + 16384, &tmQ, fb, 64, i * kRowsT, bh);
+        tma_load_3d(st + 32768, &tmDO, fb, 0, i * kRowsT, bh);
+        tma_load_3d(st + 49152, &tmDO, fb, 64, i * kRowsT, bh);
         ++issued;
       }
+      // phase 2 once every phase-1 product is done: the tiles' partials, then the totals
+      if (ok && mbar_wait(&bars[B_SLOOP], 0, abort_flag, a.status, a.wait_ns)) {
+        for (int m = 0; m <= cnt; ++m) {
+          const int sl = m & 3;
+          if (m >= 4 && !mbar_wait(&bars[B_LE + sl], ((m >> 2) - 1) & 1, abort_flag, a.status, a.wait_ns)) break;
+          uint8_t* dst = sm + OFF_ST + sl * SLOT;
+          uint64_t* fb = &bars[B_LF + sl];
+          mbar_arrive_expect_tx(fb, SLOT);
+          if (m < cnt) {
+            const int t = bh * a.nq + tile_of(m);
+            tma_load_3d(dst, &tmDHi, fb, 0, 0, t);
+            tma_load_3d(dst + 16384, &tmDHi, fb, 64, 0, t);
+          } else {
+            tma_load_3d(dst, &tmDH, fb, 0, 0, bh);
+            tma_load_3d(dst + 16384, &tmDH, fb, 64, 0, bh);
+          }
+          ++lissued;
+        }
+      }
+      // every issued copy lands before the CTA exits
       mbar_wait_drain(&bars[B_KV], 0);
-      if (issued > 0) mbar_wait_drain(&bars[B_STF], (issued - 1) & 1);
+      for (int g2 = issued > 2 ? issued - 2 : 0; g2 < issued; ++g2)
+        mbar_wait_drain(&bars[B_STF + (g2 & 1)], (g2 >> 1) & 1);
+      for (int g2 = lissued > 4 ? lissued - 4 : 0; g2 < lissued; ++g2)
+        mbar_wait_drain(&bars[B_LF + (g2 & 3)], (g2 >> 2) & 1);
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);   // Q_i K_j^T, dO_i V_j^T (bf16)
-      const uint32_t id_a = idesc_f16(0, 0, 0, 128, 64);   // phi(Q_i) phi(K_j)^T (f16)
-      const uint32_t id_t = idesc_f16(1, 1, 1, 128, 64);   // dO^T C, Q^T dS (bf16, both MN-major)
-      const uint32_t id_tp = idesc_f16(0, 1, 1, 128, 64);  // phi(Q)^T (-Bx sigma) (f16)
+      const uint32_t id_s = idesc_f16(1, 0, 0, 128, 64);   // Q_i K_j^T, dO_i V_j^T (bf16, K-major)
+      const uint32_t id_t = idesc_f16(1, 1, 1, 128, 64);   // dO^T (alpha P), Q^T dS (bf16, both MN-major)
+      const uint32_t id_lp = idesc_f16(0, 0, 0, 128, 64);  // T V16_j^T (f16, both K-major)
+      const uint32_t id_lv = idesc_f16(0, 1, 0, 128, 64);  // T^T (MN-major) phi(K_j)^T (K-major), f16
       const uint64_t dKd = sdesc_sw128(smem_u32(sm + OFF_K), 16, 1024);
       const uint64_t dStK = sdesc_sw128(smem_u32(sm + OFF_ST), 16, 1024);
       const uint64_t dStMN = sdesc_sw128(smem_u32(sm + OFF_ST), 16384, 1024);
       const uint64_t dOpsMN = sdesc_sw128(smem_u32(sm + OFF_OPS), 16, 1024);  // N = 64 fits one atom
-      bool ok = cnt > 0 && mbar_wait(&bars[B_KV], 0, abort_flag, a.status, a.wait_ns);
-      for (int n = 0; ok && n < cnt; ++n) {
-        if (!mbar_wait(&bars[B_STF], n & 1, abort_flag, a.status, a.wait_ns)) {
-          ok = false;
-          break;
-        }
+      bool ok = mbar_wait(&bars[B_KV], 0, abort_flag, a.status, a.wait_ns);
+      auto ops = [&](int m) -> bool {
+        if (!mbar_wait(&bars[B_OPF], m & 1, abort_flag, a.status, a.wait_ns)) return false;
         tc_fence_after();
-        // S, G, A: M = 128 rows, N = 64 keys, K = 128 channels
+        const uint32_t so = ((m & 1) * STAGE) >> 4;
 #pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
-          const uint32_t ob = ((k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
-          mma_f16_ss(tmem + T_S, dStK + oa, dKd + ob, id_s, k8 > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + T_G, dStK + (32768u >> 4) + oa, dKd + (16384u >> 4) + ob, id_s, k8 > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + T_A, dStK + (65536u >> 4) + oa, dKd + (32768u >> 4) + ob, id_a, k8 > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[B_SGF]);
-        if (!mbar_wait(&bars[B_OPF], n & 1, abort_flag, a.status, a.wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dV^T, dK^T, dphi(K)^T: M = 128 channels, N = 64 keys, K = 128 rows (+2048 B per 16)
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const uint32_t acc = (n > 0 || k8 > 0) ? 1u : 0u;
-          mma_f16_ss(tmem + T_DV, dStMN + (32768u >> 4) + k8 * 128u, dOpsMN + (16384u >> 4) + k8 * 128u, id_t, acc);
-          mma_f16_ss(tmem + T_DK, dStMN + k8 * 128u, dOpsMN + k8 * 128u, id_t, acc);
-          mma_f16_ss(tmem + T_DP, dStMN + (65536u >> 4) + k8 * 128u, dOpsMN + (32768u >> 4) + k8 * 128u, id_tp, acc);
+        for (int k8 = 0; k8 < 8; ++k8) {  // K = 128 rows, +2048 B per 16
+          const uint32_t acc = (m > 0 || k8 > 0) ? 1u : 0u;
+          mma_f16_ss(tmem + T_DV, dStMN + so + (32768u >> 4) + k8 * 128u, dOpsMN + (16384u >> 4) + k8 * 128u, id_t,
+                     acc);
+          mma_f16_ss(tmem + T_DK, dStMN + so + k8 * 128u, dOpsMN + k8 * 128u, id_t, acc);
         }
         mma_commit(&bars[B_OPE]);
-        mma_commit(&bars[B_STE]);
+        mma_commit(&bars[B_STE + (m & 1)]);
+        return true;
+      };
+      for (int n = 0; ok && n < cnt; ++n) {
+        const int b = n & 1;
+        if (!mbar_wait(&bars[B_STF + b], (n >> 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (n >= 2 && !mbar_wait(&bars[B_SGE + b], ((n >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t so = (b * STAGE) >> 4;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {  // M = 128 rows, N = 64 keys, K = 128 channels
+          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          const uint32_t ob = ((k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + 128 * b, dStK + so + oa, dKd + ob, id_s, k8 > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + 128 * b + 64, dStK + so + (32768u >> 4) + oa, dKd + (16384u >> 4) + ob, id_s,
+                     k8 > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[B_SGF + b]);
+        if (n >= 1 && !ops(n - 1)) {
+          ok = false;
+          break;
+        }
       }
-      mma_commit(&bars[B_DONE]);
+      if (ok && cnt > 0) ok = ops(cnt - 1);
+      if (ok) mma_commit(&bars[B_SLOOP]);
+      for (int m = 0; ok && m <= cnt; ++m) {
+        const int sl = m & 3;
+        if (!mbar_wait(&bars[B_LF + sl], (m >> 2) & 1, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t so = (sl * SLOT) >> 4;
+        const bool tot = m == cnt;
+        const uint32_t cp = tot ? T_TP : T_KP, cv = tot ? T_TV : T_KV;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {  // M = 128 (e, then c), N = 64 keys, K = 128
+          const uint32_t acc = ((!tot && m > 0) || k8 > 0) ? 1u : 0u;
+          const uint32_t oa = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
+          const uint32_t ob = ((k8 >> 2) * 8192u + (k8 & 3) * 32u) >> 4;
+          mma_f16_ss(tmem + cp, dStK + so + oa, dKd + (32768u >> 4) + ob, id_lp, acc);
+          mma_f16_ss(tmem + cv, dStMN + so + k8 * 128u, dKd + (49152u >> 4) + ob, id_lv, acc);
+        }
+        mma_commit(&bars[B_LE + sl]);
+      }
+      if (ok) mma_commit(&bars[B_DONE]);
       mma_commit(&bars[B_DRAIN]);
       mbar_wait_drain(&bars[B_DRAIN], 0);
     }
@@ -701,85 +797,146 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nvalid = (tail && j == a.nkv - 1) ? a.N - j * kBlockKV : kBlockKV;
     bool ok = true;
     uint8_t* opS = sm + OFF_OPS;
-    uint8_t* opC = sm + OFF_OPS + 16384;
-    uint8_t* opB = sm + OFF_OPS + 32768;
+    uint8_t* opP = sm + OFF_OPS + 16384;
     for (int n = 0; n < cnt; ++n) {
-      int i = il[n];
-      if (i < 0 || i >= a.nq) i = 0;
+      const int i = tile_of(n);
       const int tok = i * kRowsT + r;
       const bool valid = tok < a.N;
-      float lse2 = 0.0f, D = 0.0f, sr = 0.0f, dd = 0.0f;
+      float lse2 = 0.0f, D = 0.0f;
       if (valid) {
-        const float4 st = *reinterpret_cast<const float4*>(a.rows + (static_cast<long long>(bh) * a.N + tok) * 8);
+        const float2 st = *reinterpret_cast<const float2*>(a.rows + (static_cast<long long>(bh) * a.N + tok) * 8);
         lse2 = st.x;
         D = st.y;
-        sr = st.z;
-        dd = st.w;
       }
       const float alpha = a.alpha[static_cast<long long>(bh) * a.nq + i];
-      ok = ok && warp_wait_tc(&bars[B_SGF], n & 1, abort_flag, a.status, a.wait_ns);
-      // The products of the previous tile read the operand tiles; they were
-      // issued before this tile's S, G, A, so they are done (the wait is immediate).
-      ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
+      const int b = n & 1;
+      ok = ok && warp_wait_tc(&bars[B_SGF + b], (n >> 1) & 1, abort_flag, a.status, a.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      float sv[16], gv[16], av[16];
-      tmem_ld16(tmem + lrow + T_S + 16 * g, sv);
-      tmem_ld16(tmem + lrow + T_G + 16 * g, gv);
-      tmem_ld16(tmem + lrow + T_A + 16 * g, av);
+      float sv[16], gv[16];
+      tmem_ld16(tmem + lrow + 128 * b + 16 * g, sv);
+      tmem_ld16(tmem + lrow + 128 * b + 64 + 16 * g, gv);
       tmem_wait_ld();
-      uint32_t pS[8], pC[8], pB[8];
+      uint32_t pS[8], pP[8];
 #pragma unroll
       for (int c = 0; c < 16; c += 2) {
-        float ds[2], cv[2], bx[2];
+        float ds[2], ap[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const bool kv = valid && (16 * g + c + e < nvalid);
           const float p = kv ? ex2_approx(fmaf(sv[c + e], a.sl2, -lse2)) : 0.0f;
           ds[e] = p * fmaf(alpha, gv[c + e], -D);
-          cv[e] = kv ? fmaf(alpha, p, -sr * av[c + e]) : 0.0f;
-          bx[e] = kv ? -fmaf(sr, gv[c + e], dd) * sigma : 0.0f;
+          ap[e] = alpha * p;
         }
         pS[c / 2] = pack_bf162(ds[0], ds[1]);
-        pC[c / 2] = pack_bf162(cv[0], cv[1]);
-        pB[c / 2] = pack_half2(bx[0], bx[1]);
+        pP[c / 2] = pack_bf162(ap[0], ap[1]);
       }
+      tc_fence_before();
+      mbar_arrive(&bars[B_SGE + b]);
+      ok = ok && (n == 0 || warp_wait_tc(&bars[B_OPE], (n - 1) & 1, abort_flag, a.status, a.wait_ns));
+      if (!ok) break;
       put_unit(opS, r, 2 * g, pS[0], pS[1], pS[2], pS[3]);
       put_unit(opS, r, 2 * g + 1, pS[4], pS[5], pS[6], pS[7]);
-      put_unit(opC, r, 2 * g, pC[0], pC[1], pC[2], pC[3]);
-      put_unit(opC, r, 2 * g + 1, pC[4], pC[5], pC[6], pC[7]);
-      put_unit(opB, r, 2 * g, pB[0], pB[1], pB[2], pB[3]);
-      put_unit(opB, r, 2 * g + 1, pB[4], pB[5], pB[6], pB[7]);
-      tc_fence_before();
+      put_unit(opP, r, 2 * g, pP[0], pP[1], pP[2], pP[3]);
+      put_unit(opP, r, 2 * g + 1, pP[4], pP[5], pP[6], pP[7]);
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_OPF]);
     }
-    // epilogue: lane = channel c; keys 16 g .. of the block
-    if (cnt > 0) ok = ok && warp_wait_tc(&bars[B_DONE], 0, abort_flag, a.status, a.wait_ns);
-    if (ok) {
-      tc_fence_after();
-      const int c = r;
-      const float inv_sigma = 1.0f / sigma;
-      const long long base = (static_cast<long long>(bh) * a.N + static_cast<long long>(j) * kBlockKV) * kDPad + c;
-      float vv[16], kv[16], pv[16];
-      if (cnt > 0) {
-        tmem_ld16(tmem + lrow + T_DV + 16 * g, vv);
-        tmem_ld16(tmem + lrow + T_DK + 16 * g, kv);
-        tmem_ld16(tmem + lrow + T_DP + 16 * g, pv);
+    // epilogue: lane = channel c; keys 16 g .. of the block (the K tile read here
+    // landed on B_KV, long complete)
+    ok = ok && warp_wait_tc(&bars[B_DONE], 0, abort_flag, a.status, a.wait_ns);
+    ok = ok && warp_wait_tc(&bars[B_KV], 0, abort_flag, a.status, a.wait_ns);
+    if (ok) tc_fence_after();
+    const int c = r;
+    const bool have = cnt > 0;
+    const float inv_sigma = 1.0f / sigma, inv_tau = 1.0f / a.tau[bh];  // exact: powers of two
+    float zc = a.dztot[static_cast<long long>(bh) * kDPad + c];
+    for (int n = 0; n < cnt; ++n) zc -= a.dzpart[(static_cast<long long>(bh) * a.nq + tile_of(n)) * kDPad + c];
+    // the key values k[key][c] of this thread's 16 keys (bf16 tile in smem), and
+    // dphi(k) = (tau dH_tot) V^T / tau + (-sigma sum dH_i) V^T / sigma + dZ_tot - sum dZ_i
+    float kx[16], dphi[16];
+    {
+      float tp[16], kp[16];
+      if (ok) {
+        tmem_ld16(tmem + lrow + T_TP + 16 * g, tp);
+        tmem_ld16(tmem + lrow + T_KP + 16 * g, kp);
         tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) vv[x] = kv[x] = pv[x] = 0.0f;
       }
 #pragma unroll
       for (int x = 0; x < 16; ++x) {
         const int key = 16 * g + x;
-        if (key < nvalid) {
-          const long long o = base + static_cast<long long>(key) * kDPad;
-          a.dv[o] = vv[x];
-          a.dk[o] = kv[x] * a.scale;
-          a.dphik[o] = pv[x] * inv_sigma;
+        const __nv_bfloat16* kp16 = reinterpret_cast<const __nv_bfloat16*>(
+            sm + OFF_K + (c >> 6) * 8192u + sw128_off(key, (c & 63) >> 3)) + (c & 7);
+        kx[x] = __bfloat162float(*kp16);
+        dphi[x] = ok ? tp[x] * inv_tau + (have ? kp[x] * inv_sigma : 0.0f) + zc : 0.0f;
+      }
+    }
+    const bool smx = a.phi == SLA_PHI_SOFTMAX;
+    if (smx) {
+      // phi'(k) dphi = f (dphi - sum_c f_c dphi_c), f the softmax of the key over its
+      // 128 channels (the lanes of the four warps that share g): kx becomes f, dphi
+      // becomes phi'(k) dphi
+      float* red = reinterpret_cast<float*>(sm + OFF_OPS);  // [3][4 groups][4 quarters][16 keys]
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        float m = kx[x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[(g * 4 + q4) * 16 + x] = m;
+      }
+      named_bar_sync(1, kCompute);
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float* rr = red + g * 64 + x;
+        float e = expf(kx[x] - fmaxf(fmaxf(rr[0], rr[16]), fmaxf(rr[32], rr[48])));
+        kx[x] = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+        if (lane == 0) red[256 + (g * 4 + q4) * 16 + x] = e;
+      }
+      named_bar_sync(1, kCompute);
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float* rr = red + 256 + g * 64 + x;
+        kx[x] /= (rr[0] + rr[16]) + (rr[32] + rr[48]);
+        float dd = kx[x] * dphi[x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+        if (lane == 0) red[512 + (g * 4 + q4) * 16 + x] = dd;
+      }
+      named_bar_sync(1, kCompute);
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float* rr = red + 512 + g * 64 + x;
+        dphi[x] = kx[x] * (dphi[x] - ((rr[0] + rr[16]) + (rr[32] + rr[48])));
+      }
+    } else {
+#pragma unroll
+      for (int x = 0; x < 16; ++x) dphi[x] *= kx[x] > 0.0f ? 1.0f : expf(kx[x]);
+    }
+    if (ok) {
+      const long long base = (static_cast<long long>(bh) * a.N + static_cast<long long>(j) * kBlockKV) * kDPad + c;
+      {
+        float dkx[16];
+        tmem_ld16(tmem + lrow + T_DK + 16 * g, dkx);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int key = 16 * g + x;
+          if (key < nvalid) a.dk[base + static_cast<long long>(key) * kDPad] = (have ? dkx[x] * a.scale : 0.0f) + dphi[x];
         }
+      }
+      float dvx[16], tv[16], kv2[16];
+      tmem_ld16(tmem + lrow + T_DV + 16 * g, dvx);
+      tmem_ld16(tmem + lrow + T_TV + 16 * g, tv);
+      tmem_ld16(tmem + lrow + T_KV + 16 * g, kv2);
+      tmem_wait_ld();
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int key = 16 * g + x;
+        if (key < nvalid)
+          a.dv[base + static_cast<long long>(key) * kDPad] =
+              (have ? dvx[x] : 0.0f) + tv[x] * inv_tau + (have ? kv2[x] * inv_sigma : 0.0f);
       }
     }
   }
@@ -792,16 +949,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------- reductions
-// grid (64, BH): dH_tot[bh][e][c] and dZ_tot[bh][e] as the tiles' partials summed in tile order.
-__global__ void __launch_bounds__(256) dh_reduce_kernel(const float* __restrict__ dhpart,
-                                                        const float* __restrict__ dzpart, int nq,
+// grid (64, BH): dH_tot[bh][e][c] and dZ_tot[bh][e] as the tiles' partials summed in
+// tile order (the dH partials are -sigma dH_i in fp16).
+__global__ void __launch_bounds__(256) dh_reduce_kernel(const __half* __restrict__ dhpart,
+                                                        const float* __restrict__ dzpart,
+                                                        const float* __restrict__ sigma, int nq,
                                                         float* __restrict__ dhtot, float* __restrict__ dztot) {
   const long long bh = blockIdx.y;
   const int x = blockIdx.x * 256 + threadIdx.x;  // element of the 128 x 128 block
-  const float* src = dhpart + bh * nq * kDPad * kDPad + x;
+  const __half* src = dhpart + bh * nq * kDPad * kDPad + x;
   float t = 0.0f;
-  for (int i = 0; i < nq; ++i) t += src[static_cast<long long>(i) * kDPad * kDPad];
-  dhtot[bh * kDPad * kDPad + x] = t;
+  for (int i = 0; i < nq; ++i) t += __half2float(src[static_cast<long long>(i) * kDPad * kDPad]);
+  dhtot[bh * kDPad * kDPad + x] = -t / sigma[bh];  // exact division: sigma is a power of two
   if (blockIdx.x == 0 && threadIdx.x < kDPad) {
     const float* zs = dzpart + bh * nq * kDPad + threadIdx.x;
     float z = 0.0f;
@@ -831,183 +990,6 @@ __global__ void __launch_bounds__(256) dh_pack_kernel(const float* __restrict__ 
   const float t = m > 0.0f ? ldexpf(1.0f, 14 - ex) : 1.0f;
   if (threadIdx.x == 0) tau[bh] = t;
   for (int x = threadIdx.x; x < kDPad * kDPad; x += 256) dh16[bh * kDPad * kDPad + x] = __float2half_rn(src[x] * t);
-}
-
-// ---------------------------------------------------------------- the totals' share per key (tensor cores)
-// One CTA per 128-key tile of a head.  With dH = dH_tot (fp16, times tau):
-//   acc1 = V dH^T   (fp16 V copy x dH K-major)    -> dphi(k) = acc1 / tau + dZ_tot + kept share
-//   acc2 = phi(K) dH (fp16 phi(K) x dH MN-major)  -> dv += acc2 / tau
-// then dk += phi'(k) dphi(k).  Warps 0..3 one key row per thread, warp 4 loads and issues.
-namespace kt {
-constexpr uint32_t OFF_V = 0, OFF_PK = 32768, OFF_H = 65536, OFF_BAR = 98304, OFF_MISC = OFF_BAR + 64;
-constexpr uint32_t SMEM = OFF_MISC + 64;
-constexpr int kThreads = 160;
-enum { B_LD = 0, B_MMA = 1, NBAR = 2 };
-}  // namespace kt
-
-__global__ void __launch_bounds__(kt::kThreads)
-    bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmPK,
-                       const __grid_constant__ CUtensorMap tmH, const __nv_bfloat16* __restrict__ k, int N, int ntile,
-                       int phi, const float* __restrict__ tau, const float* __restrict__ dztot,
-                       const float* __restrict__ dphik, float* __restrict__ dk, float* __restrict__ dv, int* status,
-                       unsigned long long wait_ns) {
-  using namespace kt;
-  extern __shared__ __align__(1024) uint8_t sm[];
-  if ((smem_u32(sm) & 1023u) != 0) {
-    if (threadIdx.x == 0) report_error(status, SLA_ERR_UNSUPPORTED);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = blockIdx.x % ntile;
-  const int bh = blockIdx.x / ntile;
-  if (tid == 0) {
-    mbar_init(&bars[B_LD], 1);
-    mbar_init(&bars[B_MMA], 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 4) {
-    tmem_alloc(tmem_slot, 256);
-    tmem_relinquish();
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  if (warp == 4) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[B_LD], 98304);
-      tma_load_3d(sm + OFF_V, &tmV16, &bars[B_LD], 0, t * 128, bh);
-      tma_load_3d(sm + OFF_V + 16384, &tmV16, &bars[B_LD], 64, t * 128, bh);
-      tma_load_3d(sm + OFF_PK, &tmPK, &bars[B_LD], 0, t * 128, bh);
-      tma_load_3d(sm + OFF_PK + 16384, &tmPK, &bars[B_LD], 64, t * 128, bh);
-      tma_load_3d(sm + OFF_H, &tmH, &bars[B_LD], 0, 0, bh);
-      tma_load_3d(sm + OFF_H + 16384, &tmH, &bars[B_LD], 64, 0, bh);
-      if (mbar_wait(&bars[B_LD], 0, abort_flag, status, wait_ns)) {
-        tc_fence_after();
-        const uint32_t id1 = idesc_f16(0, 0, 0, 128, 128);
-        const uint32_t id2 = idesc_f16(0, 0, 1, 128, 128);
-        const uint64_t dVd = sdesc_sw128(smem_u32(sm + OFF_V), 16, 1024);
-        const uint64_t dPd = sdesc_sw128(smem_u32(sm + OFF_PK), 16, 1024);
-        const uint64_t dHk = sdesc_sw128(smem_u32(sm + OFF_H), 16, 1024);
-        const uint64_t dHm = sdesc_sw128(smem_u32(sm + OFF_H), 16384, 1024);
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const uint32_t o = ((k8 >> 2) * 16384u + (k8 & 3) * 32u) >> 4;
-          mma_f16_ss(tmem, dVd + o, dHk + o, id1, k8 > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + 128, dPd + o, dHm + k8 * 128u, id2, k8 > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[B_MMA]);
-      } else {
-        mbar_wait_drain(&bars[B_LD], 0);
-      }
-    }
-  } else {
-    const int r = tid, tok = t * 128 + r;
-    const bool valid = tok < N;
-    const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;
-    const bool ok = warp_wait_tc(&bars[B_MMA], 0, abort_flag, status, wait_ns);
-    if (ok) {
-      tc_fence_after();
-      const float it = 1.0f / tau[bh];  // exact: a power of two
-      const float* zt = dztot + static_cast<long long>(bh) * kDPad;
-      const long long row = static_cast<long long>(bh) * N + (valid ? tok : 0);
-      const __nv_bfloat16* kr = k + row * kDPad;
-      const float* pk = dphik + row * kDPad;
-      auto k32 = [&](int cc, float* x) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint4 w = *reinterpret_cast<const uint4*>(kr + 32 * cc + 8 * u);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf162(ww[e]);
-            x[8 * u + 2 * e] = f.x;
-            x[8 * u + 2 * e + 1] = f.y;
-          }
-        }
-      };
-      auto dphi32 = [&](int cc, float* g) {
-        float a1[32];
-        tmem_ld32(tmem + lrow + 32 * cc, a1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) g[c] = a1[c] * it + zt[32 * cc + c] + pk[32 * cc + c];
-      };
-      const bool smx = phi == SLA_PHI_SOFTMAX;
-      float mx = -INFINITY, inv_sum = 0.0f, dot = 0.0f;
-      // warp-uniform: dphi32 reads TMEM with a warp-collective load (rows past N
-      // read row 0 of the head and store nothing)
-      if (smx) {
-        float x[32];
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          k32(cc, x);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, x[c]);
-        }
-        float sum = 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          k32(cc, x);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sum += expf(x[c] - mx);
-        }
-        inv_sum = 1.0f / sum;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float g[32];
-          k32(cc, x);
-          dphi32(cc, g);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) dot = fmaf(expf(x[c] - mx) * inv_sum, g[c], dot);
-        }
-      }
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        float g[32], x[32], a2[32];
-        dphi32(cc, g);
-        tmem_ld32(tmem + lrow + 128 + 32 * cc, a2);
-        tmem_wait_ld();
-        if (valid) {
-          k32(cc, x);
-          float* dkr = dk + row * kDPad + 32 * cc;
-          float* dvr = dv + row * kDPad + 32 * cc;
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            float4 kk4 = *reinterpret_cast<float4*>(dkr + c);
-            float4 vv4 = *reinterpret_cast<float4*>(dvr + c);
-            float o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float xe = x[c + e], ge = g[c + e];
-              o[e] = smx ? expf(xe - mx) * inv_sum * (ge - dot) : ge * (xe > 0.0f ? 1.0f : expf(xe));
-            }
-            kk4.x += o[0];
-            kk4.y += o[1];
-            kk4.z += o[2];
-            kk4.w += o[3];
-            vv4.x += a2[c] * it;
-            vv4.y += a2[c + 1] * it;
-            vv4.z += a2[c + 2] * it;
-            vv4.w += a2[c + 3] * it;
-            *reinterpret_cast<float4*>(dkr + c) = kk4;
-            *reinterpret_cast<float4*>(dvr + c) = vv4;
-          }
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 4) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 256);
-  }
 }
 
 // One warp per (bh, query block): dalpha = its rows' dO . (O_s - O_l), lane-strided then a fixed tree.
@@ -1046,11 +1028,10 @@ BwdTcLayout bwd_tc_layout(const sla_shape& s) {
   L.phiq = take(BH * N * kDPad * 2);
   L.inv = take(BH * nkv * nq * 4);
   L.inv_n = take(BH * nkv * 4);
-  L.dhpart = take(BH * nq * kDPad * kDPad * 4);
+  L.dhpart = take(BH * nq * kDPad * kDPad * 2);
   L.dzpart = take(BH * nq * kDPad * 4);
   L.dhtot = take(BH * kDPad * kDPad * 4);
   L.dztot = take(BH * kDPad * 4);
-  L.dphik = take(BH * N * kDPad * 4);
   L.dh16 = take(BH * kDPad * kDPad * 2);
   L.tau = take(BH * 4);
   L.total = off;
@@ -1147,43 +1128,38 @@ cudaError_t launch_backward_tc(const sla_shape& s, const void* q, const void* k,
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.dphik = reinterpret_cast<float*>(ws + L.dphik);
-  a.dhpart = reinterpret_cast<float*>(ws + L.dhpart);
+  a.dhpart = reinterpret_cast<__half*>(ws + L.dhpart);
   a.dzpart = reinterpret_cast<float*>(ws + L.dzpart);
   a.status = reinterpret_cast<int*>(ws + L.fwd.status);
   a.wait_ns = kWaitLimitNs;
+  float* dhtot = reinterpret_cast<float*>(ws + L.dhtot);
+  float* dztot = reinterpret_cast<float*>(ws + L.dztot);
+  __half* dh16 = reinterpret_cast<__half*>(ws + L.dh16);
+  float* tau = reinterpret_cast<float*>(ws + L.tau);
+  a.dztot = dztot;
+  a.tau = tau;
 
-  // 2. dQ per query tile; dH_i, dZ_i partials
+  // 2. dQ per query tile; the tiles' -sigma dH_i (fp16) and dZ_i
   if ((e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM)) != cudaSuccess)
     return e;
   bwd_dq_kernel<<<static_cast<unsigned>(BH * nq), kTcThreads, dq::SMEM, st>>>(mq, mdo, mk, mv, mpk, mh, mpq, a);
-  // 3. kept shares of dK, dV, dphi(K) per key block
+  // 3. dH_tot, dZ_tot (tile order), tau dH_tot in fp16; dalpha
+  dh_reduce_kernel<<<dim3(kDPad * kDPad / 256, BH), 256, 0, st>>>(a.dhpart, a.dzpart, a.sigma, nq, dhtot, dztot);
+  dh_pack_kernel<<<BH, 256, 0, st>>>(dhtot, dh16, tau);
+  const long long ntile = static_cast<long long>(BH) * nq;
+  dalpha_kernel<<<static_cast<unsigned>((ntile * 32 + 255) / 256), 256, 0, st>>>(a.rows, s.N, nq, ntile, dalpha);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 4. dK, dV per key block: the sparse shares over the tiles keeping it, the linear
+  //    shares from the totals minus those tiles' partials
+  CUtensorMap mv16, mdhi, mdh;
+  if ((e = encode_map(&mv16, ws + L.fwd.v16, F16, s.N, BH, 64)) != cudaSuccess) return e;
+  if ((e = encode_map(&mdhi, a.dhpart, F16, kDPad, BH * nq, 128)) != cudaSuccess) return e;
+  if ((e = encode_map(&mdh, dh16, F16, kDPad, BH, 128)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM)) !=
       cudaSuccess)
     return e;
-  bwd_dkv_kernel<<<static_cast<unsigned>(BH * nkv), kTcThreads, dkv::SMEM, st>>>(mq, mdo, mk, mv, mpk, mpq, a);
-  // 4. dH_tot, dZ_tot; dalpha
-  float* dhtot = reinterpret_cast<float*>(ws + L.dhtot);
-  float* dztot = reinterpret_cast<float*>(ws + L.dztot);
-  dh_reduce_kernel<<<dim3(kDPad * kDPad / 256, BH), 256, 0, st>>>(a.dhpart, a.dzpart, nq, dhtot, dztot);
-  const long long ntile = static_cast<long long>(BH) * nq;
-  dalpha_kernel<<<static_cast<unsigned>((ntile * 32 + 255) / 256), 256, 0, st>>>(a.rows, s.N, nq, ntile, dalpha);
-  // 5. the totals' share of every key, on the tensor cores
-  __half* dh16 = reinterpret_cast<__half*>(ws + L.dh16);
-  float* tau = reinterpret_cast<float*>(ws + L.tau);
-  dh_pack_kernel<<<BH, 256, 0, st>>>(dhtot, dh16, tau);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  CUtensorMap mv16, mpk128, mdh;
-  if ((e = encode_map(&mv16, ws + L.fwd.v16, F16, s.N, BH, 128)) != cudaSuccess) return e;
-  if ((e = encode_map(&mpk128, ws + L.fwd.phik, F16, s.N, BH, 128)) != cudaSuccess) return e;
-  if ((e = encode_map(&mdh, dh16, F16, kDPad, BH, 128)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(bwd_keys_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kt::SMEM)) !=
-      cudaSuccess)
-    return e;
-  const int ntk = ceil_div(s.N, 128);
-  bwd_keys_tc_kernel<<<static_cast<unsigned>(BH * ntk), kt::kThreads, kt::SMEM, st>>>(
-      mv16, mpk128, mdh, static_cast<const __nv_bfloat16*>(k), s.N, ntk, phi, tau, dztot, a.dphik, dk, dv, a.status,
-      kWaitLimitNs);
+  bwd_dkv_kernel<<<static_cast<unsigned>(BH * nkv), kTcThreads, dkv::SMEM, st>>>(mq, mdo, mk, mv, mv16, mpk, mdhi,
+                                                                                  mdh, a);
   return cudaGetLastError();
 }
 

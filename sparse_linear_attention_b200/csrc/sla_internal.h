@@ -66,9 +66,8 @@ struct BwdTcLayout {
   size_t rows = 0;            // fp32 [BH * N, 8]: lse2, D, s, dden, dalpha share
   size_t phiq = 0;            // fp16 [BH, N, 128]
   size_t inv = 0, inv_n = 0;  // int32 [BH, n_kv, n_q], [BH, n_kv]
-  size_t dhpart = 0, dzpart = 0;  // fp32 [BH * n_q, 128, 128], [BH * n_q, 128]
+  size_t dhpart = 0, dzpart = 0;  // fp16 [BH * n_q, 128, 128] = -sigma dH_i, fp32 [BH * n_q, 128] = dZ_i
   size_t dhtot = 0, dztot = 0;    // fp32 [BH, 128, 128], [BH, 128]
-  size_t dphik = 0;           // fp32 [BH, N, 128]: kept blocks' share of dL/dphi(K)
   size_t dh16 = 0, tau = 0;   // fp16 [BH, 128, 128] = tau dH_tot; fp32 [BH] power-of-two scale tau
   size_t total = 0;
 };

@@ -24,12 +24,6 @@ cudaError_t launch_backward(const sla_shape& s, const void* q, const void* k, co
                             const int32_t* kept, int k_keep, const float* alpha, int phi, float* dq, float* dk,
                             float* dv, float* dalpha, char* ws, cudaStream_t st);
 
-// The per-key step of the backward (backward.cu): with dk, dv holding the
-// kept blocks' shares, adds the totals' share: dphi(k) = dphik + dH_tot v +
-// dZ_tot, dv += dH_tot^T phi(k), dk += phi'(k) dphi(k).
-cudaError_t launch_bwd_keys(const sla_shape& s, const void* k, const void* v, int phi, const float* dhtot,
-                            const float* dztot, const float* dphik, float* dk, float* dv, cudaStream_t st);
-
 // The tensor-core SLA2 backward (backward_tc.cu) for bf16 inputs, d = 128,
 // b_q = 128: same arguments as launch_backward, its own workspace layout.
 BwdTcLayout bwd_tc_layout(const sla_shape& s);

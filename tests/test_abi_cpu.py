@@ -224,8 +224,8 @@ def test_backward_workspace_layout():
     [BH, N, 128] fp32 key-side buffer, each rounded up to 256 bytes.
     Tensor-core path (bf16, d = 128, b_q = 128): the forward's SLA2 workspace,
     then the per-row statistics, phi(Q) in fp16, the inverse block lists, the
-    dH / dZ partials per query tile, dH_tot, dZ_tot, the key-side buffer, and
-    the fp16 copy of dH_tot with its per-head scale."""
+    dH (fp16) / dZ partials per query tile, dH_tot, dZ_tot, and the fp16 copy
+    of dH_tot with its per-head scale."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
     for B, H, N, d, dt in [(1, 12, 32760, 64, sla.SLA_BF16), (2, 3, 1000, 64, sla.SLA_BF16), (1, 1, 1, 8, sla.SLA_F32),
                            (1, 40, 75600, 128, sla.SLA_F32)]:
@@ -237,8 +237,8 @@ def test_backward_workspace_layout():
         s = _shape(B=B, H=H, N=N, d=128, bq=128, in_dtype=sla.SLA_BF16)
         BH, nq, nkv = B * H, -(-N // 128), -(-N // 64)
         want = (sla.sla_workspace_size(s, sla.SLA_MODE_SLA2_TOPK) + a256(BH * N * 32) + a256(BH * N * 256)
-                + a256(BH * nkv * nq * 4) + a256(BH * nkv * 4) + a256(BH * nq * 65536) + a256(BH * nq * 512)
-                + a256(BH * 65536) + a256(BH * 512) + a256(BH * N * 512) + a256(BH * 32768) + a256(BH * 4))
+                + a256(BH * nkv * nq * 4) + a256(BH * nkv * 4) + a256(BH * nq * 32768) + a256(BH * nq * 512)
+                + a256(BH * 65536) + a256(BH * 512) + a256(BH * 32768) + a256(BH * 4))
         assert sla.sla2_attn_bwd_workspace_size(s) == want, (B, H, N)
 
 

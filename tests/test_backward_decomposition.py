@@ -439,3 +439,83 @@ def test_tensor_core_arrangement_matches_oracle(N, d, bq, kk, kind):
     got = _tensor_core_arrangement(q, k, v, kept, alpha, do, bq, bkv, kind)
     for name in ref:
         assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
+
+
+def _key_block_linear_from_tile_partials(q, k, v, kept, alpha, do, bq, bkv, kind):
+    """The key side regrouped around the query tiles' linear partials: with
+    dH_i = phi(Q_i)^T (s dO_i) and dZ_i = phi(Q_i)^T dden_i per query tile i and
+    M_j = dH_tot - sum over the tiles i keeping key block j of dH_i,
+      dV_j    = sum_i (alpha_i P_ij)^T dO_i + phi(K_j) M_j
+      dphi(K_j) = V_j M_j^T + dZ_tot - sum_i dZ_i
+      dK_j    = sum_i dS_ij^T Q_i / sqrt(d) + phi'(K_j) dphi(K_j)
+    so the key-major pass needs only S, G, dS and P; the linear part comes from
+    the partials.  dQ as before (query-major)."""
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    kk = kept.shape[-1]
+    base = _tensor_core_arrangement(q, k, v, kept, alpha, do, bq, bkv, kind)  # dq, dalpha
+    dk, dv = np.zeros(k.shape), np.zeros(v.shape)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK, PQ = _phi(K, kind), _phi(Q, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            keys_of = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in range(nkv)]
+            lse, D, s, dd = np.zeros(N), np.zeros(N), np.zeros(N), np.zeros(N)
+            dH_i, dZ_i = [], []
+            for i in range(nq):
+                rows = np.arange(i * bq, min((i + 1) * bq, N))
+                a = alpha[b, h, i]
+                ks = np.concatenate([keys_of[j] for j in kept[b, h, i]]) if kk else np.zeros(0, int)
+                Os = np.zeros((len(rows), d))
+                if len(ks):
+                    S = sc * Q[rows] @ K[ks].T
+                    mx = S.max(1)
+                    lse[rows] = mx + np.log(np.exp(S - mx[:, None]).sum(1))
+                    Os = np.exp(S - lse[rows][:, None]) @ V[ks]
+                if kk < nkv:
+                    A = PQ[rows] @ PK[ks].T if len(ks) else np.zeros((len(rows), 0))
+                    den = PQ[rows] @ Zt - A.sum(1)
+                    Ol = (PQ[rows] @ Ht - A @ V[ks]) / den[:, None]
+                    s[rows] = (1 - a) / den
+                    dd[rows] = -(1 - a) * (G[rows] * Ol).sum(1) / den
+                D[rows] = a * (G[rows] * Os).sum(1)
+                dH_i.append(PQ[rows].T @ (s[rows][:, None] * G[rows]))
+                dZ_i.append(PQ[rows].T @ dd[rows])
+            dHt, dZt = np.sum(dH_i, axis=0), np.sum(dZ_i, axis=0)
+            for j in range(nkv):
+                ks = keys_of[j]
+                users = [i for i in range(nq) if j in set(int(x) for x in kept[b, h, i])]
+                M = dHt - sum((dH_i[i] for i in users), np.zeros((d, d)))
+                z = dZt - sum((dZ_i[i] for i in users), np.zeros(d))
+                dvj = PK[ks] @ M
+                dkj = np.zeros((len(ks), d))
+                for i in users:
+                    rows = np.arange(i * bq, min((i + 1) * bq, N))
+                    a = alpha[b, h, i]
+                    P = np.exp(sc * Q[rows] @ K[ks].T - lse[rows][:, None])
+                    dS = P * (a * (G[rows] @ V[ks].T) - D[rows][:, None])
+                    dvj += (a * P).T @ G[rows]
+                    dkj += sc * dS.T @ Q[rows]
+                dphi = V[ks] @ M.T + z[None, :]
+                dv[b, h, ks] = dvj
+                dk[b, h, ks] = dkj + _phi_grad(K[ks], dphi, kind)
+    return {"dq": base["dq"], "dk": dk, "dv": dv, "dalpha": base["dalpha"]}
+
+
+@pytest.mark.parametrize("N,d,bq,kk,kind", [(300, 16, 128, 2, "elu1"), (333, 8, 128, 3, "softmax"),
+                                            (130, 16, 128, 0, "elu1"), (256, 16, 128, 4, "elu1")])
+def test_key_side_from_tile_partials_matches_oracle(N, d, bq, kk, kind):
+    rng = np.random.default_rng(13 * N + kk)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kk = min(kk, nkv)
+    kept = np.array([[[np.sort(rng.choice(nkv, kk, replace=False)) for _ in range(nq)] for _ in range(H)]])
+    kept = kept.reshape(1, H, nq, kk)
+    alpha = rng.uniform(0.1, 0.9, (1, H, nq))
+    ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
+    got = _key_block_linear_from_tile_partials(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
