@@ -365,9 +365,9 @@ def backward_leg(args, w, dev, stream):
     achieved = flops / (ms * 1e-3) / 1e12
     # the SLA2 backward of bf16 inputs at d = 128, b_q = 128 runs on the tensor cores:
     # prepare (3), the attention kernel with its statistics epilogue, phi(Q), the
-    # inverse lists, dQ, dK/dV, the dH reduction, dalpha, the dH packing, the per-key step
+    # inverse lists, dQ, the dH reduction, the dH packing, dalpha, dK/dV
     tc_path = (not sla_mode) and w.dtype == "bf16" and w.d == 128 and w.bq == 128
-    launches = 6 if sla_mode else (12 if tc_path else 3)
+    launches = 6 if sla_mode else (11 if tc_path else 3)
     metric = ("SLA backward ms @Wan-1.3B shape (sla_attn_bwd: dQ, dK, dV, dW_proj)" if sla_mode else
               "SLA2 backward ms @Wan-1.3B shape (sla2_attn_bwd: dQ, dK, dV, dalpha)")
     keep_txt = f"critical={k} negligible={k_neg}/{w.n_kv}" if sla_mode else f"keep={k}/{w.n_kv}"
