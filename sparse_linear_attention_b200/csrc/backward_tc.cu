@@ -5,13 +5,17 @@
 // Transformers …" (papernotes.org) 关键设计 4: the sparse part back-propagated
 // the FlashAttention way, the linear part through dH_i, dZ_i written as totals
 // minus the kept blocks; "SLA2 深度解读 …" (jefxiong.cn) §07: gradients on
-// the unquantised inputs), with A_j = phi(Q) phi(K_j)^T, G_j = dO V_j^T,
-// s = (1 - alpha) / den, dden = -(1 - alpha) dO . O_l / den:
-//   dS_j = P_j * (alpha G_j - D),  Bx_j = s G_j + dden,  C_j = alpha P_j - s A_j
+// the unquantised inputs), with G_j = dO V_j^T, s = (1 - alpha) / den,
+// dden = -(1 - alpha) dO . O_l / den, per query tile i: dH_i = phi(Q_i)^T (s dO_i),
+// dZ_i = phi(Q_i)^T dden_i:
+//   dS_j = P_j * (alpha G_j - D),  Bx_j = s G_j + dden
 //   dQ   = dS K / sqrt(d) + phi'(Q) [ s dO H_tot^T + dden Z_tot^T - sum_j Bx_j phi(K_j) ]
-//   dK_j = dS_j^T Q / sqrt(d),  dV_j = C_j^T dO,  dphi(K_j) = -Bx_j^T phi(Q)  (kept shares)
-//   dH_tot = sum phi(Q)^T (s dO),  dZ_tot = sum phi(Q)^T dden
-// and the per-key step of backward.cu for the totals' share.
+//   dH_tot = sum_i dH_i,  dZ_tot = sum_i dZ_i
+// and per key block j, with M_j = dH_tot - sum of dH_i over the tiles i keeping j
+// (the kept blocks' linear share regrouped through the tiles' partials):
+//   dV_j = sum_i (alpha P_ij)^T dO_i + phi(K_j) M_j
+//   dphi(K_j) = V_j M_j^T + dZ_tot - sum_i dZ_i
+//   dK_j = sum_i dS_ij^T Q_i / sqrt(d) + phi'(K_j) dphi(K_j)
 //
 // The per-row quantities (the log2-sum-exp of the kept scores, D, s, dden and
 // the row's share of dalpha) come from the attention kernel itself, run once
