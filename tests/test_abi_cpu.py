@@ -338,5 +338,11 @@ def test_binding_refuses_host_tensors():
         sla.sla2_attn_fwd(shape, q, q, q, kept, 1, torch.zeros(1, 2, 1), 0, 0, torch.zeros_like(q), ws)
     with pytest.raises(ValueError, match="CUDA tensor"):
         sla.sla_read_device_status(ws)
+    g = torch.zeros(1, 2, 64, 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla2_attn_bwd(shape, q, q, q, kept, 1, torch.zeros(1, 2, 1), 0, q, g, g, g, torch.zeros(1, 2, 1), ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sla.sla_attn_bwd(shape, q, q, q, torch.zeros(1, 2, 1, 1, dtype=torch.int8),
+                         torch.zeros(64, 64, dtype=torch.bfloat16), 0, q, g, g, g, torch.zeros(64, 64), ws)
     with pytest.raises(TypeError):
         sla.sla_route(shape, "q", q, None, None, 0, 1, 0, kept, None, None, ws)
