@@ -16,10 +16,12 @@ critical and negligible blocks both taken out of the linear totals, the
 W_proj gradient) is checked against the oracle's sla_backward; backward.cu
 follows it for SLA.
 
-Two rearrangements of the SLA2 decomposition follow: a key-major one, and the
+Rearrangements of the SLA2 decomposition follow: a key-major one, the
 arrangement of the tensor-core kernels (csrc/backward_tc.cu: statistics from
-the attention kernel, query-major dQ, key-major kept shares, per-tile dH_i
-partials, power-of-two scalings), each in fp64 against the oracle.
+the attention kernel, query-major dQ, per-tile dH_i partials, power-of-two
+scalings), and the key side regrouped through those partials; then the same
+regrouping for SLA's three labels, which a tensor-core SLA backward would
+follow.  Each is checked in fp64 against the oracle.
 """
 import math
 
@@ -517,5 +519,115 @@ def test_key_side_from_tile_partials_matches_oracle(N, d, bq, kk, kind):
     alpha = rng.uniform(0.1, 0.9, (1, H, nq))
     ref = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, kind)
     got = _key_block_linear_from_tile_partials(q, k, v, kept, alpha, do, bq, bkv, kind)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
+
+
+def _sla_key_side_from_tile_partials(q, k, v, labels, wp, do, bq, bkv, kind):
+    """SLA's backward in the arrangement of the tensor-core SLA2 kernels: per
+    query tile i, E_i = dO_i W_proj^T (dO_l), den from the marginal blocks,
+    s = 1 / den, dden = -E . O_l / den, dH_i = phi(Q_i)^T (s E_i), dZ_i =
+    phi(Q_i)^T dden; per key block j, with L_j the tiles for which j is critical
+    or negligible (both leave the linear branch) and C_j those for which it is
+    critical (the softmax), M_j = dH_tot - sum over L_j of dH_i:
+      dV_j = sum over C_j of P_ij^T dO_i + phi(K_j) M_j
+      dphi(K_j) = V_j M_j^T + dZ_tot - sum over L_j of dZ_i
+      dK_j = sum over C_j of dS_ij^T Q_i / sqrt(d) + phi'(K_j) dphi(K_j)
+    with dS = P * (dO V^T - D), D = dO . O_s; dQ query-major as in SLA2 with E
+    for the linear terms; dW_proj = sum O_l^T dO."""
+    B, H, N, d = q.shape
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    sc = 1.0 / math.sqrt(d)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dwp = np.zeros(wp.shape)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = q[b, h], k[b, h], v[b, h], do[b, h]
+            PK, PQ = _phi(K, kind), _phi(Q, kind)
+            Ht, Zt = PK.T @ V, PK.sum(0)
+            keys_of = [np.arange(j * bkv, min((j + 1) * bkv, N)) for j in range(nkv)]
+            lse, D = np.zeros(N), np.zeros(N)
+            dH_i, dZ_i = [], []
+            crit_of, out_of = [], []
+            for i in range(nq):
+                rows = np.arange(i * bq, min((i + 1) * bq, N))
+                lab = labels[b, h, i]
+                crit = [int(j) for j in np.nonzero(lab == 1)[0]]
+                out = [int(j) for j in np.nonzero(lab != 0)[0]]
+                crit_of.append(set(crit))
+                out_of.append(set(out))
+                ks = np.concatenate([keys_of[j] for j in crit]) if crit else np.zeros(0, int)
+                ko = np.concatenate([keys_of[j] for j in out]) if out else np.zeros(0, int)
+                E = G[rows] @ wp.T
+                Os = np.zeros((len(rows), d))
+                if len(ks):
+                    S = sc * Q[rows] @ K[ks].T
+                    mx = S.max(1)
+                    lse[rows] = mx + np.log(np.exp(S - mx[:, None]).sum(1))
+                    Os = np.exp(S - lse[rows][:, None]) @ V[ks]
+                D[rows] = (G[rows] * Os).sum(1)
+                s_r, dd_r = np.zeros(len(rows)), np.zeros(len(rows))
+                Ol = np.zeros((len(rows), d))
+                if len(out) < nkv:
+                    A = PQ[rows] @ PK[ko].T if len(ko) else np.zeros((len(rows), 0))
+                    den = PQ[rows] @ Zt - A.sum(1)
+                    Ol = (PQ[rows] @ Ht - A @ V[ko]) / den[:, None]
+                    s_r = 1.0 / den
+                    dd_r = -(E * Ol).sum(1) / den
+                dwp += Ol.T @ G[rows]
+                dH_i.append(PQ[rows].T @ (s_r[:, None] * E))
+                dZ_i.append(PQ[rows].T @ dd_r)
+                # dQ: the sparse part over the critical blocks, the linear part with E
+                dqs = np.zeros((len(rows), d))
+                dql = s_r[:, None] * (E @ Ht.T) + dd_r[:, None] * Zt[None, :]
+                for j in out:
+                    kj = keys_of[j]
+                    Bx = s_r[:, None] * (E @ V[kj].T) + dd_r[:, None]
+                    dql -= Bx @ PK[kj]
+                    if j in crit_of[i]:
+                        P = np.exp(sc * Q[rows] @ K[kj].T - lse[rows][:, None])
+                        dS = P * (G[rows] @ V[kj].T - D[rows][:, None])
+                        dqs += sc * dS @ K[kj]
+                dq[b, h, rows] = dqs + _phi_grad(Q[rows], dql, kind)
+            dHt, dZt = np.sum(dH_i, axis=0), np.sum(dZ_i, axis=0)
+            for j in range(nkv):
+                ks = keys_of[j]
+                L = [i for i in range(nq) if j in out_of[i]]
+                Cr = [i for i in L if j in crit_of[i]]
+                M = dHt - sum((dH_i[i] for i in L), np.zeros((d, d)))
+                z = dZt - sum((dZ_i[i] for i in L), np.zeros(d))
+                dvj = PK[ks] @ M
+                dkj = np.zeros((len(ks), d))
+                for i in Cr:
+                    rows = np.arange(i * bq, min((i + 1) * bq, N))
+                    P = np.exp(sc * Q[rows] @ K[ks].T - lse[rows][:, None])
+                    dS = P * (G[rows] @ V[ks].T - D[rows][:, None])
+                    dvj += P.T @ G[rows]
+                    dkj += sc * dS.T @ Q[rows]
+                dv[b, h, ks] = dvj
+                dk[b, h, ks] = dkj + _phi_grad(K[ks], V[ks] @ M.T + z[None, :], kind)
+    return {"dq": dq, "dk": dk, "dv": dv, "dwproj": dwp}
+
+
+@pytest.mark.parametrize("N,d,bq,kind,n_crit,n_negl", [(300, 16, 128, "elu1", 1, 1), (333, 8, 128, "softmax", 2, 1),
+                                                        (130, 16, 128, "elu1", 0, 1), (256, 16, 128, "elu1", 2, 2),
+                                                        (256, 16, 128, "elu1", 4, 0)])
+def test_sla_key_side_from_tile_partials_matches_oracle(N, d, bq, kind, n_crit, n_negl):
+    """The same regrouping for SLA's three labels: critical blocks in the
+    softmax, critical and negligible blocks both out of the linear totals,
+    dO_l = dO W_proj^T; no critical block, no marginal block, every block
+    critical."""
+    rng = np.random.default_rng(3 * N + 10 * n_crit + n_negl)
+    H, bkv = 2, 64
+    q, k, v, do = (rng.standard_normal((1, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    labels = np.zeros((1, H, nq, nkv), dtype=np.int8)
+    for h, i in np.ndindex(H, nq):
+        perm = rng.permutation(nkv)
+        labels[0, h, i, perm[:n_crit]] = 1
+        labels[0, h, i, perm[n_crit:n_crit + n_negl]] = -1
+    wp = rng.standard_normal((d, d)) / math.sqrt(d)
+    ref = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv, kind)
+    got = _sla_key_side_from_tile_partials(q, k, v, labels, wp, do, bq, bkv, kind)
     for name in ref:
         assert np.allclose(got[name], ref[name], atol=1e-12, rtol=1e-10), name
