@@ -76,7 +76,6 @@ struct TcArgs {
   const float* ztot;     // [BH, 128]
   const int32_t* inv;    // [BH, nkv, nq] query blocks keeping each key block
   const int32_t* inv_n;  // [BH, nkv]
-  const __nv_bfloat16* q;
   float *dq, *dk, *dv;          // [BH, N, 128]
   __half* dhpart;               // [BH * nq, 128, 128]: -sigma dH_i per query tile
   float* dzpart;                // [BH * nq, 128]: dZ_i per query tile
@@ -974,7 +973,7 @@ __global__ void __launch_bounds__(256) dh_reduce_kernel(const __half* __restrict
 }
 
 // One block per head: tau = a power of two with tau max|dH_tot| < 2^14 (1 if dH_tot = 0)
-// and the fp16 copy tau dH_tot for the per-key products.
+// and the fp16 copy tau dH_tot for the key kernel's totals products.
 __global__ void __launch_bounds__(256) dh_pack_kernel(const float* __restrict__ dhtot, __half* __restrict__ dh16,
                                                       float* __restrict__ tau) {
   __shared__ float red[8];
@@ -1128,7 +1127,6 @@ cudaError_t launch_backward_tc(const sla_shape& s, const void* q, const void* k,
   a.ztot = reinterpret_cast<const float*>(ws + L.fwd.ztot);
   a.inv = inv;
   a.inv_n = inv_n;
-  a.q = static_cast<const __nv_bfloat16*>(q);
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
