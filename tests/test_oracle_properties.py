@@ -89,3 +89,34 @@ def test_soft_topk_budget_and_range(n, k, tau, seed):
     for idx in np.ndindex(1, 1, 2):
         o = np.argsort(s[idx])
         assert np.all(np.diff(m[idx][o]) >= -1e-12)
+
+
+def test_backward_block_shares_add_up():
+    """The backward's blocks= option (the oracle computing the share of some
+    query blocks only, as the full-size GPU checks use it) splits the gradients
+    exactly: the shares of disjoint block sets add up to the full result, for
+    SLA2 and SLA."""
+    g = np.random.default_rng(41)
+    B, H, N, d, bq, bkv = 1, 2, 300, 8, 64, 64
+    q, k, v, do = (g.standard_normal((B, H, N, d)) for _ in range(4))
+    nq, nkv = -(-N // bq), -(-N // bkv)
+    kept = np.stack([np.sort(g.choice(nkv, 2, replace=False)) for _ in range(H * nq)]).reshape(B, H, nq, 2)
+    alpha = g.uniform(0.1, 0.9, (B, H, nq))
+    labels = np.zeros((B, H, nq, nkv), dtype=np.int8)
+    for h, i in np.ndindex(H, nq):
+        perm = g.permutation(nkv)
+        labels[0, h, i, perm[:1]] = 1
+        labels[0, h, i, perm[1:2]] = -1
+    wp = g.standard_normal((d, d)) / np.sqrt(d)
+    all_blocks = [(0, h, i) for h in range(H) for i in range(nq)]
+    first, rest = all_blocks[::2], all_blocks[1::2]
+    full = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv)
+    a = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, blocks=first)
+    b = orc.sla2_backward(q, k, v, kept, alpha, do, bq, bkv, blocks=rest)
+    for name in full:
+        assert np.allclose(a[name] + b[name], full[name], atol=1e-12), name
+    full = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv)
+    a = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv, blocks=first)
+    b = orc.sla_backward(q, k, v, labels, wp, do, bq, bkv, blocks=rest)
+    for name in full:
+        assert np.allclose(a[name] + b[name], full[name], atol=1e-12), name
